@@ -1,0 +1,403 @@
+"""CPU oracle for the BATQuant W4A4 MXFP4 linear path -- TEST INFRASTRUCTURE ONLY.
+
+This is a plain, slow, obviously-correct restatement of what the path
+computes, written from the method's description.  It shares no code with the
+CUDA library and imports nothing from it.  Only the test suite, the smoke
+check and the benchmark's CPU-baseline / reference arm may import it; the
+product path never calls it.
+
+Sources (BATQuant: Outlier-resilient MXFP4 Quantization via Learnable
+Block-wise Optimization, arXiv 2603.16590), cited by page and section:
+
+* [p1] zhaoyang97.github.io daily-arxiv summary, sections "块仿射变换 (BAT)",
+  "Global-Private Kronecker (GPK) 分解", "块级可学习裁剪".
+* [p2] gist.science technical summary ("Résumé Technique"), §2.A-§2.D.
+* [p3] thelatestinai.com page: abstract, Figure 2 and Figure 3 captions,
+  Table 1.
+* MXFP4 element / scale rules: OCP Microscaling Formats (MX) v1.0 (E8M0 shared
+  scale 2^(floor(log2 amax) - emax_elem), emax_elem = 2 for E2M1; E2M1 elements
+  rounded to nearest even and saturated at +-6).  The pages state only that 32
+  elements share one E8M0 scale (p3, DuQuant++ abstract) and that values are
+  divided by the scale before rounding (p3, Figure 2 caption).
+
+Readings taken where the pages are silent (each is listed with its reason in
+the design notes):
+
+* A 32-element block x is reshaped row-major to X in R^{4x8}; with the
+  row-vector convention of Table 1 ("XP") the block transform is
+  y = x . P_i with P_i = B_i (x) A (4x4 private B_i, 8x8 global A).
+* Clip after the transform, with per-block-column ratios sigma(alpha) computed
+  in fp64 and rounded to fp32 once; min/max are per token and block.
+* lo > hi: clamp(y, lo, hi) = min(max(y, lo), hi), so hi wins.
+* All-zero block: scale byte 0x00, codes 0.  Any non-finite transformed value
+  in a block: scale byte 0xFF, codes 0.
+* An exact-zero transformed value is +0 (a sum has no sign of its own).
+* Two E2M1 codes per byte, element 2j in the low nibble; code = sign<<3 | mag.
+* Weights: W' = W . P^{-T} per block, from the fp64 Gauss-Jordan inverse of
+  the dense 32x32 P_i, rounded to fp32, then MXFP4 round-to-nearest along K
+  without clipping.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against
+closed forms, brute force and the pages' Table 1.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+G = 32  # MXFP block size g [p3 Table 1 caption]
+G1 = 8  # size of the global factor A [p3 Table 1 caption; p1 GPK]
+G2 = 4  # size of the private factor B_i [p3 Table 1 caption; p1 GPK]
+
+# E2M1 magnitudes for magnitude codes 0..7 (OCP MX v1.0, FP4 E2M1: bias 1,
+# subnormal 0.5 at exponent 0).
+E2M1_MAGNITUDE = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+# Round-to-nearest-even decision table on |q| (q = value / scale).  Each row
+# is (upper bound, bound included?, magnitude code); the first row whose bound
+# admits |q| gives the code.  Bounds are the midpoints between neighbouring
+# magnitudes; a midpoint belongs to the neighbour with an even code (mantissa
+# bit 0).  Anything above 5 rounds to 6, which also saturates (6, 8) -> 6.
+E2M1_RNE_TABLE = (
+    (0.25, True, 0),
+    (0.75, False, 1),
+    (1.25, True, 2),
+    (1.75, False, 3),
+    (2.5, True, 4),
+    (3.5, False, 5),
+    (5.0, True, 6),
+    (np.inf, True, 7),
+)
+
+
+# ---------------------------------------------------------------------------
+# Table 1: parameter counts of the transform P for each decomposition
+# ---------------------------------------------------------------------------
+
+def param_counts(N: int, g: int = G, g1: int = G1, g2: int = G2) -> dict:
+    """Number of stored parameters of P under each decomposition [p3 Table 1].
+
+    Counted from the shapes of the arrays each decomposition stores:
+    FlatQuant stores two sqrt(N) x sqrt(N) Kronecker factors (2N in Table 1);
+    "w/o" stores k dense g x g blocks; naive Kronecker stores an
+    8x8 and a 4x4 factor per block; GPK stores one shared 8x8 A and one 4x4
+    B_i per block.
+    """
+    k = N // g
+    n_side = int(round(np.sqrt(N)))
+    flat_1 = np.zeros((n_side, n_side))
+    flat_2 = np.zeros((n_side, n_side))
+    dense_blocks = np.zeros((k, g, g))
+    naive_A = np.zeros((k, g1, g1))
+    naive_B = np.zeros((k, g2, g2))
+    gpk_A = np.zeros((g1, g1))
+    gpk_B = np.zeros((k, g2, g2))
+    return {
+        "flatquant": flat_1.size + flat_2.size,
+        "wo": dense_blocks.size,
+        "naive_kronecker": naive_A.size + naive_B.size,
+        "gpk": gpk_A.size + gpk_B.size,
+    }
+
+
+# ---------------------------------------------------------------------------
+# Block-wise affine transform with the GPK decomposition
+# ---------------------------------------------------------------------------
+
+def kron_block(A: np.ndarray, Bi: np.ndarray) -> np.ndarray:
+    """Dense P_i = B_i (x) A, 32x32 in fp64, built entry by entry [p1 GPK; p2 §2.B].
+
+    P_i[8r + a, 8c + b] = B_i[r, c] * A[a, b].
+    """
+    A = np.asarray(A, dtype=np.float64)
+    Bi = np.asarray(Bi, dtype=np.float64)
+    P = np.zeros((G, G), dtype=np.float64)
+    for r in range(G2):
+        for c in range(G2):
+            for a in range(G1):
+                for b in range(G1):
+                    P[G1 * r + a, G1 * c + b] = Bi[r, c] * A[a, b]
+    return P
+
+
+def dense_blocks(A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """All k dense blocks P_i = B_i (x) A, shape (k, 32, 32), fp64 [p1 BAT: P = diag(P_1..P_k)].
+
+    Same entry-by-entry rule as ``kron_block``, applied to every block at once.
+    """
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    k = B.shape[0]
+    P = np.zeros((k, G, G), dtype=np.float64)
+    for r in range(G2):
+        for c in range(G2):
+            for a in range(G1):
+                for b in range(G1):
+                    P[:, G1 * r + a, G1 * c + b] = B[:, r, c] * A[a, b]
+    return P
+
+
+def transform_f64(X: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """y_i = x_i . P_i for every token and block, in fp64 (no rounding) [p3 Table 1 "XP"; p1 BAT]."""
+    X = np.asarray(X, dtype=np.float64)
+    S, N = X.shape
+    k = N // G
+    P = dense_blocks(A, B)
+    Xb = X.reshape(S, k, G).transpose(1, 0, 2)  # (k, S, 32)
+    Y = np.matmul(Xb, P)  # (k, S, 32): row vector times P_i
+    return Y.transpose(1, 0, 2).reshape(S, N)
+
+
+def transform(X: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """Transformed activations, computed in fp64 and rounded to fp32 once.
+
+    Exact zeros are returned as +0.
+    """
+    Y = transform_f64(X, A, B) + 0.0
+    return Y.astype(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# Block-wise learnable clipping
+# ---------------------------------------------------------------------------
+
+def clip_ratios(alpha: np.ndarray) -> np.ndarray:
+    """sigma(alpha) = 1 / (1 + exp(-alpha)) in fp64, rounded to fp32 [p1 块级可学习裁剪; p2 §2.C]."""
+    a = np.asarray(alpha, dtype=np.float64)
+    return (1.0 / (1.0 + np.exp(-a))).astype(np.float32)
+
+
+def clip_blocks(Y: np.ndarray, r_min: np.ndarray, r_max: np.ndarray):
+    """x_hat = clip(y, sigma(a_min) * min(y), sigma(a_max) * max(y)) per token and block [p1 块级可学习裁剪].
+
+    ``Y`` is fp32 (S, N); ``r_min``/``r_max`` are the fp32 ratios per block
+    column.  Returns (Y_hat fp32 (S, N), lo (S, k), hi (S, k), nonfinite (S, k)).
+    lo and hi are single-rounded fp32 products.
+    """
+    Y = np.asarray(Y, dtype=np.float32)
+    S, N = Y.shape
+    k = N // G
+    Yb = Y.reshape(S, k, G)
+    nonfinite = ~np.all(np.isfinite(Yb), axis=2)
+    with np.errstate(invalid="ignore"):
+        mn = Yb.min(axis=2)
+        mx = Yb.max(axis=2)
+        lo = (np.asarray(r_min, np.float64)[None, :] * mn.astype(np.float64)).astype(np.float32)
+        hi = (np.asarray(r_max, np.float64)[None, :] * mx.astype(np.float64)).astype(np.float32)
+        Yh = np.minimum(np.maximum(Yb, lo[:, :, None]), hi[:, :, None])
+    return Yh.reshape(S, N).astype(np.float32), lo, hi, nonfinite
+
+
+# ---------------------------------------------------------------------------
+# MXFP4: shared E8M0 scale and E2M1 elements
+# ---------------------------------------------------------------------------
+
+def e8m0_exponent(amax: np.ndarray) -> np.ndarray:
+    """Shared-scale exponent e = floor(log2 amax) - 2, clamped to [-127, 127] (OCP MX v1.0).
+
+    amax == 0 gives -127.  Uses frexp (amax = m * 2^ex with m in [0.5, 1), so
+    floor(log2 amax) = ex - 1), exact for every finite fp32 value.
+    """
+    a = np.asarray(amax, dtype=np.float64)
+    _, ex = np.frexp(a)
+    e = ex.astype(np.int64) - 1 - 2
+    e = np.where(a == 0.0, -127, e)
+    return np.clip(e, -127, 127)
+
+
+def e2m1_encode(q: np.ndarray) -> np.ndarray:
+    """4-bit E2M1 codes of q (already divided by the shared scale) by table lookup [p3 Figure 2 caption].
+
+    The sign bit (bit 3) is the sign of q, so negative values that round to 0
+    keep the sign (code 0x8).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    mag = np.abs(q)
+    code = np.full(q.shape, -1, dtype=np.int64)
+    for bound, inclusive, c in E2M1_RNE_TABLE:
+        hit = (mag <= bound) if inclusive else (mag < bound)
+        code = np.where((code < 0) & hit, c, code)
+    sign = np.signbit(q).astype(np.int64)
+    return (sign << 3) | code
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    """Value of each 4-bit code."""
+    codes = np.asarray(codes, dtype=np.int64)
+    mag = np.asarray(E2M1_MAGNITUDE, dtype=np.float64)[codes & 7]
+    return np.where(codes & 8, -mag, mag)
+
+
+def pack_nibbles(codes: np.ndarray) -> np.ndarray:
+    """(rows, N) 4-bit codes -> (rows, N/2) bytes; element 2j in the low nibble."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
+    """(rows, N/2) bytes -> (rows, N) 4-bit codes."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    rows, half = packed.shape
+    out = np.empty((rows, 2 * half), dtype=np.uint8)
+    out[:, 0::2] = packed & 0xF
+    out[:, 1::2] = packed >> 4
+    return out
+
+
+def mxfp4_quantize(V: np.ndarray, nonfinite: np.ndarray | None = None):
+    """MXFP4 of fp32 rows V (rows, N): per 32-block scale, divide, round [p3 Figure 2 caption; OCP MX].
+
+    Returns (packed codes (rows, N/2) uint8, scale bytes (rows, N/32) uint8,
+    q (rows, N) fp64 = V / 2^e before rounding).
+    """
+    V = np.asarray(V, dtype=np.float32)
+    rows, N = V.shape
+    k = N // G
+    Vb = V.reshape(rows, k, G).astype(np.float64)
+    if nonfinite is None:
+        nonfinite = ~np.all(np.isfinite(Vb), axis=2)
+    with np.errstate(invalid="ignore"):
+        amax = np.abs(Vb).max(axis=2)
+    amax = np.where(nonfinite, 0.0, amax)
+    e = e8m0_exponent(amax)
+    q = Vb * np.exp2(-e.astype(np.float64))[:, :, None]  # exact: power-of-two scaling in fp64
+    q = np.where(nonfinite[:, :, None], 0.0, q)
+    codes = e2m1_encode(q)
+    scale = (e + 127).astype(np.int64)
+    scale = np.where(nonfinite, 0xFF, scale).astype(np.uint8)
+    return pack_nibbles(codes.reshape(rows, N)), scale, q.reshape(rows, N)
+
+
+def dequantize(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """fp64 values code * 2^(byte - 127); byte 0xFF decodes to NaN."""
+    codes = unpack_nibbles(packed)
+    rows, N = codes.shape
+    k = N // G
+    vals = e2m1_decode(codes).reshape(rows, k, G)
+    s = np.asarray(scales, dtype=np.int64)
+    factor = np.where(s == 0xFF, np.nan, np.exp2((s - 127).astype(np.float64)))
+    return (vals * factor[:, :, None]).reshape(rows, N)
+
+
+# ---------------------------------------------------------------------------
+# Scale-factor layout consumed by the block-scaled tensor-core MMA
+# ---------------------------------------------------------------------------
+
+def mma_scale_offset(row: np.ndarray, kb: np.ndarray, k: int) -> np.ndarray:
+    """Byte offset of scale (row, block column kb) in the 128x4 tiled layout.
+
+    Tiles of 128 rows x 4 block columns (512 bytes) are stored row-tile major;
+    inside a tile, row r and column c sit at (r % 32) * 16 + (r // 32) * 4 + c.
+    """
+    kpad = -(-k // 4) * 4
+    row = np.asarray(row, dtype=np.int64)
+    kb = np.asarray(kb, dtype=np.int64)
+    return ((row // 128) * (kpad // 4) + kb // 4) * 512 + (row % 32) * 16 + ((row // 32) % 4) * 4 + kb % 4
+
+
+def scales_from_mma_layout(buf: np.ndarray, rows: int, k: int) -> np.ndarray:
+    """Read a (rows, k) LINEAR scale matrix back out of the tiled layout buffer."""
+    r, c = np.meshgrid(np.arange(rows), np.arange(k), indexing="ij")
+    return np.asarray(buf, dtype=np.uint8).reshape(-1)[mma_scale_offset(r, c, k)]
+
+
+def mma_layout_bytes(rows: int, k: int) -> int:
+    return (-(-rows // 128) * 128) * (-(-k // 4) * 4)
+
+
+# ---------------------------------------------------------------------------
+# Online activation side: transform + clip + MXFP4 [p2 §2.D; p3 Figure 3 caption]
+# ---------------------------------------------------------------------------
+
+def quant_act(X, A, B, alpha_min, alpha_max) -> dict:
+    """Online activation path for one linear: y = x P_i, clip, MXFP4.
+
+    Returns a dict with Y (fp32 transformed), Y_hat (clipped), codes
+    (S, N/2), scales (S, k) linear, q (fp64 pre-rounding), nonfinite (S, k).
+    """
+    Y = transform(X, A, B)
+    r_min = clip_ratios(alpha_min)
+    r_max = clip_ratios(alpha_max)
+    Yh, lo, hi, nonfinite = clip_blocks(Y, r_min, r_max)
+    codes, scales, q = mxfp4_quantize(Yh, nonfinite)
+    return {"Y": Y, "Y_hat": Yh, "codes": codes, "scales": scales, "q": q,
+            "nonfinite": nonfinite, "lo": lo, "hi": hi}
+
+
+def encode_from_transformed(Y, r_min, r_max) -> dict:
+    """Clip + MXFP4 starting from already-transformed fp32 values (steps after the transform)."""
+    Yh, lo, hi, nonfinite = clip_blocks(Y, r_min, r_max)
+    codes, scales, q = mxfp4_quantize(Yh, nonfinite)
+    return {"Y_hat": Yh, "codes": codes, "scales": scales, "q": q, "nonfinite": nonfinite}
+
+
+# ---------------------------------------------------------------------------
+# Offline weight side [p1 (weights fused offline); p2 §2.D; p3 Figure 3 caption]
+# ---------------------------------------------------------------------------
+
+def gauss_jordan_inverse(P: np.ndarray) -> np.ndarray:
+    """Inverse of a square matrix by Gauss-Jordan elimination with partial pivoting, fp64."""
+    P = np.array(P, dtype=np.float64)
+    n = P.shape[0]
+    aug = np.concatenate([P, np.eye(n)], axis=1)
+    for col in range(n):
+        piv = col + int(np.argmax(np.abs(aug[col:, col])))
+        if aug[piv, col] == 0.0:
+            raise np.linalg.LinAlgError("singular block transform")
+        if piv != col:
+            aug[[col, piv]] = aug[[piv, col]]
+        aug[col] = aug[col] / aug[col, col]
+        for row in range(n):
+            if row != col:
+                aug[row] = aug[row] - aug[row, col] * aug[col]
+    return aug[:, n:]
+
+
+def fuse_weights_f64(W: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """W' = W . P^{-T} block by block, fp64: (x P)(P^{-1} W^T) = x W^T."""
+    W = np.asarray(W, dtype=np.float64)
+    M, N = W.shape
+    k = N // G
+    out = np.empty_like(W)
+    for i in range(k):
+        Pinv = gauss_jordan_inverse(kron_block(A, B[i]))
+        out[:, G * i:G * (i + 1)] = W[:, G * i:G * (i + 1)] @ Pinv.T
+    return out
+
+
+def prepare_weights(W, A, B) -> dict:
+    """Fused weights rounded to fp32, then MXFP4 round-to-nearest along K (no clip)."""
+    Wf = fuse_weights_f64(W, A, B).astype(np.float32)
+    codes, scales, q = mxfp4_quantize(Wf)
+    return {"W_fused": Wf, "codes": codes, "scales": scales, "q": q}
+
+
+# ---------------------------------------------------------------------------
+# W4A4 block-scaled GEMM
+# ---------------------------------------------------------------------------
+
+def gemm(a_codes, a_scales, w_codes, w_scales):
+    """out[s, m] = sum_n deq(a)[s, n] * deq(w)[m, n] in fp64, plus T = sum |a||w| (tolerance scale)."""
+    Da = dequantize(a_codes, a_scales)
+    Dw = dequantize(w_codes, w_scales)
+    out = Da @ Dw.T
+    T = np.abs(Da) @ np.abs(Dw).T
+    return out, T
+
+
+def gemm_rows(a_codes, a_scales, w_codes, w_scales, rows, cols=None):
+    """Sampled outputs: only rows ``rows`` (and optionally columns ``cols``) of the fp64 GEMM."""
+    Da = dequantize(a_codes[rows], a_scales[rows])
+    if cols is None:
+        Dw = dequantize(w_codes, w_scales)
+    else:
+        Dw = dequantize(w_codes[cols], w_scales[cols])
+    return Da @ Dw.T, np.abs(Da) @ np.abs(Dw).T
+
+
+def linear(X, A, B, alpha_min, alpha_max, W):
+    """Whole W4A4 linear: activation path, weight preparation, GEMM."""
+    act = quant_act(X, A, B, alpha_min, alpha_max)
+    wp = prepare_weights(W, A, B)
+    out, T = gemm(act["codes"], act["scales"], wp["codes"], wp["scales"])
+    return out, T, act, wp

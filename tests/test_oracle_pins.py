@@ -1,0 +1,411 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix.
+
+Each test compares the oracle with something other than itself: the pages'
+Table 1 counts, a hand-derived worked example, textbook identities computed a
+different way, brute-force search, exact integer arithmetic.  A plausible slip
+in the oracle (transposed factor, swapped ratios, off-by-one exponent, wrong
+tie rule or nibble order, wrong fusion direction) fails at least one of them.
+"""
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import batq_oracle as O
+from mxfp4_w4a4_post_block_b200 import workloads as WL
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- Table 1 ----
+
+def test_table1_parameter_counts():
+    g = _golden("table1_param_counts.json")
+    got = O.param_counts(**{"N": g["setting"]["N"], "g": g["setting"]["g"],
+                            "g1": g["setting"]["g1"], "g2": g["setting"]["g2"]})
+    assert got == g["counts"]
+
+
+def test_table1_reduction_percentages():
+    g = _golden("table1_param_counts.json")
+    c = O.param_counts(4096)
+    red = g["reduction_percent"]
+    assert round(100 * (1 - c["gpk"] / c["wo"]), 1) == red["gpk_vs_wo"]
+    assert round(100 * (1 - c["gpk"] / c["flatquant"])) == red["gpk_vs_flatquant"]
+    assert round(100 * (1 - c["gpk"] / c["naive_kronecker"])) == red["gpk_vs_naive_kronecker"]
+
+
+def test_swapped_factor_sizes_do_not_reproduce_table1():
+    # A 4x4 global factor with 8x8 private factors would give a different count.
+    assert O.param_counts(4096, g1=4, g2=8)["gpk"] != 2112
+
+
+# ------------------------------------------------------- GPK transform -------
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def test_kron_block_matches_textbook_kronecker():
+    A, Bi = _rand((8, 8), 1), _rand((4, 4), 2)
+    np.testing.assert_array_equal(O.kron_block(A, Bi), np.kron(Bi, A))
+
+
+def test_vec_identity_BtXA_equals_x_times_P():
+    # vec_r(B^T X A) = x (B (x) A) with X the row-major 4x8 reshape of x.
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        A, Bi, x = rng.standard_normal((8, 8)), rng.standard_normal((4, 4)), rng.standard_normal(32)
+        lhs = (Bi.T @ x.reshape(4, 8) @ A).reshape(-1)
+        rhs = x @ O.kron_block(A, Bi)
+        np.testing.assert_allclose(rhs, lhs, rtol=0, atol=1e-13 * np.abs(x).sum() * 10)
+
+
+def test_transform_blockwise_matches_matrix_form():
+    rng = np.random.default_rng(4)
+    S, k = 5, 6
+    X = rng.standard_normal((S, 32 * k))
+    A, B = rng.standard_normal((8, 8)), rng.standard_normal((k, 4, 4))
+    Y = O.transform_f64(X, A, B)
+    for s in range(S):
+        for i in range(k):
+            Xm = X[s, 32 * i:32 * i + 32].reshape(4, 8)
+            np.testing.assert_allclose(Y[s, 32 * i:32 * i + 32], (B[i].T @ Xm @ A).reshape(-1),
+                                       rtol=1e-12, atol=1e-12)
+
+
+def test_unit_vectors_reproduce_rows_of_P():
+    A, Bi = _rand((8, 8), 5), _rand((4, 4), 6)
+    X = np.eye(32)
+    Y = O.transform_f64(X, A, Bi[None])
+    np.testing.assert_array_equal(Y, np.kron(Bi, A))
+
+
+def test_identity_transform_is_exact():
+    X = _rand((7, 128), 7).astype(np.float32)
+    B = np.broadcast_to(np.eye(4), (4, 4, 4))
+    np.testing.assert_array_equal(O.transform(X, np.eye(8), B), X)
+
+
+def test_transform_rounds_fp64_result_once_to_fp32():
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((3, 64)).astype(np.float32)
+    A, B = rng.standard_normal((8, 8)).astype(np.float32), rng.standard_normal((2, 4, 4)).astype(np.float32)
+    exact = np.zeros((3, 64), dtype=object)
+    for s in range(3):
+        for i in range(2):
+            Xm = [[Fraction(float(v)) for v in X[s, 32 * i + 8 * r:32 * i + 8 * r + 8]] for r in range(4)]
+            for c in range(4):
+                for b in range(8):
+                    acc = Fraction(0)
+                    for r in range(4):
+                        for a in range(8):
+                            acc += Fraction(float(B[i, r, c])) * Fraction(float(A[a, b])) * Xm[r][a]
+                    exact[s, 32 * i + 8 * c + b] = acc
+    want = np.array([[np.float32(float(v)) for v in row] for row in exact], dtype=np.float32)
+    got = O.transform(X, A, B)
+    # fp64 summation error is far below fp32 resolution; allow one fp32 ulp for double rounding.
+    ulps = np.abs(got.view(np.int32).astype(np.int64) - want.view(np.int32).astype(np.int64))
+    assert ulps.max() <= 1
+
+
+def test_block_locality():
+    w = WL.tiny(with_w=False)
+    base = O.quant_act(w.x, w.A, w.B, w.alpha_min, w.alpha_max)
+    X2 = w.x.copy()
+    X2[:, 32 * 3:32 * 4] *= -7.5
+    pert = O.quant_act(X2, w.A, w.B, w.alpha_min, w.alpha_max)
+    for i in range(w.k):
+        same = slice(16 * i, 16 * i + 16)
+        if i == 3:
+            continue
+        np.testing.assert_array_equal(pert["codes"][:, same], base["codes"][:, same])
+        np.testing.assert_array_equal(pert["scales"][:, i], base["scales"][:, i])
+
+
+# ------------------------------------------------------------- clipping ------
+
+def test_clip_ratio_values():
+    r = O.clip_ratios(np.array([0.0, 30.0, -30.0, 2.0, -2.0], dtype=np.float32))
+    assert r[0] == np.float32(0.5)
+    assert r[1] == np.float32(1.0)
+    assert 0 < r[2] < 1e-12
+    assert abs(float(r[3]) + float(r[4]) - 1.0) < 1e-7
+    assert r[3] == np.float32(1 / (1 + math.exp(-2.0)))
+
+
+def test_clip_with_unit_ratios_is_noop():
+    Y = _rand((9, 96), 9).astype(np.float32)
+    Yh, lo, hi, nf = O.clip_blocks(Y, np.ones(3, np.float32), np.ones(3, np.float32))
+    np.testing.assert_array_equal(Yh, Y)
+    assert not nf.any()
+
+
+def test_clip_extremes_and_bounds():
+    Y = _rand((11, 64), 10).astype(np.float32) * 5
+    rmin = np.array([0.3, 0.9], np.float32)
+    rmax = np.array([0.6, 0.1], np.float32)
+    Yh, lo, hi, _ = O.clip_blocks(Y, rmin, rmax)
+    Yb, Yhb = Y.reshape(11, 2, 32), Yh.reshape(11, 2, 32)
+    for s in range(11):
+        for i in range(2):
+            mn, mx = Yb[s, i].min(), Yb[s, i].max()
+            assert lo[s, i] == np.float32(float(rmin[i]) * float(mn))
+            assert hi[s, i] == np.float32(float(rmax[i]) * float(mx))
+            assert Yhb[s, i].min() == min(max(mn, lo[s, i]), hi[s, i])
+            assert Yhb[s, i].max() == min(max(mx, lo[s, i]), hi[s, i])
+            assert np.all(Yhb[s, i] >= min(lo[s, i], hi[s, i])) and np.all(Yhb[s, i] <= hi[s, i])
+    # monotone: order preserved
+    o = np.argsort(Yb[0, 0], kind="stable")
+    assert np.all(np.diff(Yhb[0, 0][o]) >= 0)
+
+
+def test_clip_lo_above_hi_gives_constant_hi():
+    Y = np.linspace(1.0, 2.0, 32, dtype=np.float32)[None]
+    Yh, lo, hi, _ = O.clip_blocks(Y, np.array([0.99], np.float32), np.array([0.1], np.float32))
+    assert lo[0, 0] > hi[0, 0]
+    assert np.all(Yh == hi[0, 0])
+
+
+# ------------------------------------------------------ scale + encode -------
+
+def _e2m1_value(code):
+    # E2M1: 1 sign, 2 exponent bits (bias 1), 1 mantissa bit; exponent 0 is subnormal.
+    s, e, m = (code >> 3) & 1, (code >> 1) & 3, code & 1
+    mag = m * 0.5 if e == 0 else 2.0 ** (e - 1) * (1 + m / 2)
+    return -mag if s else mag
+
+
+def test_magnitude_table_matches_format_definition():
+    assert tuple(_e2m1_value(c) for c in range(8)) == O.E2M1_MAGNITUDE
+    np.testing.assert_array_equal(O.e2m1_decode(np.arange(16)), [_e2m1_value(c) for c in range(16)])
+
+
+def _brute_code(q):
+    mags = [abs(_e2m1_value(c)) for c in range(8)]
+    a = abs(q)
+    d = [abs(a - m) for m in mags]
+    best = min(d)
+    cands = [c for c in range(8) if d[c] == best]
+    even = [c for c in cands if c % 2 == 0]
+    c = (even or cands)[0]
+    return (8 if math.copysign(1.0, q) < 0 else 0) | c
+
+
+def _brute_scale_exponent(amax):
+    if amax == 0:
+        return -127
+    e = -160
+    while not (2.0 ** (e + 2) <= amax < 2.0 ** (e + 3)):
+        e += 1
+    return max(-127, min(127, e))
+
+
+def test_encoder_matches_brute_force_nearest_even():
+    pts = [0.0, -0.0]
+    for m in (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0):
+        pts += [m, np.nextafter(m, 0), np.nextafter(m, 10)]
+    pts += list(np.linspace(0, 7.99, 4001))
+    pts = np.array(pts + [-p for p in pts])
+    got = O.e2m1_encode(pts)
+    want = np.array([_brute_code(float(p)) for p in pts])
+    np.testing.assert_array_equal(got, want)
+
+
+def test_scale_exponent_matches_brute_force():
+    rng = np.random.default_rng(11)
+    vals = np.concatenate([
+        np.float32(2.0) ** np.arange(-149, 128, dtype=np.float64),
+        (rng.random(3000) * 10.0 ** rng.uniform(-40, 38, 3000)),
+        [0.0, 1e-45, 3.4e38, 4.0, np.nextafter(4.0, 0), 0.7],
+    ]).astype(np.float32).astype(np.float64)
+    got = O.e8m0_exponent(vals)
+    want = np.array([_brute_scale_exponent(float(v)) for v in vals])
+    np.testing.assert_array_equal(got, want)
+
+
+def test_identity_transform_unit_ratios_is_plain_mxfp4_rtn():
+    rng = np.random.default_rng(12)
+    S, k = 6, 5
+    X = (rng.standard_t(3, (S, 32 * k)) * 10.0 ** rng.uniform(-3, 3, (S, 1))).astype(np.float32)
+    B = np.broadcast_to(np.eye(4, dtype=np.float32), (k, 4, 4))
+    big = np.full(k, 30.0, np.float32)  # sigma(30) rounds to exactly 1.0f
+    out = O.quant_act(X, np.eye(8, dtype=np.float32), B, big, big)
+    codes = O.unpack_nibbles(out["codes"])
+    for s in range(S):
+        for i in range(k):
+            blk = X[s, 32 * i:32 * i + 32].astype(np.float64)
+            e = _brute_scale_exponent(float(np.abs(blk).max()))
+            assert out["scales"][s, i] == e + 127
+            want = [_brute_code(float(v) / 2.0 ** e) for v in blk]
+            assert list(codes[s, 32 * i:32 * i + 32]) == want
+
+
+def test_roundtrip_of_representable_values():
+    for e in range(-20, 21):
+        vals = np.array([_e2m1_value(c) for c in range(16)] * 2, dtype=np.float64) * 2.0 ** e
+        vals[0] = 6.0 * 2.0 ** e  # pin amax so the shared exponent is e
+        packed, scale, _ = O.mxfp4_quantize(vals.astype(np.float32)[None])
+        assert scale[0, 0] == e + 127
+        np.testing.assert_array_equal(O.dequantize(packed, scale)[0], vals)
+
+
+def test_amax_element_encodes_to_magnitude_4_or_6():
+    w = WL.tiny(with_w=False)
+    out = O.quant_act(w.x, w.A, w.B, w.alpha_min, w.alpha_max)
+    codes = O.unpack_nibbles(out["codes"]).reshape(w.S, w.k, 32)
+    Yh = out["Y_hat"].reshape(w.S, w.k, 32)
+    idx = np.abs(Yh).argmax(axis=2)
+    top = np.take_along_axis(codes, idx[:, :, None], axis=2)[:, :, 0] & 7
+    assert np.all((top == 6) | (top == 7))
+
+
+def test_worked_example_bytes():
+    g = _golden("clip_encode_worked_example.json")
+    for blk in g["blocks"]:
+        y = np.zeros(32, np.float32)
+        y[:len(blk["y"])] = blk["y"]
+        Yh, _, _, nf = O.clip_blocks(y[None], np.float32([blk["r_min"]]), np.float32([blk["r_max"]]))
+        packed, scale, _ = O.mxfp4_quantize(Yh, nf)
+        assert int(scale[0, 0]) == blk["scale"]
+        assert list(packed[0]) == blk["bytes"]
+
+
+def test_zero_and_nonfinite_blocks():
+    Y = np.zeros((1, 96), np.float32)
+    Y[0, 32 + 5] = np.inf
+    Y[0, 64 + 9] = np.nan
+    Yh, _, _, nf = O.clip_blocks(Y, np.ones(3, np.float32), np.ones(3, np.float32))
+    packed, scale, _ = O.mxfp4_quantize(Yh, nf)
+    assert list(scale[0]) == [0x00, 0xFF, 0xFF]
+    assert not packed.any()
+
+
+def test_nibble_order():
+    codes = np.arange(16, dtype=np.uint8)[None].repeat(2, 0)
+    packed = O.pack_nibbles(codes)
+    assert packed[0, 0] == 0x10 and packed[0, 7] == 0xFE
+    np.testing.assert_array_equal(O.unpack_nibbles(packed), codes)
+
+
+def test_mma_scale_layout_is_a_bijection():
+    for rows, k in ((16, 8), (128, 4), (300, 10), (2048, 128)):
+        r, c = np.meshgrid(np.arange(rows), np.arange(k), indexing="ij")
+        off = O.mma_scale_offset(r, c, k).reshape(-1)
+        assert len(np.unique(off)) == off.size
+        assert off.max() < O.mma_layout_bytes(rows, k)
+
+
+# ------------------------------------------------------- weight side ---------
+
+def test_gauss_jordan_inverse_matches_kronecker_inverse():
+    rng = np.random.default_rng(13)
+    A = np.eye(8) + 0.3 * rng.standard_normal((8, 8))
+    Bi = np.eye(4) + 0.3 * rng.standard_normal((4, 4))
+    Pinv = O.gauss_jordan_inverse(O.kron_block(A, Bi))
+    np.testing.assert_allclose(Pinv, np.kron(np.linalg.inv(Bi), np.linalg.inv(A)), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(O.kron_block(A, Bi) @ Pinv, np.eye(32), rtol=0, atol=1e-12)
+
+
+def test_singular_transform_rejected():
+    with pytest.raises(np.linalg.LinAlgError):
+        O.gauss_jordan_inverse(O.kron_block(np.eye(8), np.zeros((4, 4))))
+
+
+def test_weight_fusion_invariance_before_quantization():
+    # (X P)(P^{-1} W^T) = X W^T
+    w = WL.tiny()
+    lhs = O.transform_f64(w.x, w.A, w.B) @ O.fuse_weights_f64(w.W, w.A, w.B).T
+    rhs = w.x.astype(np.float64) @ w.W.astype(np.float64).T
+    scale = np.abs(w.x).astype(np.float64) @ np.abs(w.W).astype(np.float64).T
+    assert np.max(np.abs(lhs - rhs) / scale) < 1e-12
+
+
+def test_weight_fusion_direction_matters():
+    w = WL.tiny()
+    rhs = w.x.astype(np.float64) @ w.W.astype(np.float64).T
+    # transpose error on the inverse: W P^{-1} instead of W P^{-T}
+    Wt = np.empty_like(w.W, dtype=np.float64)
+    for i in range(w.k):
+        Pinv = np.linalg.inv(O.kron_block(w.A, w.B[i]))
+        Wt[:, 32 * i:32 * i + 32] = w.W[:, 32 * i:32 * i + 32] @ Pinv
+    bad = O.transform_f64(w.x, w.A, w.B) @ Wt.T
+    assert not np.allclose(bad, rhs, rtol=1e-6)
+
+
+def test_prepare_weights_is_unclipped_rtn_of_fused_weights():
+    w = WL.tiny()
+    wp = O.prepare_weights(w.W, w.A, w.B)
+    Wf = O.fuse_weights_f64(w.W, w.A, w.B).astype(np.float32)
+    np.testing.assert_array_equal(wp["W_fused"], Wf)
+    codes = O.unpack_nibbles(wp["codes"])
+    for m in range(0, w.M, 17):
+        for i in range(w.k):
+            blk = Wf[m, 32 * i:32 * i + 32].astype(np.float64)
+            e = _brute_scale_exponent(float(np.abs(blk).max()))
+            assert wp["scales"][m, i] == e + 127
+            assert list(codes[m, 32 * i:32 * i + 32]) == [_brute_code(float(v) / 2.0 ** e) for v in blk]
+
+
+# -------------------------------------------------------------- GEMM ---------
+
+def _exact_dot(ca, sa, cw, sw):
+    """Exact sum of products of E2M1 values with E8M0 scales as a Fraction."""
+    total = Fraction(0)
+    for n in range(len(ca)):
+        va = Fraction(_e2m1_value(int(ca[n]))) * Fraction(2) ** (int(sa[n // 32]) - 127)
+        vw = Fraction(_e2m1_value(int(cw[n]))) * Fraction(2) ** (int(sw[n // 32]) - 127)
+        total += va * vw
+    return total
+
+
+def test_gemm_brute_force_tiny_shapes():
+    rng = np.random.default_rng(14)
+    for S, M in ((1, 1), (2, 3), (4, 4)):
+        a = rng.integers(0, 256, (S, 32), dtype=np.uint8)
+        b = rng.integers(0, 256, (M, 32), dtype=np.uint8)
+        sa = rng.integers(110, 140, (S, 2), dtype=np.uint8)
+        sb = rng.integers(110, 140, (M, 2), dtype=np.uint8)
+        out, T = O.gemm(a, sa, b, sb)
+        ca, cb = O.unpack_nibbles(a), O.unpack_nibbles(b)
+        for s in range(S):
+            for m in range(M):
+                ex = _exact_dot(ca[s], sa[s], cb[m], sb[m])
+                assert out[s, m] == float(ex)
+                tt = sum(abs(_e2m1_value(int(ca[s, n])) * _e2m1_value(int(cb[m, n]))) *
+                         2.0 ** (int(sa[s, n // 32]) + int(sb[m, n // 32]) - 254) for n in range(64))
+                assert T[s, m] == tt
+
+
+def test_gemm_exact_on_tiny_config():
+    w = WL.tiny()
+    act = O.quant_act(w.x, w.A, w.B, w.alpha_min, w.alpha_max)
+    wp = O.prepare_weights(w.W, w.A, w.B)
+    out, T = O.gemm(act["codes"], act["scales"], wp["codes"], wp["scales"])
+    ca, cw = O.unpack_nibbles(act["codes"]), O.unpack_nibbles(wp["codes"])
+    rng = np.random.default_rng(15)
+    for s, m in zip(rng.integers(0, w.S, 24), rng.integers(0, w.M, 24)):
+        ex = _exact_dot(ca[s], act["scales"][s], cw[m], wp["scales"][m])
+        assert abs(out[s, m] - float(ex)) <= 1e-15 * T[s, m]
+
+
+def test_gemm_linear_in_codes_order():
+    w = WL.tiny()
+    act = O.quant_act(w.x, w.A, w.B, w.alpha_min, w.alpha_max)
+    wp = O.prepare_weights(w.W, w.A, w.B)
+    out, _ = O.gemm(act["codes"], act["scales"], wp["codes"], wp["scales"])
+    # reverse the block order on both operands: same sums
+    perm = np.arange(w.k)[::-1]
+    ac = act["codes"].reshape(w.S, w.k, 16)[:, perm].reshape(w.S, -1)
+    wc = wp["codes"].reshape(w.M, w.k, 16)[:, perm].reshape(w.M, -1)
+    out2, _ = O.gemm(ac, act["scales"][:, perm], wc, wp["scales"][:, perm])
+    np.testing.assert_allclose(out2, out, rtol=1e-13, atol=1e-13)
