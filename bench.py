@@ -1,0 +1,341 @@
+"""Benchmark of the BATQuant W4A4 linear hot path on B200.
+
+One step = one pass of the whole path over one batch of the Qwen3-8B-shaped
+q_proj prefill workload (S=2048 tokens, N=4096, M=4096, bf16 activations):
+batq_quant_act (GPK transform + clip + MXFP4 into the tcgen05 scale layout)
+followed by batq_gemm_mxfp4 (block-scaled tensor-core GEMM, fp32 out).  The
+weights are prepared offline (untimed), as in the method.
+
+Prints one JSON line.  ``value`` is the step's GEMM-equivalent throughput
+(2*S*N*M flops per step / device step time, summed over ranks); the per-kernel
+numbers (quantiser GB/s, GEMM TFLOP/s, their roofline fractions) ride along.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl batq|reference]
+
+Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no data-path
+collective); times are the max over ranks.  ``--impl reference`` times the CPU
+oracle on a bounded sample of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BAT+clip+MXFP4 quant GB/s & W4A4 GEMM TFLOPS (% of HBM / FP4 roofline)"
+WORKLOAD = "q_proj prefill S=2048 N=4096 M=4096 (Qwen3-8B-shaped), bf16 X, W4A4 MXFP4"
+QUANT_BYTES_PER_ELEM = 2 + 0.5 + 1.0 / 32  # bf16 in, E2M1 codes + E8M0 scales out
+FP4_NOMINAL_OVER_BF16 = 9.0 / 2.25         # dense fp4 / dense bf16 nominal ratio
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML during the timed region."""
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self._h = None
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_power_brake": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while True:
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for n, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(n)
+            except Exception:  # noqa: BLE001
+                pass
+            if self._stop.wait(0.005):
+                break
+
+    def __enter__(self):
+        if self._h is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _oracle_step(w, rows, wp):
+    from oracle import batq_oracle as O
+    x = w.x[rows]
+    act = O.quant_act(x, w.A, w.B, w.alpha_min, w.alpha_max)
+    out, _ = O.gemm(act["codes"], act["scales"], wp["codes"], wp["scales"])
+    return out
+
+
+def _cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, wp, budget_s=12.0):
+    """Oracle timed on this host on a bounded sample of the workload (rows of X)."""
+    flops_per_row = 2.0 * w.N * w.M
+    rows = 64
+    t0 = time.perf_counter()
+    _oracle_step(w, np.arange(rows), wp)
+    t1 = time.perf_counter() - t0
+    rows = int(min(w.S, max(64, rows * budget_s / max(t1, 1e-3) * 0.5)))
+    t0 = time.perf_counter()
+    _oracle_step(w, np.arange(rows), wp)
+    dt = time.perf_counter() - t0
+    return {"value": rows * flops_per_row / dt / 1e12, "unit": "TFLOP/s", "cores": _cpu_cores(), "kind": "oracle",
+            "sample": f"{rows} of {w.S} tokens of the q_proj workload (quant_act + fp64 GEMM against all "
+                      f"{w.M} prepared weight rows), {dt:.2f} s"}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    from mxfp4_w4a4_post_block_b200 import workloads as WL
+    from oracle import batq_oracle as O
+    w = WL.q_proj()
+    wp = O.prepare_weights(w.W, w.A, w.B)
+    t0 = time.perf_counter()
+    _oracle_step(w, np.arange(16), wp)
+    t_row = (time.perf_counter() - t0) / 16
+    rows = int(max(1, min(w.S, 150.0 / (args.steps + args.warmup) / max(t_row, 1e-6))))
+    for i in range(args.warmup):
+        _oracle_step(w, np.arange(rows), wp)
+    times = []
+    for i in range(args.steps):
+        r0 = (i * rows) % max(1, w.S - rows + 1)
+        t0 = time.perf_counter()
+        _oracle_step(w, np.arange(r0, r0 + rows), wp)
+        times.append(time.perf_counter() - t0)
+    t = sum(times) / len(times)
+    value = rows * 2.0 * w.N * w.M / t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample_rows_per_step": rows},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cpu_cores(), "kind": "oracle",
+                             "sample": f"{rows} of {w.S} tokens per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_batq(args):
+    import torch
+    import torch.distributed as dist
+
+    from mxfp4_w4a4_post_block_b200 import batq as BQ
+    from mxfp4_w4a4_post_block_b200 import workloads as WL
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    w = WL.q_proj(seed=2 + rank)
+    S, N, M = w.S, w.N, w.M
+    dev = torch.device("cuda", local)
+    X = torch.from_numpy(np.ascontiguousarray(w.x_bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    B = torch.from_numpy(np.ascontiguousarray(w.B.reshape(-1))).to(dev)
+    ratios = torch.from_numpy(BQ.batq_clip_ratios(w.alpha_min, w.alpha_max)).to(dev)
+    Wd = torch.from_numpy(w.W).to(dev)
+    wc, wsc = BQ.empty_act_buffers(M, N, device=dev)
+    pws = torch.empty(BQ.batq_prepare_workspace_size(N), dtype=torch.uint8, device=dev)
+    BQ.batq_prepare_weights(Wd, w.A, w.B, wc, wsc, pws)
+    del Wd
+    codes, scales = BQ.empty_act_buffers(S, N, device=dev)
+    out = torch.empty((S, M), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    def step():
+        BQ.batq_quant_act(X, w.A, B, ratios, codes, scales, BQ.BATQ_SCALES_MMA, stream=sp)
+        BQ.batq_gemm_mxfp4(codes, scales, wc, wsc, S, M, N, out, stream=sp)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert BQ.batq_device_error() == 0
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()  # L2 flush between timed steps (not inside the timed interval)
+            ev[i][0].record(stream)
+            BQ.batq_quant_act(X, w.A, B, ratios, codes, scales, BQ.BATQ_SCALES_MMA, stream=sp)
+            ev[i][1].record(stream)
+            BQ.batq_gemm_mxfp4(codes, scales, wc, wsc, S, M, N, out, stream=sp)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    t_quant = [e[0].elapsed_time(e[1]) for e in ev]
+    t_gemm = [e[1].elapsed_time(e[2]) for e in ev]
+    t_step = [a + b for a, b in zip(t_quant, t_gemm)]
+    local_ms = float(np.mean(t_step))
+    q_ms, g_ms = float(np.mean(t_quant)), float(np.mean(t_gemm))
+    if ws > 1:
+        tt = torch.tensor([local_ms, q_ms, g_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        local_ms, q_ms, g_ms = [float(v) for v in tt.tolist()]
+    assert BQ.batq_device_error() == 0
+
+    # end to end through the public call with host buffers (pinned), copies inside the timed region
+    Xh = X.cpu().pin_memory()
+    outh = torch.empty((S, M), dtype=torch.float32).pin_memory()
+    Xd = torch.empty_like(X)
+    lws = torch.empty(BQ.batq_linear_workspace_size(S, N), dtype=torch.uint8, device=dev)
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        Xd.copy_(Xh, non_blocking=True)
+        BQ.batq_linear(Xd, w.A, B, ratios, wc, wsc, M, lws, out, stream=sp)
+        outh.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if ws > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    flops = 2.0 * S * N * M
+    qbytes = S * N * QUANT_BYTES_PER_ELEM
+    peaks = _peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_NOMINAL_OVER_BF16
+    gemm_tflops = flops / (g_ms * 1e-3) / 1e12
+    quant_gbs = qbytes / (q_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": ws * flops / (local_ms * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": local_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "S": S, "N": N, "M": M, "l2": "flushed between steps (256 MB write)",
+                   "parallelism": f"replicas x{ws} (independent batches)"},
+        "quant_gbs": quant_gbs,
+        "quant_ms": q_ms,
+        "gemm_tflops": gemm_tflops,
+        "gemm_ms": g_ms,
+        "tokens_per_s": ws * S / (local_ms * 1e-3),
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / fp4_peak, "traffic": None,
+                     "kernel": "k_gemm_mxfp4",
+                     "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16)"},
+        "roofline_quant": {"bound": "hbm", "achieved": quant_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": quant_gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "k_quant_act"},
+        "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(X.numel() * X.element_size()),
+                "d2h_bytes_per_step": int(out.numel() * out.element_size()), "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        from oracle import batq_oracle as O
+        wp = O.prepare_weights(w.W, w.A, w.B)
+        line["cpu_baseline"] = cpu_baseline(w, wp)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description="BATQuant W4A4 linear benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["batq", "reference"], default="batq")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_batq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

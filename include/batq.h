@@ -1,0 +1,196 @@
+/*
+ * libbatq -- BATQuant W4A4 MXFP4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The method: BATQuant (arXiv 2603.16590), "BATQuant: Outlier-resilient MXFP4
+ * Quantization via Learnable Block-wise Optimization".  Before every linear
+ * layer each 32-element MXFP block x_i of a token is transformed by a
+ * block-wise affine matrix P_i = B_i (x) A (Global-Private Kronecker
+ * decomposition: one 8x8 A shared by all blocks, one private 4x4 B_i per
+ * block), clipped to [sigma(a_i_min) min, sigma(a_i_max) max] and quantized to
+ * MXFP4; the weight-side inverse transform is fused into the weights offline.
+ *   - block-wise affine transform, GPK: daily-arxiv summary page
+ *     (zhaoyang97.github.io), sections "块仿射变换 (BAT)" and "GPK 分解";
+ *     gist.science technical summary, sections 2.A and 2.B.
+ *   - clip: daily-arxiv summary, section "块级可学习裁剪"; gist.science 2.C.
+ *   - weights fused offline, activation transform + clip online:
+ *     thelatestinai.com page, Figure 3 caption; gist.science 2.D.
+ *   - cost of the activation transform O(SN(g1+g2)): thelatestinai.com
+ *     page, Table 1.
+ *   - MXFP4 rules (E8M0 shared scale 2^(floor(log2 amax) - 2), E2M1 elements
+ *     rounded to nearest even and saturated at +-6): OCP Microscaling
+ *     Formats v1.0; the pages state the 32-element shared E8M0 scale and the
+ *     divide-then-round order (thelatestinai.com page, Figure 2 caption).
+ *
+ * Conventions for every call:
+ *   - All pointers named *_dev, and X / W / codes / scales / out / workspace,
+ *     are DEVICE pointers owned by the caller.  The library never allocates
+ *     device memory and never synchronises on the compute calls.
+ *   - Pointers named *_host are host pointers, read during the call only.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Compute calls are asynchronous and stream-ordered.
+ *   - Every call returns a batq_status.  Argument, shape, alignment and
+ *     architecture errors are reported before anything is launched; a failed
+ *     launch returns BATQ_ERR_CUDA.  No call aborts or prints.
+ *   - Matrices are row-major.  S = tokens, N = in-features (= K), M =
+ *     out-features, k = N / 32 blocks per row.
+ *   - Codes: two E2M1 codes per byte, element 2j in the low nibble; code =
+ *     sign << 3 | magnitude (0, 0.5, 1, 1.5, 2, 3, 4, 6).  A row of N
+ *     elements takes N/2 bytes; rows are packed (row stride N/2 bytes).
+ *   - Scales: one E8M0 byte (2^(byte - 127)) per row and 32-block.
+ *     BATQ_SCALES_LINEAR: rows x k bytes, row-major.
+ *     BATQ_SCALES_MMA: the tiled layout the block-scaled tensor-core MMA
+ *     consumes: rows padded to a multiple of 128 and k to a multiple of 4;
+ *     byte (r, c) at ((r/128)*(kpad/4) + c/4)*512 + (r%32)*16 + ((r/32)%4)*4
+ *     + c%4.  Padding bytes are written as 0x7F.
+ *   - An all-zero block gets scale byte 0x00; a block holding a non-finite
+ *     transformed value gets 0xFF and zero codes.
+ */
+#ifndef BATQ_H
+#define BATQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BATQ_API __attribute__((visibility("default")))
+#else
+#define BATQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BATQ_OK = 0,
+  BATQ_ERR_INVALID_ARG = 1, /* null pointer, bad enum, negative size */
+  BATQ_ERR_SHAPE = 2,       /* N % 64 != 0, S < 1, M % 16 != 0, ld < row length */
+  BATQ_ERR_ALIGNMENT = 3,   /* a device pointer or row stride not 16-byte aligned */
+  BATQ_ERR_SINGULAR = 4,    /* A or some B_i singular / condition number > 1e8 */
+  BATQ_ERR_ARCH = 5,        /* current device is not sm_100 */
+  BATQ_ERR_CUDA = 6,        /* a CUDA runtime / driver call failed */
+  BATQ_ERR_TIMEOUT = 7,     /* a kernel gave up waiting on a barrier (device error word set) */
+  BATQ_ERR_WORKSPACE = 8    /* workspace too small */
+} batq_status;
+
+typedef enum { BATQ_F32 = 0, BATQ_BF16 = 1 } batq_dtype;
+
+typedef enum { BATQ_SCALES_LINEAR = 0, BATQ_SCALES_MMA = 1 } batq_scale_layout;
+
+/* Text for a status code (static storage). */
+BATQ_API const char* batq_status_string(batq_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+BATQ_API int batq_version(void);
+
+/*
+ * Bytes needed for the MXFP4 codes and scales of a rows x N matrix in the
+ * given scale layout (same for activations, rows = S, and weights, rows = M).
+ * Host only; no CUDA call.
+ */
+BATQ_API batq_status batq_act_buffer_sizes(int rows, int N, batq_scale_layout layout,
+                                  size_t* code_bytes, size_t* scale_bytes);
+
+/*
+ * Clip ratios sigma(alpha) = 1 / (1 + exp(-alpha)) per block column
+ * (daily-arxiv summary, section "块级可学习裁剪": the sigmoid keeps the
+ * ratios in (0, 1)).  Evaluated in double precision and rounded to fp32 once.
+ * alpha_min_host, alpha_max_host: k floats each.  ratios_out_host: 2k floats,
+ * interleaved {r_min_0, r_max_0, r_min_1, ...}.  Host only; no CUDA call.
+ */
+BATQ_API batq_status batq_clip_ratios(const float* alpha_min_host, const float* alpha_max_host, int k,
+                             float* ratios_out_host);
+
+/*
+ * Online activation path (daily-arxiv summary, "块仿射变换 (BAT)", "GPK 分解",
+ * "块级可学习裁剪"; thelatestinai.com page, Figure 2 caption): for every token
+ * s and block i, with X_si the row-major 4x8 view of the 32 inputs,
+ *   Y = B_i^T X_si A                       (= x . (B_i (x) A), fp32)
+ *   lo = r_min_i * min(Y), hi = r_max_i * max(Y), Y_hat = min(max(Y, lo), hi)
+ *   e = clamp(floor(log2 max|Y_hat|) - 2, -127, 127), scale byte e + 127
+ *   codes = E2M1_RNE_satfinite(Y_hat * 2^-e)
+ *
+ * X: device, S rows of N elements (x_dtype), row stride ldx elements
+ *    (ldx >= N, ldx * elem_size a multiple of 16, X 16-byte aligned).
+ * A_host: host, 8x8 fp32 row-major (A[a][b] at a*8+b); copied into the launch.
+ * B_dev: device, k x 16 fp32; B_i row-major (B_i[r][c] at 16i + 4r + c).
+ * ratios_dev: device, 2k fp32 from batq_clip_ratios, or NULL for no clip.
+ * codes: device, S x N/2 bytes, 16-byte aligned.
+ * scales: device, batq_act_buffer_sizes(S, N, layout) bytes.
+ * y_debug: device S x N fp32 or NULL; receives the pre-clip Y (tests only).
+ * Errors: BATQ_ERR_SHAPE, BATQ_ERR_ALIGNMENT, BATQ_ERR_ARCH, BATQ_ERR_CUDA.
+ */
+BATQ_API batq_status batq_quant_act(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                           const float* A_host, const float* B_dev, const float* ratios_dev,
+                           uint8_t* codes, uint8_t* scales, batq_scale_layout layout,
+                           float* y_debug, void* stream);
+
+/* Device workspace bytes batq_prepare_weights needs for N in-features. Host only. */
+BATQ_API batq_status batq_prepare_workspace_size(int N, size_t* bytes);
+
+/*
+ * Offline weight side (thelatestinai.com page, Figure 3 caption: weight-side
+ * transforms fused offline into the linear layers).  Since
+ * y = x W^T = (x P)(P^-1 W^T), the fused weights are W' = W P^-T, i.e. per
+ * row and block W'_mat = B_i^-1 W_mat A^-T.  The inverses of A and every B_i
+ * are computed on the host in double precision (partial-pivot Gauss-Jordan);
+ * W' is formed on the device in fp32 and quantized to MXFP4 along K by
+ * round-to-nearest, without clipping.
+ *
+ * W: device, M x N (w_dtype), row stride ldw elements (16-byte aligned rows).
+ * A_host: 8x8 fp32; B_host: k x 16 fp32 (host).
+ * w_codes: device M x N/2 bytes; w_scales: batq_act_buffer_sizes(M, N, layout).
+ * workspace: device, batq_prepare_workspace_size(N) bytes.
+ * Errors: as batq_quant_act, plus BATQ_ERR_SINGULAR (condition number of A or
+ * some B_i above 1e8) and BATQ_ERR_WORKSPACE.  Uses a pageable host->device
+ * copy, so it must not be called during stream capture.
+ */
+BATQ_API batq_status batq_prepare_weights(const void* W, batq_dtype w_dtype, int M, int N, int ldw,
+                                 const float* A_host, const float* B_host,
+                                 uint8_t* w_codes, uint8_t* w_scales, batq_scale_layout layout,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * W4A4 MXFP4 x MXFP4 block-scaled GEMM on the tcgen05 tensor cores with fp32
+ * accumulation in tensor memory:
+ *   out[s][m] = sum_n deq(a)[s][n] * deq(w)[m][n],  deq = E2M1 value * 2^(scale - 127).
+ * a_codes: S x N/2, a_scales: MMA layout for S rows; w_codes: M x N/2,
+ * w_scales: MMA layout for M rows (all device, 16-byte aligned, K-major).
+ * out: device S x M of out_dtype (fp32 or bf16), row stride ldo elements.
+ * Errors: BATQ_ERR_SHAPE (N % 64, M % 16), BATQ_ERR_ALIGNMENT, BATQ_ERR_ARCH,
+ * BATQ_ERR_CUDA.
+ */
+BATQ_API batq_status batq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales,
+                            const uint8_t* w_codes, const uint8_t* w_scales,
+                            int S, int M, int N, batq_dtype out_dtype, void* out, int ldo,
+                            void* stream);
+
+/* Device workspace bytes batq_linear needs (activation codes + MMA-layout scales). Host only. */
+BATQ_API batq_status batq_linear_workspace_size(int S, int N, size_t* bytes);
+
+/*
+ * Whole W4A4 linear: batq_quant_act (MMA scale layout, into the workspace)
+ * followed by batq_gemm_mxfp4 on the same stream.  Arguments as in those
+ * two calls; w_codes / w_scales come from batq_prepare_weights with
+ * BATQ_SCALES_MMA.
+ */
+BATQ_API batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                        const float* A_host, const float* B_dev, const float* ratios_dev,
+                        const uint8_t* w_codes, const uint8_t* w_scales, int M,
+                        void* workspace, size_t workspace_bytes,
+                        batq_dtype out_dtype, void* out, int ldo, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word.  Kernels set bits there when a bounded wait on a barrier gives up
+ * (bit 0: data never arrived; bit 1: a stage was never released; bit 2: an
+ * MMA never completed; bit 3: the accumulator was never drained).
+ * *flags_out receives the word; returns BATQ_ERR_TIMEOUT if it was non-zero.
+ */
+BATQ_API batq_status batq_device_error(void* stream, unsigned int* flags_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BATQ_H */

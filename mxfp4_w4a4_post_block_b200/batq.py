@@ -1,0 +1,164 @@
+"""Python binding of libbatq with the C-ABI's call names (argument marshalling only).
+
+Device buffers are torch CUDA tensors (PyTorch supplies memory and streams);
+every step of the path runs in libbatq's kernels.  A non-OK status raises
+``BatqError``.  Host-side parameters (A, B for weight preparation, alpha for the
+clip ratios) may be numpy arrays or CPU tensors.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import _lib
+from ._lib import (BATQ_BF16, BATQ_F32, BATQ_OK, BATQ_SCALES_LINEAR, BATQ_SCALES_MMA)  # noqa: F401
+
+
+class BatqError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        msg = _lib.load().batq_status_string(status).decode()
+        super().__init__(f"{call}: {msg} (status {status})")
+
+
+def _check(status: int, call: str):
+    if status != BATQ_OK:
+        raise BatqError(status, call)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dev_ptr(t, name):
+    """Raw pointer of a CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not getattr(t, "is_cuda", False):
+        raise TypeError(f"{name} must be a CUDA tensor (libbatq has no CPU path)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_f32(a, count, name):
+    arr = np.ascontiguousarray(np.asarray(a.cpu() if hasattr(a, "cpu") else a, dtype=np.float32)).reshape(-1)
+    if arr.size != count:
+        raise ValueError(f"{name} must hold {count} floats, got {arr.size}")
+    return arr
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return BATQ_BF16
+    if t.dtype == torch.float32:
+        return BATQ_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: bf16 or fp32")
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(_torch().cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ----------------------------------------------------------------- host calls
+
+def batq_version() -> int:
+    return _lib.load().batq_version()
+
+
+def batq_act_buffer_sizes(rows: int, N: int, layout: int = BATQ_SCALES_MMA):
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.load().batq_act_buffer_sizes(rows, N, layout, ctypes.byref(cb), ctypes.byref(sb)),
+           "batq_act_buffer_sizes")
+    return cb.value, sb.value
+
+
+def batq_clip_ratios(alpha_min, alpha_max) -> np.ndarray:
+    amin = np.ascontiguousarray(alpha_min, dtype=np.float32)
+    amax = np.ascontiguousarray(alpha_max, dtype=np.float32)
+    out = np.empty(2 * amin.size, dtype=np.float32)
+    _check(_lib.load().batq_clip_ratios(amin.ctypes.data, amax.ctypes.data, amin.size, out.ctypes.data),
+           "batq_clip_ratios")
+    return out
+
+
+def batq_prepare_workspace_size(N: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_lib.load().batq_prepare_workspace_size(N, ctypes.byref(b)), "batq_prepare_workspace_size")
+    return b.value
+
+
+def batq_linear_workspace_size(S: int, N: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_lib.load().batq_linear_workspace_size(S, N, ctypes.byref(b)), "batq_linear_workspace_size")
+    return b.value
+
+
+# -------------------------------------------------------------- device calls
+
+def batq_quant_act(X, A, B, ratios, codes, scales, layout=BATQ_SCALES_MMA, y_debug=None, stream=None):
+    """Online activation path: transform + clip + MXFP4 of X (S x N) into codes / scales."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    _check(_lib.load().batq_quant_act(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0), a.ctypes.data,
+                                      _dev_ptr(B, "B"), _dev_ptr(ratios, "ratios"), _dev_ptr(codes, "codes"),
+                                      _dev_ptr(scales, "scales"), layout, _dev_ptr(y_debug, "y_debug"),
+                                      _stream(stream)), "batq_quant_act")
+
+
+def batq_prepare_weights(W, A, B_host, w_codes, w_scales, workspace, layout=BATQ_SCALES_MMA, stream=None):
+    """Offline: fuse W P^-T and quantize to MXFP4 along K."""
+    M, N = W.shape
+    a = _host_f32(A, 64, "A")
+    b = _host_f32(B_host, (N // 32) * 16, "B")
+    _check(_lib.load().batq_prepare_weights(_dev_ptr(W, "W"), _dtype_code(W), M, N, W.stride(0), a.ctypes.data,
+                                            b.ctypes.data, _dev_ptr(w_codes, "w_codes"),
+                                            _dev_ptr(w_scales, "w_scales"), layout,
+                                            _dev_ptr(workspace, "workspace"),
+                                            workspace.numel() * workspace.element_size(), _stream(stream)),
+           "batq_prepare_weights")
+
+
+def batq_gemm_mxfp4(a_codes, a_scales, w_codes, w_scales, S, M, N, out, stream=None):
+    """out (S x M, fp32 or bf16) = deq(a) deq(w)^T on the tensor cores."""
+    _check(_lib.load().batq_gemm_mxfp4(_dev_ptr(a_codes, "a_codes"), _dev_ptr(a_scales, "a_scales"),
+                                       _dev_ptr(w_codes, "w_codes"), _dev_ptr(w_scales, "w_scales"), S, M, N,
+                                       _dtype_code(out), _dev_ptr(out, "out"), out.stride(0), _stream(stream)),
+           "batq_gemm_mxfp4")
+
+
+def batq_linear(X, A, B, ratios, w_codes, w_scales, M, workspace, out, stream=None):
+    """Whole W4A4 linear: quantize X online, then the block-scaled GEMM against prepared weights."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    _check(_lib.load().batq_linear(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0), a.ctypes.data,
+                                   _dev_ptr(B, "B"), _dev_ptr(ratios, "ratios"), _dev_ptr(w_codes, "w_codes"),
+                                   _dev_ptr(w_scales, "w_scales"), M, _dev_ptr(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(), _dtype_code(out),
+                                   _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_linear")
+
+
+def batq_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    v = ctypes.c_uint(0)
+    st = _lib.load().batq_device_error(_stream(stream), ctypes.byref(v))
+    if st not in (BATQ_OK, _lib.BATQ_ERR_TIMEOUT):
+        raise BatqError(st, "batq_device_error")
+    return v.value
+
+
+# ------------------------------------------------------- allocation helpers
+
+def empty_act_buffers(rows: int, N: int, layout=BATQ_SCALES_MMA, device="cuda"):
+    """(codes, scales) uint8 CUDA tensors sized for a rows x N matrix."""
+    torch = _torch()
+    cb, sb = batq_act_buffer_sizes(rows, N, layout)
+    codes = torch.empty((rows, N // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty(sb, dtype=torch.uint8, device=device)
+    return codes, scales

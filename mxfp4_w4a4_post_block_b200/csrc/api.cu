@@ -1,0 +1,349 @@
+// extern "C" boundary of libbatq: argument checks, host-side preparation and launches.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "../../include/batq.h"
+#include "host_util.h"
+#include "kernels.h"
+
+namespace {
+
+// Device error word, one per device (set by kernels whose bounded waits gave up).
+__device__ unsigned int g_batq_error_word;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device must be sm_100 (B200 class).  Cached per device.
+batq_status check_arch() {
+  static int state[kMaxDevices] = {0};  // 0 unknown, 1 ok, 2 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BATQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return BATQ_ERR_ARCH;
+  if (state[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return BATQ_ERR_CUDA;
+    state[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return state[dev] == 1 ? BATQ_OK : BATQ_ERR_ARCH;
+}
+
+unsigned* error_word() {
+  static unsigned* cached[kMaxDevices] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_batq_error_word) != cudaSuccess) return nullptr;
+    cached[dev] = static_cast<unsigned*>(p);
+  }
+  return cached[dev];
+}
+
+size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
+
+size_t scale_bytes_for(int rows, int N, batq_scale_layout layout) {
+  const size_t k = (size_t)N / 32;
+  if (layout == BATQ_SCALES_MMA) return round_up((size_t)rows, 128) * round_up(k, 4);
+  return (size_t)rows * k;
+}
+
+batq_status check_mn(int rows, int N) {
+  if (rows < 1 || N < 64 || (N % 64) != 0) return BATQ_ERR_SHAPE;
+  return BATQ_OK;
+}
+
+// Inverse of an n x n matrix (row-major, double) by Gauss-Jordan elimination
+// with partial pivoting; returns false if singular or if the 1-norm condition
+// number exceeds 1e8.
+bool invert(const double* a, double* inv, int n) {
+  std::vector<double> m((size_t)n * 2 * n);
+  double norm_a = 0.0;
+  for (int c = 0; c < n; ++c) {
+    double col = 0.0;
+    for (int r = 0; r < n; ++r) col += std::fabs(a[r * n + c]);
+    norm_a = col > norm_a ? col : norm_a;
+  }
+  for (int r = 0; r < n; ++r) {
+    for (int c = 0; c < n; ++c) {
+      m[(size_t)r * 2 * n + c] = a[r * n + c];
+      m[(size_t)r * 2 * n + n + c] = (r == c) ? 1.0 : 0.0;
+    }
+  }
+  for (int col = 0; col < n; ++col) {
+    int piv = col;
+    for (int r = col + 1; r < n; ++r)
+      if (std::fabs(m[(size_t)r * 2 * n + col]) > std::fabs(m[(size_t)piv * 2 * n + col])) piv = r;
+    const double pv = m[(size_t)piv * 2 * n + col];
+    if (!(std::fabs(pv) > 0.0) || !std::isfinite(pv)) return false;
+    if (piv != col)
+      for (int c = 0; c < 2 * n; ++c) std::swap(m[(size_t)piv * 2 * n + c], m[(size_t)col * 2 * n + c]);
+    for (int c = 0; c < 2 * n; ++c) m[(size_t)col * 2 * n + c] /= pv;
+    for (int r = 0; r < n; ++r) {
+      if (r == col) continue;
+      const double f = m[(size_t)r * 2 * n + col];
+      if (f == 0.0) continue;
+      for (int c = 0; c < 2 * n; ++c) m[(size_t)r * 2 * n + c] -= f * m[(size_t)col * 2 * n + c];
+    }
+  }
+  double norm_inv = 0.0;
+  for (int c = 0; c < n; ++c) {
+    double col = 0.0;
+    for (int r = 0; r < n; ++r) {
+      inv[r * n + c] = m[(size_t)r * 2 * n + n + c];
+      col += std::fabs(inv[r * n + c]);
+    }
+    norm_inv = col > norm_inv ? col : norm_inv;
+  }
+  const double cond = norm_a * norm_inv;
+  return std::isfinite(cond) && cond <= 1e8;
+}
+
+batq_status launch_quant(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
+                         const float* B_dev, const float* ratios_dev, uint8_t* codes, uint8_t* scales,
+                         batq_scale_layout layout, float* y_debug, cudaStream_t stream) {
+  batq::QuantLaunch L;
+  L.X = X;
+  L.bf16 = (x_dtype == BATQ_BF16);
+  L.S = S;
+  L.N = N;
+  L.ldx = ldx;
+  std::memcpy(L.A, A_host, sizeof(L.A));
+  L.B = B_dev;
+  L.ratios = ratios_dev;
+  L.codes = codes;
+  L.scales = scales;
+  L.mma_layout = (layout == BATQ_SCALES_MMA);
+  L.y_debug = y_debug;
+  L.err = error_word();
+  L.stream = stream;
+  cudaError_t e = batq::launch_quant_act(L);
+  if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
+  return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
+}
+
+batq_status check_quant_args(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
+                             const float* B_dev, const float* ratios_dev, const uint8_t* codes,
+                             const uint8_t* scales, batq_scale_layout layout, const float* y_debug) {
+  if (!X || !A_host || !B_dev || !codes || !scales) return BATQ_ERR_INVALID_ARG;
+  if (x_dtype != BATQ_F32 && x_dtype != BATQ_BF16) return BATQ_ERR_INVALID_ARG;
+  if (layout != BATQ_SCALES_LINEAR && layout != BATQ_SCALES_MMA) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_mn(S, N);
+  if (st != BATQ_OK) return st;
+  if (ldx < N) return BATQ_ERR_SHAPE;
+  const size_t esz = x_dtype == BATQ_BF16 ? 2 : 4;
+  if (!aligned16(X) || ((size_t)ldx * esz) % 16 != 0 || !aligned16(codes) || !aligned16(B_dev))
+    return BATQ_ERR_ALIGNMENT;
+  if (ratios_dev && (reinterpret_cast<uintptr_t>(ratios_dev) & 7u)) return BATQ_ERR_ALIGNMENT;
+  if (y_debug && !aligned16(y_debug)) return BATQ_ERR_ALIGNMENT;
+  if (layout == BATQ_SCALES_MMA && !aligned16(scales)) return BATQ_ERR_ALIGNMENT;
+  return BATQ_OK;
+}
+
+batq_status check_gemm_args(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
+                            const uint8_t* w_scales, int S, int M, int N, batq_dtype out_dtype, const void* out,
+                            int ldo) {
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !out) return BATQ_ERR_INVALID_ARG;
+  if (out_dtype != BATQ_F32 && out_dtype != BATQ_BF16) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_mn(S, N);
+  if (st != BATQ_OK) return st;
+  if (M < 16 || (M % 16) != 0 || ldo < M) return BATQ_ERR_SHAPE;
+  const size_t esz = out_dtype == BATQ_BF16 ? 2 : 4;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(out) || ((size_t)ldo * esz) % 16 != 0)
+    return BATQ_ERR_ALIGNMENT;
+  return BATQ_OK;
+}
+
+batq_status launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
+                        const uint8_t* w_scales, int S, int M, int N, batq_dtype out_dtype, void* out, int ldo,
+                        cudaStream_t stream) {
+  batq::GemmLaunch L;
+  L.a_codes = a_codes;
+  L.a_scales = a_scales;
+  L.w_codes = w_codes;
+  L.w_scales = w_scales;
+  L.S = S;
+  L.M = M;
+  L.N = N;
+  L.out_bf16 = (out_dtype == BATQ_BF16);
+  L.out = out;
+  L.ldo = ldo;
+  L.err = error_word();
+  L.stream = stream;
+  cudaError_t e = batq::launch_gemm_mxfp4(L);
+  if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
+  return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* batq_status_string(batq_status status) {
+  switch (status) {
+    case BATQ_OK: return "ok";
+    case BATQ_ERR_INVALID_ARG: return "invalid argument";
+    case BATQ_ERR_SHAPE: return "unsupported shape";
+    case BATQ_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case BATQ_ERR_SINGULAR: return "transform factor singular or ill-conditioned";
+    case BATQ_ERR_ARCH: return "device is not sm_100";
+    case BATQ_ERR_CUDA: return "CUDA error";
+    case BATQ_ERR_TIMEOUT: return "kernel barrier wait timed out";
+    case BATQ_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+int batq_version(void) { return 100; }
+
+batq_status batq_act_buffer_sizes(int rows, int N, batq_scale_layout layout, size_t* code_bytes,
+                                  size_t* scale_bytes) {
+  if (!code_bytes || !scale_bytes) return BATQ_ERR_INVALID_ARG;
+  if (layout != BATQ_SCALES_LINEAR && layout != BATQ_SCALES_MMA) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_mn(rows, N);
+  if (st != BATQ_OK) return st;
+  *code_bytes = (size_t)rows * (size_t)(N / 2);
+  *scale_bytes = scale_bytes_for(rows, N, layout);
+  return BATQ_OK;
+}
+
+batq_status batq_clip_ratios(const float* alpha_min_host, const float* alpha_max_host, int k,
+                             float* ratios_out_host) {
+  if (!alpha_min_host || !alpha_max_host || !ratios_out_host || k < 1) return BATQ_ERR_INVALID_ARG;
+  for (int i = 0; i < k; ++i) {
+    ratios_out_host[2 * i] = (float)(1.0 / (1.0 + std::exp(-(double)alpha_min_host[i])));
+    ratios_out_host[2 * i + 1] = (float)(1.0 / (1.0 + std::exp(-(double)alpha_max_host[i])));
+  }
+  return BATQ_OK;
+}
+
+batq_status batq_quant_act(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
+                           const float* B_dev, const float* ratios_dev, uint8_t* codes, uint8_t* scales,
+                           batq_scale_layout layout, float* y_debug, void* stream) {
+  batq_status st = check_quant_args(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout,
+                                    y_debug);
+  if (st != BATQ_OK) return st;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug,
+                      static_cast<cudaStream_t>(stream));
+}
+
+batq_status batq_prepare_workspace_size(int N, size_t* bytes) {
+  if (!bytes) return BATQ_ERR_INVALID_ARG;
+  if (N < 64 || N % 64 != 0) return BATQ_ERR_SHAPE;
+  *bytes = round_up((size_t)(N / 32) * 16 * sizeof(float), 256);
+  return BATQ_OK;
+}
+
+batq_status batq_prepare_weights(const void* W, batq_dtype w_dtype, int M, int N, int ldw, const float* A_host,
+                                 const float* B_host, uint8_t* w_codes, uint8_t* w_scales,
+                                 batq_scale_layout layout, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (!B_host || !workspace) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_quant_args(W, w_dtype, M, N, ldw, A_host, reinterpret_cast<const float*>(workspace),
+                                    nullptr, w_codes, w_scales, layout, nullptr);
+  if (st != BATQ_OK) return st;
+  size_t need = 0;
+  batq_prepare_workspace_size(N, &need);
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+
+  // W'_mat = B_i^-1 W_mat A^-T: the activation kernel computes B'^T X A', so
+  // A' = A^-T and B'_i = B_i^-T.
+  const int k = N / 32;
+  double a[64], ainv[64];
+  for (int i = 0; i < 64; ++i) a[i] = A_host[i];
+  if (!invert(a, ainv, 8)) return BATQ_ERR_SINGULAR;
+  float a_fused[64];
+  for (int r = 0; r < 8; ++r)
+    for (int c = 0; c < 8; ++c) a_fused[r * 8 + c] = (float)ainv[c * 8 + r];
+  std::vector<float> b_fused((size_t)k * 16);
+  for (int i = 0; i < k; ++i) {
+    double b[16], binv[16];
+    for (int j = 0; j < 16; ++j) b[j] = B_host[(size_t)i * 16 + j];
+    if (!invert(b, binv, 4)) return BATQ_ERR_SINGULAR;
+    for (int r = 0; r < 4; ++r)
+      for (int c = 0; c < 4; ++c) b_fused[(size_t)i * 16 + r * 4 + c] = (float)binv[c * 4 + r];
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(workspace, b_fused.data(), b_fused.size() * sizeof(float), cudaMemcpyHostToDevice, s) !=
+      cudaSuccess)
+    return BATQ_ERR_CUDA;
+  // cudaMemcpyAsync from pageable memory has staged the bytes when it returns,
+  // so b_fused may be released.
+  return launch_quant(W, w_dtype, M, N, ldw, a_fused, reinterpret_cast<const float*>(workspace), nullptr, w_codes,
+                      w_scales, layout, nullptr, s);
+}
+
+batq_status batq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
+                            const uint8_t* w_scales, int S, int M, int N, batq_dtype out_dtype, void* out, int ldo,
+                            void* stream) {
+  batq_status st = check_gemm_args(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo);
+  if (st != BATQ_OK) return st;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo,
+                     static_cast<cudaStream_t>(stream));
+}
+
+batq_status batq_linear_workspace_size(int S, int N, size_t* bytes) {
+  if (!bytes) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_mn(S, N);
+  if (st != BATQ_OK) return st;
+  *bytes = round_up((size_t)S * (N / 2), 256) + scale_bytes_for(S, N, BATQ_SCALES_MMA);
+  return BATQ_OK;
+}
+
+batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
+                        const float* B_dev, const float* ratios_dev, const uint8_t* w_codes,
+                        const uint8_t* w_scales, int M, void* workspace, size_t workspace_bytes,
+                        batq_dtype out_dtype, void* out, int ldo, void* stream) {
+  if (!workspace) return BATQ_ERR_INVALID_ARG;
+  size_t need = 0;
+  batq_status st = batq_linear_workspace_size(S, N, &need);
+  if (st != BATQ_OK) return st;
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BATQ_ERR_ALIGNMENT;
+  uint8_t* a_codes = static_cast<uint8_t*>(workspace);
+  uint8_t* a_scales = a_codes + round_up((size_t)S * (N / 2), 256);
+  st = check_quant_args(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA,
+                        nullptr);
+  if (st != BATQ_OK) return st;
+  st = check_gemm_args(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo);
+  if (st != BATQ_OK) return st;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA, nullptr,
+                    s);
+  if (st != BATQ_OK) return st;
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, s);
+}
+
+batq_status batq_device_error(void* stream, unsigned int* flags_out) {
+  if (!flags_out) return BATQ_ERR_INVALID_ARG;
+  unsigned* word = error_word();
+  if (!word) return BATQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BATQ_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return BATQ_ERR_CUDA;
+  if (v != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return BATQ_ERR_CUDA;
+  }
+  *flags_out = v;
+  return v ? BATQ_ERR_TIMEOUT : BATQ_OK;
+}
+
+}  // extern "C"

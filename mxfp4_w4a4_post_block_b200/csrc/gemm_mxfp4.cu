@@ -1,0 +1,357 @@
+// k_gemm_mxfp4: W4A4 MXFP4 x MXFP4 block-scaled GEMM on the sm_100a tensor cores.
+//
+// D[i][j] = sum_k P[i][k] Q[j][k] with P, Q packed E2M1 (K-major, two codes per
+// byte) and one E8M0 scale per 32 K elements, fp32 accumulation in tensor
+// memory (TMEM).  The W4A4 linear of BATQuant (daily-arxiv summary: weight-side
+// transform fused into the weights offline, activation side online; MXFP4 =
+// 32 elements sharing one E8M0 scale, thelatestinai.com page, DuQuant++
+// abstract) maps onto it as
+//   * prefill: P = activations (S rows), Q = fused weights (M rows),
+//     out[i][j] = D[i][j], tiles of 128 x 256;
+//   * decode (S <= 64): P = weights, Q = activations ("swap"), out[j][i] =
+//     D[i][j], tiles of 128 x {16, 32, 64}, so the weight stream fills the
+//     128-row MMA and the narrow activation side sits in N.
+//
+// One CTA computes one output tile:
+//   warp 0     TMA producer: per stage a 128 x 256-element P tile, a BN x 256
+//              Q tile (both 128-byte swizzled) and their scale atoms (1-D bulk
+//              copies of the 512-byte 128x4 scale tiles);
+//   warp 1     TMEM allocator and MMA issuer: copies the stage's scales into
+//              TMEM (tcgen05.cp 32x128b.warpx4) and issues four
+//              tcgen05.mma kind::mxf4.block_scale (K = 64 each), then commits
+//              the stage back to the producer;
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator quadrant of each warp,
+//              staged through shared memory and written with TMA stores
+//              (prefill) or stored directly, coalesced along i (decode).
+#include <cstdint>
+
+#include "host_util.h"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace batq {
+namespace {
+
+constexpr int kBM = 128;          // MMA M (rows of P per tile, TMEM lanes)
+constexpr int kBKBytes = 128;     // bytes of K per stage and row (= 256 E2M1 codes)
+constexpr int kBK = 2 * kBKBytes; // K elements per stage
+constexpr int kKPerMma = 64;      // K of one kind::mxf4 MMA
+constexpr int kMmasPerStage = kBK / kKPerMma;
+constexpr int kThreads = 192;     // 6 warps
+constexpr int kSfAtom = 512;      // bytes of one 128-row x 4-scale tile
+
+template <int BN, bool kSwap, int kStages>
+struct GemmCfg {
+  static constexpr int kPBytes = kBM * kBKBytes;
+  static constexpr int kQBytes = BN * kBKBytes;
+  static constexpr int kQRowAtoms = BN > 128 ? 2 : 1;           // 128-row scale atoms covering Q rows
+  static constexpr int kSfPBytes = 2 * kSfAtom;                  // 2 K-atoms per stage
+  static constexpr int kSfQBytes = 2 * kQRowAtoms * kSfAtom;
+  static constexpr int kStageBytes = kPBytes + kQBytes + kSfPBytes + kSfQBytes;
+  static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
+  // TMEM columns: accumulator, then per stage 8 columns of P scales and
+  // 4 * kQRowAtoms * 2 columns of Q scales.
+  static constexpr int kSfPCols = 8;
+  static constexpr int kSfQCols = 8 * kQRowAtoms;
+  static constexpr int kTmemUsed = BN + kStages * (kSfPCols + kSfQCols);
+  static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
+                                 : kTmemUsed <= 256 ? 256 : 512;
+  static_assert(kTmemUsed <= 512, "TMEM budget");
+  static constexpr int kBarBytes = 64 * 8;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
+};
+
+struct GemmArgs {
+  const uint8_t* p_scales;  // MMA layout of P rows
+  const uint8_t* q_scales;  // MMA layout of Q rows
+  void* out;
+  unsigned* err;
+  int rows_p, rows_q;       // valid rows of P and Q
+  int rows_p_pad, rows_q_pad;
+  int N;                    // K elements
+  int kpad;                 // scale columns per row (k rounded up to 4)
+  int ldo;
+  int tiles_q;              // tiles along Q
+  int num_kstages;          // ceil(N / 256)
+};
+
+template <int BN, bool kSwap, int kStages, bool kOutBF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_mxfp4(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
+                 const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ GemmArgs g) {
+  using C = GemmCfg<BN, kSwap, kStages>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tile_p = blockIdx.x / g.tiles_q;
+  const int tile_q = blockIdx.x % g.tiles_q;
+  const int p0 = tile_p * kBM;
+  const int q0 = tile_q * BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t t_acc = tmem;
+  const uint32_t t_sfp = tmem + BN;
+  const uint32_t t_sfq = tmem + BN + kStages * C::kSfPCols;
+
+  const int nks = g.num_kstages;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      tma_prefetch_map(&tm_p);
+      tma_prefetch_map(&tm_q);
+      const int p_tile_atom = p0 >> 7;  // 128-row scale tile of P
+      const int q_tile_atom = q0 >> 7;
+      const int q_atoms_valid = min(C::kQRowAtoms, (g.rows_q_pad >> 7) - q_tile_atom);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int ks = 0; ks < nks; ++ks) {
+        if (!mbar_wait(&empty[s], ph ^ 1)) {
+          set_error(g.err, kErrReleaseTimeout);
+          break;
+        }
+        uint8_t* st = smem + s * C::kStageBytes;
+        const int katom0 = ks * 2;  // first 4-scale atom of this stage
+        const int katoms = min(2, (g.kpad >> 2) - katom0);
+        const uint32_t sf_bytes = (uint32_t)katoms * kSfAtom;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(C::kPBytes + C::kQBytes) + sf_bytes * (1 + q_atoms_valid));
+        tma_load_2d(st, &tm_p, &full[s], ks * kBKBytes, p0);
+        tma_load_2d(st + C::kPBytes, &tm_q, &full[s], ks * kBKBytes, q0);
+        const size_t row_stride = (size_t)(g.kpad >> 2) * kSfAtom;
+        bulk_load(st + C::kPBytes + C::kQBytes, g.p_scales + (size_t)p_tile_atom * row_stride + katom0 * kSfAtom,
+                  sf_bytes, &full[s]);
+        for (int a = 0; a < q_atoms_valid; ++a) {
+          bulk_load(st + C::kPBytes + C::kQBytes + C::kSfPBytes + a * 2 * kSfAtom,
+                    g.q_scales + (size_t)(q_tile_atom + a) * row_stride + katom0 * kSfAtom, sf_bytes, &full[s]);
+        }
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int ks = 0; ks < nks && ok; ++ks) {
+        if (!mbar_wait(&full[s], ph)) {
+          set_error(g.err, kErrDataTimeout);
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        uint8_t* st = smem + s * C::kStageBytes;
+        const uint32_t sp = smem_u32(st);
+        const uint32_t sq = sp + C::kPBytes;
+        const uint32_t ssfp = sq + C::kQBytes;
+        const uint32_t ssfq = ssfp + C::kSfPBytes;
+        const int kleft = g.N - ks * kBK;
+        const int nmma = kleft >= kBK ? kMmasPerStage : kleft / kKPerMma;
+        const int katoms = (nmma + 1) / 2;
+        // Scale factors of this stage into TMEM.
+        for (int a = 0; a < katoms; ++a) {
+          tc_cp_32x128b_warpx4(t_sfp + s * C::kSfPCols + a * 4, sdesc_sf_atom(ssfp + a * kSfAtom));
+#pragma unroll
+          for (int r = 0; r < C::kQRowAtoms; ++r) {
+            tc_cp_32x128b_warpx4(t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms + r * 4,
+                                 sdesc_sf_atom(ssfq + (r * 2 + a) * kSfAtom));
+          }
+        }
+        const uint64_t dp = sdesc_kmajor_sw128(sp);
+        const uint64_t dq = sdesc_kmajor_sw128(sq);
+        for (int j = 0; j < nmma; ++j) {
+          const int a = j >> 1;
+          const int sf_id = (j & 1) * 2;
+          const uint32_t idesc = idesc_mxf4(BN, sf_id, sf_id);
+          // Advance K by 64 codes = 32 bytes inside the 128-byte swizzle atom.
+          tc_mma_mxf4(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc,
+                      t_sfp + s * C::kSfPCols + a * 4, t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms,
+                      (ks > 0 || j > 0) ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+      // Signal the epilogue once every issued MMA has completed (also on error).
+      tc_commit(acc_full);
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31 are this warp's
+    if (!mbar_wait(acc_full, 0)) set_error(g.err, kErrMmaTimeout);
+    tc_fence_after_sync();
+    const uint32_t t_row = t_acc + ((uint32_t)(32 * quad) << 16);
+    if constexpr (kSwap) {
+      // D[i][j]: i = weight row (this lane), j = token.  out[j][i]: lanes write consecutive i.
+      const int i = p0 + 32 * quad + lane;
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_16cols(t_row + c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int tok = q0 + c0 + j;
+          if (tok < g.rows_q && i < g.rows_p) {
+            if constexpr (kOutBF16) {
+              const uint32_t pk = pack_bf16x2(__uint_as_float(r[j]), 0.0f);
+              reinterpret_cast<uint16_t*>(g.out)[(size_t)tok * g.ldo + i] = (uint16_t)(pk & 0xFFFFu);
+            } else {
+              reinterpret_cast<float*>(g.out)[(size_t)tok * g.ldo + i] = __uint_as_float(r[j]);
+            }
+          }
+        }
+      }
+    } else {
+      // Stage the warp's 32 rows through shared memory (pipeline buffers are
+      // idle once the accumulator is complete) and write 32-row boxes with TMA.
+      constexpr int kColsPerBox = kOutBF16 ? 64 : 32;  // 128 bytes per box row
+      constexpr int kBoxes = BN / kColsPerBox;
+      uint8_t* stage_out = smem + (size_t)quad * kBoxes * 4096;
+#pragma unroll 1
+      for (int bx = 0; bx < kBoxes; ++bx) {
+        uint8_t* box = stage_out + bx * 4096;
+        uint8_t* rowp = box + lane * 128;
+        if constexpr (kOutBF16) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32cols(t_row + bx * 64, r0);
+          tmem_ld_32cols(t_row + bx * 64 + 32, r1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t* r = c < 4 ? r0 : r1;
+            const int o = (c & 3) * 8;
+            uint4 v = make_uint4(pack_bf16x2(__uint_as_float(r[o + 0]), __uint_as_float(r[o + 1])),
+                                 pack_bf16x2(__uint_as_float(r[o + 2]), __uint_as_float(r[o + 3])),
+                                 pack_bf16x2(__uint_as_float(r[o + 4]), __uint_as_float(r[o + 5])),
+                                 pack_bf16x2(__uint_as_float(r[o + 6]), __uint_as_float(r[o + 7])));
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) = v;
+          }
+        } else {
+          uint32_t r[32];
+          tmem_ld_32cols(t_row + bx * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        for (int bx = 0; bx < kBoxes; ++bx) {
+          tma_store_2d(&tm_out, stage_out + bx * 4096, q0 + bx * kColsPerBox, p0 + 32 * quad);
+        }
+        tma_store_commit();
+        tma_store_wait_read_all();
+      }
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int BN, bool kSwap, int kStages, bool kOutBF16>
+cudaError_t launch_cfg(const GemmLaunch& L) {
+  using C = GemmCfg<BN, kSwap, kStages>;
+  const int rows_p = kSwap ? L.M : L.S;
+  const int rows_q = kSwap ? L.S : L.M;
+  const uint8_t* codes_p = kSwap ? L.w_codes : L.a_codes;
+  const uint8_t* codes_q = kSwap ? L.a_codes : L.w_codes;
+  const uint64_t row_bytes = (uint64_t)(L.N / 2);
+
+  CUtensorMap tm_p, tm_q, tm_out;
+  if (!make_map_2d(&tm_p, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_p, row_bytes, (uint64_t)rows_p, row_bytes, kBKBytes,
+                   kBM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_map_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_q, row_bytes, (uint64_t)rows_q, row_bytes, kBKBytes,
+                   BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!kSwap) {
+    const uint32_t esz = kOutBF16 ? 2 : 4;
+    if (!make_map_2d(&tm_out, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
+                     (uint64_t)L.M, (uint64_t)L.S, (uint64_t)L.ldo * esz, 128 / esz, 32,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  } else {
+    tm_out = tm_q;  // unused in the decode epilogue
+  }
+
+  GemmArgs g;
+  g.p_scales = kSwap ? L.w_scales : L.a_scales;
+  g.q_scales = kSwap ? L.a_scales : L.w_scales;
+  g.out = L.out;
+  g.err = L.err;
+  g.rows_p = rows_p;
+  g.rows_q = rows_q;
+  g.rows_p_pad = (rows_p + 127) / 128 * 128;
+  g.rows_q_pad = (rows_q + 127) / 128 * 128;
+  g.N = L.N;
+  g.kpad = (L.N / 32 + 3) / 4 * 4;
+  g.ldo = L.ldo;
+  g.tiles_q = (rows_q + BN - 1) / BN;
+  g.num_kstages = (L.N + kBK - 1) / kBK;
+  const int tiles_p = (rows_p + kBM - 1) / kBM;
+
+  auto kern = k_gemm_mxfp4<BN, kSwap, kStages, kOutBF16>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  kern<<<tiles_p * g.tiles_q, kThreads, C::kSmemBytes, L.stream>>>(tm_p, tm_q, tm_out, g);
+  return cudaGetLastError();
+}
+
+template <bool kOutBF16>
+cudaError_t launch_dtype(const GemmLaunch& L) {
+  if (L.S <= 16) return launch_cfg<16, true, 4, kOutBF16>(L);
+  if (L.S <= 32) return launch_cfg<32, true, 4, kOutBF16>(L);
+  if (L.S <= 64) return launch_cfg<64, true, 4, kOutBF16>(L);
+  return launch_cfg<256, false, 4, kOutBF16>(L);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_mxfp4(const GemmLaunch& L) {
+  return L.out_bf16 ? launch_dtype<true>(L) : launch_dtype<false>(L);
+}
+
+}  // namespace batq

@@ -1,0 +1,42 @@
+// Launchers of the device kernels (internal to libbatq).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace batq {
+
+struct QuantLaunch {
+  const void* X;
+  bool bf16;
+  int S, N, ldx;
+  float A[64];          // 8x8 row-major, passed by value into the launch
+  const float* B;       // device, k x 16
+  const float* ratios;  // device, 2k, or nullptr (no clip)
+  uint8_t* codes;       // device, S x N/2
+  uint8_t* scales;      // device
+  bool mma_layout;
+  float* y_debug;       // device S x N or nullptr
+  unsigned* err;        // device error word
+  cudaStream_t stream;
+};
+
+// Returns cudaErrorInvalidValue when the tensor map cannot be encoded.
+cudaError_t launch_quant_act(const QuantLaunch& L);
+
+struct GemmLaunch {
+  const uint8_t* a_codes;
+  const uint8_t* a_scales;  // MMA layout, S rows
+  const uint8_t* w_codes;
+  const uint8_t* w_scales;  // MMA layout, M rows
+  int S, M, N;
+  bool out_bf16;
+  void* out;
+  int ldo;
+  unsigned* err;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_gemm_mxfp4(const GemmLaunch& L);
+
+}  // namespace batq

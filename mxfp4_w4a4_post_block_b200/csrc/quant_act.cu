@@ -1,0 +1,315 @@
+// k_quant_act: BATQuant online activation path on sm_100a.
+//
+// For every token and 32-element block: Y = B_i^T X A (GPK block-wise affine
+// transform), per-block clip to [r_min * min Y, r_max * max Y], E8M0 shared
+// scale and E2M1 codes (BATQuant daily-arxiv summary, sections "块仿射变换",
+// "GPK 分解", "块级可学习裁剪"; thelatestinai.com page, Figure 2 caption for
+// the divide-then-round order; OCP MX v1.0 for the scale rule).
+//
+// Memory-bound design:
+//   * one producer warp streams tiles of 32 tokens x 8 blocks into a 4-stage
+//     shared-memory ring with TMA (one 32-row box per block column, swizzled
+//     so the per-lane row reads below are bank-conflict free);
+//   * eight consumer warps, warp w owning block column c0 + w of the tile and
+//     lane l owning token r0 + l, so B_i and the clip ratios are warp-uniform
+//     and A is read from the kernel's parameter (constant) bank;
+//   * the block extrema are in-thread (the whole block lives in one thread),
+//     the clipped amax is max(|clamp(min)|, |clamp(max)|) (clamp is
+//     monotone), and the scale comes from the exponent bits of amax.
+#include <cfloat>
+#include <cstdint>
+
+#include "host_util.h"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace batq {
+namespace {
+
+constexpr int kRows = 32;         // tokens per tile (one per lane)
+constexpr int kCols = 8;          // 32-blocks per tile (one per consumer warp)
+constexpr int kStages = 4;        // shared-memory ring depth
+constexpr int kConsumerWarps = kCols;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr uint8_t kPadScale = 0x7F;
+
+template <bool kBF16>
+struct Tile {
+  static constexpr int kBlockBytes = kBF16 ? 64 : 128;      // one 32-element block row
+  static constexpr int kBoxBytes = kRows * kBlockBytes;     // one TMA box (32 tokens x 1 block)
+  static constexpr int kStageBytes = kCols * kBoxBytes;     // one tile
+  static constexpr int kSmemBytes = kStages * kStageBytes + 2 * kStages * 8 + 1024;
+};
+
+struct QuantArgs {
+  float A[64];
+  const float* B;
+  const float* ratios;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* y_debug;
+  unsigned* err;
+  int S, N, k, kpad;
+  int rows_out;  // rows whose scales are written (S, or S rounded up to 128 in MMA layout)
+  int mma_layout;
+  int tiles_r, tiles_c;
+};
+
+__device__ __forceinline__ uint32_t mma_scale_offset(int row, int kb, int kpad) {
+  return (uint32_t)(((row >> 7) * (kpad >> 2) + (kb >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (kb & 3));
+}
+
+// One token's 32-element block from the swizzled tile.  bf16 boxes use the
+// 64-byte swizzle (16-byte chunk c of row t stored at chunk c ^ ((t >> 1) & 3)),
+// fp32 boxes the 128-byte swizzle (chunk c ^ (t & 7)).
+template <bool kBF16>
+__device__ __forceinline__ void load_block(const uint8_t* box, int lane, float x[32]) {
+  if constexpr (kBF16) {
+    const uint8_t* row = box + lane * 64;
+    const int sw = (lane >> 1) & 3;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        x[c * 8 + 2 * j] = __uint_as_float(w[j] << 16);
+        x[c * 8 + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+    }
+  } else {
+    const uint8_t* row = box + lane * 128;
+    const int sw = lane & 7;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 v = *reinterpret_cast<const float4*>(row + ((c ^ sw) << 4));
+      x[c * 4 + 0] = v.x;
+      x[c * 4 + 1] = v.y;
+      x[c * 4 + 2] = v.z;
+      x[c * 4 + 3] = v.w;
+    }
+  }
+}
+
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_quant_act(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
+  using T = Tile<kBF16>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * T::kStageBytes);
+  uint64_t* empty = full + kStages;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int ntiles = p.tiles_r * p.tiles_c;
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: one thread issues the TMA boxes ----------------
+    if (lane == 0) {
+      tma_prefetch_map(&tmx);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        if (!mbar_wait(&empty[s], ph ^ 1)) {
+          set_error(p.err, kErrReleaseTimeout);
+          break;
+        }
+        const int r0 = (t / p.tiles_c) * kRows;
+        const int c0 = (t % p.tiles_c) * kCols;
+        if (r0 < p.S) {
+          const int nb = min(kCols, p.k - c0);
+          uint8_t* dst = smem + s * T::kStageBytes;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(nb * T::kBoxBytes));
+          for (int j = 0; j < nb; ++j) tma_load_2d(dst + j * T::kBoxBytes, &tmx, &full[s], (c0 + j) * 32, r0);
+        } else {
+          mbar_arrive(&full[s]);  // padding rows only: nothing to load
+        }
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  int s = 0;
+  uint32_t ph = 0;
+  for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int r0 = (t / p.tiles_c) * kRows;
+    const int c0 = (t % p.tiles_c) * kCols;
+    const int b = c0 + warp;
+    const int row = r0 + lane;
+    if (!mbar_wait(&full[s], ph)) {
+      set_error(p.err, kErrDataTimeout);
+      break;
+    }
+    if (r0 < p.S && b < p.k) {
+      float x[32];
+      load_block<kBF16>(smem + s * T::kStageBytes + warp * T::kBoxBytes, lane, x);
+
+      // B_i (row-major 4x4) and the clip ratios are the same for the whole warp.
+      float Bm[16];
+      const float4* bp = reinterpret_cast<const float4*>(p.B + 16 * b);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 v = __ldg(bp + q);
+        Bm[4 * q + 0] = v.x;
+        Bm[4 * q + 1] = v.y;
+        Bm[4 * q + 2] = v.z;
+        Bm[4 * q + 3] = v.w;
+      }
+      float r_min = 1.0f, r_max = 1.0f;
+      if (p.ratios != nullptr) {
+        const float2 r = __ldg(reinterpret_cast<const float2*>(p.ratios) + b);
+        r_min = r.x;
+        r_max = r.y;
+      }
+
+      // T = X A  (X is the row-major 4x8 view of the block), then Y = B^T T.
+      float tm[32];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float acc = 0.0f;
+#pragma unroll
+          for (int a = 0; a < 8; ++a) acc = fmaf(x[8 * r + a], p.A[8 * a + c], acc);
+          tm[8 * r + c] = acc;
+        }
+      }
+      float y[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float acc = 0.0f;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) acc = fmaf(Bm[4 * r + c], tm[8 * r + j], acc);
+          y[8 * c + j] = acc;
+        }
+      }
+
+      // Block extrema (NaN-propagating), clip bounds, clipped amax.
+      float mn = y[0], mx = y[0];
+#pragma unroll
+      for (int j = 1; j < 32; ++j) {
+        mn = fmin_nan(mn, y[j]);
+        mx = fmax_nan(mx, y[j]);
+      }
+      const bool finite = (fabsf(mn) <= FLT_MAX) && (fabsf(mx) <= FLT_MAX);
+      const float lo = r_min * mn;
+      const float hi = r_max * mx;
+      const float cmn = fminf(fmaxf(mn, lo), hi);
+      const float cmx = fminf(fmaxf(mx, lo), hi);
+      const float amax = fmaxf(fabsf(cmn), fabsf(cmx));
+
+      // Shared scale: floor(log2 amax) = biased exponent - 127, so the scale
+      // byte e + 127 = biased exponent - 2 (clamped at 0, which also covers
+      // amax == 0 and subnormal amax).  2^-e is built from exponent bits.
+      const uint32_t ebits = __float_as_uint(amax) >> 23;
+      uint32_t sbyte = ebits > 2u ? ebits - 2u : 0u;
+      const float inv_scale = __uint_as_float((254u - sbyte) << 23);
+
+      uint32_t words[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        float q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) q[j] = fminf(fmaxf(y[8 * w + j], lo), hi) * inv_scale;
+        words[w] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+      }
+      if (!finite) {
+        sbyte = 0xFFu;
+        words[0] = words[1] = words[2] = words[3] = 0u;
+      }
+
+      if (row < p.S) {
+        uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (size_t)(p.N >> 1) + (size_t)b * 16);
+        *dst = make_uint4(words[0], words[1], words[2], words[3]);
+        if (p.mma_layout)
+          p.scales[mma_scale_offset(row, b, p.kpad)] = (uint8_t)sbyte;
+        else
+          p.scales[(size_t)row * p.k + b] = (uint8_t)sbyte;
+        if (p.y_debug != nullptr) {
+          float4* yd = reinterpret_cast<float4*>(p.y_debug + (size_t)row * p.N + (size_t)b * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) yd[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+        }
+      } else if (p.mma_layout && row < p.rows_out) {
+        p.scales[mma_scale_offset(row, b, p.kpad)] = kPadScale;
+      }
+    } else if (p.mma_layout && b < p.kpad && row < p.rows_out) {
+      p.scales[mma_scale_offset(row, b, p.kpad)] = kPadScale;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == kStages) {
+      s = 0;
+      ph ^= 1;
+    }
+  }
+}
+
+template <bool kBF16>
+cudaError_t launch_impl(const QuantLaunch& L) {
+  using T = Tile<kBF16>;
+  CUtensorMap map;
+  const uint64_t stride = (uint64_t)L.ldx * (kBF16 ? 2u : 4u);
+  if (!make_map_2d(&map, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.X,
+                   (uint64_t)L.N, (uint64_t)L.S, stride, 32, kRows,
+                   kBF16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) {
+    return cudaErrorInvalidValue;
+  }
+  QuantArgs a;
+  for (int i = 0; i < 64; ++i) a.A[i] = L.A[i];
+  a.B = L.B;
+  a.ratios = L.ratios;
+  a.codes = L.codes;
+  a.scales = L.scales;
+  a.y_debug = L.y_debug;
+  a.err = L.err;
+  a.S = L.S;
+  a.N = L.N;
+  a.k = L.N / 32;
+  a.kpad = (a.k + 3) / 4 * 4;
+  a.mma_layout = L.mma_layout ? 1 : 0;
+  a.rows_out = L.mma_layout ? (L.S + 127) / 128 * 128 : L.S;
+  a.tiles_r = (a.rows_out + kRows - 1) / kRows;
+  a.tiles_c = (a.k + kCols - 1) / kCols;
+
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         T::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int ntiles = a.tiles_r * a.tiles_c;
+  const int per_sm = kBF16 ? 2 : 1;
+  const int grid = ntiles < sm_count() * per_sm ? ntiles : sm_count() * per_sm;
+  k_quant_act<kBF16><<<grid, kThreads, T::kSmemBytes, L.stream>>>(map, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quant_act(const QuantLaunch& L) {
+  return L.bf16 ? launch_impl<true>(L) : launch_impl<false>(L);
+}
+
+}  // namespace batq

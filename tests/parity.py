@@ -1,0 +1,96 @@
+"""Parity rules shared by the GPU tests (CUDA path vs the CPU oracle).
+
+Tolerances:
+* transformed activations Y: |y_gpu - y_ref| <= 1e-5 * sum_j |x_j| |P_ji|
+  (the condition-scaled reading of "within 1e-5 relative": a plain relative
+  error is ill-posed for entries near cancellation);
+* FP4 codes and E8M0 scales bit-exact, except elements whose pre-rounding value
+  q lies within 1e-5 relative of an E2M1 rounding boundary (midpoints 0.25,
+  0.75, 1.25, 1.75, 2.5, 3.5, 5) and whole blocks whose clipped amax lies
+  within 1e-5 relative of a power of two (the shared exponent may flip); the
+  mismatching elements must number fewer than 1e-4 of all elements;
+* GEMM: |out_gpu - out_ref| <= 1e-4 * sum_n |a_n| |w_n| against the oracle's
+  fp64 product of the same codes.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import batq_oracle as O
+
+MIDPOINTS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+REL = 1e-5
+
+
+def condition_scale(X, A, B):
+    """sum_j |x_j| |P_ji| per output element (fp64)."""
+    X = np.abs(np.asarray(X, np.float64))
+    S, N = X.shape
+    k = N // 32
+    P = np.abs(O.dense_blocks(A, B))
+    return np.matmul(X.reshape(S, k, 32).transpose(1, 0, 2), P).transpose(1, 0, 2).reshape(S, N)
+
+
+def check_y(y_gpu, X, A, B, y_ref):
+    scale = condition_scale(X, A, B)
+    err = np.abs(y_gpu.astype(np.float64) - y_ref.astype(np.float64))
+    bad = err > REL * scale
+    return int(bad.sum()), float(np.max(err / np.maximum(scale, 1e-300)))
+
+
+def exempt_mask(ref):
+    """Boolean (S, N): elements whose code may legitimately differ."""
+    q = np.abs(ref["q"])
+    near_mid = np.zeros(q.shape, dtype=bool)
+    for m in MIDPOINTS:
+        near_mid |= np.abs(q - m) <= REL * m
+    S, N = q.shape
+    k = N // 32
+    amax = np.abs(ref["Y_hat"].astype(np.float64)).reshape(S, k, 32).max(axis=2)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        p2 = np.exp2(np.round(np.log2(np.where(amax > 0, amax, 1.0))))
+    near_pow2 = (amax > 0) & (np.abs(amax - p2) <= REL * p2)
+    return near_mid | np.repeat(near_pow2, 32, axis=1), near_pow2
+
+
+def compare_codes(codes_gpu, scales_gpu_linear, ref):
+    """Returns dict(mismatch, unexplained, scale_mismatch, scale_unexplained, total)."""
+    cg = O.unpack_nibbles(codes_gpu)
+    cr = O.unpack_nibbles(ref["codes"])
+    ex, ex_blk = exempt_mask(ref)
+    diff = cg != cr
+    sdiff = np.asarray(scales_gpu_linear) != ref["scales"]
+    S, N = cg.shape
+    # every element of a block whose scale differs counts as mismatching
+    diff_all = diff | np.repeat(sdiff, 32, axis=1)
+    return {
+        "mismatch": int(diff_all.sum()),
+        "unexplained": int((diff_all & ~ex).sum()),
+        "scale_mismatch": int(sdiff.sum()),
+        "scale_unexplained": int((sdiff & ~ex_blk).sum()),
+        "total": S * N,
+    }
+
+
+def assert_quant_parity(codes_gpu, scales_gpu_linear, ref, label=""):
+    r = compare_codes(codes_gpu, scales_gpu_linear, ref)
+    assert r["unexplained"] == 0 and r["scale_unexplained"] == 0, f"{label}: {r}"
+    assert r["mismatch"] < 1e-4 * r["total"], f"{label}: too many boundary mismatches {r}"
+    return r
+
+
+def assert_gemm_parity(out_gpu, out_ref, T, label=""):
+    out_gpu = np.asarray(out_gpu, np.float64)
+    err = np.abs(out_gpu - out_ref)
+    bad = err > 1e-4 * T
+    assert not bad.any(), f"{label}: {int(bad.sum())} outputs out of tolerance, worst {np.max(err / np.maximum(T, 1e-300))}"
+    return float(np.max(err / np.maximum(T, 1e-300)))
+
+
+def to_mma_layout(scales_linear, rows, k, pad=0x7F):
+    """Place a (rows, k) linear scale matrix into the tiled MMA layout buffer (test-side helper)."""
+    buf = np.full(O.mma_layout_bytes(rows, k), pad, dtype=np.uint8)
+    r, c = np.meshgrid(np.arange(rows), np.arange(k), indexing="ij")
+    buf[O.mma_scale_offset(r, c, k)] = np.asarray(scales_linear, np.uint8)
+    return buf

@@ -1,0 +1,122 @@
+"""The C-ABI library loads and exports every declared symbol; host-only calls and
+argument checks work without a GPU (no compute call is made here)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from mxfp4_w4a4_post_block_b200 import _lib
+from oracle import batq_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "batq.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"BATQ_API\s+[\w\s\*]*?\b(batq_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(_lib.LIB_PATH):
+        from mxfp4_w4a4_post_block_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def test_header_declares_expected_calls():
+    names = _declared()
+    for n in ("batq_quant_act", "batq_prepare_weights", "batq_gemm_mxfp4", "batq_linear"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert set(_declared()) == set(_lib.SIGNATURES), "binding signatures out of sync with the header"
+
+
+def test_status_strings_and_version(L):
+    assert L.batq_status_string(0) == b"ok"
+    assert b"aligned" in L.batq_status_string(3)
+    assert L.batq_version() >= 100
+
+
+def test_buffer_sizes(L):
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.batq_act_buffer_sizes(2048, 4096, 1, ctypes.byref(cb), ctypes.byref(sb)) == 0
+    assert cb.value == 2048 * 2048 and sb.value == 2048 * 128
+    assert L.batq_act_buffer_sizes(16, 320, 1, ctypes.byref(cb), ctypes.byref(sb)) == 0
+    assert sb.value == O.mma_layout_bytes(16, 10) == 128 * 12
+    assert L.batq_act_buffer_sizes(16, 320, 0, ctypes.byref(cb), ctypes.byref(sb)) == 0
+    assert sb.value == 16 * 10
+    assert L.batq_act_buffer_sizes(16, 100, 0, ctypes.byref(cb), ctypes.byref(sb)) == _lib.BATQ_ERR_SHAPE
+    assert L.batq_act_buffer_sizes(0, 256, 0, ctypes.byref(cb), ctypes.byref(sb)) == _lib.BATQ_ERR_SHAPE
+    assert L.batq_act_buffer_sizes(16, 256, 7, ctypes.byref(cb), ctypes.byref(sb)) == _lib.BATQ_ERR_INVALID_ARG
+
+
+def test_clip_ratios_match_oracle(L):
+    rng = np.random.default_rng(0)
+    amin = (rng.standard_normal(384) * 3).astype(np.float32)
+    amax = (rng.standard_normal(384) * 3).astype(np.float32)
+    out = np.empty(768, np.float32)
+    assert L.batq_clip_ratios(amin.ctypes.data, amax.ctypes.data, 384, out.ctypes.data) == 0
+    np.testing.assert_array_equal(out[0::2], O.clip_ratios(amin))
+    np.testing.assert_array_equal(out[1::2], O.clip_ratios(amax))
+
+
+def test_workspace_sizes(L):
+    b = ctypes.c_size_t()
+    assert L.batq_linear_workspace_size(2048, 4096, ctypes.byref(b)) == 0
+    assert b.value >= 2048 * 2048 + 2048 * 128
+    assert L.batq_prepare_workspace_size(4096, ctypes.byref(b)) == 0
+    assert b.value >= 128 * 64
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails in host-side validation
+
+
+def test_quant_argument_checks_fail_before_any_launch(L):
+    A = np.eye(8, dtype=np.float32)
+    qa = L.batq_quant_act
+    # null pointer
+    assert qa(None, 1, 16, 256, 256, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, None, None) == _lib.BATQ_ERR_INVALID_ARG
+    # N not a multiple of 64
+    assert qa(FAKE, 1, 16, 250, 256, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, None, None) == _lib.BATQ_ERR_SHAPE
+    # ldx < N
+    assert qa(FAKE, 1, 16, 256, 128, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, None, None) == _lib.BATQ_ERR_SHAPE
+    # misaligned X
+    assert qa(FAKE + 2, 1, 16, 256, 256, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, None, None) == _lib.BATQ_ERR_ALIGNMENT
+    # bf16 row stride not a multiple of 16 bytes
+    assert qa(FAKE, 1, 16, 256, 260, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, None, None) == _lib.BATQ_ERR_ALIGNMENT
+    # bad dtype / layout
+    assert qa(FAKE, 5, 16, 256, 256, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, None, None) == _lib.BATQ_ERR_INVALID_ARG
+    assert qa(FAKE, 1, 16, 256, 256, A.ctypes.data, FAKE, None, FAKE, FAKE, 9, None, None) == _lib.BATQ_ERR_INVALID_ARG
+
+
+def test_gemm_argument_checks_fail_before_any_launch(L):
+    g = L.batq_gemm_mxfp4
+    assert g(FAKE, FAKE, FAKE, FAKE, 16, 100, 256, 0, FAKE, 100, None) == _lib.BATQ_ERR_SHAPE  # M % 16
+    assert g(FAKE, FAKE, FAKE, FAKE, 16, 128, 96, 0, FAKE, 128, None) == _lib.BATQ_ERR_SHAPE   # N % 64
+    assert g(FAKE, FAKE, FAKE, FAKE, 0, 128, 256, 0, FAKE, 128, None) == _lib.BATQ_ERR_SHAPE   # S < 1
+    assert g(FAKE, FAKE, FAKE + 8, FAKE, 16, 128, 256, 0, FAKE, 128, None) == _lib.BATQ_ERR_ALIGNMENT
+    assert g(FAKE, FAKE, FAKE, FAKE, 16, 128, 256, 0, FAKE, 130, None) == _lib.BATQ_ERR_ALIGNMENT  # ldo*4 % 16
+    assert g(None, FAKE, FAKE, FAKE, 16, 128, 256, 0, FAKE, 128, None) == _lib.BATQ_ERR_INVALID_ARG
+
+
+def test_linear_workspace_checks(L):
+    A = np.eye(8, dtype=np.float32)
+    st = L.batq_linear(FAKE, 1, 16, 256, 256, A.ctypes.data, FAKE, None, FAKE, FAKE, 128, FAKE, 16, 0, FAKE, 128,
+                       None)
+    assert st == _lib.BATQ_ERR_WORKSPACE
+
+
+def test_prepare_checks(L):
+    A = np.eye(8, dtype=np.float32)
+    B = np.tile(np.eye(4, dtype=np.float32), (8, 1, 1))
+    st = L.batq_prepare_weights(FAKE, 0, 128, 256, 256, A.ctypes.data, B.ctypes.data, FAKE, FAKE, 1, FAKE, 1, None)
+    assert st == _lib.BATQ_ERR_WORKSPACE

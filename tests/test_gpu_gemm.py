@@ -1,0 +1,167 @@
+"""GPU parity of batq_gemm_mxfp4, batq_prepare_weights and batq_linear against the oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from mxfp4_w4a4_post_block_b200 import batq as BQ
+from mxfp4_w4a4_post_block_b200 import workloads as WL
+from oracle import batq_oracle as O
+import gpu_util as GU
+import parity as PT
+
+pytestmark = pytest.mark.gpu
+
+
+def _random_operands(S, M, N, seed):
+    """Random MXFP4 operands: every code value (incl. -0) and scales over a wide range."""
+    rng = np.random.default_rng(seed)
+    k = N // 32
+    a = rng.integers(0, 256, (S, N // 2), dtype=np.uint8)
+    w = rng.integers(0, 256, (M, N // 2), dtype=np.uint8)
+    sa = rng.integers(100, 150, (S, k), dtype=np.uint8)
+    sw = rng.integers(100, 150, (M, k), dtype=np.uint8)
+    return a, sa, w, sw
+
+
+def _run(a, sa, w, sw, out_dtype=torch.float32):
+    S, M, N = a.shape[0], w.shape[0], 2 * a.shape[1]
+    k = N // 32
+    out = GU.gpu_gemm(GU.to_dev_u8(a), GU.to_dev_u8(PT.to_mma_layout(sa, S, k)), GU.to_dev_u8(w),
+                      GU.to_dev_u8(PT.to_mma_layout(sw, M, k)), S, M, N, out_dtype)
+    return out.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("S,M,N", [
+    (16, 128, 256),     # decode path (activations in N), one K stage
+    (4, 64, 64),        # M below one 128-row tile, single MMA
+    (1, 272, 320),      # partial K stage, M not a multiple of 128
+    (33, 160, 512),     # N = 64 decode tile
+    (64, 256, 1024),
+    (65, 256, 512),     # smallest prefill-path S
+    (128, 256, 256),
+    (200, 272, 320),    # ragged everything on the prefill path
+    (300, 1024, 768),
+])
+def test_gemm_random_operands(S, M, N):
+    a, sa, w, sw = _random_operands(S, M, N, S * 7 + M + N)
+    out = _run(a, sa, w, sw)
+    ref, T = O.gemm(a, sa, w, sw)
+    PT.assert_gemm_parity(out, ref, T, f"{S}x{M}x{N}")
+
+
+@pytest.mark.parametrize("S", [16, 200])
+def test_gemm_bf16_output(S):
+    a, sa, w, sw = _random_operands(S, 256, 512, 3 + S)
+    out = _run(a, sa, w, sw, torch.bfloat16)
+    ref, T = O.gemm(a, sa, w, sw)
+    # bf16 output: the fp32 result is rounded once more (relative 2^-8 of |out| <= T).
+    err = np.abs(out - ref)
+    assert np.all(err <= 1e-4 * T + 2.0 ** -8 * np.abs(ref) + 1e-30)
+
+
+def test_gemm_tiny_config_oracle_codes():
+    w = WL.tiny()
+    act = O.quant_act(w.x, w.A, w.B, w.alpha_min, w.alpha_max)
+    wp = O.prepare_weights(w.W, w.A, w.B)
+    out = _run(act["codes"], act["scales"], wp["codes"], wp["scales"])
+    ref, T = O.gemm(act["codes"], act["scales"], wp["codes"], wp["scales"])
+    PT.assert_gemm_parity(out, ref, T, "tiny")
+
+
+def test_gemm_q_proj_full_sampled_rows():
+    w = WL.q_proj()
+    act = O.quant_act(w.x, w.A, w.B, w.alpha_min, w.alpha_max)
+    wp = O.prepare_weights(w.W, w.A, w.B)
+    out = _run(act["codes"], act["scales"], wp["codes"], wp["scales"])
+    rows = np.sort(np.random.default_rng(21).choice(w.S, 96, replace=False))
+    ref, T = O.gemm_rows(act["codes"], act["scales"], wp["codes"], wp["scales"], rows)
+    PT.assert_gemm_parity(out[rows], ref, T, "q_proj")
+
+
+@pytest.mark.parametrize("S", [1, 4, 16])
+def test_gemm_decode_full(S):
+    w = WL.decode(S, with_w=False)
+    rng = np.random.default_rng(30 + S)
+    act = O.quant_act(w.x, w.A, w.B, w.alpha_min, w.alpha_max)
+    wc = rng.integers(0, 256, (w.M, w.N // 2), dtype=np.uint8)
+    ws = rng.integers(110, 135, (w.M, w.k), dtype=np.uint8)
+    out = _run(act["codes"], act["scales"], wc, ws)
+    ref, T = O.gemm(act["codes"], act["scales"], wc, ws)
+    PT.assert_gemm_parity(out, ref, T, f"decode{S}")
+
+
+# ------------------------------------------------------------ weight side ----
+
+@pytest.mark.parametrize("maker", [WL.tiny, lambda: WL.custom(48, 320, 272, 41)])
+def test_prepare_weights_parity(maker):
+    w = maker()
+    codes, scales = GU.gpu_prepare(w)
+    ref = O.prepare_weights(w.W, w.A, w.B)
+    lin = O.scales_from_mma_layout(scales.cpu().numpy(), w.M, w.k)
+    r = PT.assert_quant_parity(codes.cpu().numpy(), lin, {"q": ref["q"], "Y_hat": ref["W_fused"],
+                                                          "codes": ref["codes"], "scales": ref["scales"]},
+                               "prepare")
+    print("prepare mismatches", r)
+
+
+def test_prepare_weights_q_proj():
+    w = WL.q_proj()
+    codes, scales = GU.gpu_prepare(w)
+    ref = O.prepare_weights(w.W, w.A, w.B)
+    lin = O.scales_from_mma_layout(scales.cpu().numpy(), w.M, w.k)
+    r = PT.assert_quant_parity(codes.cpu().numpy(), lin, {"q": ref["q"], "Y_hat": ref["W_fused"],
+                                                          "codes": ref["codes"], "scales": ref["scales"]},
+                               "prepare q_proj")
+    print("prepare q_proj mismatches", r)
+
+
+def test_prepare_rejects_singular_transform():
+    w = WL.tiny()
+    w.B[3] = 0.0
+    with pytest.raises(BQ.BatqError) as ei:
+        GU.gpu_prepare(w)
+    assert ei.value.status == 4
+
+
+# ---------------------------------------------------------------- linear ----
+
+def _linear(w, out_dtype=torch.float32):
+    X = GU.x_tensor(w)
+    B, ratios = GU.params(w)
+    wc, wsc = GU.gpu_prepare(w)
+    ws = torch.empty(BQ.batq_linear_workspace_size(w.S, w.N), dtype=torch.uint8, device="cuda")
+    out = torch.empty((w.S, w.M), dtype=out_dtype, device="cuda")
+    BQ.batq_linear(X, w.A, B, ratios, wc, wsc, w.M, ws, out)
+    assert BQ.batq_device_error() == 0
+    return out, wc, wsc
+
+
+@pytest.mark.parametrize("maker", [WL.tiny, lambda: WL.custom(200, 320, 272, 51),
+                                   lambda: WL.q_proj(), lambda: WL.decode(4)])
+def test_linear_matches_quant_then_gemm_and_oracle(maker):
+    w = maker()
+    out, wc, wsc = _linear(w)
+    # composition: identical to the two calls made separately
+    codes, lin, _, raw = GU.gpu_quant(w, BQ.BATQ_SCALES_MMA, y_debug=False)
+    out2 = GU.gpu_gemm(GU.to_dev_u8(codes), GU.to_dev_u8(raw), wc, wsc, w.S, w.M, w.N)
+    assert torch.equal(out, out2)
+    # oracle GEMM on the same operands (sampled rows for the large case)
+    rows = np.arange(w.S) if w.S <= 256 else np.sort(np.random.default_rng(5).choice(w.S, 64, replace=False))
+    wl = O.scales_from_mma_layout(wsc.cpu().numpy(), w.M, w.k)
+    ref, T = O.gemm_rows(codes, lin, wc.cpu().numpy(), wl, rows)
+    PT.assert_gemm_parity(out.cpu().numpy()[rows], ref, T, "linear")
+    # and the activations themselves match the oracle's (boundary exemptions only)
+    act = O.quant_act(w.x[rows], w.A, w.B, w.alpha_min, w.alpha_max)
+    PT.assert_quant_parity(codes[rows], lin[rows], act, "linear act")
+
+
+def test_linear_error_vs_unquantised_matches_oracle():
+    """The W4A4 output's distance from the unquantised x W^T is the oracle's."""
+    w = WL.tiny()
+    out, _, _ = _linear(w)
+    exact = w.x.astype(np.float64) @ w.W.astype(np.float64).T
+    ref, _, _, _ = O.linear(w.x, w.A, w.B, w.alpha_min, w.alpha_max, w.W)
+    rel_gpu = np.linalg.norm(out.cpu().numpy() - exact) / np.linalg.norm(exact)
+    rel_ref = np.linalg.norm(ref - exact) / np.linalg.norm(exact)
+    assert abs(rel_gpu - rel_ref) < 1e-3 * rel_ref + 1e-6, (rel_gpu, rel_ref)
