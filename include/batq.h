@@ -70,8 +70,12 @@ typedef enum {
   BATQ_ERR_ARCH = 5,        /* current device is not sm_100 */
   BATQ_ERR_CUDA = 6,        /* a CUDA runtime / driver call failed */
   BATQ_ERR_TIMEOUT = 7,     /* a kernel gave up waiting on a barrier (device error word set) */
-  BATQ_ERR_WORKSPACE = 8    /* workspace too small */
+  BATQ_ERR_WORKSPACE = 8,   /* workspace too small */
+  BATQ_ERR_SCRATCH_LIMIT = 9 /* problem needs more scratch than batq_linear_no_alloc's fixed array */
 } batq_status;
+
+/* Size of the fixed device scratch array used by batq_linear_no_alloc (16 MiB). */
+#define BATQ_NO_ALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
 typedef enum { BATQ_F32 = 0, BATQ_BF16 = 1 } batq_dtype;
 
@@ -179,6 +183,31 @@ BATQ_API batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N
                         const uint8_t* w_codes, const uint8_t* w_scales, int M,
                         void* workspace, size_t workspace_bytes,
                         batq_dtype out_dtype, void* out, int ldo, void* stream);
+
+/*
+ * batq_linear without a caller-provided workspace, for callers that cannot
+ * allocate device memory (for example a plugin running in a process whose
+ * device memory is fully reserved by another allocator, or a path where the
+ * device synchronisation cudaMalloc / cudaFree may cause is not allowed).  The
+ * method has no counterpart of this call: it only changes where the scratch
+ * lives.  Arguments, results and errors are those of batq_linear.
+ *
+ * The scratch is a fixed array of BATQ_NO_ALLOC_SCRATCH_BYTES in the
+ * library's own device memory; every GPU that loads the library holds it
+ * until the process exits.  Problems whose batq_linear_workspace_size exceeds
+ * it return BATQ_ERR_SCRATCH_LIMIT before anything is launched (for N = 4096,
+ * up to 7704 tokens fit).  The call allocates nothing.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  All calls
+ * share the one array and it keeps the last call's contents (every byte the
+ * GEMM reads is rewritten by each call, so stale contents are never used), so
+ * calls that can overlap on the GPU (different streams, or several host
+ * threads) race on it and must be serialised by the caller.
+ */
+BATQ_API batq_status batq_linear_no_alloc(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                                          const float* A_host, const float* B_dev, const float* ratios_dev,
+                                          const uint8_t* w_codes, const uint8_t* w_scales, int M,
+                                          batq_dtype out_dtype, void* out, int ldo, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's error

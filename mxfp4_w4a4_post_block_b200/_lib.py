@@ -16,6 +16,8 @@ BATQ_ERR_ARCH = 5
 BATQ_ERR_CUDA = 6
 BATQ_ERR_TIMEOUT = 7
 BATQ_ERR_WORKSPACE = 8
+BATQ_ERR_SCRATCH_LIMIT = 9
+NO_ALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 BATQ_F32 = 0
 BATQ_BF16 = 1
@@ -38,6 +40,8 @@ SIGNATURES = {
     "batq_linear_workspace_size": (_c_int, [_c_int, _c_int, _c_size_p]),
     "batq_linear": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
                              ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
+    "batq_linear_no_alloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_int,
+                                      _c_int, _vp, _c_int, _vp]),
     "batq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint)]),
 }
 

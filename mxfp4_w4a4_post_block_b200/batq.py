@@ -144,6 +144,19 @@ def batq_linear(X, A, B, ratios, w_codes, w_scales, M, workspace, out, stream=No
                                    _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_linear")
 
 
+def batq_linear_no_alloc(X, A, B, ratios, w_codes, w_scales, M, out, stream=None):
+    """batq_linear for callers that cannot allocate device memory: the scratch for the
+    quantised activations comes from a fixed array inside the library (see
+    include/batq.h for its size, sharing and ordering rules)."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    _check(_lib.load().batq_linear_no_alloc(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0), a.ctypes.data,
+                                            _dev_ptr(B, "B"), _dev_ptr(ratios, "ratios"),
+                                            _dev_ptr(w_codes, "w_codes"), _dev_ptr(w_scales, "w_scales"), M,
+                                            _dtype_code(out), _dev_ptr(out, "out"), out.stride(0),
+                                            _stream(stream)), "batq_linear_no_alloc")
+
+
 def batq_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device error word."""
     v = ctypes.c_uint(0)

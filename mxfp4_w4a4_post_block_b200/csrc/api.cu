@@ -198,6 +198,7 @@ const char* batq_status_string(batq_status status) {
     case BATQ_ERR_CUDA: return "CUDA error";
     case BATQ_ERR_TIMEOUT: return "kernel barrier wait timed out";
     case BATQ_ERR_WORKSPACE: return "workspace too small";
+    case BATQ_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the fixed no-allocation array holds";
   }
   return "unknown status";
 }
