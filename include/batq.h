@@ -117,8 +117,10 @@ BATQ_API batq_status batq_clip_ratios(const float* alpha_min_host, const float* 
  * X: device, S rows of N elements (x_dtype), row stride ldx elements
  *    (ldx >= N, ldx * elem_size a multiple of 16, X 16-byte aligned).
  * A_host: host, 8x8 fp32 row-major (A[a][b] at a*8+b); copied into the launch.
- * B_dev: device, k x 16 fp32; B_i row-major (B_i[r][c] at 16i + 4r + c).
- * ratios_dev: device, 2k fp32 from batq_clip_ratios, or NULL for no clip.
+ * B_dev: device, k x 16 fp32, 16-byte aligned; B_i row-major (B_i[r][c] at
+ *    16i + 4r + c).
+ * ratios_dev: device, 2k fp32 from batq_clip_ratios (16-byte aligned), or NULL
+ *    for no clip.
  * codes: device, S x N/2 bytes, 16-byte aligned.
  * scales: device, batq_act_buffer_sizes(S, N, layout) bytes.
  * y_debug: device S x N fp32 or NULL; receives the pre-clip Y (tests only).

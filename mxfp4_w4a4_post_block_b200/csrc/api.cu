@@ -141,7 +141,7 @@ batq_status check_quant_args(const void* X, batq_dtype x_dtype, int S, int N, in
   const size_t esz = x_dtype == BATQ_BF16 ? 2 : 4;
   if (!aligned16(X) || ((size_t)ldx * esz) % 16 != 0 || !aligned16(codes) || !aligned16(B_dev))
     return BATQ_ERR_ALIGNMENT;
-  if (ratios_dev && (reinterpret_cast<uintptr_t>(ratios_dev) & 7u)) return BATQ_ERR_ALIGNMENT;
+  if (ratios_dev && !aligned16(ratios_dev)) return BATQ_ERR_ALIGNMENT;
   if (y_debug && !aligned16(y_debug)) return BATQ_ERR_ALIGNMENT;
   if (layout == BATQ_SCALES_MMA && !aligned16(scales)) return BATQ_ERR_ALIGNMENT;
   return BATQ_OK;

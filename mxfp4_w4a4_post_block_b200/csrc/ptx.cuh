@@ -122,6 +122,18 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
   return d;
 }
 
+// Three-input forms (sm_100): one instruction per two comparisons.
+__device__ __forceinline__ float fmin3_nan(float a, float b, float c) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Four E2M1 pairs -> one 32-bit word of codes.  For each pair (lo, hi) the
 // conversion rounds to nearest even with saturation to +-6 and places `lo`
 // in the low nibble of its byte.

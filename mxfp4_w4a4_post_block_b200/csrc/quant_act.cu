@@ -10,9 +10,15 @@
 //   * one producer warp streams tiles of 32 tokens x 8 blocks into a 4-stage
 //     shared-memory ring with TMA (one 32-row box per block column, swizzled
 //     so the per-lane row reads below are bank-conflict free);
+//   * the producer also stages the tile's eight B_i and clip ratios with
+//     1-D bulk copies, so consumers read them from shared memory (broadcast);
 //   * eight consumer warps, warp w owning block column c0 + w of the tile and
 //     lane l owning token r0 + l, so B_i and the clip ratios are warp-uniform
 //     and A is read from the kernel's parameter (constant) bank;
+//   * the transform runs on packed fp32x2 FMAs: T = X A produces column
+//     pairs (T[r][2j], T[r][2j+1]) from a duplicated x value and an A row
+//     pair, then Y = B^T T reuses those column pairs with a duplicated B
+//     entry, so 384 scalar FMAs per block become 192 packed ones;
 //   * the block extrema are in-thread (the whole block lives in one thread),
 //     the clipped amax is max(|clamp(min)|, |clamp(max)|) (clamp is
 //     monotone), and the scale comes from the exponent bits of amax.
@@ -37,7 +43,10 @@ template <bool kBF16>
 struct Tile {
   static constexpr int kBlockBytes = kBF16 ? 64 : 128;      // one 32-element block row
   static constexpr int kBoxBytes = kRows * kBlockBytes;     // one TMA box (32 tokens x 1 block)
-  static constexpr int kStageBytes = kCols * kBoxBytes;     // one tile
+  static constexpr int kXBytes = kCols * kBoxBytes;         // activations of one tile
+  static constexpr int kBOffset = kXBytes;                  // kCols x 16 fp32 B_i
+  static constexpr int kROffset = kXBytes + kCols * 64;     // kCols x 2 fp32 clip ratios
+  static constexpr int kStageBytes = (kROffset + kCols * 8 + 1023) / 1024 * 1024;
   static constexpr int kSmemBytes = kStages * kStageBytes + 2 * kStages * 8 + 1024;
 };
 
@@ -128,10 +137,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int r0 = (t / p.tiles_c) * kRows;
         const int c0 = (t % p.tiles_c) * kCols;
         if (r0 < p.S) {
-          const int nb = min(kCols, p.k - c0);
+          const int nb = min(kCols, p.k - c0);  // even: k is even and c0 a multiple of 8
           uint8_t* dst = smem + s * T::kStageBytes;
-          mbar_arrive_expect_tx(&full[s], (uint32_t)(nb * T::kBoxBytes));
+          const uint32_t pbytes = (uint32_t)nb * 64u + (p.ratios != nullptr ? (uint32_t)nb * 8u : 0u);
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(nb * T::kBoxBytes) + pbytes);
           for (int j = 0; j < nb; ++j) tma_load_2d(dst + j * T::kBoxBytes, &tmx, &full[s], (c0 + j) * 32, r0);
+          bulk_load(dst + T::kBOffset, p.B + (size_t)c0 * 16, (uint32_t)nb * 64u, &full[s]);
+          if (p.ratios != nullptr) bulk_load(dst + T::kROffset, p.ratios + (size_t)c0 * 2, (uint32_t)nb * 8u, &full[s]);
         } else {
           mbar_arrive(&full[s]);  // padding rows only: nothing to load
         }
@@ -157,58 +169,69 @@ __global__ void __launch_bounds__(kThreads, 2)
       break;
     }
     if (r0 < p.S && b < p.k) {
+      const uint8_t* st = smem + s * T::kStageBytes;
       float x[32];
-      load_block<kBF16>(smem + s * T::kStageBytes + warp * T::kBoxBytes, lane, x);
+      load_block<kBF16>(st + warp * T::kBoxBytes, lane, x);
 
-      // B_i (row-major 4x4) and the clip ratios are the same for the whole warp.
-      float Bm[16];
-      const float4* bp = reinterpret_cast<const float4*>(p.B + 16 * b);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 v = __ldg(bp + q);
-        Bm[4 * q + 0] = v.x;
-        Bm[4 * q + 1] = v.y;
-        Bm[4 * q + 2] = v.z;
-        Bm[4 * q + 3] = v.w;
-      }
+      // B_i (row-major 4x4) and the clip ratios: the same for the whole warp.
+      const float4* bp = reinterpret_cast<const float4*>(st + T::kBOffset) + 4 * warp;
+      const float4 b0 = bp[0], b1 = bp[1], b2 = bp[2], b3 = bp[3];
+      const float Bm[16] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w,
+                            b2.x, b2.y, b2.z, b2.w, b3.x, b3.y, b3.z, b3.w};
       float r_min = 1.0f, r_max = 1.0f;
       if (p.ratios != nullptr) {
-        const float2 r = __ldg(reinterpret_cast<const float2*>(p.ratios) + b);
+        const float2 r = reinterpret_cast<const float2*>(st + T::kROffset)[warp];
         r_min = r.x;
         r_max = r.y;
       }
 
-      // T = X A  (X is the row-major 4x8 view of the block), then Y = B^T T.
-      float tm[32];
+      // T = X A  (X is the row-major 4x8 view of the block): column pairs
+      // (T[r][2j], T[r][2j+1]) += (x[r][a], x[r][a]) * (A[a][2j], A[a][2j+1]).
+      float2 tm[16];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float acc = 0.0f;
+        for (int j = 0; j < 4; ++j) {
+          float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-          for (int a = 0; a < 8; ++a) acc = fmaf(x[8 * r + a], p.A[8 * a + c], acc);
-          tm[8 * r + c] = acc;
+          for (int a = 0; a < 8; ++a) {
+            const float xv = x[8 * r + a];
+            acc = __ffma2_rn(make_float2(xv, xv), make_float2(p.A[8 * a + 2 * j], p.A[8 * a + 2 * j + 1]), acc);
+          }
+          tm[4 * r + j] = acc;
+        }
+      }
+      // Y = B^T T: (Y[c][2j], Y[c][2j+1]) += (B[r][c], B[r][c]) * (T[r][2j], T[r][2j+1]).
+      float2 y2[16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const float bv = Bm[4 * r + c];
+            acc = __ffma2_rn(make_float2(bv, bv), tm[4 * r + j], acc);
+          }
+          y2[4 * c + j] = acc;
         }
       }
       float y[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float acc = 0.0f;
-#pragma unroll
-          for (int r = 0; r < 4; ++r) acc = fmaf(Bm[4 * r + c], tm[8 * r + j], acc);
-          y[8 * c + j] = acc;
-        }
+      for (int i = 0; i < 16; ++i) {
+        y[2 * i] = y2[i].x;
+        y[2 * i + 1] = y2[i].y;
       }
 
       // Block extrema (NaN-propagating), clip bounds, clipped amax.
-      float mn = y[0], mx = y[0];
+      float mn = fmin3_nan(y[0], y[1], y[2]), mx = fmax3_nan(y[0], y[1], y[2]);
 #pragma unroll
-      for (int j = 1; j < 32; ++j) {
-        mn = fmin_nan(mn, y[j]);
-        mx = fmax_nan(mx, y[j]);
+      for (int j = 3; j < 31; j += 2) {
+        mn = fmin3_nan(mn, y[j], y[j + 1]);
+        mx = fmax3_nan(mx, y[j], y[j + 1]);
       }
+      mn = fmin_nan(mn, y[31]);
+      mx = fmax_nan(mx, y[31]);
       const bool finite = (fabsf(mn) <= FLT_MAX) && (fabsf(mx) <= FLT_MAX);
       const float lo = r_min * mn;
       const float hi = r_max * mx;
@@ -223,13 +246,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t sbyte = ebits > 2u ? ebits - 2u : 0u;
       const float inv_scale = __uint_as_float((254u - sbyte) << 23);
 
+      // Clip, then divide by the shared scale (an exact power-of-two multiply,
+      // two elements per packed multiply), then round to E2M1.
+      const float2 inv2 = make_float2(inv_scale, inv_scale);
       uint32_t words[4];
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        float q[8];
+        float2 q[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) q[j] = fminf(fmaxf(y[8 * w + j], lo), hi) * inv_scale;
-        words[w] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+        for (int j = 0; j < 4; ++j) {
+          const float2 c2 = make_float2(fminf(fmaxf(y[8 * w + 2 * j], lo), hi),
+                                        fminf(fmaxf(y[8 * w + 2 * j + 1], lo), hi));
+          q[j] = __fmul2_rn(c2, inv2);
+        }
+        words[w] = e2m1x8(q[0].x, q[0].y, q[1].x, q[1].y, q[2].x, q[2].y, q[3].x, q[3].y);
       }
       if (!finite) {
         sbyte = 0xFFu;
