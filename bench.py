@@ -38,6 +38,13 @@ WORKLOAD = "q_proj prefill S=2048 N=4096 M=4096 (Qwen3-8B-shaped), bf16 X, W4A4 
 QUANT_BYTES_PER_ELEM = 2 + 0.5 + 1.0 / 32  # bf16 in, E2M1 codes + E8M0 scales out
 FP4_NOMINAL_OVER_BF16 = 9.0 / 2.25         # dense fp4 / dense bf16 nominal ratio
 
+# DRAM bytes (read + write) per launch from the ncu captures summarised under profiles/, for the
+# kernel versions those captures measured; None once a kernel changes until it is re-captured.
+NCU_TRAFFIC_BYTES = {
+    "k_gemm_mxfp4": 13.42e6,   # profiles/k_gemm_mxfp4_q_proj_2048x4096x4096.md
+    "k_quant_act": 16.81e6,    # profiles/k_quant_act_q_proj_2048x4096.md
+}
+
 
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -301,11 +308,12 @@ def run_batq(args):
         "gemm_ms": g_ms,
         "tokens_per_s": ws * S / (local_ms * 1e-3),
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp4_peak, "traffic": None,
+                     "frac": gemm_tflops / fp4_peak, "traffic": NCU_TRAFFIC_BYTES["k_gemm_mxfp4"],
                      "kernel": "k_gemm_mxfp4",
                      "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16)"},
         "roofline_quant": {"bound": "hbm", "achieved": quant_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": quant_gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "k_quant_act"},
+                           "frac": quant_gbs / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC_BYTES["k_quant_act"],
+                           "kernel": "k_quant_act"},
         "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(X.numel() * X.element_size()),
                 "d2h_bytes_per_step": int(out.numel() * out.element_size()), "ms_per_step": e2e_ms},
