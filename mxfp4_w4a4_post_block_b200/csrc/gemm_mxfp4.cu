@@ -345,7 +345,8 @@ cudaError_t launch_dtype(const GemmLaunch& L) {
   if (L.S <= 16) return launch_cfg<16, true, 4, kOutBF16>(L);
   if (L.S <= 32) return launch_cfg<32, true, 4, kOutBF16>(L);
   if (L.S <= 64) return launch_cfg<64, true, 4, kOutBF16>(L);
-  return launch_cfg<256, false, 4, kOutBF16>(L);
+  if (L.S <= 128) return launch_cfg<256, false, 4, kOutBF16>(L);
+  return launch_gemm_pair(L);
 }
 
 }  // namespace

@@ -1,0 +1,370 @@
+// k_gemm_pair: W4A4 MXFP4 GEMM for prefill shapes on CTA pairs (tcgen05 cta_group::2).
+//
+// Same product as k_gemm_mxfp4 (out[s][m] = sum_n deq(a)[s][n] deq(w)[m][n],
+// fp32 accumulation in TMEM), computed by persistent clusters of two CTAs on
+// neighbouring SMs.  A pair owns a 256 (tokens) x 256 (out-features) tile:
+//   * each CTA loads its own 128 token rows of activation codes and its own
+//     128-row half of the weight tile, so one SM moves 64 bytes of operands per
+//     tensor-core cycle instead of the 96 a single-CTA 128x256 tile needs;
+//   * the leader CTA (rank 0) issues one M=256 x N=256 x K=64 block-scaled MMA
+//     per K step for both SMs; its TMA loads and its peer's count on the
+//     leader's stage barrier, and its commits arrive on both CTAs' barriers;
+//   * each CTA keeps the activation scales of its own rows and the weight
+//     scales of all 256 columns in its TMEM (128-row x 4-scale tiles copied
+//     with tcgen05.cp 32x128b.warpx4); a dedicated thread issues those copies
+//     and signals the MMA thread per stage, because copies issued by the MMA
+//     thread itself serialise with its MMAs in the tensor pipe (a stage of
+//     six copies and four MMAs takes ~990 cycles inline, ~700 when split);
+//   * eight epilogue warps per CTA read their 128 accumulator columns into
+//     registers, release TMEM for the next tile at once, and write the output
+//     through a small per-warp shared-memory box (32 rows x 32 bytes) with TMA
+//     stores while the next tile's MMAs run;
+//   * six 35 KB stages keep ~210 KB of operand loads in flight per SM: under
+//     full load the L2-to-SM latency is ~1.5 us, and this tile needs 64 bytes
+//     per SM per tensor-core cycle.
+// Every barrier wait is bounded; on expiry a bit is set in the device error
+// word and the waiting loop ends (TMEM is released and both CTAs still meet
+// at the closing cluster barrier).
+#include <cstdint>
+
+#include "host_util.h"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace batq {
+namespace {
+
+constexpr int kRowsPerCta = 128;       // token rows per CTA (TMEM lanes)
+constexpr int kTileM = 256;            // token rows per pair
+constexpr int kTileN = 256;            // out-features per pair (MMA N)
+constexpr int kHalfN = kTileN / 2;     // weight rows loaded by each CTA
+constexpr int kBKBytes = 128;          // bytes of K per stage and row (256 codes)
+constexpr int kBK = 2 * kBKBytes;
+constexpr int kKPerMma = 64;
+constexpr int kStages = 6;             // ~210 KB of operands in flight per SM (L2 latency ~1.5 us)
+constexpr int kSfAtom = 512;           // 128 rows x 4 scales
+constexpr int kEpiWarps = 8;
+constexpr int kSfWarp = 2 + kEpiWarps;          // issues the scale-factor copies
+constexpr int kThreads = (3 + kEpiWarps) * 32;
+
+constexpr int kABytes = kRowsPerCta * kBKBytes;             // 16 KB
+constexpr int kBBytes = kHalfN * kBKBytes;                  // 16 KB
+constexpr int kSfaBytes = 2 * kSfAtom;                      // 2 K atoms of own rows
+constexpr int kSfbBytes = 2 * 2 * kSfAtom;                  // 2 row atoms x 2 K atoms
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+static_assert(kStageBytes % 1024 == 0, "stage alignment");
+constexpr int kStageTxBytes = kStageBytes;                  // bytes one CTA's loads deliver per stage
+constexpr int kBoxBytes = 1024;                             // one epilogue store box: 32 rows x 32 bytes
+constexpr int kStagingBytes = kEpiWarps * kBoxBytes;
+constexpr int kBarOffset = kStages * kStageBytes + kStagingBytes;
+constexpr int kSmemBytes = kBarOffset + 512 + 1024;
+
+// TMEM columns: accumulator [0, 256), then per stage 8 columns of activation
+// scales (2 K atoms x 4) and 16 of weight scales (2 K atoms x 2 row atoms x 4).
+constexpr int kSfaCols = 8;
+constexpr int kSfbCols = 16;
+constexpr int kTmemCols = 512;
+static_assert(kTileN + kStages * (kSfaCols + kSfbCols) <= kTmemCols, "TMEM budget");
+
+struct PairArgs {
+  void* out;
+  unsigned* err;
+  int S, M, N;
+  int ldo;
+  int tiles_m, tiles_n;     // pair tiles along tokens / out-features
+  int num_kstages;
+};
+
+template <bool kOutBF16>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
+                const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfw,
+                const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ PairArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* sf_ready = acc_empty + 1;  // [kStages], leader only: scales of the stage are in TMEM
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_ready + kStages);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int cluster_id = blockIdx.x >> 1;
+  const int num_clusters = gridDim.x >> 1;
+  const int num_tiles = g.tiles_m * g.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * kEpiWarps);
+    for (int st = 0; st < kStages; ++st) mbar_init(&sf_ready[st], 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before_sync();
+  __syncwarp();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated in both
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t t_acc = tmem;
+  const uint32_t t_sfa = tmem + kTileN;
+  const uint32_t t_sfb = tmem + kTileN + kStages * kSfaCols;
+  const int nks = g.num_kstages;
+
+  if (warp == 0) {
+    // ------------------------------ producer (both CTAs) ------------------------------
+    if (lane == 0) {
+      tma_prefetch_map(&tm_a);
+      tma_prefetch_map(&tm_w);
+      tma_prefetch_map(&tm_sfa);
+      tma_prefetch_map(&tm_sfw);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = cluster_id; t < num_tiles && ok; t += num_clusters) {
+        const int a_row = (t / g.tiles_n) * kTileM + (int)rank * kRowsPerCta;
+        const int w_row0 = (t % g.tiles_n) * kTileN;
+        for (int ks = 0; ks < nks; ++ks) {
+          if (!mbar_wait(&empty[s], ph ^ 1)) {
+            set_error(g.err, kErrReleaseTimeout);
+            ok = false;
+            break;
+          }
+          const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2u * kStageTxBytes);
+          uint8_t* st = smem + s * kStageBytes;
+          tma_load_2d_pair(st, &tm_a, bar, ks * kBKBytes, a_row);
+          tma_load_2d_pair(st + kABytes, &tm_w, bar, ks * kBKBytes, w_row0 + (int)rank * kHalfN);
+          // scale tiles: {256-byte chunk, K chunk (2 per 4-scale atom), 128-row tile}
+          tma_load_3d_pair(st + kABytes + kBBytes, &tm_sfa, bar, 0, ks * 4, a_row / kRowsPerCta);
+          tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &tm_sfw, bar, 0, ks * 4, w_row0 / kRowsPerCta);
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer (leader only) ------------------------------
+    // The stages of all of this cluster's tiles form one sequence g = 0, 1, ...;
+    // stage g's scales are already in TMEM slot g % kStages when sf_ready fires.
+    if (leader && lane == 0) {
+      const int my_tiles = cluster_id < num_tiles ? (num_tiles - 1 - cluster_id) / num_clusters + 1 : 0;
+      const int total = my_tiles * nks;
+      for (int gi = 0; gi < total; ++gi) {
+        const int ks = gi % nks;
+        const uint32_t tile_iter = (uint32_t)(gi / nks);
+        if (ks == 0) {
+          // The accumulator must have been drained by both CTAs' epilogues.
+          if (!mbar_wait(acc_empty, (tile_iter & 1) ^ 1)) {
+            set_error(g.err, kErrDrainTimeout);
+            break;
+          }
+          tc_fence_after_sync();
+        }
+        const int st_idx = gi % kStages;
+        if (!mbar_wait(&sf_ready[st_idx], (uint32_t)((gi / kStages) & 1))) {
+          set_error(g.err, kErrDataTimeout);
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t sa = smem_u32(smem + st_idx * kStageBytes);
+        const uint32_t sb = sa + kABytes;
+        const int kleft = g.N - ks * kBK;
+        const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
+        const uint64_t da = sdesc_kmajor_sw128(sa);
+        const uint64_t db = sdesc_kmajor_sw128(sb);
+        for (int j = 0; j < nmma; ++j) {
+          const int a = j >> 1;
+          const int sf_id = (j & 1) * 2;
+          tc_mma_pair_mxf4(t_acc, da + (uint64_t)(j * 2), db + (uint64_t)(j * 2), idesc_mxf4_m256(kTileN, sf_id, sf_id),
+                           t_sfa + st_idx * kSfaCols + a * 4, t_sfb + st_idx * kSfbCols + a * 8,
+                           (ks > 0 || j > 0) ? 1u : 0u);
+        }
+        tc_commit_pair(&empty[st_idx], 0x3);
+        // Both epilogues may read the accumulator once every MMA of the tile has completed.
+        if (ks == nks - 1) tc_commit_pair(acc_full, 0x3);
+      }
+    }
+  } else if (warp == kSfWarp) {
+    // ---------------------- scale-factor copies (leader only) ----------------------
+    // Stage g's data has landed (full) -> copy its scale tiles into TMEM slot
+    // g % kStages in both CTAs -> sf_ready.  The slot's previous contents were
+    // consumed by the MMAs of stage g - kStages, which completed before the
+    // producer could refill the stage.
+    if (leader && lane == 0) {
+      const int my_tiles = cluster_id < num_tiles ? (num_tiles - 1 - cluster_id) / num_clusters + 1 : 0;
+      const int total = my_tiles * nks;
+      for (int gi = 0; gi < total; ++gi) {
+        const int st_idx = gi % kStages;
+        if (!mbar_wait(&full[st_idx], (uint32_t)((gi / kStages) & 1))) {
+          set_error(g.err, kErrDataTimeout);
+          break;
+        }
+        tc_fence_after_sync();
+        const int ks = gi % nks;
+        const int kleft = g.N - ks * kBK;
+        const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
+        const uint32_t ssfa = smem_u32(smem + st_idx * kStageBytes) + kABytes + kBBytes;
+        const uint32_t ssfb = ssfa + kSfaBytes;
+        for (int a = 0; a < (nmma + 1) / 2; ++a) {
+          tc_cp_pair_32x128b_warpx4(t_sfa + st_idx * kSfaCols + a * 4, sdesc_sf_atom(ssfa + a * kSfAtom));
+          // weight-scale box is {2 row tiles} x {2 K atoms}: row tile r, atom a at (2r + a) * 512
+          tc_cp_pair_32x128b_warpx4(t_sfb + st_idx * kSfbCols + a * 8, sdesc_sf_atom(ssfb + a * kSfAtom));
+          tc_cp_pair_32x128b_warpx4(t_sfb + st_idx * kSfbCols + a * 8 + 4, sdesc_sf_atom(ssfb + (2 + a) * kSfAtom));
+        }
+        tc_commit_pair_local(&sf_ready[st_idx]);
+      }
+    }
+  } else if (warp >= 2 && warp < 2 + kEpiWarps) {
+    // ------------------------------ epilogue (both CTAs) ------------------------------
+    const int ew = warp - 2;
+    const int quad = warp & 3;                // TMEM lanes 32*quad .. 32*quad+31
+    const int col0 = (ew >> 2) * 128;          // this warp's 128 accumulator columns
+    uint8_t* box = smem + kStages * kStageBytes + ew * kBoxBytes;
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+    uint32_t tile_iter = 0;
+    bool store_pending = false;
+    for (int t = cluster_id; t < num_tiles; t += num_clusters, ++tile_iter) {
+      const int row0 = (t / g.tiles_n) * kTileM + (int)rank * kRowsPerCta + 32 * quad;
+      const int n0 = (t % g.tiles_n) * kTileN + col0;
+      if (!mbar_wait(acc_full, tile_iter & 1)) {
+        set_error(g.err, kErrMmaTimeout);
+        break;
+      }
+      __syncwarp();
+      tc_fence_after_sync();
+      uint32_t v[4][32];
+      const uint32_t taddr = t_acc + ((uint32_t)(32 * quad) << 16) + col0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32cols(taddr + 32 * c, v[c]);
+      tmem_ld_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // TMEM free for the next tile
+
+      // 32-byte box rows: 8 fp32 or 16 bf16 columns; 32-byte swizzle (16-byte
+      // chunk c of row r stored at chunk c ^ ((r >> 2) & 1)).
+      constexpr int kColsPerBox = kOutBF16 ? 16 : 8;
+      uint8_t* rowp = box + lane * 32;
+      const int sw = (lane >> 2) & 1;
+#pragma unroll
+      for (int bx = 0; bx < 128 / kColsPerBox; ++bx) {
+        if (store_pending) {
+          if (lane == 0) tma_store_wait_read_all();
+          __syncwarp();
+        }
+        if constexpr (kOutBF16) {
+          const uint32_t* r = v[bx >> 1] + (bx & 1) * 16;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int o = c * 8;
+            *reinterpret_cast<uint4*>(rowp + ((c ^ sw) << 4)) =
+                make_uint4(pack_bf16x2(__uint_as_float(r[o + 0]), __uint_as_float(r[o + 1])),
+                           pack_bf16x2(__uint_as_float(r[o + 2]), __uint_as_float(r[o + 3])),
+                           pack_bf16x2(__uint_as_float(r[o + 4]), __uint_as_float(r[o + 5])),
+                           pack_bf16x2(__uint_as_float(r[o + 6]), __uint_as_float(r[o + 7])));
+          }
+        } else {
+          const uint32_t* r = v[bx >> 2] + (bx & 3) * 8;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            *reinterpret_cast<uint4*>(rowp + ((c ^ sw) << 4)) =
+                make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int x = n0 + bx * kColsPerBox;
+        if (lane == 0 && row0 < g.S && x < g.M) {
+          tma_store_2d(&tm_out, box, x, row0);
+          tma_store_commit();
+        }
+        store_pending = true;
+      }
+    }
+    if (lane == 0) tma_store_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before_sync();
+  __syncwarp();
+  cluster_sync_all();  // all MMAs done and all TMEM reads finished in both CTAs
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+template <bool kOutBF16>
+cudaError_t launch_pair_impl(const GemmLaunch& L) {
+  const uint64_t row_bytes = (uint64_t)(L.N / 2);
+  const int kpad = (L.N / 32 + 3) / 4 * 4;
+  const uint64_t sf_row_tile_bytes = (uint64_t)(kpad / 4) * kSfAtom;
+  const uint64_t a_tiles = (uint64_t)(L.S + 127) / 128;
+  const uint64_t w_tiles = (uint64_t)(L.M + 127) / 128;
+
+  CUtensorMap tm_a, tm_w, tm_sfa, tm_sfw, tm_out;
+  if (!make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_codes, row_bytes, (uint64_t)L.S, row_bytes, kBKBytes,
+                   kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_codes, row_bytes, (uint64_t)L.M, row_bytes, kBKBytes,
+                   kHalfN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  // Scale tiles as {256-byte chunks, chunks per row tile, row tiles}; one box = 2 K atoms (x 2 row tiles).
+  if (!make_map_3d(&tm_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_scales, 256, sf_row_tile_bytes / 256, a_tiles, 256,
+                   sf_row_tile_bytes, 256, 4, 1))
+    return cudaErrorInvalidValue;
+  if (!make_map_3d(&tm_sfw, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_scales, 256, sf_row_tile_bytes / 256, w_tiles, 256,
+                   sf_row_tile_bytes, 256, 4, 2))
+    return cudaErrorInvalidValue;
+  const uint32_t esz = kOutBF16 ? 2 : 4;
+  if (!make_map_2d(&tm_out, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
+                   (uint64_t)L.M, (uint64_t)L.S, (uint64_t)L.ldo * esz, 32 / esz, 32, CU_TENSOR_MAP_SWIZZLE_32B))
+    return cudaErrorInvalidValue;
+
+  PairArgs g;
+  g.out = L.out;
+  g.err = L.err;
+  g.S = L.S;
+  g.M = L.M;
+  g.N = L.N;
+  g.ldo = L.ldo;
+  g.tiles_m = (L.S + kTileM - 1) / kTileM;
+  g.tiles_n = (L.M + kTileN - 1) / kTileN;
+  g.num_kstages = (L.N + kBK - 1) / kBK;
+
+  auto kern = k_gemm_pair<kOutBF16>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int tiles = g.tiles_m * g.tiles_n;
+  const int max_clusters = sm_count() / 2;
+  const int clusters = tiles < max_clusters ? tiles : max_clusters;
+  kern<<<2 * clusters, kThreads, kSmemBytes, L.stream>>>(tm_a, tm_w, tm_sfa, tm_sfw, tm_out, g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_pair(const GemmLaunch& L) {
+  return L.out_bf16 ? launch_pair_impl<true>(L) : launch_pair_impl<false>(L);
+}
+
+}  // namespace batq

@@ -19,6 +19,10 @@ EncodeTiledFn encode_tiled_fn();
 bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
                  uint64_t outer_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
+// 3-D tensor map (no swizzle): dims {d0, d1, d2} in elements, strides of dims 1 and 2 in bytes.
+bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                 uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

@@ -39,4 +39,7 @@ struct GemmLaunch {
 
 cudaError_t launch_gemm_mxfp4(const GemmLaunch& L);
 
+// Prefill-shape GEMM on CTA pairs (tcgen05 cta_group::2); used for S > 128.
+cudaError_t launch_gemm_pair(const GemmLaunch& L);
+
 }  // namespace batq

@@ -42,6 +42,9 @@ def _run(a, sa, w, sw, out_dtype=torch.float32):
     (128, 256, 256),
     (200, 272, 320),    # ragged everything on the prefill path
     (300, 1024, 768),
+    (129, 256, 256),    # smallest CTA-pair path, second CTA nearly empty
+    (1000, 1280, 512),  # several pair tiles per cluster row
+    (520, 4096, 256),   # more pair tiles than co-resident clusters
 ])
 def test_gemm_random_operands(S, M, N):
     a, sa, w, sw = _random_operands(S, M, N, S * 7 + M + N)
