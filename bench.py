@@ -41,8 +41,8 @@ FP4_NOMINAL_OVER_BF16 = 9.0 / 2.25         # dense fp4 / dense bf16 nominal rati
 # DRAM bytes (read + write) per launch from the ncu captures summarised under profiles/, for the
 # kernel versions those captures measured; None once a kernel changes until it is re-captured.
 NCU_TRAFFIC_BYTES = {
-    "k_gemm_mxfp4": 13.42e6,   # profiles/k_gemm_mxfp4_q_proj_2048x4096x4096.md
-    "k_quant_act": 16.81e6,    # profiles/k_quant_act_q_proj_2048x4096.md
+    "k_gemm_pair": None,
+    "k_quant_act": None,
 }
 
 
@@ -218,9 +218,12 @@ def run_batq(args):
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
+    lws = torch.empty(BQ.batq_linear_workspace_size(S, N), dtype=torch.uint8, device=dev)
+
     def step():
-        BQ.batq_quant_act(X, w.A, B, ratios, codes, scales, BQ.BATQ_SCALES_MMA, stream=sp)
-        BQ.batq_gemm_mxfp4(codes, scales, wc, wsc, S, M, N, out, stream=sp)
+        # one pass of the whole path: online quantisation + block-scaled GEMM
+        # (batq_linear launches the GEMM as a programmatic dependent of the quantiser)
+        BQ.batq_linear(X, w.A, B, ratios, wc, wsc, M, lws, out, stream=sp)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -228,7 +231,8 @@ def run_batq(args):
     torch.cuda.synchronize()
     assert BQ.batq_device_error() == 0
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # timed region 1: whole steps (-> value)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -236,16 +240,26 @@ def run_batq(args):
         for i in range(args.steps):
             flush.zero_()  # L2 flush between timed steps (not inside the timed interval)
             ev[i][0].record(stream)
-            BQ.batq_quant_act(X, w.A, B, ratios, codes, scales, BQ.BATQ_SCALES_MMA, stream=sp)
+            step()
             ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        # timed region 2: each kernel alone (-> per-kernel throughput and roofline)
+        kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            kev[i][0].record(stream)
+            BQ.batq_quant_act(X, w.A, B, ratios, codes, scales, BQ.BATQ_SCALES_MMA, stream=sp)
+            kev[i][1].record(stream)
+            flush.zero_()
+            kev[i][2].record(stream)
             BQ.batq_gemm_mxfp4(codes, scales, wc, wsc, S, M, N, out, stream=sp)
-            ev[i][2].record(stream)
+            kev[i][3].record(stream)
         torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
-    t_quant = [e[0].elapsed_time(e[1]) for e in ev]
-    t_gemm = [e[1].elapsed_time(e[2]) for e in ev]
-    t_step = [a + b for a, b in zip(t_quant, t_gemm)]
+    t_step = [e[0].elapsed_time(e[1]) for e in ev]
+    t_quant = [e[0].elapsed_time(e[1]) for e in kev]
+    t_gemm = [e[2].elapsed_time(e[3]) for e in kev]
     local_ms = float(np.mean(t_step))
     q_ms, g_ms = float(np.mean(t_quant)), float(np.mean(t_gemm))
     if ws > 1:
@@ -258,7 +272,6 @@ def run_batq(args):
     Xh = X.cpu().pin_memory()
     outh = torch.empty((S, M), dtype=torch.float32).pin_memory()
     Xd = torch.empty_like(X)
-    lws = torch.empty(BQ.batq_linear_workspace_size(S, N), dtype=torch.uint8, device=dev)
     e2e_steps = max(3, min(args.steps, 50))
 
     def e2e_step():
@@ -308,8 +321,8 @@ def run_batq(args):
         "gemm_ms": g_ms,
         "tokens_per_s": ws * S / (local_ms * 1e-3),
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp4_peak, "traffic": NCU_TRAFFIC_BYTES["k_gemm_mxfp4"],
-                     "kernel": "k_gemm_mxfp4",
+                     "frac": gemm_tflops / fp4_peak, "traffic": NCU_TRAFFIC_BYTES["k_gemm_pair"],
+                     "kernel": "k_gemm_pair",
                      "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16)"},
         "roofline_quant": {"bound": "hbm", "achieved": quant_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                            "frac": quant_gbs / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC_BYTES["k_quant_act"],
@@ -317,7 +330,9 @@ def run_batq(args):
         "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(X.numel() * X.element_size()),
                 "d2h_bytes_per_step": int(out.numel() * out.element_size()), "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 4 * args.steps,
+        "timing": "value: whole steps (batq_linear) with L2 flushed before each; per-kernel figures and roofline: "
+                  "each kernel timed alone in a second loop over the same steps, L2 flushed before each launch",
         "clocks": clk.summary(),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

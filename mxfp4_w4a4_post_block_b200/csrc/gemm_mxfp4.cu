@@ -121,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_map(&tm_p);
       tma_prefetch_map(&tm_q);
+      griddep_wait();  // operands may come from the grid just before this one
       const int p_tile_atom = p0 >> 7;  // 128-row scale tile of P
       const int q_tile_atom = q0 >> 7;
       const int q_atoms_valid = min(C::kQRowAtoms, (g.rows_q_pad >> 7) - q_tile_atom);
@@ -336,8 +337,17 @@ cudaError_t launch_cfg(const GemmLaunch& L) {
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  kern<<<tiles_p * g.tiles_q, kThreads, C::kSmemBytes, L.stream>>>(tm_p, tm_q, tm_out, g);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles_p * g.tiles_q);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tm_p, tm_q, tm_out, g);
 }
 
 template <bool kOutBF16>

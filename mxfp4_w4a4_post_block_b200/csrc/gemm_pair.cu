@@ -79,7 +79,8 @@ template <bool kOutBF16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfw,
-                const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ PairArgs g) {
+                const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_out_wide,
+                const __grid_constant__ PairArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
@@ -120,6 +121,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t t_sfa = tmem + kTileN;
   const uint32_t t_sfb = tmem + kTileN + kStages * kSfaCols;
   const int nks = g.num_kstages;
+  const int my_tiles = cluster_id < num_tiles ? (num_tiles - 1 - cluster_id) / num_clusters + 1 : 0;
 
   if (warp == 0) {
     // ------------------------------ producer (both CTAs) ------------------------------
@@ -128,30 +130,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tma_prefetch_map(&tm_w);
       tma_prefetch_map(&tm_sfa);
       tma_prefetch_map(&tm_sfw);
-      int s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      for (int t = cluster_id; t < num_tiles && ok; t += num_clusters) {
-        const int a_row = (t / g.tiles_n) * kTileM + (int)rank * kRowsPerCta;
-        const int w_row0 = (t % g.tiles_n) * kTileN;
-        for (int ks = 0; ks < nks; ++ks) {
-          if (!mbar_wait(&empty[s], ph ^ 1)) {
-            set_error(g.err, kErrReleaseTimeout);
-            ok = false;
-            break;
-          }
-          const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[s], 2u * kStageTxBytes);
-          uint8_t* st = smem + s * kStageBytes;
-          tma_load_2d_pair(st, &tm_a, bar, ks * kBKBytes, a_row);
-          tma_load_2d_pair(st + kABytes, &tm_w, bar, ks * kBKBytes, w_row0 + (int)rank * kHalfN);
-          // scale tiles: {256-byte chunk, K chunk (2 per 4-scale atom), 128-row tile}
-          tma_load_3d_pair(st + kABytes + kBBytes, &tm_sfa, bar, 0, ks * 4, a_row / kRowsPerCta);
-          tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &tm_sfw, bar, 0, ks * 4, w_row0 / kRowsPerCta);
-          if (++s == kStages) {
-            s = 0;
-            ph ^= 1;
-          }
+      // Stage g of this cluster's sequence: tile cluster_id + (g / nks) * num_clusters, K step g % nks.
+      const int total = my_tiles * nks;
+      auto a_row_of = [&](int gi) { return ((cluster_id + (gi / nks) * num_clusters) / g.tiles_n) * kTileM + (int)rank * kRowsPerCta; };
+      auto w_row_of = [&](int gi) { return ((cluster_id + (gi / nks) * num_clusters) % g.tiles_n) * kTileN; };
+      auto issue_weights = [&](int gi) {
+        const int st_idx = gi % kStages;
+        uint8_t* st = smem + st_idx * kStageBytes;
+        const uint32_t bar = mapa_shared(smem_u32(&full[st_idx]), 0);
+        const int ks = gi % nks;
+        tma_load_2d_pair(st + kABytes, &tm_w, bar, ks * kBKBytes, w_row_of(gi) + (int)rank * kHalfN);
+        tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &tm_sfw, bar, 0, ks * 4, w_row_of(gi) / kRowsPerCta);
+      };
+      auto issue_activations = [&](int gi) {
+        const int st_idx = gi % kStages;
+        uint8_t* st = smem + st_idx * kStageBytes;
+        const uint32_t bar = mapa_shared(smem_u32(&full[st_idx]), 0);
+        const int ks = gi % nks;
+        tma_load_2d_pair(st, &tm_a, bar, ks * kBKBytes, a_row_of(gi));
+        // scale tiles: {256-byte chunk, K chunk (2 per 4-scale atom), 128-row tile}
+        tma_load_3d_pair(st + kABytes + kBBytes, &tm_sfa, bar, 0, ks * 4, a_row_of(gi) / kRowsPerCta);
+      };
+      // The weights do not depend on the preceding grid (the quantiser): load the
+      // first ring's weights before waiting for it, then the activations.
+      const int prologue = total < kStages ? total : kStages;
+      for (int gi = 0; gi < prologue; ++gi) {
+        if (leader) mbar_arrive_expect_tx(&full[gi], 2u * kStageTxBytes);
+        issue_weights(gi);
+      }
+      griddep_wait();
+      for (int gi = 0; gi < prologue; ++gi) issue_activations(gi);
+      int s = prologue % kStages;
+      uint32_t ph = prologue == kStages ? 1u : 0u;
+      for (int gi = prologue; gi < total; ++gi) {
+        if (!mbar_wait(&empty[s], ph ^ 1)) {
+          set_error(g.err, kErrReleaseTimeout);
+          break;
+        }
+        if (leader) mbar_arrive_expect_tx(&full[s], 2u * kStageTxBytes);
+        issue_weights(gi);
+        issue_activations(gi);
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1;
         }
       }
     }
@@ -160,7 +181,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // The stages of all of this cluster's tiles form one sequence g = 0, 1, ...;
     // stage g's scales are already in TMEM slot g % kStages when sf_ready fires.
     if (leader && lane == 0) {
-      const int my_tiles = cluster_id < num_tiles ? (num_tiles - 1 - cluster_id) / num_clusters + 1 : 0;
       const int total = my_tiles * nks;
       for (int gi = 0; gi < total; ++gi) {
         const int ks = gi % nks;
@@ -204,7 +224,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // consumed by the MMAs of stage g - kStages, which completed before the
     // producer could refill the stage.
     if (leader && lane == 0) {
-      const int my_tiles = cluster_id < num_tiles ? (num_tiles - 1 - cluster_id) / num_clusters + 1 : 0;
       const int total = my_tiles * nks;
       for (int gi = 0; gi < total; ++gi) {
         const int st_idx = gi % kStages;
@@ -253,6 +272,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // TMEM free for the next tile
+
+      const bool last_tile = (t + num_clusters >= num_tiles);
+      if (last_tile) {
+        // Nothing is loaded after the last tile, and its MMAs have completed,
+        // so the operand stages are idle: each warp stages its whole 32 x 128
+        // block there (128-byte rows, 128-byte swizzle) and issues all of its
+        // stores at once instead of one small box at a time.
+        if (store_pending) {
+          if (lane == 0) tma_store_wait_read_all();
+          __syncwarp();
+        }
+        constexpr int kWideCols = kOutBF16 ? 64 : 32;   // 128-byte box rows
+        constexpr int kWideBoxes = 128 / kWideCols;
+        uint8_t* wide = smem + ew * (kWideBoxes * 4096);
+#pragma unroll
+        for (int bx = 0; bx < kWideBoxes; ++bx) {
+          uint8_t* wrow = wide + bx * 4096 + lane * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 q;
+            if constexpr (kOutBF16) {
+              const uint32_t* r = v[2 * bx + (c >> 2)] + (c & 3) * 8;
+              q = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                             pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                             pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                             pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+            } else {
+              const uint32_t* r = v[bx] + 4 * c;
+              q = make_uint4(r[0], r[1], r[2], r[3]);
+            }
+            *reinterpret_cast<uint4*>(wrow + ((c ^ (lane & 7)) << 4)) = q;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < g.S) {
+          for (int bx = 0; bx < kWideBoxes; ++bx) {
+            const int x = n0 + bx * kWideCols;
+            if (x < g.M) tma_store_2d(&tm_out_wide, wide + bx * 4096, x, row0);
+          }
+          tma_store_commit();
+        }
+        store_pending = true;
+        continue;
+      }
 
       // 32-byte box rows: 8 fp32 or 16 bf16 columns; 32-byte swizzle (16-byte
       // chunk c of row r stored at chunk c ^ ((r >> 2) & 1)).
@@ -315,7 +379,7 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   const uint64_t a_tiles = (uint64_t)(L.S + 127) / 128;
   const uint64_t w_tiles = (uint64_t)(L.M + 127) / 128;
 
-  CUtensorMap tm_a, tm_w, tm_sfa, tm_sfw, tm_out;
+  CUtensorMap tm_a, tm_w, tm_sfa, tm_sfw, tm_out, tm_out_wide;
   if (!make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_codes, row_bytes, (uint64_t)L.S, row_bytes, kBKBytes,
                    kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
@@ -332,6 +396,9 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   const uint32_t esz = kOutBF16 ? 2 : 4;
   if (!make_map_2d(&tm_out, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
                    (uint64_t)L.M, (uint64_t)L.S, (uint64_t)L.ldo * esz, 32 / esz, 32, CU_TENSOR_MAP_SWIZZLE_32B))
+    return cudaErrorInvalidValue;
+  if (!make_map_2d(&tm_out_wide, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
+                   (uint64_t)L.M, (uint64_t)L.S, (uint64_t)L.ldo * esz, 128 / esz, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
 
   PairArgs g;
@@ -357,8 +424,19 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   const int tiles = g.tiles_m * g.tiles_n;
   const int max_clusters = sm_count() / 2;
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
-  kern<<<2 * clusters, kThreads, kSmemBytes, L.stream>>>(tm_a, tm_w, tm_sfa, tm_sfw, tm_out, g);
-  return cudaGetLastError();
+  // Launched as a programmatic dependent of the preceding grid: set-up and
+  // weight loads overlap the quantiser's tail; activations wait for it.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tm_a, tm_w, tm_sfa, tm_sfw, tm_out, tm_out_wide, g);
 }
 
 }  // namespace

@@ -62,7 +62,12 @@ struct QuantArgs {
   int rows_out;  // rows whose scales are written (S, or S rounded up to 128 in MMA layout)
   int mma_layout;
   int tiles_r, tiles_c;
+  unsigned long long tiles_c_magic;  // ceil(2^40 / tiles_c): t / tiles_c = (t * magic) >> 40 for t < 2^24
 };
+
+__device__ __forceinline__ int tile_row(int t, const QuantArgs& p) {
+  return (int)(((unsigned long long)(unsigned)t * p.tiles_c_magic) >> 40);
+}
 
 __device__ __forceinline__ uint32_t mma_scale_offset(int row, int kb, int kpad) {
   return (uint32_t)(((row >> 7) * (kpad >> 2) + (kb >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (kb & 3));
@@ -101,7 +106,7 @@ __device__ __forceinline__ void load_block(const uint8_t* box, int lane, float x
 }
 
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kBF16 ? 3 : 1)
     k_quant_act(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
   using T = Tile<kBF16>;
   extern __shared__ uint8_t smem_raw[];
@@ -118,6 +123,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&empty[s], kConsumerWarps);
     }
     fence_barrier_init();
+    // The GEMM that consumes these codes may start its set-up (and its weight
+    // loads) while this grid runs; it waits for this grid before reading codes.
+    griddep_launch_dependents();
   }
   __syncthreads();
 
@@ -134,8 +142,9 @@ __global__ void __launch_bounds__(kThreads, 2)
           set_error(p.err, kErrReleaseTimeout);
           break;
         }
-        const int r0 = (t / p.tiles_c) * kRows;
-        const int c0 = (t % p.tiles_c) * kCols;
+        const int tr = tile_row(t, p);
+        const int r0 = tr * kRows;
+        const int c0 = (t - tr * p.tiles_c) * kCols;
         if (r0 < p.S) {
           const int nb = min(kCols, p.k - c0);  // even: k is even and c0 a multiple of 8
           uint8_t* dst = smem + s * T::kStageBytes;
@@ -160,8 +169,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   int s = 0;
   uint32_t ph = 0;
   for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-    const int r0 = (t / p.tiles_c) * kRows;
-    const int c0 = (t % p.tiles_c) * kCols;
+    const int tr = tile_row(t, p);
+    const int r0 = tr * kRows;
+    const int c0 = (t - tr * p.tiles_c) * kCols;
     const int b = c0 + warp;
     const int row = r0 + lane;
     if (!mbar_wait(&full[s], ph)) {
@@ -319,6 +329,7 @@ cudaError_t launch_impl(const QuantLaunch& L) {
   a.rows_out = L.mma_layout ? (L.S + 127) / 128 * 128 : L.S;
   a.tiles_r = (a.rows_out + kRows - 1) / kRows;
   a.tiles_c = (a.k + kCols - 1) / kCols;
+  a.tiles_c_magic = ((1ull << 40) + (unsigned long long)a.tiles_c - 1) / (unsigned long long)a.tiles_c;
 
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -330,7 +341,7 @@ cudaError_t launch_impl(const QuantLaunch& L) {
     attr_set[dev] = true;
   }
   const int ntiles = a.tiles_r * a.tiles_c;
-  const int per_sm = kBF16 ? 2 : 1;
+  const int per_sm = kBF16 ? 3 : 1;
   const int grid = ntiles < sm_count() * per_sm ? ntiles : sm_count() * per_sm;
   k_quant_act<kBF16><<<grid, kThreads, T::kSmemBytes, L.stream>>>(map, a);
   return cudaGetLastError();
