@@ -212,6 +212,18 @@ BATQ_API batq_status batq_linear_no_alloc(const void* X, batq_dtype x_dtype, int
                                           batq_dtype out_dtype, void* out, int ldo, void* stream);
 
 /*
+ * Failure-path self-test: launches a one-thread kernel that waits on a
+ * barrier nothing ever arrives on, with a bounded wait of `limit_us`
+ * microseconds (1 .. 1e6) -- the same bounded wait every libbatq kernel uses
+ * for its pipeline barriers.  The wait expires, the kernel sets bit 0 of the
+ * device error word and returns; the context stays usable.  Follow with
+ * batq_device_error to read (and clear) the word.  The method has no
+ * counterpart of this call.  Errors: BATQ_ERR_INVALID_ARG, BATQ_ERR_ARCH,
+ * BATQ_ERR_CUDA.
+ */
+BATQ_API batq_status batq_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error
  * word.  Kernels set bits there when a bounded wait on a barrier gives up
  * (bit 0: data never arrived; bit 1: a stage was never released; bit 2: an

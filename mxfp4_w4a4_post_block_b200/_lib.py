@@ -42,6 +42,7 @@ SIGNATURES = {
                              ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
     "batq_linear_no_alloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_int,
                                       _c_int, _vp, _c_int, _vp]),
+    "batq_selftest_wait_timeout": (_c_int, [ctypes.c_uint, _vp]),
     "batq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint)]),
 }
 

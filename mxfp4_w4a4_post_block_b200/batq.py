@@ -157,6 +157,11 @@ def batq_linear_no_alloc(X, A, B, ratios, w_codes, w_scales, M, out, stream=None
                                             _stream(stream)), "batq_linear_no_alloc")
 
 
+def batq_selftest_wait_timeout(limit_us: int, stream=None):
+    """Launch the bounded-wait self-test kernel (its wait always expires)."""
+    _check(_lib.load().batq_selftest_wait_timeout(limit_us, _stream(stream)), "batq_selftest_wait_timeout")
+
+
 def batq_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device error word."""
     v = ctypes.c_uint(0)

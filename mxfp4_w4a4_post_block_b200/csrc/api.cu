@@ -331,6 +331,16 @@ batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx
   return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, s);
 }
 
+batq_status batq_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_arch();
+  if (st != BATQ_OK) return st;
+  unsigned* err = error_word();
+  if (!err) return BATQ_ERR_CUDA;
+  cudaError_t e = batq::launch_wait_selftest((uint64_t)limit_us * 1000ull, err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
+}
+
 batq_status batq_device_error(void* stream, unsigned int* flags_out) {
   if (!flags_out) return BATQ_ERR_INVALID_ARG;
   unsigned* word = error_word();

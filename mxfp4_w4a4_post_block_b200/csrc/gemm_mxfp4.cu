@@ -16,10 +16,12 @@
 //   warp 0     TMA producer: per stage a 128 x 256-element P tile, a BN x 256
 //              Q tile (both 128-byte swizzled) and their scale atoms (1-D bulk
 //              copies of the 512-byte 128x4 scale tiles);
-//   warp 1     TMEM allocator and MMA issuer: copies the stage's scales into
-//              TMEM (tcgen05.cp 32x128b.warpx4) and issues four
-//              tcgen05.mma kind::mxf4.block_scale (K = 64 each), then commits
+//   warp 1     TMEM allocator and MMA issuer: four tcgen05.mma
+//              kind::mxf4.block_scale (K = 64 each) per stage, then commits
 //              the stage back to the producer;
+//   warp 6     copies each stage's scales into TMEM (tcgen05.cp 32x128b.warpx4)
+//              and signals the MMA thread (copies issued by the MMA thread
+//              itself would serialise with its MMAs);
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator quadrant of each warp,
 //              staged through shared memory and written with TMA stores
 //              (prefill) or stored directly, coalesced along i (decode).
@@ -37,7 +39,8 @@ constexpr int kBKBytes = 128;     // bytes of K per stage and row (= 256 E2M1 co
 constexpr int kBK = 2 * kBKBytes; // K elements per stage
 constexpr int kKPerMma = 64;      // K of one kind::mxf4 MMA
 constexpr int kMmasPerStage = kBK / kKPerMma;
-constexpr int kThreads = 192;     // 6 warps
+constexpr int kThreads = 224;     // 7 warps: producer, MMA, 4 epilogue, scale copies
+constexpr int kSfWarp = 6;
 constexpr int kSfAtom = 512;      // bytes of one 128-row x 4-scale tile
 
 template <int BN, bool kSwap, int kStages>
@@ -85,7 +88,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::kStageBytes);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* sf_ready = acc_full + 1;  // [kStages] scales of the stage are in TMEM
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_ready + kStages);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -100,6 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(&sf_ready[s], 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -159,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0;
       bool ok = true;
       for (int ks = 0; ks < nks && ok; ++ks) {
-        if (!mbar_wait(&full[s], ph)) {
+        if (!mbar_wait(&sf_ready[s], ph)) {
           set_error(g.err, kErrDataTimeout);
           ok = false;
           break;
@@ -168,20 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* st = smem + s * C::kStageBytes;
         const uint32_t sp = smem_u32(st);
         const uint32_t sq = sp + C::kPBytes;
-        const uint32_t ssfp = sq + C::kQBytes;
-        const uint32_t ssfq = ssfp + C::kSfPBytes;
         const int kleft = g.N - ks * kBK;
         const int nmma = kleft >= kBK ? kMmasPerStage : kleft / kKPerMma;
-        const int katoms = (nmma + 1) / 2;
-        // Scale factors of this stage into TMEM.
-        for (int a = 0; a < katoms; ++a) {
-          tc_cp_32x128b_warpx4(t_sfp + s * C::kSfPCols + a * 4, sdesc_sf_atom(ssfp + a * kSfAtom));
-#pragma unroll
-          for (int r = 0; r < C::kQRowAtoms; ++r) {
-            tc_cp_32x128b_warpx4(t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms + r * 4,
-                                 sdesc_sf_atom(ssfq + (r * 2 + a) * kSfAtom));
-          }
-        }
         const uint64_t dp = sdesc_kmajor_sw128(sp);
         const uint64_t dq = sdesc_kmajor_sw128(sq);
         for (int j = 0; j < nmma; ++j) {
@@ -201,6 +194,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Signal the epilogue once every issued MMA has completed (also on error).
       tc_commit(acc_full);
+    }
+  } else if (warp == kSfWarp) {
+    // ------------------------------ scale copies ------------------------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int ks = 0; ks < nks; ++ks) {
+        if (!mbar_wait(&full[s], ph)) {
+          set_error(g.err, kErrDataTimeout);
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t ssfp = smem_u32(smem + s * C::kStageBytes) + C::kPBytes + C::kQBytes;
+        const uint32_t ssfq = ssfp + C::kSfPBytes;
+        const int kleft = g.N - ks * kBK;
+        const int nmma = kleft >= kBK ? kMmasPerStage : kleft / kKPerMma;
+        for (int a = 0; a < (nmma + 1) / 2; ++a) {
+          tc_cp_32x128b_warpx4(t_sfp + s * C::kSfPCols + a * 4, sdesc_sf_atom(ssfp + a * kSfAtom));
+#pragma unroll
+          for (int r = 0; r < C::kQRowAtoms; ++r) {
+            tc_cp_32x128b_warpx4(t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms + r * 4,
+                                 sdesc_sf_atom(ssfq + (r * 2 + a) * kSfAtom));
+          }
+        }
+        tc_commit(&sf_ready[s]);
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
     }
   } else {
     // ------------------------------ epilogue ------------------------------

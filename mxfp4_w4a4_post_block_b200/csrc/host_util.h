@@ -23,6 +23,11 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, 
 bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                  uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 
+// 3-D tensor map with a swizzle mode (strides need not be increasing).
+bool make_map_3d_swizzled(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1,
+                          uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                          uint32_t b2, CUtensorMapSwizzle swizzle);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

@@ -42,4 +42,7 @@ cudaError_t launch_gemm_mxfp4(const GemmLaunch& L);
 // Prefill-shape GEMM on CTA pairs (tcgen05 cta_group::2); used for S > 128.
 cudaError_t launch_gemm_pair(const GemmLaunch& L);
 
+// One-thread kernel whose barrier wait always expires after limit_ns.
+cudaError_t launch_wait_selftest(uint64_t limit_ns, unsigned* err, cudaStream_t stream);
+
 }  // namespace batq

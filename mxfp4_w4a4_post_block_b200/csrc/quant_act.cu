@@ -8,8 +8,9 @@
 //
 // Memory-bound design:
 //   * one producer warp streams tiles of 32 tokens x 8 blocks into a 4-stage
-//     shared-memory ring with TMA (one 32-row box per block column, swizzled
-//     so the per-lane row reads below are bank-conflict free);
+//     shared-memory ring with one 3-D TMA box per tile ({32 elements, 32
+//     tokens, 8 blocks}: each block column lands as a 32-row slab, swizzled so
+//     the per-lane row reads below are bank-conflict free);
 //   * the producer also stages the tile's eight B_i and clip ratios with
 //     1-D bulk copies, so consumers read them from shared memory (broadcast);
 //   * eight consumer warps, warp w owning block column c0 + w of the tile and
@@ -149,8 +150,9 @@ __global__ void __launch_bounds__(kThreads, kBF16 ? 3 : 1)
           const int nb = min(kCols, p.k - c0);  // even: k is even and c0 a multiple of 8
           uint8_t* dst = smem + s * T::kStageBytes;
           const uint32_t pbytes = (uint32_t)nb * 64u + (p.ratios != nullptr ? (uint32_t)nb * 8u : 0u);
-          mbar_arrive_expect_tx(&full[s], (uint32_t)(nb * T::kBoxBytes) + pbytes);
-          for (int j = 0; j < nb; ++j) tma_load_2d(dst + j * T::kBoxBytes, &tmx, &full[s], (c0 + j) * 32, r0);
+          // the box always delivers all 8 block columns (zero-filled past k)
+          mbar_arrive_expect_tx(&full[s], (uint32_t)T::kXBytes + pbytes);
+          tma_load_3d(dst, &tmx, &full[s], 0, r0, c0);
           bulk_load(dst + T::kBOffset, p.B + (size_t)c0 * 16, (uint32_t)nb * 64u, &full[s]);
           if (p.ratios != nullptr) bulk_load(dst + T::kROffset, p.ratios + (size_t)c0 * 2, (uint32_t)nb * 8u, &full[s]);
         } else {
@@ -306,11 +308,12 @@ __global__ void __launch_bounds__(kThreads, kBF16 ? 3 : 1)
 template <bool kBF16>
 cudaError_t launch_impl(const QuantLaunch& L) {
   using T = Tile<kBF16>;
+  // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
   CUtensorMap map;
-  const uint64_t stride = (uint64_t)L.ldx * (kBF16 ? 2u : 4u);
-  if (!make_map_2d(&map, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.X,
-                   (uint64_t)L.N, (uint64_t)L.S, stride, 32, kRows,
-                   kBF16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) {
+  const uint64_t esz = kBF16 ? 2u : 4u;
+  if (!make_map_3d_swizzled(&map, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.X,
+                            32, (uint64_t)L.S, (uint64_t)(L.N / 32), (uint64_t)L.ldx * esz, 32 * esz, 32, kRows,
+                            kCols, kBF16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) {
     return cudaErrorInvalidValue;
   }
   QuantArgs a;
