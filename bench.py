@@ -37,6 +37,7 @@ METRIC = "BAT+clip+MXFP4 quant GB/s & W4A4 GEMM TFLOPS (% of HBM / FP4 roofline)
 WORKLOAD = "q_proj prefill S=2048 N=4096 M=4096 (Qwen3-8B-shaped), bf16 X, W4A4 MXFP4"
 QUANT_BYTES_PER_ELEM = 2 + 0.5 + 1.0 / 32  # bf16 in, E2M1 codes + E8M0 scales out
 FP4_NOMINAL_OVER_BF16 = 9.0 / 2.25         # dense fp4 / dense bf16 nominal ratio
+ROT = 10                                   # rotating input/output sets (see run_batq)
 
 # DRAM bytes (read + write) per launch from the ncu captures summarised under profiles/, for the
 # kernel versions those captures measured; None once a kernel changes until it is re-captured.
@@ -204,91 +205,124 @@ def run_batq(args):
     w = WL.q_proj(seed=2 + rank)
     S, N, M = w.S, w.N, w.M
     dev = torch.device("cuda", local)
-    X = torch.from_numpy(np.ascontiguousarray(w.x_bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    X0 = torch.from_numpy(np.ascontiguousarray(w.x_bits).view(np.int16)).view(torch.bfloat16).to(dev)
     B = torch.from_numpy(np.ascontiguousarray(w.B.reshape(-1))).to(dev)
     ratios = torch.from_numpy(BQ.batq_clip_ratios(w.alpha_min, w.alpha_max)).to(dev)
     Wd = torch.from_numpy(w.W).to(dev)
-    wc, wsc = BQ.empty_act_buffers(M, N, device=dev)
+    wc0, wsc0 = BQ.empty_act_buffers(M, N, device=dev)
     pws = torch.empty(BQ.batq_prepare_workspace_size(N), dtype=torch.uint8, device=dev)
-    BQ.batq_prepare_weights(Wd, w.A, w.B, wc, wsc, pws)
-    del Wd
-    codes, scales = BQ.empty_act_buffers(S, N, device=dev)
-    out = torch.empty((S, M), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    BQ.batq_prepare_weights(Wd, w.A, w.B, wc0, wsc0, pws)
+    del Wd, pws
+    lws_bytes = BQ.batq_linear_workspace_size(S, N)
+    code_bytes = -(-S * (N // 2) // 256) * 256
+
+    # ROT independent sets (activations, prepared weights, workspace, output), visited
+    # round-robin: between two uses of a set every other set streams through L2, so each
+    # step reads its inputs from HBM (far more than the 126 MB L2 in between).
+    sets = []
+    for _ in range(ROT):
+        ws_buf = torch.empty(lws_bytes, dtype=torch.uint8, device=dev)
+        sets.append({
+            "X": X0.clone(), "wc": wc0.clone(), "wsc": wsc0.clone(), "lws": ws_buf,
+            "codes": ws_buf[:S * (N // 2)].view(S, N // 2), "scales": ws_buf[code_bytes:],
+            "out": torch.empty((S, M), dtype=torch.float32, device=dev),
+        })
+    set_bytes = sum(t.numel() * t.element_size() for t in
+                    (sets[0]["X"], sets[0]["wc"], sets[0]["wsc"], sets[0]["lws"], sets[0]["out"]))
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
-    lws = torch.empty(BQ.batq_linear_workspace_size(S, N), dtype=torch.uint8, device=dev)
-
-    def step():
+    def step(i):
         # one pass of the whole path: online quantisation + block-scaled GEMM
         # (batq_linear launches the GEMM as a programmatic dependent of the quantiser)
-        BQ.batq_linear(X, w.A, B, ratios, wc, wsc, M, lws, out, stream=sp)
+        z = sets[i % ROT]
+        BQ.batq_linear(z["X"], w.A, B, ratios, z["wc"], z["wsc"], M, z["lws"], z["out"], stream=sp)
 
-    for _ in range(max(3, args.warmup)):
-        flush.zero_()
-        step()
+    def quant(i):
+        z = sets[i % ROT]
+        BQ.batq_quant_act(z["X"], w.A, B, ratios, z["codes"], z["scales"], BQ.BATQ_SCALES_MMA, stream=sp)
+
+    def gemm(i):
+        z = sets[i % ROT]
+        BQ.batq_gemm_mxfp4(z["codes"], z["scales"], z["wc"], z["wsc"], S, M, N, z["out"], stream=sp)
+
+    def timed(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    warm = max(3, args.warmup)
+    for i in range(ROT):
+        quant(i)  # every set's workspace holds valid codes before the GEMM-only loop
+    for fn in (step, quant, gemm):
+        for i in range(warm):
+            fn(i)
     torch.cuda.synchronize()
     assert BQ.batq_device_error() == 0
 
-    # timed region 1: whole steps (-> value)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            flush.zero_()  # L2 flush between timed steps (not inside the timed interval)
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        # timed region 2: each kernel alone (-> per-kernel throughput and roofline)
-        kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-        for i in range(args.steps):
-            flush.zero_()
-            kev[i][0].record(stream)
-            BQ.batq_quant_act(X, w.A, B, ratios, codes, scales, BQ.BATQ_SCALES_MMA, stream=sp)
-            kev[i][1].record(stream)
-            flush.zero_()
-            kev[i][2].record(stream)
-            BQ.batq_gemm_mxfp4(codes, scales, wc, wsc, S, M, N, out, stream=sp)
-            kev[i][3].record(stream)
-        torch.cuda.synchronize()
+        # timed region 1: whole steps back to back (-> value)
+        local_ms = timed(step, args.steps)
+        # timed region 2: each kernel alone, back to back over the same rotation
+        # (-> per-kernel throughput and roofline)
+        q_ms = timed(quant, args.steps)
+        g_ms = timed(gemm, args.steps)
     if ws > 1:
         dist.barrier()
-    t_step = [e[0].elapsed_time(e[1]) for e in ev]
-    t_quant = [e[0].elapsed_time(e[1]) for e in kev]
-    t_gemm = [e[2].elapsed_time(e[3]) for e in kev]
-    local_ms = float(np.mean(t_step))
-    q_ms, g_ms = float(np.mean(t_quant)), float(np.mean(t_gemm))
-    if ws > 1:
         tt = torch.tensor([local_ms, q_ms, g_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         local_ms, q_ms, g_ms = [float(v) for v in tt.tolist()]
     assert BQ.batq_device_error() == 0
 
-    # end to end through the public call with host buffers (pinned), copies inside the timed region
-    Xh = X.cpu().pin_memory()
-    outh = torch.empty((S, M), dtype=torch.float32).pin_memory()
-    Xd = torch.empty_like(X)
-    e2e_steps = max(3, min(args.steps, 50))
+    # End to end through the public call with host buffers: pinned host X in, fp32 result
+    # out, every step.  Copies in both directions run on their own streams so that step
+    # i's upload, step i-1's compute and step i-2's download overlap (double-buffered).
+    Xh = X0.cpu().pin_memory()
+    outh = [torch.empty((S, M), dtype=torch.float32).pin_memory() for _ in range(2)]
+    z0 = sets[0]
+    Xd = [torch.empty_like(X0) for _ in range(2)]
+    outd = [torch.empty((S, M), dtype=torch.float32, device=dev) for _ in range(2)]
+    s_up, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    e2e_steps = max(4, min(args.steps, 50))
 
-    def e2e_step():
-        Xd.copy_(Xh, non_blocking=True)
-        BQ.batq_linear(Xd, w.A, B, ratios, wc, wsc, M, lws, out, stream=sp)
-        outh.copy_(out, non_blocking=True)
+    def e2e_run(n):
+        up = [torch.cuda.Event() for _ in range(n)]
+        done = [torch.cuda.Event() for _ in range(n)]
+        dn = [torch.cuda.Event() for _ in range(n)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s_up)
+        stream.wait_event(e0)
+        s_dn.wait_event(e0)
+        for i in range(n):
+            j = i % 2
+            if i >= 2:
+                s_up.wait_event(done[i - 2])      # Xd[j] no longer read
+            with torch.cuda.stream(s_up):
+                Xd[j].copy_(Xh, non_blocking=True)
+            up[i].record(s_up)
+            stream.wait_event(up[i])
+            if i >= 2:
+                stream.wait_event(dn[i - 2])      # outd[j] already downloaded
+            BQ.batq_linear(Xd[j], w.A, B, ratios, z0["wc"], z0["wsc"], M, z0["lws"], outd[j], stream=sp)
+            done[i].record(stream)
+            s_dn.wait_event(done[i])
+            with torch.cuda.stream(s_dn):
+                outh[j].copy_(outd[j], non_blocking=True)
+            dn[i].record(s_dn)
+        s_up.wait_event(dn[n - 1])
+        e1.record(s_up)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
 
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_run(3)
+    e2e_ms = e2e_run(e2e_steps)
     if ws > 1:
         tt = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -306,14 +340,16 @@ def run_batq(args):
         "unit": "TFLOP/s",
         "n_gpus": ws,
         "steps": args.steps,
-        "warmup": max(3, args.warmup),
+        "warmup": warm,
         "ms_per_step": local_ms,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "e2m1",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "S": S, "N": N, "M": M, "l2": "flushed between steps (256 MB write)",
+        "config": {"workload": WORKLOAD, "S": S, "N": N, "M": M,
+                   "l2": f"inputs larger than L2: {ROT} rotating sets of X, prepared weights, workspace and "
+                         f"output ({ROT * set_bytes / 2**20:.0f} MiB) visited round-robin, steps back to back",
                    "parallelism": f"replicas x{ws} (independent batches)"},
         "quant_gbs": quant_gbs,
         "quant_ms": q_ms,
@@ -328,11 +364,14 @@ def run_batq(args):
                            "frac": quant_gbs / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC_BYTES["k_quant_act"],
                            "kernel": "k_quant_act"},
         "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(X.numel() * X.element_size()),
-                "d2h_bytes_per_step": int(out.numel() * out.element_size()), "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
+                "d2h_bytes_per_step": int(outh[0].numel() * outh[0].element_size()), "ms_per_step": e2e_ms,
+                "note": "batq_linear on pinned host buffers; upload, compute and download on three streams, "
+                        "double-buffered"},
         "gpu_launches": 4 * args.steps,
-        "timing": "value: whole steps (batq_linear) with L2 flushed before each; per-kernel figures and roofline: "
-                  "each kernel timed alone in a second loop over the same steps, L2 flushed before each launch",
+        "timing": "CUDA events on the launching stream around K back-to-back launches; value: whole steps "
+                  "(batq_linear: quantiser + GEMM); per-kernel figures and roofline: K quantiser launches, then K "
+                  "GEMM launches, each over the same rotation; gpu_launches counts these three loops",
         "clocks": clk.summary(),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

@@ -164,7 +164,7 @@ batq_status check_gemm_args(const uint8_t* a_codes, const uint8_t* a_scales, con
 
 batq_status launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
                         const uint8_t* w_scales, int S, int M, int N, batq_dtype out_dtype, void* out, int ldo,
-                        cudaStream_t stream) {
+                        bool weights_ready, cudaStream_t stream) {
   batq::GemmLaunch L;
   L.a_codes = a_codes;
   L.a_scales = a_scales;
@@ -178,6 +178,7 @@ batq_status launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const u
   L.ldo = ldo;
   L.err = error_word();
   L.stream = stream;
+  L.weights_ready = weights_ready;
   cudaError_t e = batq::launch_gemm_mxfp4(L);
   if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
   return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
@@ -293,7 +294,9 @@ batq_status batq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, con
   if (st != BATQ_OK) return st;
   st = check_arch();
   if (st != BATQ_OK) return st;
-  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo,
+  // The preceding grid may be anything (e.g. the weight quantiser of
+  // batq_prepare_weights): wait for it before reading any operand.
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, false,
                      static_cast<cudaStream_t>(stream));
 }
 
@@ -328,7 +331,10 @@ batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx
   st = launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA, nullptr,
                     s);
   if (st != BATQ_OK) return st;
-  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, s);
+  // The quantiser just launched writes only the workspace and starts its
+  // dependents after every earlier grid has finished, so the GEMM may fetch
+  // weights while the quantiser runs.
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, s);
 }
 
 batq_status batq_selftest_wait_timeout(unsigned int limit_us, void* stream) {

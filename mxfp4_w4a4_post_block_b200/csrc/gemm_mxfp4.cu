@@ -106,6 +106,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_full, 1);
     for (int s = 0; s < kStages; ++s) mbar_init(&sf_ready[s], 1);
     fence_barrier_init();
+    // The next grid in the stream may start its set-up now; it waits for this
+    // grid to finish before it touches memory.
+    griddep_launch_dependents();
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::kTmemCols);

@@ -73,6 +73,7 @@ struct PairArgs {
   int ldo;
   int tiles_m, tiles_n;     // pair tiles along tokens / out-features
   int num_kstages;
+  int early_weights;        // weights may be read before waiting for the preceding grid
 };
 
 template <bool kOutBF16>
@@ -107,6 +108,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(acc_empty, 2 * kEpiWarps);
     for (int st = 0; st < kStages; ++st) mbar_init(&sf_ready[st], 1);
     fence_barrier_init();
+    // The next grid in the stream may start its set-up now; it waits for this
+    // grid to finish before it touches memory.
+    griddep_launch_dependents();
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, kTmemCols);
@@ -151,14 +155,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // scale tiles: {256-byte chunk, K chunk (2 per 4-scale atom), 128-row tile}
         tma_load_3d_pair(st + kABytes + kBBytes, &tm_sfa, bar, 0, ks * 4, a_row_of(gi) / kRowsPerCta);
       };
-      // The weights do not depend on the preceding grid (the quantiser): load the
-      // first ring's weights before waiting for it, then the activations.
+      // When the preceding grid is known not to write the weights (the linear
+      // layer's own quantiser), the first ring's weights are loaded before
+      // waiting for that grid; the activations always come after the wait.
       const int prologue = total < kStages ? total : kStages;
+      if (!g.early_weights) griddep_wait();
       for (int gi = 0; gi < prologue; ++gi) {
         if (leader) mbar_arrive_expect_tx(&full[gi], 2u * kStageTxBytes);
         issue_weights(gi);
       }
-      griddep_wait();
+      if (g.early_weights) griddep_wait();
       for (int gi = 0; gi < prologue; ++gi) issue_activations(gi);
       int s = prologue % kStages;
       uint32_t ph = prologue == kStages ? 1u : 0u;
@@ -411,6 +417,7 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   g.tiles_m = (L.S + kTileM - 1) / kTileM;
   g.tiles_n = (L.M + kTileN - 1) / kTileN;
   g.num_kstages = (L.N + kBK - 1) / kBK;
+  g.early_weights = L.weights_ready ? 1 : 0;
 
   auto kern = k_gemm_pair<kOutBF16>;
   static bool attr_set[64] = {false};

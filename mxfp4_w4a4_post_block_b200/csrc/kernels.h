@@ -22,6 +22,10 @@ struct QuantLaunch {
 };
 
 // Returns cudaErrorInvalidValue when the tensor map cannot be encoded.
+// All kernels are launched as programmatic dependents of the preceding grid in
+// the stream: each waits for that grid before touching memory it may write
+// (the GEMM's weights excepted when GemmLaunch::weights_ready is set), and
+// lets its own dependents start early.
 cudaError_t launch_quant_act(const QuantLaunch& L);
 
 struct GemmLaunch {
@@ -35,6 +39,10 @@ struct GemmLaunch {
   int ldo;
   unsigned* err;
   cudaStream_t stream;
+  // The grid launched just before this one in the stream does not write the
+  // weights, so they may be read before waiting for it (set by the linear
+  // layer, whose preceding grid is its own quantiser).
+  bool weights_ready;
 };
 
 cudaError_t launch_gemm_mxfp4(const GemmLaunch& L);

@@ -124,9 +124,6 @@ __global__ void __launch_bounds__(kThreads, kBF16 ? 3 : 1)
       mbar_init(&empty[s], kConsumerWarps);
     }
     fence_barrier_init();
-    // The GEMM that consumes these codes may start its set-up (and its weight
-    // loads) while this grid runs; it waits for this grid before reading codes.
-    griddep_launch_dependents();
   }
   __syncthreads();
 
@@ -136,6 +133,13 @@ __global__ void __launch_bounds__(kThreads, kBF16 ? 3 : 1)
     // ---------------- producer: one thread issues the TMA boxes ----------------
     if (lane == 0) {
       tma_prefetch_map(&tmx);
+      // Launched as a programmatic dependent: X (and the outputs, which the
+      // preceding grid may still read) are touched only after that grid has
+      // finished.  Consumers access memory only after this thread's loads.
+      griddep_wait();
+      // Every grid before this one is complete from here on, so the dependent
+      // GEMM may start (and fetch weights) while the codes are produced.
+      griddep_launch_dependents();
       int s = 0;
       uint32_t ph = 0;
       for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -346,8 +350,17 @@ cudaError_t launch_impl(const QuantLaunch& L) {
   const int ntiles = a.tiles_r * a.tiles_c;
   const int per_sm = kBF16 ? 3 : 1;
   const int grid = ntiles < sm_count() * per_sm ? ntiles : sm_count() * per_sm;
-  k_quant_act<kBF16><<<grid, kThreads, T::kSmemBytes, L.stream>>>(map, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = T::kSmemBytes;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16>, map, a);
 }
 
 }  // namespace
