@@ -42,8 +42,8 @@ ROT = 10                                   # rotating input/output sets (see run
 # DRAM bytes (read + write) per launch from the ncu captures summarised under profiles/, for the
 # kernel versions those captures measured; None once a kernel changes until it is re-captured.
 NCU_TRAFFIC_BYTES = {
-    "k_gemm_pair": None,
-    "k_quant_act": None,
+    "k_gemm_pair": 13_465_600,
+    "k_quant_act": 16_802_304,
 }
 
 
