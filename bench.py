@@ -188,6 +188,97 @@ def run_reference(args):
     return 0
 
 
+def per_config(dev, peaks):
+    """Kernel-alone throughput on the other workloads (down_proj prefill, decode S=16, the seven
+    linears of one S=8192 layer), each timed over back-to-back launches whose inputs rotate through
+    more than the 126 MB L2.  Activation codes come from the quantiser; weight codes are random
+    bytes with unit scales (timing does not depend on their values)."""
+    import torch
+
+    from mxfp4_w4a4_post_block_b200 import batq as BQ
+    from mxfp4_w4a4_post_block_b200 import workloads as WL
+
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    fp4_peak = peaks["bf16_tflops"] * FP4_NOMINAL_OVER_BF16
+
+    def timed(fns, reps):
+        for f in fns:
+            f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            for f in fns:
+                f()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * len(fns))
+
+    def linear_sets(w, copies):
+        S, N, M = w.S, w.N, w.M
+        X = torch.from_numpy(np.ascontiguousarray(w.x_bits).view(np.int16)).view(torch.bfloat16).to(dev)
+        B = torch.from_numpy(np.ascontiguousarray(w.B.reshape(-1))).to(dev)
+        ratios = torch.from_numpy(BQ.batq_clip_ratios(w.alpha_min, w.alpha_max)).to(dev)
+        g = torch.Generator(device=dev).manual_seed(w.seed)
+        out = []
+        for c in range(copies):
+            codes, scales = BQ.empty_act_buffers(S, N, device=dev)
+            wc, wsc = BQ.empty_act_buffers(M, N, device=dev)
+            wc.random_(0, 256, generator=g)
+            wsc.fill_(127)
+            out.append({"X": X if c == 0 else X.clone(), "B": B, "ratios": ratios, "A": w.A, "codes": codes,
+                        "scales": scales, "wc": wc, "wsc": wsc, "S": S, "N": N, "M": M,
+                        "out": torch.empty((S, M), dtype=torch.float32, device=dev)})
+        return out
+
+    def q_fn(z):
+        return lambda: BQ.batq_quant_act(z["X"], z["A"], z["B"], z["ratios"], z["codes"], z["scales"],
+                                         BQ.BATQ_SCALES_MMA, stream=sp)
+
+    def g_fn(z):
+        return lambda: BQ.batq_gemm_mxfp4(z["codes"], z["scales"], z["wc"], z["wsc"], z["S"], z["M"], z["N"],
+                                          z["out"], stream=sp)
+
+    res = {}
+    # down_proj prefill: S=4096, N=12288, M=4096 (three copies: 300 MB of activations)
+    zs = linear_sets(WL.down_proj(with_w=False), 3)
+    q_ms = timed([q_fn(z) for z in zs], 10)
+    g_ms = timed([g_fn(z) for z in zs], 10)
+    S, N, M = zs[0]["S"], zs[0]["N"], zs[0]["M"]
+    qb = S * N * QUANT_BYTES_PER_ELEM
+    res["down_proj_4096x12288x4096"] = {
+        "quant_us": q_ms * 1e3, "quant_gbs": qb / q_ms / 1e6, "quant_frac_hbm": qb / q_ms / 1e6 / peaks["hbm_gbs"],
+        "gemm_us": g_ms * 1e3, "gemm_tflops": 2.0 * S * N * M / g_ms / 1e9,
+        "gemm_frac_fp4": 2.0 * S * N * M / g_ms / 1e9 / fp4_peak}
+    del zs
+    # decode: S=16, N=4096, M=24576; the GEMM streams the prepared weights (three copies: 160 MB)
+    zs = linear_sets(WL.decode(16, with_w=False), 3)
+    q_ms = timed([q_fn(z) for z in zs], 30)
+    g_ms = timed([g_fn(z) for z in zs], 30)
+    S, N, M = zs[0]["S"], zs[0]["N"], zs[0]["M"]
+    wb = M * N * (0.5 + 1.0 / 32)
+    res["decode_16x4096x24576"] = {
+        "quant_us": q_ms * 1e3, "gemm_us": g_ms * 1e3, "gemm_weight_gbs": wb / g_ms / 1e6,
+        "gemm_frac_hbm": wb / g_ms / 1e6 / peaks["hbm_gbs"], "note": "launch-bound quantiser (128 KB); "
+        "GEMM judged on weight bytes against HBM"}
+    del zs
+    # the seven linears of one S=8192 layer, one after another (each launch reads new inputs)
+    zs = []
+    for j in range(7):
+        zs += linear_sets(WL.layer_linear(j, with_w=False), 1)
+    q_ms = timed([q_fn(z) for z in zs], 3) * 7
+    g_ms = timed([g_fn(z) for z in zs], 3) * 7
+    qb = sum(z["S"] * z["N"] for z in zs) * QUANT_BYTES_PER_ELEM
+    fl = sum(2.0 * z["S"] * z["N"] * z["M"] for z in zs)
+    res["layer_S8192_7_linears"] = {
+        "quant_us": q_ms * 1e3, "quant_gbs": qb / q_ms / 1e6, "quant_frac_hbm": qb / q_ms / 1e6 / peaks["hbm_gbs"],
+        "gemm_us": g_ms * 1e3, "gemm_tflops": fl / g_ms / 1e9, "gemm_frac_fp4": fl / g_ms / 1e9 / fp4_peak}
+    del zs
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_batq(args):
     import torch
     import torch.distributed as dist
@@ -374,6 +465,8 @@ def run_batq(args):
                   "GEMM launches, each over the same rotation; gpu_launches counts these three loops",
         "clocks": clk.summary(),
     }
+    if rank == 0 and not args.no_configs:
+        line["per_config"] = per_config(dev, peaks)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         from oracle import batq_oracle as O
         wp = O.prepare_weights(w.W, w.A, w.B)
@@ -393,6 +486,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["batq", "reference"], default="batq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload kernel timings")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

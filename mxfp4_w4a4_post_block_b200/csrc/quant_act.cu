@@ -7,15 +7,18 @@
 // the divide-then-round order; OCP MX v1.0 for the scale rule).
 //
 // Memory-bound design:
-//   * one producer warp streams tiles of 32 tokens x 8 blocks into a 4-stage
-//     shared-memory ring with one 3-D TMA box per tile ({32 elements, 32
-//     tokens, 8 blocks}: each block column lands as a 32-row slab, swizzled so
-//     the per-lane row reads below are bank-conflict free);
+//   * one CTA per SM, each owning a contiguous, equal share of the tiles (so
+//     no SM is left with more work than another); one producer warp streams
+//     tiles of 32 tokens x 8 blocks into a shared-memory ring with one 3-D TMA
+//     box per tile ({32 elements, 32 tokens, 8 blocks}: each block column lands
+//     as a 32-row slab, swizzled so the per-lane row reads below are
+//     bank-conflict free);
 //   * the producer also stages the tile's eight B_i and clip ratios with
 //     1-D bulk copies, so consumers read them from shared memory (broadcast);
-//   * eight consumer warps, warp w owning block column c0 + w of the tile and
-//     lane l owning token r0 + l, so B_i and the clip ratios are warp-uniform
-//     and A is read from the kernel's parameter (constant) bank;
+//   * consumer groups of eight warps take the CTA's tiles in turn (three
+//     groups for bf16 input); in a group, warp w owns block column c0 + w of
+//     the tile and lane l owns token r0 + l, so B_i and the clip ratios are
+//     warp-uniform and A is read from the kernel's parameter (constant) bank;
 //   * the transform runs on packed fp32x2 FMAs: T = X A produces column
 //     pairs (T[r][2j], T[r][2j+1]) from a duplicated x value and an A row
 //     pair, then Y = B^T T reuses those column pairs with a duplicated B
@@ -34,14 +37,15 @@ namespace batq {
 namespace {
 
 constexpr int kRows = 32;         // tokens per tile (one per lane)
-constexpr int kCols = 8;          // 32-blocks per tile (one per consumer warp)
-constexpr int kStages = 4;        // shared-memory ring depth
-constexpr int kConsumerWarps = kCols;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kCols = 8;          // 32-blocks per tile (one per warp of a consumer group)
 constexpr uint8_t kPadScale = 0x7F;
 
 template <bool kBF16>
 struct Tile {
+  static constexpr int kGroups = kBF16 ? 3 : 1;          // consumer groups per CTA
+  static constexpr int kStages = kGroups * (kBF16 ? 3 : 4);  // ring depth (a multiple of kGroups)
+  static constexpr int kConsumerWarps = kGroups * kCols;
+  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
   static constexpr int kBlockBytes = kBF16 ? 64 : 128;      // one 32-element block row
   static constexpr int kBoxBytes = kRows * kBlockBytes;     // one TMA box (32 tokens x 1 block)
   static constexpr int kXBytes = kCols * kBoxBytes;         // activations of one tile
@@ -74,17 +78,28 @@ __device__ __forceinline__ uint32_t mma_scale_offset(int row, int kb, int kpad) 
   return (uint32_t)(((row >> 7) * (kpad >> 2) + (kb >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (kb & 3));
 }
 
-// One token's 32-element block from the swizzled tile.  bf16 boxes use the
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float2 lds64f(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
+// One token's 32-element block from the swizzled tile (box = shared address of its slab).  bf16 boxes use the
 // 64-byte swizzle (16-byte chunk c of row t stored at chunk c ^ ((t >> 1) & 3)),
 // fp32 boxes the 128-byte swizzle (chunk c ^ (t & 7)).
 template <bool kBF16>
-__device__ __forceinline__ void load_block(const uint8_t* box, int lane, float x[32]) {
+__device__ __forceinline__ void load_block(uint32_t box, int lane, float x[32]) {
   if constexpr (kBF16) {
-    const uint8_t* row = box + lane * 64;
+    const uint32_t row = box + lane * 64;
     const int sw = (lane >> 1) & 3;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
+      const uint4 v = lds128(row + ((c ^ sw) << 4));
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -93,43 +108,49 @@ __device__ __forceinline__ void load_block(const uint8_t* box, int lane, float x
       }
     }
   } else {
-    const uint8_t* row = box + lane * 128;
+    const uint32_t row = box + lane * 128;
     const int sw = lane & 7;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      const float4 v = *reinterpret_cast<const float4*>(row + ((c ^ sw) << 4));
-      x[c * 4 + 0] = v.x;
-      x[c * 4 + 1] = v.y;
-      x[c * 4 + 2] = v.z;
-      x[c * 4 + 3] = v.w;
+      const uint4 v = lds128(row + ((c ^ sw) << 4));
+      x[c * 4 + 0] = __uint_as_float(v.x);
+      x[c * 4 + 1] = __uint_as_float(v.y);
+      x[c * 4 + 2] = __uint_as_float(v.z);
+      x[c * 4 + 3] = __uint_as_float(v.w);
     }
   }
 }
 
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads, kBF16 ? 3 : 1)
+__global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
     k_quant_act(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
   using T = Tile<kBF16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * T::kStageBytes);
-  uint64_t* empty = full + kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::kStages * T::kStageBytes);
+  uint64_t* empty = full + T::kStages;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < T::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], kCols);  // the eight warps of the group that consumed it
     }
     fence_barrier_init();
   }
   __syncthreads();
 
-  const int ntiles = p.tiles_r * p.tiles_c;
+  // This CTA's contiguous share of the tiles (one CTA per SM, shares differ by
+  // at most one tile).  Local tile i sits in stage i % kStages; consumer group
+  // i % kGroups processes it (kStages is a multiple of kGroups, so each stage
+  // always serves the same group).
+  const long long ntiles = (long long)p.tiles_r * p.tiles_c;
+  const int t_begin = (int)((long long)blockIdx.x * ntiles / gridDim.x);
+  const int nloc = (int)((long long)(blockIdx.x + 1) * ntiles / gridDim.x) - t_begin;
 
-  if (warp == kConsumerWarps) {
+  if (warp == T::kConsumerWarps) {
     // ---------------- producer: one thread issues the TMA boxes ----------------
     if (lane == 0) {
       tma_prefetch_map(&tmx);
@@ -140,13 +161,13 @@ __global__ void __launch_bounds__(kThreads, kBF16 ? 3 : 1)
       // Every grid before this one is complete from here on, so the dependent
       // GEMM may start (and fetch weights) while the codes are produced.
       griddep_launch_dependents();
-      int s = 0;
-      uint32_t ph = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        if (!mbar_wait(&empty[s], ph ^ 1)) {
+      for (int i = 0; i < nloc; ++i) {
+        const int s = i % T::kStages;
+        if (!mbar_wait(&empty[s], ((i / T::kStages) & 1) ^ 1)) {
           set_error(p.err, kErrReleaseTimeout);
           break;
         }
+        const int t = t_begin + i;
         const int tr = tile_row(t, p);
         const int r0 = tr * kRows;
         const int c0 = (t - tr * p.tiles_c) * kCols;
@@ -162,41 +183,41 @@ __global__ void __launch_bounds__(kThreads, kBF16 ? 3 : 1)
         } else {
           mbar_arrive(&full[s]);  // padding rows only: nothing to load
         }
-        if (++s == kStages) {
-          s = 0;
-          ph ^= 1;
-        }
       }
     }
     return;
   }
 
   // ---------------- consumers ----------------
-  int s = 0;
-  uint32_t ph = 0;
-  for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+  const int grp = warp / kCols;
+  const int wc = warp % kCols;  // block column of the tile owned by this warp
+  for (int i = grp; i < nloc; i += T::kGroups) {
+    const int s = i % T::kStages;
+    const int t = t_begin + i;
     const int tr = tile_row(t, p);
     const int r0 = tr * kRows;
     const int c0 = (t - tr * p.tiles_c) * kCols;
-    const int b = c0 + warp;
+    const int b = c0 + wc;
     const int row = r0 + lane;
-    if (!mbar_wait(&full[s], ph)) {
+    if (!mbar_wait(&full[s], (i / T::kStages) & 1)) {
       set_error(p.err, kErrDataTimeout);
       break;
     }
     if (r0 < p.S && b < p.k) {
-      const uint8_t* st = smem + s * T::kStageBytes;
+      const uint32_t st = smem_u32(smem) + s * T::kStageBytes;
       float x[32];
-      load_block<kBF16>(st + warp * T::kBoxBytes, lane, x);
+      load_block<kBF16>(st + wc * T::kBoxBytes, lane, x);
 
       // B_i (row-major 4x4) and the clip ratios: the same for the whole warp.
-      const float4* bp = reinterpret_cast<const float4*>(st + T::kBOffset) + 4 * warp;
-      const float4 b0 = bp[0], b1 = bp[1], b2 = bp[2], b3 = bp[3];
-      const float Bm[16] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w,
-                            b2.x, b2.y, b2.z, b2.w, b3.x, b3.y, b3.z, b3.w};
+      const uint32_t bp = st + T::kBOffset + wc * 64;
+      const uint4 b0 = lds128(bp), b1 = lds128(bp + 16), b2 = lds128(bp + 32), b3 = lds128(bp + 48);
+      const float Bm[16] = {__uint_as_float(b0.x), __uint_as_float(b0.y), __uint_as_float(b0.z), __uint_as_float(b0.w),
+                            __uint_as_float(b1.x), __uint_as_float(b1.y), __uint_as_float(b1.z), __uint_as_float(b1.w),
+                            __uint_as_float(b2.x), __uint_as_float(b2.y), __uint_as_float(b2.z), __uint_as_float(b2.w),
+                            __uint_as_float(b3.x), __uint_as_float(b3.y), __uint_as_float(b3.z), __uint_as_float(b3.w)};
       float r_min = 1.0f, r_max = 1.0f;
       if (p.ratios != nullptr) {
-        const float2 r = reinterpret_cast<const float2*>(st + T::kROffset)[warp];
+        const float2 r = lds64f(st + T::kROffset + wc * 8);
         r_min = r.x;
         r_max = r.y;
       }
@@ -302,10 +323,6 @@ __global__ void __launch_bounds__(kThreads, kBF16 ? 3 : 1)
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-    if (++s == kStages) {
-      s = 0;
-      ph ^= 1;
-    }
   }
 }
 
@@ -348,11 +365,10 @@ cudaError_t launch_impl(const QuantLaunch& L) {
     attr_set[dev] = true;
   }
   const int ntiles = a.tiles_r * a.tiles_c;
-  const int per_sm = kBF16 ? 3 : 1;
-  const int grid = ntiles < sm_count() * per_sm ? ntiles : sm_count() * per_sm;
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();  // one CTA per SM
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(T::kThreads);
   cfg.dynamicSmemBytes = T::kSmemBytes;
   cfg.stream = L.stream;
   cudaLaunchAttribute attr[1];
