@@ -257,11 +257,20 @@ def per_config(dev, peaks):
     q_ms = timed([q_fn(z) for z in zs], 30)
     g_ms = timed([g_fn(z) for z in zs], 30)
     S, N, M = zs[0]["S"], zs[0]["N"], zs[0]["M"]
+    lws = [torch.empty(BQ.batq_linear_workspace_size(S, N), dtype=torch.uint8, device=dev) for _ in zs]
+
+    def l_fn(z, ws_buf):
+        return lambda: BQ.batq_linear(z["X"], z["A"], z["B"], z["ratios"], z["wc"], z["wsc"], M, ws_buf, z["out"],
+                                      stream=sp)
+
+    l_ms = timed([l_fn(z, b) for z, b in zip(zs, lws)], 30)
     wb = M * N * (0.5 + 1.0 / 32)
     res["decode_16x4096x24576"] = {
         "quant_us": q_ms * 1e3, "gemm_us": g_ms * 1e3, "gemm_weight_gbs": wb / g_ms / 1e6,
-        "gemm_frac_hbm": wb / g_ms / 1e6 / peaks["hbm_gbs"], "note": "launch-bound quantiser (128 KB); "
-        "GEMM judged on weight bytes against HBM"}
+        "gemm_frac_hbm": wb / g_ms / 1e6 / peaks["hbm_gbs"], "linear_us": l_ms * 1e3,
+        "linear_weight_gbs": wb / l_ms / 1e6,
+        "note": "launch-bound quantiser (128 KB); GEMM judged on weight bytes against HBM; linear = "
+                "batq_linear (the GEMM prefetches its weights into L2 while the quantiser runs)"}
     del zs
     # the seven linears of one S=8192 layer, one after another (each launch reads new inputs)
     zs = []

@@ -76,6 +76,9 @@ struct GemmArgs {
   int ldo;
   int tiles_q;              // tiles along Q
   int num_kstages;          // ceil(N / 256)
+  const uint8_t* w_codes;   // the weight operand (P when swapped, else Q), for the L2 prefetch
+  int w_rows;               // its valid rows
+  int early_w;              // the preceding grid does not write the weights: prefetch them before waiting
 };
 
 template <int BN, bool kSwap, int kStages, bool kOutBF16>
@@ -91,6 +94,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* sf_ready = acc_full + 1;  // [kStages] scales of the stage are in TMEM
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_ready + kStages);
 
+  // Fetch the TMA descriptors while the barriers and TMEM are set up.
+  if (threadIdx.x == 0) {
+    tma_prefetch_map(&tm_p);
+    tma_prefetch_map(&tm_q);
+    tma_prefetch_map(&tm_out);
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int tile_p = blockIdx.x / g.tiles_q;
@@ -127,8 +136,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
     if (lane == 0) {
-      tma_prefetch_map(&tm_p);
-      tma_prefetch_map(&tm_q);
+      if (g.early_w) {
+        // This CTA's weight rows (contiguous) and their scale tiles go to L2 while
+        // the preceding grid (the linear layer's quantiser) still runs.
+        const int w0 = kSwap ? p0 : q0;
+        const int wn = min(kSwap ? kBM : BN, g.w_rows - w0);
+        const size_t row_bytes = (size_t)(g.N >> 1);
+        const uint8_t* wbase = g.w_codes + (size_t)w0 * row_bytes;
+        const size_t wbytes = (size_t)wn * row_bytes;
+        for (size_t off = 0; off < wbytes; off += 65536)
+          bulk_prefetch_l2(wbase + off, (uint32_t)(wbytes - off < 65536 ? wbytes - off : 65536));
+        const size_t sf_tile = (size_t)(g.kpad >> 2) * kSfAtom;  // one 128-row scale tile
+        const uint8_t* wsf = kSwap ? g.p_scales : g.q_scales;
+        for (int a = 0; a < (wn + 127) / 128; ++a) bulk_prefetch_l2(wsf + (size_t)((w0 >> 7) + a) * sf_tile, (uint32_t)sf_tile);
+      }
       griddep_wait();  // operands may come from the grid just before this one
       const int p_tile_atom = p0 >> 7;  // 128-row scale tile of P
       const int q_tile_atom = q0 >> 7;
@@ -352,6 +373,9 @@ cudaError_t launch_cfg(const GemmLaunch& L) {
   g.ldo = L.ldo;
   g.tiles_q = (rows_q + BN - 1) / BN;
   g.num_kstages = (L.N + kBK - 1) / kBK;
+  g.w_codes = L.w_codes;
+  g.w_rows = L.M;
+  g.early_w = L.weights_ready ? 1 : 0;
   const int tiles_p = (rows_p + kBM - 1) / kBM;
 
   auto kern = k_gemm_mxfp4<BN, kSwap, kStages, kOutBF16>;

@@ -91,6 +91,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* sf_ready = acc_empty + 1;  // [kStages], leader only: scales of the stage are in TMEM
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_ready + kStages);
 
+  // Fetch the TMA descriptors while the barriers and TMEM are set up.
+  if (threadIdx.x == 0) {
+    tma_prefetch_map(&tm_a);
+    tma_prefetch_map(&tm_w);
+    tma_prefetch_map(&tm_sfa);
+    tma_prefetch_map(&tm_sfw);
+    tma_prefetch_map(&tm_out);
+    tma_prefetch_map(&tm_out_wide);
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -130,10 +139,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------ producer (both CTAs) ------------------------------
     if (lane == 0) {
-      tma_prefetch_map(&tm_a);
-      tma_prefetch_map(&tm_w);
-      tma_prefetch_map(&tm_sfa);
-      tma_prefetch_map(&tm_sfw);
       // Stage g of this cluster's sequence: tile cluster_id + (g / nks) * num_clusters, K step g % nks.
       const int total = my_tiles * nks;
       auto a_row_of = [&](int gi) { return ((cluster_id + (gi / nks) * num_clusters) / g.tiles_n) * kTileM + (int)rank * kRowsPerCta; };

@@ -192,6 +192,11 @@ __device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v
 // ------------------------------------------------------------ bulk copies
 
 // 1-D bulk copy global -> shared (both 16-byte aligned, size a multiple of 16).
+// Prefetch `bytes` of global memory into L2 (16-byte aligned address, size a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),

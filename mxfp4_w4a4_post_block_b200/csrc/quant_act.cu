@@ -129,6 +129,10 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::kStages * T::kStageBytes);
   uint64_t* empty = full + T::kStages;
+  // Fetch the TMA descriptors while the barriers and TMEM are set up.
+  if (threadIdx.x == 0) {
+    tma_prefetch_map(&tmx);
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -153,7 +157,6 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
   if (warp == T::kConsumerWarps) {
     // ---------------- producer: one thread issues the TMA boxes ----------------
     if (lane == 0) {
-      tma_prefetch_map(&tmx);
       // Launched as a programmatic dependent: X (and the outputs, which the
       // preceding grid may still read) are touched only after that grid has
       // finished.  Consumers access memory only after this thread's loads.

@@ -141,7 +141,8 @@ def _linear(w, out_dtype=torch.float32):
 
 
 @pytest.mark.parametrize("maker", [WL.tiny, lambda: WL.custom(200, 320, 272, 51),
-                                   lambda: WL.q_proj(), lambda: WL.decode(4)])
+                                   lambda: WL.custom(100, 320, 272, 52),
+                                   lambda: WL.q_proj(), lambda: WL.decode(4), lambda: WL.decode(16)])
 def test_linear_matches_quant_then_gemm_and_oracle(maker):
     w = maker()
     out, wc, wsc = _linear(w)
