@@ -141,3 +141,48 @@ def test_zero_and_nonfinite_blocks():
     ref = O.quant_act(X, w.A, w.B, w.alpha_min, w.alpha_max)
     np.testing.assert_array_equal(scales, ref["scales"])
     PT.assert_quant_parity(codes, scales, ref, "zero/nonfinite")
+
+
+def test_clip_lo_above_hi_gives_constant_block():
+    """Same-sign blocks with r_min > r_max: lo = r_min*mn exceeds hi = r_max*mx, so
+    min(max(y, lo), hi) is hi everywhere (the clamp order the oracle fixes)."""
+    rng = np.random.default_rng(21)
+    S, N = 40, 128
+    k = N // 32
+    X = (5.0 + 0.5 * rng.standard_normal((S, N))).astype(np.float32)
+    X[S // 2:] *= -1.0  # negative blocks too
+    w = WL.Workload("lo_gt_hi", 21, S, N, 16, "f32", X, X, np.eye(8, dtype=np.float32),
+                    np.tile(np.eye(4, dtype=np.float32), (k, 1, 1)), np.full(k, 3.0, np.float32),
+                    np.full(k, -3.0, np.float32), None)
+    codes, scales, y, _ = GU.gpu_quant(w, BQ.BATQ_SCALES_LINEAR)
+    ref = O.quant_act(X, w.A, w.B, w.alpha_min, w.alpha_max)
+    np.testing.assert_array_equal(scales, ref["scales"])
+    np.testing.assert_array_equal(codes, ref["codes"])
+    # every positive block collapses to a single code (its hi, the clipped amax)
+    u = O.unpack_nibbles(codes[: S // 2]).reshape(S // 2, k, 32)
+    assert (u == u[:, :, :1]).all()
+
+
+def test_subnormal_blocks_and_smallest_scale():
+    """Blocks whose values are E2M1 grid points times 2^-127 (many of them fp32
+    subnormals): the shared exponent clamps at -127 (byte 0) and every code is exact."""
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], np.float64)
+    rng = np.random.default_rng(22)
+    S, N = 24, 64
+    k = N // 32
+    X = np.empty((S, N), np.float32)
+    for r in range(S):
+        v = rng.choice(grid, N) * rng.choice([-1.0, 1.0], N)
+        v[0] = 6.0  # every block's amax is 6 * 2^-127 -> e = -127
+        v[32] = -6.0
+        X[r] = (v * 2.0 ** -127).astype(np.float32)
+    assert (np.abs(X[X != 0]) < 2.0 ** -126).any()  # subnormal inputs present
+    w = WL.Workload("subnormal", 22, S, N, 16, "f32", X, X, np.eye(8, dtype=np.float32),
+                    np.tile(np.eye(4, dtype=np.float32), (k, 1, 1)), np.full(k, 40, np.float32),
+                    np.full(k, 40, np.float32), None)
+    codes, scales, y, _ = GU.gpu_quant(w, BQ.BATQ_SCALES_LINEAR)
+    np.testing.assert_array_equal(y, X)
+    ref = O.quant_act(X, w.A, w.B, w.alpha_min, w.alpha_max)
+    assert (ref["scales"] == 0).all()
+    np.testing.assert_array_equal(scales, ref["scales"])
+    np.testing.assert_array_equal(codes, ref["codes"])
