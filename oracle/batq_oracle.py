@@ -37,6 +37,18 @@ the design notes):
   the dense 32x32 P_i, rounded to fp32, then MXFP4 round-to-nearest along K
   without clipping.
 
+W4A8 variant (the pages' second main setting, MXFP8 activations against the
+MXFP4 weights; p3 abstract and Table 2):
+
+* E4M3 elements (bias 7, 3 mantissa bits, subnormals m * 2^-9, largest 448),
+  shared scale 2^(floor(log2 amax) - 8) (OCP MX v1.0, emax_elem = 8), round to
+  nearest even, and magnitudes above 448 saturate to 448 (the scaled amax lies
+  in [256, 512), so the largest elements of a block can saturate; OCP leaves
+  overflow to the implementation, and saturation is the reading taken).
+* The same clip, zero-block and non-finite rules as MXFP4.
+* The MXFP4 weights are consumed from one-byte E4M3 containers that hold the
+  same E2M1 values exactly (every E2M1 value is an E4M3 value).
+
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 closed forms, brute force and the pages' Table 1.
 """
@@ -401,3 +413,122 @@ def linear(X, A, B, alpha_min, alpha_max, W):
     wp = prepare_weights(W, A, B)
     out, T = gemm(act["codes"], act["scales"], wp["codes"], wp["scales"])
     return out, T, act, wp
+
+
+# ---------------------------------------------------------------------------
+# W4A8 variant: MXFP8 (E4M3) activations against the MXFP4 weights
+# [p3 abstract and Table 2 (W4A8 rows); OCP MX v1.0 for FP8 E4M3]
+# ---------------------------------------------------------------------------
+
+def _e4m3_magnitudes() -> np.ndarray:
+    """Values of the 127 finite non-negative E4M3 codes 0x00..0x7E (0x7F is NaN).
+
+    Exponent bias 7, 3 mantissa bits; exponent field 0 holds the subnormals
+    m * 2^-9.  The largest value is 1.75 * 2^8 = 448.
+    """
+    vals = []
+    for c in range(0x7F):
+        ex, m = c >> 3, c & 7
+        vals.append(m * 2.0 ** -9 if ex == 0 else (1.0 + m / 8.0) * 2.0 ** (ex - 7))
+    return np.asarray(vals, dtype=np.float64)
+
+
+E4M3_MAGNITUDE = _e4m3_magnitudes()
+E4M3_MAX = 448.0
+E4M3_EMAX = 8  # exponent of the largest normal (OCP MX v1.0: emax_elem for E4M3)
+
+
+def e8m0_exponent_e4m3(amax: np.ndarray) -> np.ndarray:
+    """Shared-scale exponent for E4M3 elements: floor(log2 amax) - 8, clamped to [-127, 127]."""
+    a = np.asarray(amax, dtype=np.float64)
+    _, ex = np.frexp(a)
+    e = ex.astype(np.int64) - 1 - E4M3_EMAX
+    e = np.where(a == 0.0, -127, e)
+    return np.clip(e, -127, 127)
+
+
+def e4m3_encode(q: np.ndarray) -> np.ndarray:
+    """8-bit E4M3 codes of q by round-to-nearest-even over the value table, saturating at +-448.
+
+    For each |q| the two neighbouring table entries are found; the nearer one
+    wins, and an exact midpoint goes to the even code (mantissa bit 0).
+    Magnitudes above 448 give 448 (no NaN is produced).  The sign bit (bit 7)
+    is the sign of q, so negative values that round to zero give 0x80.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    mag = np.minimum(np.abs(q), E4M3_MAX)
+    hi = np.searchsorted(E4M3_MAGNITUDE, mag, side="left")  # first entry >= mag
+    hi = np.clip(hi, 0, len(E4M3_MAGNITUDE) - 1)
+    lo = np.clip(hi - 1, 0, len(E4M3_MAGNITUDE) - 1)
+    d_lo = mag - E4M3_MAGNITUDE[lo]
+    d_hi = E4M3_MAGNITUDE[hi] - mag
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(mag == E4M3_MAGNITUDE[hi], hi, code)
+    sign = np.signbit(q).astype(np.int64)
+    return (sign << 7) | code
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Value of each finite 8-bit E4M3 code (0x7F / 0xFF would be NaN; never produced here)."""
+    codes = np.asarray(codes, dtype=np.int64)
+    mag = E4M3_MAGNITUDE[np.minimum(codes & 0x7F, 0x7E)]
+    mag = np.where((codes & 0x7F) == 0x7F, np.nan, mag)
+    return np.where(codes & 0x80, -mag, mag)
+
+
+def mxfp8_quantize(V: np.ndarray, nonfinite: np.ndarray | None = None):
+    """MXFP8 (E4M3) of fp32 rows V: per 32-block scale 2^(floor(log2 amax) - 8), divide, round.
+
+    Returns (codes (rows, N) uint8, scale bytes (rows, N/32) uint8, q (rows, N)
+    fp64 before rounding).  A block with a non-finite value gets scale 0xFF and
+    zero codes, as in the MXFP4 path.
+    """
+    V = np.asarray(V, dtype=np.float32)
+    rows, N = V.shape
+    k = N // G
+    Vb = V.reshape(rows, k, G).astype(np.float64)
+    if nonfinite is None:
+        nonfinite = ~np.all(np.isfinite(Vb), axis=2)
+    with np.errstate(invalid="ignore"):
+        amax = np.abs(Vb).max(axis=2)
+    amax = np.where(nonfinite, 0.0, amax)
+    e = e8m0_exponent_e4m3(amax)
+    q = Vb * np.exp2(-e.astype(np.float64))[:, :, None]  # exact: power-of-two scaling in fp64
+    q = np.where(nonfinite[:, :, None], 0.0, q)
+    codes = e4m3_encode(q).reshape(rows, N)
+    codes = np.where(np.repeat(nonfinite, G, axis=1), 0, codes).astype(np.uint8)
+    scale = np.where(nonfinite, 0xFF, e + 127).astype(np.uint8)
+    return codes, scale, q.reshape(rows, N)
+
+
+def dequantize_e4m3(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """fp64 values code * 2^(byte - 127) for (rows, N) E4M3 codes; byte 0xFF decodes to NaN."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    rows, N = codes.shape
+    k = N // G
+    vals = e4m3_decode(codes).reshape(rows, k, G)
+    s = np.asarray(scales, dtype=np.int64)
+    factor = np.where(s == 0xFF, np.nan, np.exp2((s - 127).astype(np.float64)))
+    return (vals * factor[:, :, None]).reshape(rows, N)
+
+
+def quant_act_mxfp8(X, A, B, alpha_min, alpha_max) -> dict:
+    """Online activation path of the W4A8 variant: y = x P_i, the same clip, MXFP8 (E4M3)."""
+    Y = transform(X, A, B)
+    Yh, lo, hi, nonfinite = clip_blocks(Y, clip_ratios(alpha_min), clip_ratios(alpha_max))
+    codes, scales, q = mxfp8_quantize(Yh, nonfinite)
+    return {"Y": Y, "Y_hat": Yh, "codes": codes, "scales": scales, "q": q,
+            "nonfinite": nonfinite, "lo": lo, "hi": hi}
+
+
+def e4m3_containers_from_e2m1(packed: np.ndarray) -> np.ndarray:
+    """(rows, N/2) packed E2M1 codes -> (rows, N) E4M3 bytes holding the same values (exact)."""
+    return e4m3_encode(e2m1_decode(unpack_nibbles(packed))).astype(np.uint8)
+
+
+def gemm_w4a8(a_codes8, a_scales, w_codes8, w_scales):
+    """out = deq(a) deq(w)^T in fp64 for E4M3 activation and weight codes, plus T = sum |a||w|."""
+    Da = dequantize_e4m3(a_codes8, a_scales)
+    Dw = dequantize_e4m3(w_codes8, w_scales)
+    return Da @ Dw.T, np.abs(Da) @ np.abs(Dw).T

@@ -409,3 +409,121 @@ def test_gemm_linear_in_codes_order():
     wc = wp["codes"].reshape(w.M, w.k, 16)[:, perm].reshape(w.M, -1)
     out2, _ = O.gemm(ac, act["scales"][:, perm], wc, wp["scales"][:, perm])
     np.testing.assert_allclose(out2, out, rtol=1e-13, atol=1e-13)
+
+
+# ------------------------------------------------- W4A8 (MXFP8 E4M3) ----
+
+def _e4m3_value_from_bits(c):
+    """E4M3 from its bit fields, written independently of the oracle's table:
+    sign bit 7, exponent bits 6..3 (bias 7), mantissa bits 2..0; exponent 0 is subnormal."""
+    s = -1.0 if c & 0x80 else 1.0
+    e = (c >> 3) & 0xF
+    m = c & 7
+    if e == 0xF and m == 7:
+        return math.nan
+    return s * (m / 8.0 * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7))
+
+
+def test_e4m3_table_matches_bit_fields_and_extremes():
+    vals = [_e4m3_value_from_bits(c) for c in range(0x7F)]
+    np.testing.assert_array_equal(O.E4M3_MAGNITUDE, vals)
+    assert O.E4M3_MAGNITUDE[0x7E] == 448.0 and O.E4M3_MAGNITUDE[1] == 2.0 ** -9
+    assert O.E4M3_MAGNITUDE[8] == 2.0 ** -6  # smallest normal
+    for c in range(256):
+        if (c & 0x7F) != 0x7F:
+            v = O.e4m3_decode(np.array([c]))[0]
+            assert v == _e4m3_value_from_bits(c) or (v == 0 and _e4m3_value_from_bits(c) == 0)
+
+
+def test_e4m3_encode_brute_force_nearest_even_saturating():
+    """Against a search over all finite codes: nearest value, ties to the even code,
+    |q| > 448 saturates, sign from the sign of q."""
+    rng = np.random.default_rng(7)
+    mags = np.concatenate([rng.uniform(0, 500, 3000), np.exp2(rng.uniform(-12, 9, 3000)),
+                           (O.E4M3_MAGNITUDE[:-1] + O.E4M3_MAGNITUDE[1:]) / 2,  # every midpoint
+                           O.E4M3_MAGNITUDE, [448.0, 456.0, 464.0, 470.0, 1e6]])
+    q = mags * rng.choice([-1.0, 1.0], len(mags))
+    table = np.array([_e4m3_value_from_bits(c) for c in range(0x7F)])
+    got = O.e4m3_encode(q)
+    for qi, ci in zip(q, got):
+        a = min(abs(qi), 448.0)
+        d = np.abs(table - a)
+        best = np.flatnonzero(d == d.min())
+        want = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        assert ci == (want | (0x80 if np.signbit(qi) else 0)), (qi, ci, want)
+
+
+def test_e4m3_round_trip_and_sign_of_zero():
+    for c in range(256):
+        if (c & 0x7F) == 0x7F:
+            continue
+        v = _e4m3_value_from_bits(c)
+        want = c if not (c == 0x80) else 0x80
+        assert O.e4m3_encode(np.array([v if c != 0x80 else -0.0]))[0] == want
+    assert O.e4m3_encode(np.array([-1e-9]))[0] == 0x80
+
+
+def test_mxfp8_scale_rule_and_amax_range():
+    """e = floor(log2 amax) - 8: the scaled amax lies in [256, 512) and encodes to a
+    magnitude in [256, 448] (saturating above 448)."""
+    rng = np.random.default_rng(8)
+    V = (rng.standard_normal((64, 256)) * np.exp2(rng.integers(-20, 20, (64, 1)))).astype(np.float32)
+    codes, scales, q = O.mxfp8_quantize(V)
+    amax = np.abs(V.reshape(64, 8, 32).astype(np.float64)).max(axis=2)
+    e = scales.astype(np.int64) - 127
+    np.testing.assert_array_equal(e, np.floor(np.log2(amax)).astype(np.int64) - 8)
+    qa = amax * np.exp2(-e)
+    assert (qa >= 256).all() and (qa < 512).all()
+    mag_codes = codes.reshape(64, 8, 32) & 0x7F
+    top = np.take_along_axis(mag_codes, np.abs(V.reshape(64, 8, 32)).argmax(axis=2)[:, :, None], axis=2)[:, :, 0]
+    assert (O.E4M3_MAGNITUDE[top] >= 256).all() and (O.E4M3_MAGNITUDE[top] <= 448).all()
+
+
+def test_mxfp8_identity_transform_reduces_to_plain_rtn():
+    w = WL.custom(8, 128, 16, 31, x_dtype="f32", with_w=False)
+    k = 4
+    A, B = np.eye(8), np.tile(np.eye(4), (k, 1, 1))
+    act = O.quant_act_mxfp8(w.x, A, B, np.full(k, 40.0), np.full(k, 40.0))
+    codes, scales, _ = O.mxfp8_quantize(w.x)
+    np.testing.assert_array_equal(act["codes"], codes)
+    np.testing.assert_array_equal(act["scales"], scales)
+    # dequantized values: within half an E4M3 step of x (relative 2^-4, or 2^-10 of the
+    # scale among the subnormals), except that |q| > 448 saturates to exactly 448 * scale
+    deq = O.dequantize_e4m3(codes, scales).reshape(8, k, 32)
+    x = w.x.astype(np.float64).reshape(8, k, 32)
+    s = np.exp2(scales.astype(np.float64) - 127)[:, :, None]
+    sat = np.abs(x) / s > 448
+    assert (np.abs(deq[sat]) == (448 * np.broadcast_to(s, x.shape))[sat]).all()
+    half = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * s)
+    assert (np.abs(deq - x)[~sat] <= half[~sat]).all()
+
+
+def test_e4m3_containers_hold_the_e2m1_values_exactly():
+    packed = O.pack_nibbles(np.arange(16, dtype=np.uint8).reshape(1, 16))
+    c8 = O.e4m3_containers_from_e2m1(packed)
+    np.testing.assert_array_equal(O.e4m3_decode(c8)[0], O.e2m1_decode(np.arange(16)))
+    # positive E2M1 values sit at E4M3 bytes 0x00, 0x30, 0x38, 0x3C, 0x40, 0x44, 0x48, 0x4C
+    assert c8[0, :8].tolist() == [0x00, 0x30, 0x38, 0x3C, 0x40, 0x44, 0x48, 0x4C]
+
+
+def test_gemm_w4a8_exact_on_small_random_codes():
+    """The fp64 GEMM equals an exact rational sum of the dequantized products."""
+    rng = np.random.default_rng(9)
+    S, M, N = 3, 4, 64
+    a8 = rng.integers(0, 256, (S, N)).astype(np.uint8)
+    a8[(a8 & 0x7F) == 0x7F] = 0x11
+    w4 = rng.integers(0, 256, (M, N // 2)).astype(np.uint8)
+    w8 = O.e4m3_containers_from_e2m1(w4)
+    sa = rng.integers(110, 140, (S, 2)).astype(np.uint8)
+    sw = rng.integers(110, 140, (M, 2)).astype(np.uint8)
+    out, T = O.gemm_w4a8(a8, sa, w8, sw)
+    for s in range(S):
+        for m in range(M):
+            tot = Fraction(0)
+            for n in range(N):
+                va = Fraction(_e4m3_value_from_bits(int(a8[s, n]))) * Fraction(2) ** (int(sa[s, n // 32]) - 127)
+                vw = Fraction(O.e2m1_decode(np.array([int(O.unpack_nibbles(w4)[m, n])]))[0]) \
+                    * Fraction(2) ** (int(sw[m, n // 32]) - 127)
+                tot += va * vw
+            # fp64 accumulation of 64 terms: within n * 2^-53 of the sum of magnitudes
+            assert abs(Fraction(float(out[s, m])) - tot) <= Fraction(N, 2 ** 53) * Fraction(float(T[s, m]))
