@@ -186,6 +186,70 @@ BATQ_API batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N
                         void* workspace, size_t workspace_bytes,
                         batq_dtype out_dtype, void* out, int ldo, void* stream);
 
+/* ------------------------------------------------------------------ W4A8 variant
+ * The pages' second setting (BATQuant thelatestinai.com page, abstract and
+ * Table 2, W4A8 rows): the same transform and clip with MXFP8 activations,
+ * E4M3 elements under the E8M0 shared scale 2^(floor(log2 amax) - 8) (OCP MX
+ * v1.0), round to nearest even, magnitudes above 448 saturated to 448.  The
+ * weights stay MXFP4 (same values and scales as batq_prepare_weights); for the
+ * E4M3 x E4M3 block-scaled MMA (tcgen05 kind::mxf8f6f4) each E2M1 weight code
+ * is held in one E4M3 byte of the same value.
+ */
+
+/* Bytes of MXFP8 codes (rows x N, one per element) and of scales. Host only. */
+BATQ_API batq_status batq_mxfp8_buffer_sizes(int rows, int N, batq_scale_layout layout, size_t* code_bytes,
+                                    size_t* scale_bytes);
+
+/*
+ * As batq_quant_act, but the codes are E4M3 bytes: codes is device S x N
+ * bytes (16-byte aligned), element n of row s at s * N + n.  Scales as in
+ * batq_quant_act.  Errors as batq_quant_act.
+ */
+BATQ_API batq_status batq_quant_act_mxfp8(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                                 const float* A_host, const float* B_dev, const float* ratios_dev,
+                                 uint8_t* codes, uint8_t* scales, batq_scale_layout layout,
+                                 float* y_debug, void* stream);
+
+/* Device workspace bytes batq_prepare_weights_w4a8 needs. Host only. */
+BATQ_API batq_status batq_prepare_weights_w4a8_workspace_size(int M, int N, size_t* bytes);
+
+/*
+ * batq_prepare_weights, then each E2M1 code widened to the E4M3 byte of the
+ * same value: w_codes8 is device M x N bytes (16-byte aligned); w_scales as in
+ * batq_prepare_weights.  workspace: batq_prepare_weights_w4a8_workspace_size
+ * bytes (it also holds the packed MXFP4 codes on the way).  Errors as
+ * batq_prepare_weights.
+ */
+BATQ_API batq_status batq_prepare_weights_w4a8(const void* W, batq_dtype w_dtype, int M, int N, int ldw,
+                                      const float* A_host, const float* B_host,
+                                      uint8_t* w_codes8, uint8_t* w_scales, batq_scale_layout layout,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * W4A8 block-scaled GEMM: out = deq(a) deq(w)^T with E4M3 codes on both sides
+ * (a_codes8 S x N from batq_quant_act_mxfp8, w_codes8 M x N from
+ * batq_prepare_weights_w4a8), MMA-layout scales, fp32 accumulation in tensor
+ * memory.  Shapes, alignment and errors as batq_gemm_mxfp4.
+ */
+BATQ_API batq_status batq_gemm_w4a8(const uint8_t* a_codes8, const uint8_t* a_scales,
+                           const uint8_t* w_codes8, const uint8_t* w_scales,
+                           int S, int M, int N, batq_dtype out_dtype, void* out, int ldo,
+                           void* stream);
+
+/* Device workspace bytes batq_linear_w4a8 needs (E4M3 codes + MMA-layout scales). Host only. */
+BATQ_API batq_status batq_linear_w4a8_workspace_size(int S, int N, size_t* bytes);
+
+/*
+ * Whole W4A8 linear: batq_quant_act_mxfp8 (MMA scale layout, into the
+ * workspace) followed by batq_gemm_w4a8 on the same stream.  Arguments as
+ * batq_linear, with the weights from batq_prepare_weights_w4a8.
+ */
+BATQ_API batq_status batq_linear_w4a8(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                             const float* A_host, const float* B_dev, const float* ratios_dev,
+                             const uint8_t* w_codes8, const uint8_t* w_scales, int M,
+                             void* workspace, size_t workspace_bytes,
+                             batq_dtype out_dtype, void* out, int ldo, void* stream);
+
 /*
  * batq_linear without a caller-provided workspace, for callers that cannot
  * allocate device memory (for example a plugin running in a process whose

@@ -157,6 +157,71 @@ def batq_linear_no_alloc(X, A, B, ratios, w_codes, w_scales, M, out, stream=None
                                             _stream(stream)), "batq_linear_no_alloc")
 
 
+# ------------------------------------------------------ W4A8 variant calls
+
+def batq_mxfp8_buffer_sizes(rows: int, N: int, layout: int = BATQ_SCALES_MMA):
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.load().batq_mxfp8_buffer_sizes(rows, N, layout, ctypes.byref(cb), ctypes.byref(sb)),
+           "batq_mxfp8_buffer_sizes")
+    return cb.value, sb.value
+
+
+def batq_prepare_weights_w4a8_workspace_size(M: int, N: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_lib.load().batq_prepare_weights_w4a8_workspace_size(M, N, ctypes.byref(b)),
+           "batq_prepare_weights_w4a8_workspace_size")
+    return b.value
+
+
+def batq_linear_w4a8_workspace_size(S: int, N: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_lib.load().batq_linear_w4a8_workspace_size(S, N, ctypes.byref(b)), "batq_linear_w4a8_workspace_size")
+    return b.value
+
+
+def batq_quant_act_mxfp8(X, A, B, ratios, codes, scales, layout=BATQ_SCALES_MMA, y_debug=None, stream=None):
+    """W4A8 activation path: transform + clip + MXFP8 (E4M3) of X (S x N) into codes (S x N) / scales."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    _check(_lib.load().batq_quant_act_mxfp8(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0), a.ctypes.data,
+                                            _dev_ptr(B, "B"), _dev_ptr(ratios, "ratios"), _dev_ptr(codes, "codes"),
+                                            _dev_ptr(scales, "scales"), layout, _dev_ptr(y_debug, "y_debug"),
+                                            _stream(stream)), "batq_quant_act_mxfp8")
+
+
+def batq_prepare_weights_w4a8(W, A, B_host, w_codes8, w_scales, workspace, layout=BATQ_SCALES_MMA, stream=None):
+    """Offline: the MXFP4 weights of batq_prepare_weights, each code held in one E4M3 byte (M x N)."""
+    M, N = W.shape
+    a = _host_f32(A, 64, "A")
+    b = _host_f32(B_host, (N // 32) * 16, "B")
+    _check(_lib.load().batq_prepare_weights_w4a8(_dev_ptr(W, "W"), _dtype_code(W), M, N, W.stride(0),
+                                                 a.ctypes.data, b.ctypes.data, _dev_ptr(w_codes8, "w_codes8"),
+                                                 _dev_ptr(w_scales, "w_scales"), layout,
+                                                 _dev_ptr(workspace, "workspace"),
+                                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "batq_prepare_weights_w4a8")
+
+
+def batq_gemm_w4a8(a_codes8, a_scales, w_codes8, w_scales, S, M, N, out, stream=None):
+    """out (S x M) = deq(a) deq(w)^T with E4M3 codes on both sides."""
+    _check(_lib.load().batq_gemm_w4a8(_dev_ptr(a_codes8, "a_codes8"), _dev_ptr(a_scales, "a_scales"),
+                                      _dev_ptr(w_codes8, "w_codes8"), _dev_ptr(w_scales, "w_scales"), S, M, N,
+                                      _dtype_code(out), _dev_ptr(out, "out"), out.stride(0), _stream(stream)),
+           "batq_gemm_w4a8")
+
+
+def batq_linear_w4a8(X, A, B, ratios, w_codes8, w_scales, M, workspace, out, stream=None):
+    """Whole W4A8 linear: MXFP8 activations online, then the E4M3 x E4M3 block-scaled GEMM."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    _check(_lib.load().batq_linear_w4a8(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0), a.ctypes.data,
+                                        _dev_ptr(B, "B"), _dev_ptr(ratios, "ratios"),
+                                        _dev_ptr(w_codes8, "w_codes8"), _dev_ptr(w_scales, "w_scales"), M,
+                                        _dev_ptr(workspace, "workspace"),
+                                        workspace.numel() * workspace.element_size(), _dtype_code(out),
+                                        _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_linear_w4a8")
+
+
 def batq_selftest_wait_timeout(limit_us: int, stream=None):
     """Launch the bounded-wait self-test kernel (its wait always expires)."""
     _check(_lib.load().batq_selftest_wait_timeout(limit_us, _stream(stream)), "batq_selftest_wait_timeout")
@@ -178,5 +243,14 @@ def empty_act_buffers(rows: int, N: int, layout=BATQ_SCALES_MMA, device="cuda"):
     torch = _torch()
     cb, sb = batq_act_buffer_sizes(rows, N, layout)
     codes = torch.empty((rows, N // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty(sb, dtype=torch.uint8, device=device)
+    return codes, scales
+
+
+def empty_mxfp8_buffers(rows: int, N: int, layout=BATQ_SCALES_MMA, device="cuda"):
+    """(codes, scales) uint8 CUDA tensors for MXFP8 (one byte per element) of a rows x N matrix."""
+    torch = _torch()
+    cb, sb = batq_mxfp8_buffer_sizes(rows, N, layout)
+    codes = torch.empty((rows, N), dtype=torch.uint8, device=device)
     scales = torch.empty(sb, dtype=torch.uint8, device=device)
     return codes, scales

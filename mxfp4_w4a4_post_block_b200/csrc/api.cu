@@ -108,7 +108,7 @@ bool invert(const double* a, double* inv, int n) {
 
 batq_status launch_quant(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
                          const float* B_dev, const float* ratios_dev, uint8_t* codes, uint8_t* scales,
-                         batq_scale_layout layout, float* y_debug, cudaStream_t stream) {
+                         batq_scale_layout layout, float* y_debug, bool fp8, cudaStream_t stream) {
   batq::QuantLaunch L;
   L.X = X;
   L.bf16 = (x_dtype == BATQ_BF16);
@@ -124,6 +124,7 @@ batq_status launch_quant(const void* X, batq_dtype x_dtype, int S, int N, int ld
   L.y_debug = y_debug;
   L.err = error_word();
   L.stream = stream;
+  L.fp8 = fp8;
   cudaError_t e = batq::launch_quant_act(L);
   if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
   return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
@@ -164,7 +165,7 @@ batq_status check_gemm_args(const uint8_t* a_codes, const uint8_t* a_scales, con
 
 batq_status launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
                         const uint8_t* w_scales, int S, int M, int N, batq_dtype out_dtype, void* out, int ldo,
-                        bool weights_ready, cudaStream_t stream) {
+                        bool weights_ready, bool fp8, cudaStream_t stream) {
   batq::GemmLaunch L;
   L.a_codes = a_codes;
   L.a_scales = a_scales;
@@ -179,6 +180,7 @@ batq_status launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const u
   L.err = error_word();
   L.stream = stream;
   L.weights_ready = weights_ready;
+  L.fp8 = fp8;
   cudaError_t e = batq::launch_gemm_mxfp4(L);
   if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
   return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
@@ -235,7 +237,7 @@ batq_status batq_quant_act(const void* X, batq_dtype x_dtype, int S, int N, int 
   if (st != BATQ_OK) return st;
   st = check_arch();
   if (st != BATQ_OK) return st;
-  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug,
+  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug, false,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -284,7 +286,7 @@ batq_status batq_prepare_weights(const void* W, batq_dtype w_dtype, int M, int N
   // cudaMemcpyAsync from pageable memory has staged the bytes when it returns,
   // so b_fused may be released.
   return launch_quant(W, w_dtype, M, N, ldw, a_fused, reinterpret_cast<const float*>(workspace), nullptr, w_codes,
-                      w_scales, layout, nullptr, s);
+                      w_scales, layout, nullptr, false, s);
 }
 
 batq_status batq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
@@ -296,7 +298,7 @@ batq_status batq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, con
   if (st != BATQ_OK) return st;
   // The preceding grid may be anything (e.g. the weight quantiser of
   // batq_prepare_weights): wait for it before reading any operand.
-  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, false,
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, false, false,
                      static_cast<cudaStream_t>(stream));
 }
 
@@ -329,12 +331,114 @@ batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx
   if (st != BATQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA, nullptr,
-                    s);
+                    false, s);
   if (st != BATQ_OK) return st;
   // The quantiser just launched writes only the workspace and starts its
   // dependents after every earlier grid has finished, so the GEMM may fetch
   // weights while the quantiser runs.
-  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, s);
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, false, s);
+}
+
+// ------------------------------------------------------------------ W4A8 variant
+
+batq_status batq_mxfp8_buffer_sizes(int rows, int N, batq_scale_layout layout, size_t* code_bytes,
+                                    size_t* scale_bytes) {
+  if (!code_bytes || !scale_bytes) return BATQ_ERR_INVALID_ARG;
+  if (layout != BATQ_SCALES_LINEAR && layout != BATQ_SCALES_MMA) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_mn(rows, N);
+  if (st != BATQ_OK) return st;
+  *code_bytes = (size_t)rows * (size_t)N;
+  *scale_bytes = scale_bytes_for(rows, N, layout);
+  return BATQ_OK;
+}
+
+batq_status batq_quant_act_mxfp8(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
+                                 const float* B_dev, const float* ratios_dev, uint8_t* codes, uint8_t* scales,
+                                 batq_scale_layout layout, float* y_debug, void* stream) {
+  batq_status st = check_quant_args(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout,
+                                    y_debug);
+  if (st != BATQ_OK) return st;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug, true,
+                      static_cast<cudaStream_t>(stream));
+}
+
+batq_status batq_prepare_weights_w4a8_workspace_size(int M, int N, size_t* bytes) {
+  if (!bytes) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_mn(M, N);
+  if (st != BATQ_OK) return st;
+  size_t base = 0;
+  batq_prepare_workspace_size(N, &base);
+  *bytes = base + round_up((size_t)M * (size_t)(N / 2), 256);
+  return BATQ_OK;
+}
+
+batq_status batq_prepare_weights_w4a8(const void* W, batq_dtype w_dtype, int M, int N, int ldw,
+                                      const float* A_host, const float* B_host, uint8_t* w_codes8,
+                                      uint8_t* w_scales, batq_scale_layout layout, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!workspace || !w_codes8) return BATQ_ERR_INVALID_ARG;
+  size_t need = 0, base = 0;
+  batq_status st = batq_prepare_weights_w4a8_workspace_size(M, N, &need);
+  if (st != BATQ_OK) return st;
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  if (!aligned16(workspace) || !aligned16(w_codes8)) return BATQ_ERR_ALIGNMENT;
+  batq_prepare_workspace_size(N, &base);
+  // The MXFP4 weights go to the workspace first (packed), then are widened
+  // into the caller's E4M3 containers.
+  uint8_t* packed = static_cast<uint8_t*>(workspace) + base;
+  st = batq_prepare_weights(W, w_dtype, M, N, ldw, A_host, B_host, packed, w_scales, layout, workspace, base,
+                            stream);
+  if (st != BATQ_OK) return st;
+  cudaError_t e = batq::launch_e2m1_to_e4m3(packed, w_codes8, (size_t)M * (size_t)(N / 2),
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
+}
+
+batq_status batq_gemm_w4a8(const uint8_t* a_codes8, const uint8_t* a_scales, const uint8_t* w_codes8,
+                           const uint8_t* w_scales, int S, int M, int N, batq_dtype out_dtype, void* out, int ldo,
+                           void* stream) {
+  batq_status st = check_gemm_args(a_codes8, a_scales, w_codes8, w_scales, S, M, N, out_dtype, out, ldo);
+  if (st != BATQ_OK) return st;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  return launch_gemm(a_codes8, a_scales, w_codes8, w_scales, S, M, N, out_dtype, out, ldo, false, true,
+                     static_cast<cudaStream_t>(stream));
+}
+
+batq_status batq_linear_w4a8_workspace_size(int S, int N, size_t* bytes) {
+  if (!bytes) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_mn(S, N);
+  if (st != BATQ_OK) return st;
+  *bytes = round_up((size_t)S * (size_t)N, 256) + scale_bytes_for(S, N, BATQ_SCALES_MMA);
+  return BATQ_OK;
+}
+
+batq_status batq_linear_w4a8(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
+                             const float* B_dev, const float* ratios_dev, const uint8_t* w_codes8,
+                             const uint8_t* w_scales, int M, void* workspace, size_t workspace_bytes,
+                             batq_dtype out_dtype, void* out, int ldo, void* stream) {
+  if (!workspace) return BATQ_ERR_INVALID_ARG;
+  size_t need = 0;
+  batq_status st = batq_linear_w4a8_workspace_size(S, N, &need);
+  if (st != BATQ_OK) return st;
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BATQ_ERR_ALIGNMENT;
+  uint8_t* a_codes = static_cast<uint8_t*>(workspace);
+  uint8_t* a_scales = a_codes + round_up((size_t)S * (size_t)N, 256);
+  st = check_quant_args(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA,
+                        nullptr);
+  if (st != BATQ_OK) return st;
+  st = check_gemm_args(a_codes, a_scales, w_codes8, w_scales, S, M, N, out_dtype, out, ldo);
+  if (st != BATQ_OK) return st;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA, nullptr,
+                    true, s);
+  if (st != BATQ_OK) return st;
+  return launch_gemm(a_codes, a_scales, w_codes8, w_scales, S, M, N, out_dtype, out, ldo, true, true, s);
 }
 
 batq_status batq_selftest_wait_timeout(unsigned int limit_us, void* stream) {

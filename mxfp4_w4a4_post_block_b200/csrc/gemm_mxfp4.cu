@@ -35,27 +35,28 @@ namespace batq {
 namespace {
 
 constexpr int kBM = 128;          // MMA M (rows of P per tile, TMEM lanes)
-constexpr int kBKBytes = 128;     // bytes of K per stage and row (= 256 E2M1 codes)
-constexpr int kBK = 2 * kBKBytes; // K elements per stage
-constexpr int kKPerMma = 64;      // K of one kind::mxf4 MMA
-constexpr int kMmasPerStage = kBK / kKPerMma;
+constexpr int kBKBytes = 128;     // bytes of K per stage and row (256 E2M1 or 128 E4M3 codes)
+constexpr int kMmasPerStage = 4;  // an MMA consumes 32 bytes of K per row
 constexpr int kThreads = 224;     // 7 warps: producer, MMA, 4 epilogue, scale copies
 constexpr int kSfWarp = 6;
 constexpr int kSfAtom = 512;      // bytes of one 128-row x 4-scale tile
 
-template <int BN, bool kSwap, int kStages>
+// kFp8: both operands are E4M3 bytes (the W4A8 variant), else packed E2M1.
+template <int BN, bool kSwap, int kStages, bool kFp8>
 struct GemmCfg {
+  static constexpr int kBK = kFp8 ? kBKBytes : 2 * kBKBytes;     // K elements per stage
+  static constexpr int kKPerMma = kFp8 ? 32 : 64;                // K elements per MMA
+  static constexpr int kAtoms = kBK / 128;                       // 4-scale atoms per row and stage
   static constexpr int kPBytes = kBM * kBKBytes;
   static constexpr int kQBytes = BN * kBKBytes;
   static constexpr int kQRowAtoms = BN > 128 ? 2 : 1;           // 128-row scale atoms covering Q rows
-  static constexpr int kSfPBytes = 2 * kSfAtom;                  // 2 K-atoms per stage
-  static constexpr int kSfQBytes = 2 * kQRowAtoms * kSfAtom;
-  static constexpr int kStageBytes = kPBytes + kQBytes + kSfPBytes + kSfQBytes;
-  static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
-  // TMEM columns: accumulator, then per stage 8 columns of P scales and
-  // 4 * kQRowAtoms * 2 columns of Q scales.
-  static constexpr int kSfPCols = 8;
-  static constexpr int kSfQCols = 8 * kQRowAtoms;
+  static constexpr int kSfPBytes = kAtoms * kSfAtom;
+  static constexpr int kSfQBytes = kAtoms * kQRowAtoms * kSfAtom;
+  static constexpr int kStageBytes = (kPBytes + kQBytes + kSfPBytes + kSfQBytes + 1023) / 1024 * 1024;
+  // TMEM columns: accumulator, then per stage 4 columns per K atom of P
+  // scales and 4 * kQRowAtoms per K atom of Q scales.
+  static constexpr int kSfPCols = 4 * kAtoms;
+  static constexpr int kSfQCols = 4 * kAtoms * kQRowAtoms;
   static constexpr int kTmemUsed = BN + kStages * (kSfPCols + kSfQCols);
   static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                  : kTmemUsed <= 256 ? 256 : 512;
@@ -81,11 +82,12 @@ struct GemmArgs {
   int early_w;              // the preceding grid does not write the weights: prefetch them before waiting
 };
 
-template <int BN, bool kSwap, int kStages, bool kOutBF16>
+template <int BN, bool kSwap, int kStages, bool kOutBF16, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_mxfp4(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ GemmArgs g) {
-  using C = GemmCfg<BN, kSwap, kStages>;
+  using C = GemmCfg<BN, kSwap, kStages, kFp8>;
+  constexpr int kBK = C::kBK, kKPerMma = C::kKPerMma;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::kStageBytes);
@@ -141,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the preceding grid (the linear layer's quantiser) still runs.
         const int w0 = kSwap ? p0 : q0;
         const int wn = min(kSwap ? kBM : BN, g.w_rows - w0);
-        const size_t row_bytes = (size_t)(g.N >> 1);
+        const size_t row_bytes = (size_t)(kFp8 ? g.N : g.N >> 1);
         const uint8_t* wbase = g.w_codes + (size_t)w0 * row_bytes;
         const size_t wbytes = (size_t)wn * row_bytes;
         for (size_t off = 0; off < wbytes; off += 65536)
@@ -162,8 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t* st = smem + s * C::kStageBytes;
-        const int katom0 = ks * 2;  // first 4-scale atom of this stage
-        const int katoms = min(2, (g.kpad >> 2) - katom0);
+        const int katom0 = ks * C::kAtoms;  // first 4-scale atom of this stage
+        const int katoms = min(C::kAtoms, (g.kpad >> 2) - katom0);
         const uint32_t sf_bytes = (uint32_t)katoms * kSfAtom;
         mbar_arrive_expect_tx(&full[s], (uint32_t)(C::kPBytes + C::kQBytes) + sf_bytes * (1 + q_atoms_valid));
         tma_load_2d(st, &tm_p, &full[s], ks * kBKBytes, p0);
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(st + C::kPBytes + C::kQBytes, g.p_scales + (size_t)p_tile_atom * row_stride + katom0 * kSfAtom,
                   sf_bytes, &full[s]);
         for (int a = 0; a < q_atoms_valid; ++a) {
-          bulk_load(st + C::kPBytes + C::kQBytes + C::kSfPBytes + a * 2 * kSfAtom,
+          bulk_load(st + C::kPBytes + C::kQBytes + C::kSfPBytes + a * C::kAtoms * kSfAtom,
                     g.q_scales + (size_t)(q_tile_atom + a) * row_stride + katom0 * kSfAtom, sf_bytes, &full[s]);
         }
         if (++s == kStages) {
@@ -202,13 +204,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dp = sdesc_kmajor_sw128(sp);
         const uint64_t dq = sdesc_kmajor_sw128(sq);
         for (int j = 0; j < nmma; ++j) {
-          const int a = j >> 1;
-          const int sf_id = (j & 1) * 2;
-          const uint32_t idesc = idesc_mxf4(BN, sf_id, sf_id);
-          // Advance K by 64 codes = 32 bytes inside the 128-byte swizzle atom.
-          tc_mma_mxf4(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc,
-                      t_sfp + s * C::kSfPCols + a * 4, t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms,
-                      (ks > 0 || j > 0) ? 1u : 0u);
+          // MMA j covers 32-element scale blocks kb.. of the stage: atom kb / 4,
+          // byte kb % 4 of each 4-scale TMEM column.
+          const int kb = j * (kKPerMma / 32);
+          const int a = kb >> 2;
+          const int sf_id = kb & 3;
+          // Advance K by 32 bytes inside the 128-byte swizzle atom.
+          if constexpr (kFp8)
+            tc_mma_mxf8(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc_mxf8(kBM, BN, sf_id, sf_id),
+                        t_sfp + s * C::kSfPCols + a * 4, t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms,
+                        (ks > 0 || j > 0) ? 1u : 0u);
+          else
+            tc_mma_mxf4(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc_mxf4(BN, sf_id, sf_id),
+                        t_sfp + s * C::kSfPCols + a * 4, t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms,
+                        (ks > 0 || j > 0) ? 1u : 0u);
         }
         tc_commit(&empty[s]);
         if (++s == kStages) {
@@ -234,12 +243,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ssfq = ssfp + C::kSfPBytes;
         const int kleft = g.N - ks * kBK;
         const int nmma = kleft >= kBK ? kMmasPerStage : kleft / kKPerMma;
-        for (int a = 0; a < (nmma + 1) / 2; ++a) {
+        const int atoms = ((nmma - 1) * (kKPerMma / 32)) / 4 + 1;  // atoms the stage's MMAs read
+        for (int a = 0; a < atoms; ++a) {
           tc_cp_32x128b_warpx4(t_sfp + s * C::kSfPCols + a * 4, sdesc_sf_atom(ssfp + a * kSfAtom));
 #pragma unroll
           for (int r = 0; r < C::kQRowAtoms; ++r) {
             tc_cp_32x128b_warpx4(t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms + r * 4,
-                                 sdesc_sf_atom(ssfq + (r * 2 + a) * kSfAtom));
+                                 sdesc_sf_atom(ssfq + (r * C::kAtoms + a) * kSfAtom));
           }
         }
         tc_commit(&sf_ready[s]);
@@ -333,14 +343,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BN, bool kSwap, int kStages, bool kOutBF16>
+template <int BN, bool kSwap, int kStages, bool kOutBF16, bool kFp8>
 cudaError_t launch_cfg(const GemmLaunch& L) {
-  using C = GemmCfg<BN, kSwap, kStages>;
+  using C = GemmCfg<BN, kSwap, kStages, kFp8>;
   const int rows_p = kSwap ? L.M : L.S;
   const int rows_q = kSwap ? L.S : L.M;
   const uint8_t* codes_p = kSwap ? L.w_codes : L.a_codes;
   const uint8_t* codes_q = kSwap ? L.a_codes : L.w_codes;
-  const uint64_t row_bytes = (uint64_t)(L.N / 2);
+  const uint64_t row_bytes = (uint64_t)(kFp8 ? L.N : L.N / 2);
 
   CUtensorMap tm_p, tm_q, tm_out;
   if (!make_map_2d(&tm_p, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_p, row_bytes, (uint64_t)rows_p, row_bytes, kBKBytes,
@@ -372,13 +382,13 @@ cudaError_t launch_cfg(const GemmLaunch& L) {
   g.kpad = (L.N / 32 + 3) / 4 * 4;
   g.ldo = L.ldo;
   g.tiles_q = (rows_q + BN - 1) / BN;
-  g.num_kstages = (L.N + kBK - 1) / kBK;
+  g.num_kstages = (L.N + C::kBK - 1) / C::kBK;
   g.w_codes = L.w_codes;
   g.w_rows = L.M;
   g.early_w = L.weights_ready ? 1 : 0;
   const int tiles_p = (rows_p + kBM - 1) / kBM;
 
-  auto kern = k_gemm_mxfp4<BN, kSwap, kStages, kOutBF16>;
+  auto kern = k_gemm_mxfp4<BN, kSwap, kStages, kOutBF16, kFp8>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -400,19 +410,20 @@ cudaError_t launch_cfg(const GemmLaunch& L) {
   return cudaLaunchKernelEx(&cfg, kern, tm_p, tm_q, tm_out, g);
 }
 
-template <bool kOutBF16>
+template <bool kOutBF16, bool kFp8>
 cudaError_t launch_dtype(const GemmLaunch& L) {
-  if (L.S <= 16) return launch_cfg<16, true, 4, kOutBF16>(L);
-  if (L.S <= 32) return launch_cfg<32, true, 4, kOutBF16>(L);
-  if (L.S <= 64) return launch_cfg<64, true, 4, kOutBF16>(L);
-  if (L.S <= 128) return launch_cfg<256, false, 4, kOutBF16>(L);
+  if (L.S <= 16) return launch_cfg<16, true, 4, kOutBF16, kFp8>(L);
+  if (L.S <= 32) return launch_cfg<32, true, 4, kOutBF16, kFp8>(L);
+  if (L.S <= 64) return launch_cfg<64, true, 4, kOutBF16, kFp8>(L);
+  if (L.S <= 128) return launch_cfg<256, false, 4, kOutBF16, kFp8>(L);
   return launch_gemm_pair(L);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_mxfp4(const GemmLaunch& L) {
-  return L.out_bf16 ? launch_dtype<true>(L) : launch_dtype<false>(L);
+  if (L.fp8) return L.out_bf16 ? launch_dtype<true, true>(L) : launch_dtype<false, true>(L);
+  return L.out_bf16 ? launch_dtype<true, false>(L) : launch_dtype<false, false>(L);
 }
 
 }  // namespace batq

@@ -39,8 +39,6 @@ constexpr int kTileM = 256;            // token rows per pair
 constexpr int kTileN = 256;            // out-features per pair (MMA N)
 constexpr int kHalfN = kTileN / 2;     // weight rows loaded by each CTA
 constexpr int kBKBytes = 128;          // bytes of K per stage and row (256 codes)
-constexpr int kBK = 2 * kBKBytes;
-constexpr int kKPerMma = 64;
 constexpr int kStages = 6;             // ~210 KB of operands in flight per SM (L2 latency ~1.5 us)
 constexpr int kSfAtom = 512;           // 128 rows x 4 scales
 constexpr int kEpiWarps = 8;
@@ -49,22 +47,30 @@ constexpr int kThreads = (3 + kEpiWarps) * 32;
 
 constexpr int kABytes = kRowsPerCta * kBKBytes;             // 16 KB
 constexpr int kBBytes = kHalfN * kBKBytes;                  // 16 KB
-constexpr int kSfaBytes = 2 * kSfAtom;                      // 2 K atoms of own rows
-constexpr int kSfbBytes = 2 * 2 * kSfAtom;                  // 2 row atoms x 2 K atoms
-constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-static_assert(kStageBytes % 1024 == 0, "stage alignment");
-constexpr int kStageTxBytes = kStageBytes;                  // bytes one CTA's loads deliver per stage
 constexpr int kBoxBytes = 1024;                             // one epilogue store box: 32 rows x 32 bytes
 constexpr int kStagingBytes = kEpiWarps * kBoxBytes;
-constexpr int kBarOffset = kStages * kStageBytes + kStagingBytes;
-constexpr int kSmemBytes = kBarOffset + 512 + 1024;
-
-// TMEM columns: accumulator [0, 256), then per stage 8 columns of activation
-// scales (2 K atoms x 4) and 16 of weight scales (2 K atoms x 2 row atoms x 4).
-constexpr int kSfaCols = 8;
-constexpr int kSfbCols = 16;
 constexpr int kTmemCols = 512;
-static_assert(kTileN + kStages * (kSfaCols + kSfbCols) <= kTmemCols, "TMEM budget");
+
+// Per element format (kFp8: E4M3 bytes, the W4A8 variant; else packed E2M1).
+// A stage always holds 128 bytes of K per row; an MMA consumes 32 of them.
+template <bool kFp8>
+struct PairCfg {
+  static constexpr int kBK = kFp8 ? kBKBytes : 2 * kBKBytes;  // K elements per stage
+  static constexpr int kKPerMma = kFp8 ? 32 : 64;             // K elements per MMA
+  static constexpr int kAtoms = kBK / 128;                    // 4-scale atoms per row and stage
+  static constexpr int kSfaBytes = kAtoms * kSfAtom;          // K atoms of own rows
+  static constexpr int kSfbBytes = 2 * kAtoms * kSfAtom;      // 2 row atoms x K atoms
+  static constexpr int kStageTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // bytes one CTA's loads deliver
+  static constexpr int kStageBytes = (kStageTxBytes + 1023) / 1024 * 1024;
+  static constexpr int kBarOffset = kStages * kStageBytes + kStagingBytes;
+  static constexpr int kSmemBytes = kBarOffset + 512 + 1024;
+  // TMEM columns: accumulator [0, 256), then per stage 4 columns per atom of
+  // activation scales and 8 per atom of weight scales (2 row atoms).
+  static constexpr int kSfaCols = 4 * kAtoms;
+  static constexpr int kSfbCols = 8 * kAtoms;
+  static_assert(kTileN + kStages * (kSfaCols + kSfbCols) <= kTmemCols, "TMEM budget");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 struct PairArgs {
   void* out;
@@ -76,7 +82,7 @@ struct PairArgs {
   int early_weights;        // weights may be read before waiting for the preceding grid
 };
 
-template <bool kOutBF16>
+template <bool kOutBF16, bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfw,
@@ -84,7 +90,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const __grid_constant__ PairArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+  using C = PairCfg<kFp8>;
+  constexpr int kStageBytes = C::kStageBytes, kSfaBytes = C::kSfaBytes, kSfaCols = C::kSfaCols,
+                kSfbCols = C::kSfbCols, kBK = C::kBK, kKPerMma = C::kKPerMma;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 1;
@@ -149,7 +158,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t bar = mapa_shared(smem_u32(&full[st_idx]), 0);
         const int ks = gi % nks;
         tma_load_2d_pair(st + kABytes, &tm_w, bar, ks * kBKBytes, w_row_of(gi) + (int)rank * kHalfN);
-        tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &tm_sfw, bar, 0, ks * 4, w_row_of(gi) / kRowsPerCta);
+        tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &tm_sfw, bar, 0, ks * 2 * C::kAtoms,
+                         w_row_of(gi) / kRowsPerCta);
       };
       auto issue_activations = [&](int gi) {
         const int st_idx = gi % kStages;
@@ -158,7 +168,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int ks = gi % nks;
         tma_load_2d_pair(st, &tm_a, bar, ks * kBKBytes, a_row_of(gi));
         // scale tiles: {256-byte chunk, K chunk (2 per 4-scale atom), 128-row tile}
-        tma_load_3d_pair(st + kABytes + kBBytes, &tm_sfa, bar, 0, ks * 4, a_row_of(gi) / kRowsPerCta);
+        tma_load_3d_pair(st + kABytes + kBBytes, &tm_sfa, bar, 0, ks * 2 * C::kAtoms, a_row_of(gi) / kRowsPerCta);
       };
       // When the preceding grid is known not to write the weights (the linear
       // layer's own quantiser), the first ring's weights are loaded before
@@ -166,7 +176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int prologue = total < kStages ? total : kStages;
       if (!g.early_weights) griddep_wait();
       for (int gi = 0; gi < prologue; ++gi) {
-        if (leader) mbar_arrive_expect_tx(&full[gi], 2u * kStageTxBytes);
+        if (leader) mbar_arrive_expect_tx(&full[gi], 2u * C::kStageTxBytes);
         issue_weights(gi);
       }
       if (g.early_weights) griddep_wait();
@@ -178,7 +188,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           set_error(g.err, kErrReleaseTimeout);
           break;
         }
-        if (leader) mbar_arrive_expect_tx(&full[s], 2u * kStageTxBytes);
+        if (leader) mbar_arrive_expect_tx(&full[s], 2u * C::kStageTxBytes);
         issue_weights(gi);
         issue_activations(gi);
         if (++s == kStages) {
@@ -217,11 +227,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint64_t da = sdesc_kmajor_sw128(sa);
         const uint64_t db = sdesc_kmajor_sw128(sb);
         for (int j = 0; j < nmma; ++j) {
-          const int a = j >> 1;
-          const int sf_id = (j & 1) * 2;
-          tc_mma_pair_mxf4(t_acc, da + (uint64_t)(j * 2), db + (uint64_t)(j * 2), idesc_mxf4_m256(kTileN, sf_id, sf_id),
-                           t_sfa + st_idx * kSfaCols + a * 4, t_sfb + st_idx * kSfbCols + a * 8,
-                           (ks > 0 || j > 0) ? 1u : 0u);
+          // MMA j covers 32-element scale blocks kb.. of the stage: atom kb / 4,
+          // byte kb % 4 of each 4-scale TMEM column.
+          const int kb = j * (kKPerMma / 32);
+          const int a = kb >> 2;
+          const int sf_id = kb & 3;
+          // Advance K by 32 bytes inside the 128-byte swizzle atom.
+          if constexpr (kFp8)
+            tc_mma_pair_mxf8(t_acc, da + (uint64_t)(j * 2), db + (uint64_t)(j * 2), idesc_mxf8(256, kTileN, sf_id, sf_id),
+                             t_sfa + st_idx * kSfaCols + a * 4, t_sfb + st_idx * kSfbCols + a * 8,
+                             (ks > 0 || j > 0) ? 1u : 0u);
+          else
+            tc_mma_pair_mxf4(t_acc, da + (uint64_t)(j * 2), db + (uint64_t)(j * 2),
+                             idesc_mxf4_m256(kTileN, sf_id, sf_id), t_sfa + st_idx * kSfaCols + a * 4,
+                             t_sfb + st_idx * kSfbCols + a * 8, (ks > 0 || j > 0) ? 1u : 0u);
         }
         tc_commit_pair(&empty[st_idx], 0x3);
         // Both epilogues may read the accumulator once every MMA of the tile has completed.
@@ -248,11 +267,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
         const uint32_t ssfa = smem_u32(smem + st_idx * kStageBytes) + kABytes + kBBytes;
         const uint32_t ssfb = ssfa + kSfaBytes;
-        for (int a = 0; a < (nmma + 1) / 2; ++a) {
+        const int atoms = ((nmma - 1) * (kKPerMma / 32)) / 4 + 1;  // atoms the stage's MMAs read
+        for (int a = 0; a < atoms; ++a) {
           tc_cp_pair_32x128b_warpx4(t_sfa + st_idx * kSfaCols + a * 4, sdesc_sf_atom(ssfa + a * kSfAtom));
-          // weight-scale box is {2 row tiles} x {2 K atoms}: row tile r, atom a at (2r + a) * 512
+          // weight-scale box is {2 row tiles} x {K atoms}: row tile r, atom a at (r * kAtoms + a) * 512
           tc_cp_pair_32x128b_warpx4(t_sfb + st_idx * kSfbCols + a * 8, sdesc_sf_atom(ssfb + a * kSfAtom));
-          tc_cp_pair_32x128b_warpx4(t_sfb + st_idx * kSfbCols + a * 8 + 4, sdesc_sf_atom(ssfb + (2 + a) * kSfAtom));
+          tc_cp_pair_32x128b_warpx4(t_sfb + st_idx * kSfbCols + a * 8 + 4,
+                                    sdesc_sf_atom(ssfb + (C::kAtoms + a) * kSfAtom));
         }
         tc_commit_pair_local(&sf_ready[st_idx]);
       }
@@ -382,9 +403,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool kOutBF16>
+template <bool kOutBF16, bool kFp8>
 cudaError_t launch_pair_impl(const GemmLaunch& L) {
-  const uint64_t row_bytes = (uint64_t)(L.N / 2);
+  using C = PairCfg<kFp8>;
+  const uint64_t row_bytes = (uint64_t)(kFp8 ? L.N : L.N / 2);
   const int kpad = (L.N / 32 + 3) / 4 * 4;
   const uint64_t sf_row_tile_bytes = (uint64_t)(kpad / 4) * kSfAtom;
   const uint64_t a_tiles = (uint64_t)(L.S + 127) / 128;
@@ -399,10 +421,10 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
     return cudaErrorInvalidValue;
   // Scale tiles as {256-byte chunks, chunks per row tile, row tiles}; one box = 2 K atoms (x 2 row tiles).
   if (!make_map_3d(&tm_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_scales, 256, sf_row_tile_bytes / 256, a_tiles, 256,
-                   sf_row_tile_bytes, 256, 4, 1))
+                   sf_row_tile_bytes, 256, 2 * C::kAtoms, 1))
     return cudaErrorInvalidValue;
   if (!make_map_3d(&tm_sfw, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_scales, 256, sf_row_tile_bytes / 256, w_tiles, 256,
-                   sf_row_tile_bytes, 256, 4, 2))
+                   sf_row_tile_bytes, 256, 2 * C::kAtoms, 2))
     return cudaErrorInvalidValue;
   const uint32_t esz = kOutBF16 ? 2 : 4;
   if (!make_map_2d(&tm_out, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
@@ -421,15 +443,15 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   g.ldo = L.ldo;
   g.tiles_m = (L.S + kTileM - 1) / kTileM;
   g.tiles_n = (L.M + kTileN - 1) / kTileN;
-  g.num_kstages = (L.N + kBK - 1) / kBK;
+  g.num_kstages = (L.N + C::kBK - 1) / C::kBK;
   g.early_weights = L.weights_ready ? 1 : 0;
 
-  auto kern = k_gemm_pair<kOutBF16>;
+  auto kern = k_gemm_pair<kOutBF16, kFp8>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -441,7 +463,7 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = L.stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -454,7 +476,8 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
 }  // namespace
 
 cudaError_t launch_gemm_pair(const GemmLaunch& L) {
-  return L.out_bf16 ? launch_pair_impl<true>(L) : launch_pair_impl<false>(L);
+  if (L.fp8) return L.out_bf16 ? launch_pair_impl<true, true>(L) : launch_pair_impl<false, true>(L);
+  return L.out_bf16 ? launch_pair_impl<true, false>(L) : launch_pair_impl<false, false>(L);
 }
 
 }  // namespace batq

@@ -19,6 +19,7 @@ struct QuantLaunch {
   float* y_debug;       // device S x N or nullptr
   unsigned* err;        // device error word
   cudaStream_t stream;
+  bool fp8;             // E4M3 elements (MXFP8, one byte each) instead of packed E2M1
 };
 
 // Returns cudaErrorInvalidValue when the tensor map cannot be encoded.
@@ -43,12 +44,20 @@ struct GemmLaunch {
   // weights, so they may be read before waiting for it (set by the linear
   // layer, whose preceding grid is its own quantiser).
   bool weights_ready;
+  // Both operands are E4M3 bytes (the W4A8 variant: MXFP8 activations, MXFP4
+  // weights in E4M3 containers) instead of packed E2M1.
+  bool fp8;
 };
 
 cudaError_t launch_gemm_mxfp4(const GemmLaunch& L);
 
 // Prefill-shape GEMM on CTA pairs (tcgen05 cta_group::2); used for S > 128.
 cudaError_t launch_gemm_pair(const GemmLaunch& L);
+
+// Widen packed E2M1 codes (element 2j in the low nibble) to one E4M3 byte per
+// element holding the same value; packed_bytes must be a multiple of 16 and
+// both pointers 16-byte aligned.
+cudaError_t launch_e2m1_to_e4m3(const uint8_t* packed, uint8_t* out, size_t packed_bytes, cudaStream_t stream);
 
 // One-thread kernel whose barrier wait always expires after limit_ns.
 cudaError_t launch_wait_selftest(uint64_t limit_ns, unsigned* err, cudaStream_t stream);

@@ -188,15 +188,27 @@ __device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v
   return out;
 }
 
+// Four E4M3 codes (round to nearest even, saturating at +-448): v0 in the
+// lowest byte.
+__device__ __forceinline__ uint32_t e4m3x4(float v0, float v1, float v2, float v3) {
+  uint32_t out;
+  asm("{\n\t.reg .b16 h0, h1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h1, %4, %3;\n\t"
+      "mov.b32 %0, {h0, h1};\n\t}"
+      : "=r"(out)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+  return out;
+}
 
 // ------------------------------------------------------------ bulk copies
 
-// 1-D bulk copy global -> shared (both 16-byte aligned, size a multiple of 16).
 // Prefetch `bytes` of global memory into L2 (16-byte aligned address, size a multiple of 16).
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// 1-D bulk copy global -> shared (both 16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
@@ -240,6 +252,18 @@ __device__ __forceinline__ void tc_mma_mxf4(uint32_t tacc, uint64_t adesc, uint6
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// As tc_mma_mxf4 for E4M3 x E4M3 operands (kind::mxf8f6f4, K = 32 per MMA,
+// one E8M0 scale per 32 K, i.e. one scale byte of each 4-scale TMEM column).
+__device__ __forceinline__ void tc_mma_mxf8(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
       : "memory");
 }
@@ -292,6 +316,14 @@ __device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_mxf4(int n, int sf_id_a, int sf_id_b) {
   return ((uint32_t)(sf_id_b & 3) << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
          ((uint32_t)(128 >> 4) << 24) | ((uint32_t)(sf_id_a & 3) << 29);
+}
+
+// Instruction descriptor of kind::mxf8f6f4 block-scaled MMA with E4M3 A and B
+// (format code 0 in bits 7-9 and 10-12), E8M0 scales, K-major, M = m, N = n,
+// dense K = 32 (bit 31 clear); scale ids as for idesc_mxf4.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int m, int n, int sf_id_a, int sf_id_b) {
+  return ((uint32_t)(sf_id_b & 3) << 4) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(m >> 4) << 24) |
+         ((uint32_t)(sf_id_a & 3) << 29);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -382,6 +414,17 @@ __device__ __forceinline__ void tc_mma_pair_mxf4(uint32_t tacc, uint64_t adesc, 
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Pair MMA of kind::mxf8f6f4 (E4M3 x E4M3), otherwise as tc_mma_pair_mxf4.
+__device__ __forceinline__ void tc_mma_pair_mxf8(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
       : "memory");
 }

@@ -121,7 +121,8 @@ __device__ __forceinline__ void load_block(uint32_t box, int lane, float x[32]) 
   }
 }
 
-template <bool kBF16>
+// kFp8: E4M3 elements (MXFP8, the W4A8 variant's activations) instead of E2M1.
+template <bool kBF16, bool kFp8>
 __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
     k_quant_act(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
   using T = Tile<kBF16>;
@@ -280,16 +281,19 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
       const float amax = fmaxf(fabsf(cmn), fabsf(cmx));
 
       // Shared scale: floor(log2 amax) = biased exponent - 127, so the scale
-      // byte e + 127 = biased exponent - 2 (clamped at 0, which also covers
-      // amax == 0 and subnormal amax).  2^-e is built from exponent bits.
+      // byte e + 127 = biased exponent - emax (emax = 2 for E2M1, 8 for E4M3;
+      // clamped at 0, which also covers amax == 0 and subnormal amax).  2^-e
+      // is built from exponent bits.
+      constexpr uint32_t kEmax = kFp8 ? 8u : 2u;
       const uint32_t ebits = __float_as_uint(amax) >> 23;
-      uint32_t sbyte = ebits > 2u ? ebits - 2u : 0u;
+      uint32_t sbyte = ebits > kEmax ? ebits - kEmax : 0u;
       const float inv_scale = __uint_as_float((254u - sbyte) << 23);
 
       // Clip, then divide by the shared scale (an exact power-of-two multiply,
-      // two elements per packed multiply), then round to E2M1.
+      // two elements per packed multiply), then round to E2M1 or E4M3.
       const float2 inv2 = make_float2(inv_scale, inv_scale);
-      uint32_t words[4];
+      constexpr int kWords = kFp8 ? 8 : 4;  // 32 codes of 4 or 8 bits
+      uint32_t words[kWords];
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         float2 q[4];
@@ -299,16 +303,25 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
                                         fminf(fmaxf(y[8 * w + 2 * j + 1], lo), hi));
           q[j] = __fmul2_rn(c2, inv2);
         }
-        words[w] = e2m1x8(q[0].x, q[0].y, q[1].x, q[1].y, q[2].x, q[2].y, q[3].x, q[3].y);
+        if constexpr (kFp8) {
+          words[2 * w] = e4m3x4(q[0].x, q[0].y, q[1].x, q[1].y);
+          words[2 * w + 1] = e4m3x4(q[2].x, q[2].y, q[3].x, q[3].y);
+        } else {
+          words[w] = e2m1x8(q[0].x, q[0].y, q[1].x, q[1].y, q[2].x, q[2].y, q[3].x, q[3].y);
+        }
       }
       if (!finite) {
         sbyte = 0xFFu;
-        words[0] = words[1] = words[2] = words[3] = 0u;
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) words[w] = 0u;
       }
 
       if (row < p.S) {
-        uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (size_t)(p.N >> 1) + (size_t)b * 16);
-        *dst = make_uint4(words[0], words[1], words[2], words[3]);
+        constexpr int kBlockCodeBytes = kWords * 4;
+        uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (size_t)(kFp8 ? p.N : p.N >> 1) +
+                                              (size_t)b * kBlockCodeBytes);
+        dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+        if constexpr (kFp8) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
         if (p.mma_layout)
           p.scales[mma_scale_offset(row, b, p.kpad)] = (uint8_t)sbyte;
         else
@@ -329,7 +342,7 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
   }
 }
 
-template <bool kBF16>
+template <bool kBF16, bool kFp8>
 cudaError_t launch_impl(const QuantLaunch& L) {
   using T = Tile<kBF16>;
   // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
@@ -362,7 +375,7 @@ cudaError_t launch_impl(const QuantLaunch& L) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          T::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -379,13 +392,14 @@ cudaError_t launch_impl(const QuantLaunch& L) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16>, map, a);
+  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16, kFp8>, map, a);
 }
 
 }  // namespace
 
 cudaError_t launch_quant_act(const QuantLaunch& L) {
-  return L.bf16 ? launch_impl<true>(L) : launch_impl<false>(L);
+  if (L.fp8) return L.bf16 ? launch_impl<true, true>(L) : launch_impl<false, true>(L);
+  return L.bf16 ? launch_impl<true, false>(L) : launch_impl<false, false>(L);
 }
 
 }  // namespace batq

@@ -11,6 +11,11 @@ Tolerances:
   mismatching elements must number fewer than 1e-4 of all elements;
 * GEMM: |out_gpu - out_ref| <= 1e-4 * sum_n |a_n| |w_n| against the oracle's
   fp64 product of the same codes.
+* W4A8 (E4M3 codes): as for FP4, except that the band around each rounding
+  boundary is the Y tolerance itself, 1e-5 * max(|y|, sum_j |x_j| |P_ji|),
+  carried into scaled units (E4M3 boundaries are 1/16 apart down to the
+  subnormals, so an element with cancellation can cross one within the fp32
+  error of the transform).
 """
 
 from __future__ import annotations
@@ -94,3 +99,52 @@ def to_mma_layout(scales_linear, rows, k, pad=0x7F):
     r, c = np.meshgrid(np.arange(rows), np.arange(k), indexing="ij")
     buf[O.mma_scale_offset(r, c, k)] = np.asarray(scales_linear, np.uint8)
     return buf
+
+
+# ------------------------------------------------------- W4A8 (MXFP8 E4M3) ----
+
+E4M3_MIDPOINTS = (O.E4M3_MAGNITUDE[:-1] + O.E4M3_MAGNITUDE[1:]) / 2
+
+
+def exempt_mask_e4m3(ref, X, A, B):
+    """Elements whose E4M3 code may legitimately differ from the oracle's.
+
+    E4M3 has a rounding boundary every 1/16 (relative) all the way down to the
+    subnormals, so an element whose transformed value suffers cancellation can
+    cross one within the fp32 error of the transform, which is bounded relative
+    to the condition scale sum_j |x_j| |P_ji|, not to |y|.  The band is therefore
+    that of the Y tolerance: a code may differ if a midpoint of neighbouring E4M3
+    magnitudes lies within 1e-5 * max(|y|, condition scale) * 2^-e of the
+    oracle's pre-rounding value q.  Whole blocks may differ in scale when the
+    clipped amax lies within 1e-5 * max(amax, largest condition scale of the
+    block) of a power of two.
+    """
+    q = np.abs(ref["q"])
+    S, N = q.shape
+    k = N // 32
+    cond = condition_scale(X, A, B)
+    e = ref["scales"].astype(np.int64) - 127
+    inv = np.repeat(np.exp2(-np.clip(e, -127, 127).astype(np.float64)), 32, axis=1)
+    band = REL * np.maximum(np.abs(ref["Y_hat"].astype(np.float64)), cond) * inv
+    idx = np.clip(np.searchsorted(E4M3_MIDPOINTS, q), 1, len(E4M3_MIDPOINTS) - 1)
+    near = np.minimum(np.abs(q - E4M3_MIDPOINTS[idx - 1]), np.abs(q - E4M3_MIDPOINTS[idx]))
+    near_mid = near <= band
+    amax = np.abs(ref["Y_hat"].astype(np.float64)).reshape(S, k, 32).max(axis=2)
+    cmax = cond.reshape(S, k, 32).max(axis=2)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        p2 = np.exp2(np.round(np.log2(np.where(amax > 0, amax, 1.0))))
+    near_pow2 = (amax > 0) & (np.abs(amax - p2) <= REL * np.maximum(p2, cmax))
+    return near_mid | np.repeat(near_pow2, 32, axis=1), near_pow2
+
+
+def assert_quant_parity_e4m3(codes_gpu, scales_gpu_linear, ref, X, A, B, label=""):
+    """E4M3 codes and E8M0 scales bit-exact outside the exemptions; exempt mismatches < 1e-4."""
+    ex, ex_blk = exempt_mask_e4m3(ref, X, A, B)
+    diff = np.asarray(codes_gpu) != ref["codes"]
+    sdiff = np.asarray(scales_gpu_linear) != ref["scales"]
+    diff_all = diff | np.repeat(sdiff, 32, axis=1)
+    r = {"mismatch": int(diff_all.sum()), "unexplained": int((diff_all & ~ex).sum()),
+         "scale_unexplained": int((sdiff & ~ex_blk).sum()), "total": diff.size}
+    assert r["unexplained"] == 0 and r["scale_unexplained"] == 0, f"{label}: {r}"
+    assert r["mismatch"] < 1e-4 * r["total"], f"{label}: too many boundary mismatches {r}"
+    return r
