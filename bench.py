@@ -272,6 +272,37 @@ def per_config(dev, peaks):
         "note": "launch-bound quantiser (128 KB); GEMM judged on weight bytes against HBM; linear = "
                 "batq_linear (the GEMM prefetches its weights into L2 while the quantiser runs)"}
     del zs
+    # W4A8 variant on q_proj: MXFP8 activations (3.03 B per element moved) and the E4M3 x E4M3
+    # block-scaled GEMM, whose roofline is the dense FP8 rate (measured bf16 x 2)
+    w8 = WL.q_proj(with_w=False)
+    S, N, M = w8.S, w8.N, w8.M
+    X8 = torch.from_numpy(np.ascontiguousarray(w8.x_bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    B8 = torch.from_numpy(np.ascontiguousarray(w8.B.reshape(-1))).to(dev)
+    r8 = torch.from_numpy(BQ.batq_clip_ratios(w8.alpha_min, w8.alpha_max)).to(dev)
+    g8 = torch.Generator(device=dev).manual_seed(7)
+    sets8 = []
+    for c in range(6):  # 6 x (16.8 MB X + 8.4 + 16.8 MB codes + 33.5 MB out) rotate through L2
+        codes8, sc8 = BQ.empty_mxfp8_buffers(S, N, device=dev)
+        wc8 = torch.empty((M, N), dtype=torch.uint8, device=dev).random_(0, 128, generator=g8)
+        wc8[(wc8 & 0x7F) == 0x7F] = 0x38  # no NaN codes
+        _, wsb = BQ.batq_mxfp8_buffer_sizes(M, N)
+        sets8.append({"X": X8 if c == 0 else X8.clone(), "codes": codes8, "scales": sc8, "wc": wc8,
+                      "wsc": torch.full((wsb,), 127, dtype=torch.uint8, device=dev),
+                      "out": torch.empty((S, M), dtype=torch.float32, device=dev)})
+    q8 = [lambda z=z: BQ.batq_quant_act_mxfp8(z["X"], w8.A, B8, r8, z["codes"], z["scales"], stream=sp)
+          for z in sets8]
+    g8f = [lambda z=z: BQ.batq_gemm_w4a8(z["codes"], z["scales"], z["wc"], z["wsc"], S, M, N, z["out"], stream=sp)
+           for z in sets8]
+    q_ms = timed(q8, 10)
+    g_ms = timed(g8f, 10)
+    qb = S * N * (2 + 1 + 1.0 / 32)
+    fp8_peak = peaks["bf16_tflops"] * 2.0
+    res["w4a8_q_proj_2048x4096x4096"] = {
+        "quant_us": q_ms * 1e3, "quant_gbs": qb / q_ms / 1e6, "quant_frac_hbm": qb / q_ms / 1e6 / peaks["hbm_gbs"],
+        "gemm_us": g_ms * 1e3, "gemm_tflops": 2.0 * S * N * M / g_ms / 1e9,
+        "gemm_frac_fp8": 2.0 * S * N * M / g_ms / 1e9 / fp8_peak,
+        "note": "MXFP8 activations x MXFP4 weights in E4M3 containers (kind::mxf8f6f4); FP8 peak = measured bf16 x 2"}
+    del sets8
     # the seven linears of one S=8192 layer, one after another (each launch reads new inputs)
     zs = []
     for j in range(7):
