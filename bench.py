@@ -122,6 +122,24 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(values, device=None):
+    """Each value's maximum over all ranks (unchanged with one rank): a multi-GPU time is the
+    slowest rank's.  Every rank must call this the same number of times."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_tflops(world_size, flops_per_rank_step, ms_per_step):
+    """Whole-job throughput: every rank processes its own batch of flops_per_rank_step in the
+    (max-over-ranks) step time (weak scaling)."""
+    return world_size * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 def _oracle_step(w, rows, wp):
     from oracle import batq_oracle as O
     x = w.x[rows]
@@ -407,9 +425,7 @@ def run_batq(args):
         g_ms = timed(gemm, args.steps)
     if ws > 1:
         dist.barrier()
-        tt = torch.tensor([local_ms, q_ms, g_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        local_ms, q_ms, g_ms = [float(v) for v in tt.tolist()]
+    local_ms, q_ms, g_ms = max_over_ranks([local_ms, q_ms, g_ms], device=dev)
     assert BQ.batq_device_error() == 0
 
     # End to end through the public call with host buffers: pinned host X in, fp32 result
@@ -454,10 +470,7 @@ def run_batq(args):
 
     e2e_run(3)
     e2e_ms = e2e_run(e2e_steps)
-    if ws > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    (e2e_ms,) = max_over_ranks([e2e_ms], device=dev)
 
     flops = 2.0 * S * N * M
     qbytes = S * N * QUANT_BYTES_PER_ELEM
@@ -467,7 +480,7 @@ def run_batq(args):
     quant_gbs = qbytes / (q_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC,
-        "value": ws * flops / (local_ms * 1e-3) / 1e12,
+        "value": whole_job_tflops(ws, flops, local_ms),
         "unit": "TFLOP/s",
         "n_gpus": ws,
         "steps": args.steps,
@@ -494,7 +507,7 @@ def run_batq(args):
         "roofline_quant": {"bound": "hbm", "achieved": quant_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                            "frac": quant_gbs / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC_BYTES["k_quant_act"],
                            "kernel": "k_quant_act"},
-        "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": whole_job_tflops(ws, flops, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
                 "d2h_bytes_per_step": int(outh[0].numel() * outh[0].element_size()), "ms_per_step": e2e_ms,
                 "note": "batq_linear on pinned host buffers; upload, compute and download on three streams, "
