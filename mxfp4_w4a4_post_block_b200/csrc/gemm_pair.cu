@@ -38,15 +38,17 @@ constexpr int kRowsPerCta = 128;       // token rows per CTA (TMEM lanes)
 constexpr int kTileM = 256;            // token rows per pair
 constexpr int kTileN = 256;            // out-features per pair (MMA N)
 constexpr int kHalfN = kTileN / 2;     // weight rows loaded by each CTA
-constexpr int kBKBytes = 128;          // bytes of K per stage and row (256 codes)
-constexpr int kStages = 6;             // ~210 KB of operands in flight per SM (L2 latency ~1.5 us)
+constexpr int kSwAtoms = 2;            // 128-byte swizzle atoms along K per stage
+constexpr int kBKBytes = 128 * kSwAtoms; // bytes of K per stage and row
+constexpr int kStages = 6 / kSwAtoms;  // ~210 KB of operands in flight per SM (L2 latency ~1.5 us)
+constexpr int kSwTile = 128 * 128;     // one 128-row x 128-byte swizzled operand tile
 constexpr int kSfAtom = 512;           // 128 rows x 4 scales
 constexpr int kEpiWarps = 8;
 constexpr int kSfWarp = 2 + kEpiWarps;          // issues the scale-factor copies
 constexpr int kThreads = (3 + kEpiWarps) * 32;
 
-constexpr int kABytes = kRowsPerCta * kBKBytes;             // 16 KB
-constexpr int kBBytes = kHalfN * kBKBytes;                  // 16 KB
+constexpr int kABytes = kRowsPerCta * kBKBytes;             // 32 KB (kSwAtoms swizzle tiles)
+constexpr int kBBytes = kHalfN * kBKBytes;                  // 32 KB
 constexpr int kBoxBytes = 1024;                             // one epilogue store box: 32 rows x 32 bytes
 constexpr int kStagingBytes = kEpiWarps * kBoxBytes;
 constexpr int kTmemCols = 512;
@@ -80,6 +82,7 @@ struct PairArgs {
   int tiles_m, tiles_n;     // pair tiles along tokens / out-features
   int num_kstages;
   int early_weights;        // weights may be read before waiting for the preceding grid
+  int sf_box_chunks;        // 256-byte scale chunks per row tile in one stage's box (<= 2 * kAtoms)
 };
 
 template <bool kOutBF16, bool kFp8>
@@ -148,6 +151,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------ producer (both CTAs) ------------------------------
     if (lane == 0) {
+      // Bytes one CTA's loads deliver per stage: the code tiles and the scale boxes
+      // (one box of own activation scales, one of two weight row tiles).
+      const uint32_t stage_tx = (uint32_t)(kABytes + kBBytes) + 3u * (uint32_t)g.sf_box_chunks * 256u;
       // Stage g of this cluster's sequence: tile cluster_id + (g / nks) * num_clusters, K step g % nks.
       const int total = my_tiles * nks;
       auto a_row_of = [&](int gi) { return ((cluster_id + (gi / nks) * num_clusters) / g.tiles_n) * kTileM + (int)rank * kRowsPerCta; };
@@ -157,16 +163,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint8_t* st = smem + st_idx * kStageBytes;
         const uint32_t bar = mapa_shared(smem_u32(&full[st_idx]), 0);
         const int ks = gi % nks;
-        tma_load_2d_pair(st + kABytes, &tm_w, bar, ks * kBKBytes, w_row_of(gi) + (int)rank * kHalfN);
+#pragma unroll
+        for (int t = 0; t < kSwAtoms; ++t)
+          tma_load_2d_pair(st + kABytes + t * kSwTile, &tm_w, bar, ks * kBKBytes + t * 128,
+                           w_row_of(gi) + (int)rank * kHalfN);
         tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &tm_sfw, bar, 0, ks * 2 * C::kAtoms,
-                         w_row_of(gi) / kRowsPerCta);
+                         w_row_of(gi) / kRowsPerCta);  // {2 row tiles} x {sf_box_chunks}
       };
       auto issue_activations = [&](int gi) {
         const int st_idx = gi % kStages;
         uint8_t* st = smem + st_idx * kStageBytes;
         const uint32_t bar = mapa_shared(smem_u32(&full[st_idx]), 0);
         const int ks = gi % nks;
-        tma_load_2d_pair(st, &tm_a, bar, ks * kBKBytes, a_row_of(gi));
+#pragma unroll
+        for (int t = 0; t < kSwAtoms; ++t)
+          tma_load_2d_pair(st + t * kSwTile, &tm_a, bar, ks * kBKBytes + t * 128, a_row_of(gi));
         // scale tiles: {256-byte chunk, K chunk (2 per 4-scale atom), 128-row tile}
         tma_load_3d_pair(st + kABytes + kBBytes, &tm_sfa, bar, 0, ks * 2 * C::kAtoms, a_row_of(gi) / kRowsPerCta);
       };
@@ -176,7 +187,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int prologue = total < kStages ? total : kStages;
       if (!g.early_weights) griddep_wait();
       for (int gi = 0; gi < prologue; ++gi) {
-        if (leader) mbar_arrive_expect_tx(&full[gi], 2u * C::kStageTxBytes);
+        if (leader) mbar_arrive_expect_tx(&full[gi], 2u * stage_tx);
         issue_weights(gi);
       }
       if (g.early_weights) griddep_wait();
@@ -188,7 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           set_error(g.err, kErrReleaseTimeout);
           break;
         }
-        if (leader) mbar_arrive_expect_tx(&full[s], 2u * C::kStageTxBytes);
+        if (leader) mbar_arrive_expect_tx(&full[s], 2u * stage_tx);
         issue_weights(gi);
         issue_activations(gi);
         if (++s == kStages) {
@@ -224,22 +235,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t sb = sa + kABytes;
         const int kleft = g.N - ks * kBK;
         const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
-        const uint64_t da = sdesc_kmajor_sw128(sa);
-        const uint64_t db = sdesc_kmajor_sw128(sb);
         for (int j = 0; j < nmma; ++j) {
           // MMA j covers 32-element scale blocks kb.. of the stage: atom kb / 4,
           // byte kb % 4 of each 4-scale TMEM column.
           const int kb = j * (kKPerMma / 32);
           const int a = kb >> 2;
           const int sf_id = kb & 3;
-          // Advance K by 32 bytes inside the 128-byte swizzle atom.
+          // Bytes 32j.. of the stage's K: swizzle tile j / 4, then 32 bytes per
+          // MMA inside its 128-byte swizzle atom.
+          const uint64_t da = sdesc_kmajor_sw128(sa + (j >> 2) * kSwTile) + (uint64_t)((j & 3) * 2);
+          const uint64_t db = sdesc_kmajor_sw128(sb + (j >> 2) * kSwTile) + (uint64_t)((j & 3) * 2);
           if constexpr (kFp8)
-            tc_mma_pair_mxf8(t_acc, da + (uint64_t)(j * 2), db + (uint64_t)(j * 2), idesc_mxf8(256, kTileN, sf_id, sf_id),
+            tc_mma_pair_mxf8(t_acc, da, db, idesc_mxf8(256, kTileN, sf_id, sf_id),
                              t_sfa + st_idx * kSfaCols + a * 4, t_sfb + st_idx * kSfbCols + a * 8,
                              (ks > 0 || j > 0) ? 1u : 0u);
           else
-            tc_mma_pair_mxf4(t_acc, da + (uint64_t)(j * 2), db + (uint64_t)(j * 2),
-                             idesc_mxf4_m256(kTileN, sf_id, sf_id), t_sfa + st_idx * kSfaCols + a * 4,
+            tc_mma_pair_mxf4(t_acc, da, db, idesc_mxf4_m256(kTileN, sf_id, sf_id), t_sfa + st_idx * kSfaCols + a * 4,
                              t_sfb + st_idx * kSfbCols + a * 8, (ks > 0 || j > 0) ? 1u : 0u);
         }
         tc_commit_pair(&empty[st_idx], 0x3);
@@ -270,10 +281,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int atoms = ((nmma - 1) * (kKPerMma / 32)) / 4 + 1;  // atoms the stage's MMAs read
         for (int a = 0; a < atoms; ++a) {
           tc_cp_pair_32x128b_warpx4(t_sfa + st_idx * kSfaCols + a * 4, sdesc_sf_atom(ssfa + a * kSfAtom));
-          // weight-scale box is {2 row tiles} x {K atoms}: row tile r, atom a at (r * kAtoms + a) * 512
+          // weight-scale box is {2 row tiles} x {sf_box_chunks}: row tile r, atom a at
+          // r * sf_box_chunks * 256 + a * 512
           tc_cp_pair_32x128b_warpx4(t_sfb + st_idx * kSfbCols + a * 8, sdesc_sf_atom(ssfb + a * kSfAtom));
           tc_cp_pair_32x128b_warpx4(t_sfb + st_idx * kSfbCols + a * 8 + 4,
-                                    sdesc_sf_atom(ssfb + (C::kAtoms + a) * kSfAtom));
+                                    sdesc_sf_atom(ssfb + g.sf_box_chunks * 256 + a * kSfAtom));
         }
         tc_commit_pair_local(&sf_ready[st_idx]);
       }
@@ -407,24 +419,28 @@ template <bool kOutBF16, bool kFp8>
 cudaError_t launch_pair_impl(const GemmLaunch& L) {
   using C = PairCfg<kFp8>;
   const uint64_t row_bytes = (uint64_t)(kFp8 ? L.N : L.N / 2);
+  // Code tiles: boxes of 128 rows x 128 bytes (one swizzle atom); a stage takes kSwAtoms of them.
   const int kpad = (L.N / 32 + 3) / 4 * 4;
   const uint64_t sf_row_tile_bytes = (uint64_t)(kpad / 4) * kSfAtom;
   const uint64_t a_tiles = (uint64_t)(L.S + 127) / 128;
   const uint64_t w_tiles = (uint64_t)(L.M + 127) / 128;
 
   CUtensorMap tm_a, tm_w, tm_sfa, tm_sfw, tm_out, tm_out_wide;
-  if (!make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_codes, row_bytes, (uint64_t)L.S, row_bytes, kBKBytes,
+  if (!make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_codes, row_bytes, (uint64_t)L.S, row_bytes, 128,
                    kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (!make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_codes, row_bytes, (uint64_t)L.M, row_bytes, kBKBytes,
+  if (!make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_codes, row_bytes, (uint64_t)L.M, row_bytes, 128,
                    kHalfN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  // Scale tiles as {256-byte chunks, chunks per row tile, row tiles}; one box = 2 K atoms (x 2 row tiles).
-  if (!make_map_3d(&tm_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_scales, 256, sf_row_tile_bytes / 256, a_tiles, 256,
-                   sf_row_tile_bytes, 256, 2 * C::kAtoms, 1))
+  // Scale tiles as {256-byte chunks, chunks per row tile, row tiles}; one box = the stage's K
+  // atoms (x 2 row tiles for the weights), clamped to the row tile when all of K is shorter.
+  const uint64_t chunks = sf_row_tile_bytes / 256;
+  const int box_chunks = (int)(chunks < (uint64_t)(2 * C::kAtoms) ? chunks : (uint64_t)(2 * C::kAtoms));
+  if (!make_map_3d(&tm_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_scales, 256, chunks, a_tiles, 256,
+                   sf_row_tile_bytes, 256, box_chunks, 1))
     return cudaErrorInvalidValue;
-  if (!make_map_3d(&tm_sfw, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_scales, 256, sf_row_tile_bytes / 256, w_tiles, 256,
-                   sf_row_tile_bytes, 256, 2 * C::kAtoms, 2))
+  if (!make_map_3d(&tm_sfw, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_scales, 256, chunks, w_tiles, 256,
+                   sf_row_tile_bytes, 256, box_chunks, 2))
     return cudaErrorInvalidValue;
   const uint32_t esz = kOutBF16 ? 2 : 4;
   if (!make_map_2d(&tm_out, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
@@ -445,6 +461,7 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   g.tiles_n = (L.M + kTileN - 1) / kTileN;
   g.num_kstages = (L.N + C::kBK - 1) / C::kBK;
   g.early_weights = L.weights_ready ? 1 : 0;
+  g.sf_box_chunks = box_chunks;
 
   auto kern = k_gemm_pair<kOutBF16, kFp8>;
   static bool attr_set[64] = {false};
