@@ -49,6 +49,23 @@ MXFP4 weights; p3 abstract and Table 2):
 * The MXFP4 weights are consumed from one-byte E4M3 containers that hold the
   same E2M1 values exactly (every E2M1 value is an E4M3 value).
 
+NVFP4 output variant (format named on the ARCQuant page: 16 E2M1 elements
+share one E4M3 scale; the pages give no other rule, so these are readings):
+
+* The transform and the clip stay on 32-element blocks (the method's own
+  granularity); each clipped block is then stored as two 16-element groups.
+* Per-tensor fp32 encode scale gs (decoded value = code * scale / gs), as the
+  block-scaled FP4 tensor-core GEMM consumes only the group scales and applies
+  a per-tensor factor afterwards; gs = 1 is the format with no tensor scale.
+  For weights gs = fp32(448 * 6 / amax of the fused fp32 weights).
+* Group scale = E4M3 of fp32(fp32(amax * gs) / 6), nearest even, saturating at
+  448; element q = fp32(v * fp32(gs / scale)) (0 multiplier for a zero scale),
+  then the E2M1 table.  All steps are fp32 operations so that the CUDA path
+  can take the same decisions in the same precision.
+* A non-finite 32-block gives scale byte 0x7F (E4M3 NaN) to both groups and
+  zero codes.
+* GEMM: out = fp32(1 / fp32(gs_a * gs_w)) * sum (code_a s_a)(code_w s_w).
+
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 closed forms, brute force and the pages' Table 1.
 """
@@ -532,3 +549,122 @@ def gemm_w4a8(a_codes8, a_scales, w_codes8, w_scales):
     Da = dequantize_e4m3(a_codes8, a_scales)
     Dw = dequantize_e4m3(w_codes8, w_scales)
     return Da @ Dw.T, np.abs(Da) @ np.abs(Dw).T
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 output variant: 16-element groups sharing one E4M3 scale
+# [ARCQuant page (zhihu-style summary), section "背景：为什么 W4A4 在 NVFP4 上很难":
+#  every 16 E2M1 elements share one E4M3 scale factor]
+# ---------------------------------------------------------------------------
+
+NV_G = 16                 # elements per NVFP4 scale group
+NV_SCALE_NAN = 0x7F       # E4M3 NaN: scale byte of a group whose 32-block is non-finite
+NV_GLOBAL_NUMERATOR = 448.0 * 6.0  # largest E4M3 scale x largest E2M1 magnitude
+
+
+def f32(v):
+    """Round fp64 values to fp32 (one IEEE round-to-nearest-even).
+
+    Every fp32 operation below is written as the exact (or fp64) result
+    rounded once to fp32.  A product of two fp32 values is exact in fp64; for
+    a quotient, fp64 rounding followed by fp32 rounding equals the correctly
+    rounded fp32 quotient because 53 >= 2 * 24 + 2 (double rounding is
+    innocuous for one operation in that case).
+    """
+    return np.asarray(v, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+def nvfp4_group_scale(amax, gs):
+    """E4M3 scale byte, its value, and the element multiplier of 16-element groups.
+
+    amax: clipped group amax (fp32 values); gs: per-tensor fp32 encode scale
+    (decoded tensor = code * scale / gs).  Steps, each rounded to fp32:
+    t = amax * gs, u = t / 6, scale = E4M3(u) (nearest even, saturating at 448),
+    multiplier = gs / scale (0 when the scale is 0).
+    """
+    amax = np.asarray(amax, dtype=np.float64)
+    gs = float(np.float32(gs))
+    t = f32(amax * gs)
+    u = f32(t / 6.0)
+    byte = e4m3_encode(u).astype(np.int64)            # u >= 0: sign bit clear
+    sval = e4m3_decode(byte)
+    with np.errstate(divide="ignore"):
+        mult = np.where(sval == 0.0, 0.0, f32(gs / np.where(sval == 0.0, 1.0, sval)))
+    return byte, sval, mult
+
+
+def nvfp4_quantize(V: np.ndarray, gs: float = 1.0, nonfinite: np.ndarray | None = None):
+    """NVFP4 of fp32 rows V (rows, N): 16-element groups, E4M3 scale, E2M1 codes.
+
+    Each element: q = fp32(v * multiplier), then the E2M1 table (nearest even,
+    saturating at 6, sign kept on zero).  ``nonfinite`` flags 32-element
+    blocks (rows, N/32) holding a non-finite value: both of their groups get
+    scale byte 0x7F and codes 0.  Returns (packed codes (rows, N/2), scale
+    bytes (rows, N/16) uint8, q (rows, N) fp64).
+    """
+    V = np.asarray(V, dtype=np.float32)
+    rows, N = V.shape
+    k16 = N // NV_G
+    Vg = V.reshape(rows, k16, NV_G).astype(np.float64)
+    if nonfinite is None:
+        nonfinite = ~np.all(np.isfinite(V.reshape(rows, N // G, G)), axis=2)
+    nf16 = np.repeat(nonfinite, G // NV_G, axis=1)
+    with np.errstate(invalid="ignore"):
+        amax = np.abs(Vg).max(axis=2)
+    amax = np.where(nf16, 0.0, amax)
+    byte, _, mult = nvfp4_group_scale(amax, gs)
+    with np.errstate(invalid="ignore"):
+        q = f32(Vg * mult[:, :, None])
+    q = np.where(nf16[:, :, None], 0.0, q)
+    codes = e2m1_encode(q).reshape(rows, N)
+    codes = np.where(np.repeat(nf16, NV_G, axis=1), 0, codes)
+    scale = np.where(nf16, NV_SCALE_NAN, byte).astype(np.uint8)
+    return pack_nibbles(codes), scale, q.reshape(rows, N)
+
+
+def dequantize_nvfp4(packed: np.ndarray, scales: np.ndarray, gs: float = 1.0) -> np.ndarray:
+    """fp64 values code * E4M3(scale) / gs; a 0x7F scale decodes to NaN."""
+    codes = unpack_nibbles(packed)
+    rows, N = codes.shape
+    vals = e2m1_decode(codes).reshape(rows, N // NV_G, NV_G)
+    sval = e4m3_decode(np.asarray(scales, dtype=np.int64))
+    return (vals * sval[:, :, None]).reshape(rows, N) / float(np.float32(gs))
+
+
+def quant_act_nvfp4(X, A, B, alpha_min, alpha_max, gs: float = 1.0) -> dict:
+    """Online activation path with NVFP4 output: y = x P_i and the clip on 32-blocks, then NVFP4."""
+    Y = transform(X, A, B)
+    Yh, lo, hi, nonfinite = clip_blocks(Y, clip_ratios(alpha_min), clip_ratios(alpha_max))
+    codes, scales, q = nvfp4_quantize(Yh, gs, nonfinite)
+    return {"Y": Y, "Y_hat": Yh, "codes": codes, "scales": scales, "q": q,
+            "nonfinite": nonfinite, "lo": lo, "hi": hi, "gs": float(np.float32(gs))}
+
+
+def nvfp4_global_scale(amax: float) -> float:
+    """Per-tensor encode scale fp32(448 * 6 / amax), 1 for an all-zero (or too small) tensor."""
+    a = float(np.float32(amax))
+    if not a > 0.0:
+        return 1.0
+    g = float(f32(NV_GLOBAL_NUMERATOR / a))
+    return g if np.isfinite(g) else 1.0
+
+
+def prepare_weights_nvfp4(W, A, B) -> dict:
+    """Fused weights rounded to fp32, per-tensor scale from their amax, NVFP4 along K (no clip)."""
+    Wf = fuse_weights_f64(W, A, B).astype(np.float32)
+    gs = nvfp4_global_scale(np.max(np.abs(Wf)))
+    codes, scales, q = nvfp4_quantize(Wf, gs)
+    return {"W_fused": Wf, "codes": codes, "scales": scales, "q": q, "gs": gs}
+
+
+def nvfp4_alpha(gs_a: float, gs_w: float) -> float:
+    """Epilogue factor fp32(1 / fp32(gs_a * gs_w)) undoing both per-tensor scales."""
+    return float(f32(1.0 / f32(float(np.float32(gs_a)) * float(np.float32(gs_w)))))
+
+
+def gemm_nvfp4(a_codes, a_scales, w_codes, w_scales, alpha: float = 1.0):
+    """out = alpha * sum_n (code_a s_a)(code_w s_w) in fp64, plus T = |alpha| sum |a||w|."""
+    Da = dequantize_nvfp4(a_codes, a_scales)
+    Dw = dequantize_nvfp4(w_codes, w_scales)
+    al = float(np.float32(alpha))
+    return al * (Da @ Dw.T), abs(al) * (np.abs(Da) @ np.abs(Dw).T)
