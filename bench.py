@@ -207,8 +207,8 @@ def run_reference(args):
 
 
 def per_config(dev, peaks):
-    """Kernel-alone throughput on the other workloads (down_proj prefill, decode S=16, the seven
-    linears of one S=8192 layer), each timed over back-to-back launches whose inputs rotate through
+    """Kernel-alone throughput on the other workloads (down_proj prefill, decode S=16, the W4A8 and
+    NVFP4 variants on q_proj, the seven linears of one S=8192 layer), each timed over back-to-back launches whose inputs rotate through
     more than the 126 MB L2.  Activation codes come from the quantiser; weight codes are random
     bytes with unit scales (timing does not depend on their values)."""
     import torch
@@ -321,6 +321,31 @@ def per_config(dev, peaks):
         "gemm_frac_fp8": 2.0 * S * N * M / g_ms / 1e9 / fp8_peak,
         "note": "MXFP8 activations x MXFP4 weights in E4M3 containers (kind::mxf8f6f4); FP8 peak = measured bf16 x 2"}
     del sets8
+    # NVFP4 output on q_proj: E4M3 scale per 16 elements (2.5625 B per element moved; per-tensor
+    # encode scale 2.0 from the device) and the kind::mxf4nvf4 GEMM, judged against the FP4 peak
+    gsn = torch.full((1,), 2.0, dtype=torch.float32, device=dev)
+    gn = torch.Generator(device=dev).manual_seed(11)
+    setsn = []
+    for c in range(6):  # 6 x (16.8 MB X + 4.2 + 8.4 MB codes + 33.5 MB out) rotate through L2
+        cn, sn = BQ.empty_nvfp4_buffers(S, N, device=dev)
+        wcn, wsn = BQ.empty_nvfp4_buffers(M, N, device=dev)
+        wcn.random_(0, 256, generator=gn)
+        wsn.fill_(0x38)  # E4M3 1.0
+        setsn.append({"X": X8 if c == 0 else X8.clone(), "codes": cn, "scales": sn, "wc": wcn, "wsc": wsn,
+                      "out": torch.empty((S, M), dtype=torch.float32, device=dev)})
+    qn = [lambda z=z: BQ.batq_quant_act_nvfp4(z["X"], w8.A, B8, r8, z["codes"], z["scales"], gs=gsn, stream=sp)
+          for z in setsn]
+    gnf = [lambda z=z: BQ.batq_gemm_nvfp4(z["codes"], z["scales"], gsn, z["wc"], z["wsc"], None, S, M, N, z["out"],
+                                          stream=sp) for z in setsn]
+    q_ms = timed(qn, 10)
+    g_ms = timed(gnf, 10)
+    qb = S * N * (2 + 0.5 + 1.0 / 16)
+    res["nvfp4_q_proj_2048x4096x4096"] = {
+        "quant_us": q_ms * 1e3, "quant_gbs": qb / q_ms / 1e6, "quant_frac_hbm": qb / q_ms / 1e6 / peaks["hbm_gbs"],
+        "gemm_us": g_ms * 1e3, "gemm_tflops": 2.0 * S * N * M / g_ms / 1e9,
+        "gemm_frac_fp4": 2.0 * S * N * M / g_ms / 1e9 / fp4_peak,
+        "note": "NVFP4 activations and weights (E4M3 scale per 16, per-tensor encode scale; kind::mxf4nvf4 block16)"}
+    del setsn
     # the seven linears of one S=8192 layer, one after another (each launch reads new inputs)
     zs = []
     for j in range(7):

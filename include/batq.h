@@ -250,6 +250,86 @@ BATQ_API batq_status batq_linear_w4a8(const void* X, batq_dtype x_dtype, int S, 
                              void* workspace, size_t workspace_bytes,
                              batq_dtype out_dtype, void* out, int ldo, void* stream);
 
+/* ------------------------------------------------------------------------
+ * NVFP4 output variant.  The format is the one the ARCQuant page names
+ * (section "背景：为什么 W4A4 在 NVFP4 上很难"): 16 E2M1 elements share one
+ * E4M3 scale.  The transform and the clip stay on the method's 32-element
+ * blocks (BATQuant daily-arxiv summary, "块仿射变换" and "块级可学习裁剪");
+ * each clipped block is stored as two 16-element groups.  A per-tensor fp32
+ * encode scale gs (decoded value = code x group scale / gs) widens the range
+ * of the E4M3 group scales; gs = 1 is the format with no tensor scale.
+ * Every step is an IEEE fp32 operation:
+ *   group scale  s = E4M3(fp32(fp32(amax_group * gs) / 6)), nearest even,
+ *                saturating at 448 (amax of the clipped group);
+ *   element      q = fp32(y_hat * fp32(gs / s)) (multiplier 0 when s = 0),
+ *                then E2M1 nearest even, saturating at 6, sign kept on zero.
+ * A 32-block holding a non-finite value gets scale byte 0x7F (E4M3 NaN) in
+ * both groups and zero codes.  Codes are packed as in batq_quant_act.  Scales
+ * are one byte per row and group: LINEAR layout rows x N/16, row-major; MMA
+ * layout the 128-row x 4-column tiles of batq_quant_act with N/16 columns
+ * (N/16 is a multiple of 4) and rows padded to 128 with the byte 0x38 (1.0).
+ * All scale pointers must be 16-byte aligned, gs pointers 4-byte aligned.
+ * ------------------------------------------------------------------------ */
+
+/* Sizes of an NVFP4 operand: rows x N/2 code bytes; scale bytes as above. Host only. */
+BATQ_API batq_status batq_nvfp4_buffer_sizes(int rows, int N, batq_scale_layout layout, size_t* code_bytes,
+                                    size_t* scale_bytes);
+
+/*
+ * As batq_quant_act with NVFP4 output.  gs_dev: device float holding the
+ * per-tensor encode scale (finite and > 0; a static calibration value), or
+ * NULL for 1.  It is read after the preceding grid in the stream finishes.
+ * Errors as batq_quant_act; BATQ_ERR_ALIGNMENT also for a misaligned scales
+ * or gs_dev pointer.
+ */
+BATQ_API batq_status batq_quant_act_nvfp4(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                                 const float* A_host, const float* B_dev, const float* ratios_dev,
+                                 const float* gs_dev, uint8_t* codes, uint8_t* scales,
+                                 batq_scale_layout layout, float* y_debug, void* stream);
+
+/* Device workspace bytes batq_prepare_weights_nvfp4 needs. Host only. */
+BATQ_API batq_status batq_prepare_weights_nvfp4_workspace_size(int N, size_t* bytes);
+
+/*
+ * Offline weight side with NVFP4 output: the fused weights W' = W P^-T
+ * (as batq_prepare_weights) are measured once for their largest magnitude
+ * amax, then quantised (no clip) with gs = fp32(448 * 6 / amax) (1 for
+ * all-zero weights), which is written to the device float *gs_out_dev for the
+ * GEMM.  Two kernel launches and a 4-byte memset on `stream`, nothing
+ * synchronised.  Errors as batq_prepare_weights (BATQ_ERR_INVALID_ARG also
+ * for a NULL gs_out_dev).
+ */
+BATQ_API batq_status batq_prepare_weights_nvfp4(const void* W, batq_dtype w_dtype, int M, int N, int ldw,
+                                       const float* A_host, const float* B_host, uint8_t* w_codes,
+                                       uint8_t* w_scales, batq_scale_layout layout, float* gs_out_dev,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * NVFP4 block-scaled GEMM (tcgen05 kind::mxf4nvf4, one E4M3 scale per 16 K):
+ * out = fp32(1 / fp32(gs_a * gs_w)) x sum_n (code_a s_a)(code_w s_w), fp32
+ * accumulation in tensor memory.  a_gs_dev / w_gs_dev: device floats (NULL
+ * for 1), read after the preceding grid finishes.  Scales in MMA layout.
+ * Shapes and errors as batq_gemm_mxfp4.
+ */
+BATQ_API batq_status batq_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_gs_dev,
+                            const uint8_t* w_codes, const uint8_t* w_scales, const float* w_gs_dev,
+                            int S, int M, int N, batq_dtype out_dtype, void* out, int ldo, void* stream);
+
+/* Device workspace bytes batq_linear_nvfp4 needs (codes + MMA-layout scales). Host only. */
+BATQ_API batq_status batq_linear_nvfp4_workspace_size(int S, int N, size_t* bytes);
+
+/*
+ * Whole NVFP4 linear: batq_quant_act_nvfp4 (gs from a_gs_dev, MMA layout,
+ * into the workspace) followed by batq_gemm_nvfp4 on the same stream, with
+ * the weights and w_gs_dev from batq_prepare_weights_nvfp4.  Other arguments
+ * and errors as batq_linear.
+ */
+BATQ_API batq_status batq_linear_nvfp4(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                              const float* A_host, const float* B_dev, const float* ratios_dev,
+                              const float* a_gs_dev, const uint8_t* w_codes, const uint8_t* w_scales,
+                              const float* w_gs_dev, int M, void* workspace, size_t workspace_bytes,
+                              batq_dtype out_dtype, void* out, int ldo, void* stream);
+
 /*
  * batq_linear without a caller-provided workspace, for callers that cannot
  * allocate device memory (for example a plugin running in a process whose

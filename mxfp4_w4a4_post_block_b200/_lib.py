@@ -52,6 +52,16 @@ SIGNATURES = {
     "batq_linear_w4a8_workspace_size": (_c_int, [_c_int, _c_int, _c_size_p]),
     "batq_linear_w4a8": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
                                   ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
+    "batq_nvfp4_buffer_sizes": (_c_int, [_c_int, _c_int, _c_int, _c_size_p, _c_size_p]),
+    "batq_quant_act_nvfp4": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
+                                      _vp, _vp]),
+    "batq_prepare_weights_nvfp4_workspace_size": (_c_int, [_c_int, _c_size_p]),
+    "batq_prepare_weights_nvfp4": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _vp,
+                                            _vp, ctypes.c_size_t, _vp]),
+    "batq_gemm_nvfp4": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_int, _vp]),
+    "batq_linear_nvfp4_workspace_size": (_c_int, [_c_int, _c_int, _c_size_p]),
+    "batq_linear_nvfp4": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
+                                   _vp, ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
     "batq_selftest_wait_timeout": (_c_int, [ctypes.c_uint, _vp]),
     "batq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint)]),
 }

@@ -222,6 +222,74 @@ def batq_linear_w4a8(X, A, B, ratios, w_codes8, w_scales, M, workspace, out, str
                                         _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_linear_w4a8")
 
 
+# ------------------------------------------------------ NVFP4 output calls
+
+def batq_nvfp4_buffer_sizes(rows: int, N: int, layout: int = BATQ_SCALES_MMA):
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.load().batq_nvfp4_buffer_sizes(rows, N, layout, ctypes.byref(cb), ctypes.byref(sb)),
+           "batq_nvfp4_buffer_sizes")
+    return cb.value, sb.value
+
+
+def batq_prepare_weights_nvfp4_workspace_size(N: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_lib.load().batq_prepare_weights_nvfp4_workspace_size(N, ctypes.byref(b)),
+           "batq_prepare_weights_nvfp4_workspace_size")
+    return b.value
+
+
+def batq_linear_nvfp4_workspace_size(S: int, N: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_lib.load().batq_linear_nvfp4_workspace_size(S, N, ctypes.byref(b)), "batq_linear_nvfp4_workspace_size")
+    return b.value
+
+
+def batq_quant_act_nvfp4(X, A, B, ratios, codes, scales, gs=None, layout=BATQ_SCALES_MMA, y_debug=None,
+                         stream=None):
+    """Transform + clip (32-blocks) + NVFP4 (E4M3 scale per 16) of X (S x N); gs: 1-element CUDA float or None."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    _check(_lib.load().batq_quant_act_nvfp4(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0), a.ctypes.data,
+                                            _dev_ptr(B, "B"), _dev_ptr(ratios, "ratios"), _dev_ptr(gs, "gs"),
+                                            _dev_ptr(codes, "codes"), _dev_ptr(scales, "scales"), layout,
+                                            _dev_ptr(y_debug, "y_debug"), _stream(stream)), "batq_quant_act_nvfp4")
+
+
+def batq_prepare_weights_nvfp4(W, A, B_host, w_codes, w_scales, gs_out, workspace, layout=BATQ_SCALES_MMA,
+                               stream=None):
+    """Offline: fused weights measured for their amax, then NVFP4 with gs = 448*6/amax written to gs_out."""
+    M, N = W.shape
+    a = _host_f32(A, 64, "A")
+    b = _host_f32(B_host, (N // 32) * 16, "B")
+    _check(_lib.load().batq_prepare_weights_nvfp4(_dev_ptr(W, "W"), _dtype_code(W), M, N, W.stride(0),
+                                                  a.ctypes.data, b.ctypes.data, _dev_ptr(w_codes, "w_codes"),
+                                                  _dev_ptr(w_scales, "w_scales"), layout, _dev_ptr(gs_out, "gs_out"),
+                                                  _dev_ptr(workspace, "workspace"),
+                                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+           "batq_prepare_weights_nvfp4")
+
+
+def batq_gemm_nvfp4(a_codes, a_scales, a_gs, w_codes, w_scales, w_gs, S, M, N, out, stream=None):
+    """out (S x M) = fp32(1/(gs_a gs_w)) x deq(a) deq(w)^T for NVFP4 operands (gs tensors or None)."""
+    _check(_lib.load().batq_gemm_nvfp4(_dev_ptr(a_codes, "a_codes"), _dev_ptr(a_scales, "a_scales"),
+                                       _dev_ptr(a_gs, "a_gs"), _dev_ptr(w_codes, "w_codes"),
+                                       _dev_ptr(w_scales, "w_scales"), _dev_ptr(w_gs, "w_gs"), S, M, N,
+                                       _dtype_code(out), _dev_ptr(out, "out"), out.stride(0), _stream(stream)),
+           "batq_gemm_nvfp4")
+
+
+def batq_linear_nvfp4(X, A, B, ratios, a_gs, w_codes, w_scales, w_gs, M, workspace, out, stream=None):
+    """Whole NVFP4 linear: NVFP4 activations online, then the kind::mxf4nvf4 block-scaled GEMM."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    _check(_lib.load().batq_linear_nvfp4(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0), a.ctypes.data,
+                                         _dev_ptr(B, "B"), _dev_ptr(ratios, "ratios"), _dev_ptr(a_gs, "a_gs"),
+                                         _dev_ptr(w_codes, "w_codes"), _dev_ptr(w_scales, "w_scales"),
+                                         _dev_ptr(w_gs, "w_gs"), M, _dev_ptr(workspace, "workspace"),
+                                         workspace.numel() * workspace.element_size(), _dtype_code(out),
+                                         _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_linear_nvfp4")
+
+
 def batq_selftest_wait_timeout(limit_us: int, stream=None):
     """Launch the bounded-wait self-test kernel (its wait always expires)."""
     _check(_lib.load().batq_selftest_wait_timeout(limit_us, _stream(stream)), "batq_selftest_wait_timeout")
@@ -252,5 +320,14 @@ def empty_mxfp8_buffers(rows: int, N: int, layout=BATQ_SCALES_MMA, device="cuda"
     torch = _torch()
     cb, sb = batq_mxfp8_buffer_sizes(rows, N, layout)
     codes = torch.empty((rows, N), dtype=torch.uint8, device=device)
+    scales = torch.empty(sb, dtype=torch.uint8, device=device)
+    return codes, scales
+
+
+def empty_nvfp4_buffers(rows: int, N: int, layout=BATQ_SCALES_MMA, device="cuda"):
+    """(codes, scales) uint8 CUDA tensors for NVFP4 (packed E2M1, one scale per 16) of a rows x N matrix."""
+    torch = _torch()
+    cb, sb = batq_nvfp4_buffer_sizes(rows, N, layout)
+    codes = torch.empty((rows, N // 2), dtype=torch.uint8, device=device)
     scales = torch.empty(sb, dtype=torch.uint8, device=device)
     return codes, scales

@@ -106,9 +106,13 @@ bool invert(const double* a, double* inv, int n) {
   return std::isfinite(cond) && cond <= 1e8;
 }
 
+// gs / gs_amax / gs_out / amax_out: the NVFP4 per-tensor scale sources and
+// outputs of batq::QuantLaunch (nullptr for the MX formats).
 batq_status launch_quant(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
                          const float* B_dev, const float* ratios_dev, uint8_t* codes, uint8_t* scales,
-                         batq_scale_layout layout, float* y_debug, bool fp8, cudaStream_t stream) {
+                         batq_scale_layout layout, float* y_debug, int fmt, cudaStream_t stream,
+                         const float* gs = nullptr, const unsigned* gs_amax = nullptr, float* gs_out = nullptr,
+                         unsigned* amax_out = nullptr) {
   batq::QuantLaunch L;
   L.X = X;
   L.bf16 = (x_dtype == BATQ_BF16);
@@ -124,7 +128,11 @@ batq_status launch_quant(const void* X, batq_dtype x_dtype, int S, int N, int ld
   L.y_debug = y_debug;
   L.err = error_word();
   L.stream = stream;
-  L.fp8 = fp8;
+  L.fmt = fmt;
+  L.gs = gs;
+  L.gs_amax = gs_amax;
+  L.gs_out = gs_out;
+  L.amax_out = amax_out;
   cudaError_t e = batq::launch_quant_act(L);
   if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
   return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
@@ -165,7 +173,8 @@ batq_status check_gemm_args(const uint8_t* a_codes, const uint8_t* a_scales, con
 
 batq_status launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
                         const uint8_t* w_scales, int S, int M, int N, batq_dtype out_dtype, void* out, int ldo,
-                        bool weights_ready, bool fp8, cudaStream_t stream) {
+                        bool weights_ready, int fmt, cudaStream_t stream, const float* gs_a = nullptr,
+                        const float* gs_w = nullptr) {
   batq::GemmLaunch L;
   L.a_codes = a_codes;
   L.a_scales = a_scales;
@@ -180,11 +189,48 @@ batq_status launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const u
   L.err = error_word();
   L.stream = stream;
   L.weights_ready = weights_ready;
-  L.fp8 = fp8;
+  L.fmt = fmt;
+  L.gs_a = gs_a;
+  L.gs_w = gs_w;
   cudaError_t e = batq::launch_gemm_mxfp4(L);
   if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
   return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
 }
+
+// Transform of the fused weights: W'_mat = B_i^-1 W_mat A^-T, and the
+// activation kernel computes B'^T X A', so A' = A^-T (to a_fused, host) and
+// B'_i = B_i^-T (k x 16 floats copied to the start of `workspace`, device).
+batq_status fused_transform(const float* A_host, const float* B_host, int N, void* workspace, float a_fused[64],
+                            cudaStream_t s) {
+  const int k = N / 32;
+  double a[64], ainv[64];
+  for (int i = 0; i < 64; ++i) a[i] = A_host[i];
+  if (!invert(a, ainv, 8)) return BATQ_ERR_SINGULAR;
+  for (int r = 0; r < 8; ++r)
+    for (int c = 0; c < 8; ++c) a_fused[r * 8 + c] = (float)ainv[c * 8 + r];
+  std::vector<float> b_fused((size_t)k * 16);
+  for (int i = 0; i < k; ++i) {
+    double b[16], binv[16];
+    for (int j = 0; j < 16; ++j) b[j] = B_host[(size_t)i * 16 + j];
+    if (!invert(b, binv, 4)) return BATQ_ERR_SINGULAR;
+    for (int r = 0; r < 4; ++r)
+      for (int c = 0; c < 4; ++c) b_fused[(size_t)i * 16 + r * 4 + c] = (float)binv[c * 4 + r];
+  }
+  if (cudaMemcpyAsync(workspace, b_fused.data(), b_fused.size() * sizeof(float), cudaMemcpyHostToDevice, s) !=
+      cudaSuccess)
+    return BATQ_ERR_CUDA;
+  // cudaMemcpyAsync from pageable memory has staged the bytes when it returns,
+  // so b_fused may be released.
+  return BATQ_OK;
+}
+
+size_t nv_scale_bytes_for(int rows, int N, batq_scale_layout layout) {
+  const size_t cols = (size_t)N / 16;  // a multiple of 4 for N % 64 == 0
+  if (layout == BATQ_SCALES_MMA) return round_up((size_t)rows, 128) * cols;
+  return (size_t)rows * cols;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 }  // namespace
 
@@ -237,8 +283,8 @@ batq_status batq_quant_act(const void* X, batq_dtype x_dtype, int S, int N, int 
   if (st != BATQ_OK) return st;
   st = check_arch();
   if (st != BATQ_OK) return st;
-  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug, false,
-                      static_cast<cudaStream_t>(stream));
+  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug,
+                      batq::kFmtMxfp4, static_cast<cudaStream_t>(stream));
 }
 
 batq_status batq_prepare_workspace_size(int N, size_t* bytes) {
@@ -262,31 +308,12 @@ batq_status batq_prepare_weights(const void* W, batq_dtype w_dtype, int M, int N
   st = check_arch();
   if (st != BATQ_OK) return st;
 
-  // W'_mat = B_i^-1 W_mat A^-T: the activation kernel computes B'^T X A', so
-  // A' = A^-T and B'_i = B_i^-T.
-  const int k = N / 32;
-  double a[64], ainv[64];
-  for (int i = 0; i < 64; ++i) a[i] = A_host[i];
-  if (!invert(a, ainv, 8)) return BATQ_ERR_SINGULAR;
   float a_fused[64];
-  for (int r = 0; r < 8; ++r)
-    for (int c = 0; c < 8; ++c) a_fused[r * 8 + c] = (float)ainv[c * 8 + r];
-  std::vector<float> b_fused((size_t)k * 16);
-  for (int i = 0; i < k; ++i) {
-    double b[16], binv[16];
-    for (int j = 0; j < 16; ++j) b[j] = B_host[(size_t)i * 16 + j];
-    if (!invert(b, binv, 4)) return BATQ_ERR_SINGULAR;
-    for (int r = 0; r < 4; ++r)
-      for (int c = 0; c < 4; ++c) b_fused[(size_t)i * 16 + r * 4 + c] = (float)binv[c * 4 + r];
-  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(workspace, b_fused.data(), b_fused.size() * sizeof(float), cudaMemcpyHostToDevice, s) !=
-      cudaSuccess)
-    return BATQ_ERR_CUDA;
-  // cudaMemcpyAsync from pageable memory has staged the bytes when it returns,
-  // so b_fused may be released.
+  st = fused_transform(A_host, B_host, N, workspace, a_fused, s);
+  if (st != BATQ_OK) return st;
   return launch_quant(W, w_dtype, M, N, ldw, a_fused, reinterpret_cast<const float*>(workspace), nullptr, w_codes,
-                      w_scales, layout, nullptr, false, s);
+                      w_scales, layout, nullptr, batq::kFmtMxfp4, s);
 }
 
 batq_status batq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
@@ -298,7 +325,7 @@ batq_status batq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, con
   if (st != BATQ_OK) return st;
   // The preceding grid may be anything (e.g. the weight quantiser of
   // batq_prepare_weights): wait for it before reading any operand.
-  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, false, false,
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, false, batq::kFmtMxfp4,
                      static_cast<cudaStream_t>(stream));
 }
 
@@ -331,12 +358,12 @@ batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx
   if (st != BATQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA, nullptr,
-                    false, s);
+                    batq::kFmtMxfp4, s);
   if (st != BATQ_OK) return st;
   // The quantiser just launched writes only the workspace and starts its
   // dependents after every earlier grid has finished, so the GEMM may fetch
   // weights while the quantiser runs.
-  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, false, s);
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, batq::kFmtMxfp4, s);
 }
 
 // ------------------------------------------------------------------ W4A8 variant
@@ -360,8 +387,8 @@ batq_status batq_quant_act_mxfp8(const void* X, batq_dtype x_dtype, int S, int N
   if (st != BATQ_OK) return st;
   st = check_arch();
   if (st != BATQ_OK) return st;
-  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug, true,
-                      static_cast<cudaStream_t>(stream));
+  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug,
+                      batq::kFmtMxfp8, static_cast<cudaStream_t>(stream));
 }
 
 batq_status batq_prepare_weights_w4a8_workspace_size(int M, int N, size_t* bytes) {
@@ -403,7 +430,7 @@ batq_status batq_gemm_w4a8(const uint8_t* a_codes8, const uint8_t* a_scales, con
   if (st != BATQ_OK) return st;
   st = check_arch();
   if (st != BATQ_OK) return st;
-  return launch_gemm(a_codes8, a_scales, w_codes8, w_scales, S, M, N, out_dtype, out, ldo, false, true,
+  return launch_gemm(a_codes8, a_scales, w_codes8, w_scales, S, M, N, out_dtype, out, ldo, false, batq::kFmtMxfp8,
                      static_cast<cudaStream_t>(stream));
 }
 
@@ -436,9 +463,124 @@ batq_status batq_linear_w4a8(const void* X, batq_dtype x_dtype, int S, int N, in
   if (st != BATQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA, nullptr,
-                    true, s);
+                    batq::kFmtMxfp8, s);
   if (st != BATQ_OK) return st;
-  return launch_gemm(a_codes, a_scales, w_codes8, w_scales, S, M, N, out_dtype, out, ldo, true, true, s);
+  return launch_gemm(a_codes, a_scales, w_codes8, w_scales, S, M, N, out_dtype, out, ldo, true, batq::kFmtMxfp8, s);
+}
+
+// ------------------------------------------------------------------ NVFP4 output variant
+
+batq_status batq_nvfp4_buffer_sizes(int rows, int N, batq_scale_layout layout, size_t* code_bytes,
+                                    size_t* scale_bytes) {
+  if (!code_bytes || !scale_bytes) return BATQ_ERR_INVALID_ARG;
+  if (layout != BATQ_SCALES_LINEAR && layout != BATQ_SCALES_MMA) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_mn(rows, N);
+  if (st != BATQ_OK) return st;
+  *code_bytes = (size_t)rows * (size_t)(N / 2);
+  *scale_bytes = nv_scale_bytes_for(rows, N, layout);
+  return BATQ_OK;
+}
+
+batq_status batq_quant_act_nvfp4(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
+                                 const float* B_dev, const float* ratios_dev, const float* gs_dev, uint8_t* codes,
+                                 uint8_t* scales, batq_scale_layout layout, float* y_debug, void* stream) {
+  batq_status st = check_quant_args(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout,
+                                    y_debug);
+  if (st != BATQ_OK) return st;
+  if (!aligned16(scales) || (gs_dev && !aligned4(gs_dev))) return BATQ_ERR_ALIGNMENT;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug,
+                      batq::kFmtNvfp4, static_cast<cudaStream_t>(stream), gs_dev);
+}
+
+batq_status batq_prepare_weights_nvfp4_workspace_size(int N, size_t* bytes) {
+  if (!bytes) return BATQ_ERR_INVALID_ARG;
+  size_t base = 0;
+  batq_status st = batq_prepare_workspace_size(N, &base);
+  if (st != BATQ_OK) return st;
+  *bytes = base + 256;  // + the amax word of the measuring pass
+  return BATQ_OK;
+}
+
+batq_status batq_prepare_weights_nvfp4(const void* W, batq_dtype w_dtype, int M, int N, int ldw, const float* A_host,
+                                       const float* B_host, uint8_t* w_codes, uint8_t* w_scales,
+                                       batq_scale_layout layout, float* gs_out_dev, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (!B_host || !workspace || !gs_out_dev) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_quant_args(W, w_dtype, M, N, ldw, A_host, reinterpret_cast<const float*>(workspace),
+                                    nullptr, w_codes, w_scales, layout, nullptr);
+  if (st != BATQ_OK) return st;
+  if (!aligned16(w_scales) || !aligned4(gs_out_dev)) return BATQ_ERR_ALIGNMENT;
+  size_t need = 0, base = 0;
+  batq_prepare_weights_nvfp4_workspace_size(N, &need);
+  batq_prepare_workspace_size(N, &base);
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  float a_fused[64];
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = fused_transform(A_host, B_host, N, workspace, a_fused, s);
+  if (st != BATQ_OK) return st;
+  // Pass 1 measures the amax of the fused weights, pass 2 quantises them with
+  // gs = 448 * 6 / amax and publishes gs.
+  unsigned* amax_word = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + base);
+  if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned), s) != cudaSuccess) return BATQ_ERR_CUDA;
+  const float* b_fused = reinterpret_cast<const float*>(workspace);
+  st = launch_quant(W, w_dtype, M, N, ldw, a_fused, b_fused, nullptr, w_codes, w_scales, layout, nullptr,
+                    batq::kFmtNvfp4, s, nullptr, nullptr, nullptr, amax_word);
+  if (st != BATQ_OK) return st;
+  return launch_quant(W, w_dtype, M, N, ldw, a_fused, b_fused, nullptr, w_codes, w_scales, layout, nullptr,
+                      batq::kFmtNvfp4, s, nullptr, amax_word, gs_out_dev, nullptr);
+}
+
+batq_status batq_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_gs_dev,
+                            const uint8_t* w_codes, const uint8_t* w_scales, const float* w_gs_dev, int S, int M,
+                            int N, batq_dtype out_dtype, void* out, int ldo, void* stream) {
+  batq_status st = check_gemm_args(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo);
+  if (st != BATQ_OK) return st;
+  if ((a_gs_dev && !aligned4(a_gs_dev)) || (w_gs_dev && !aligned4(w_gs_dev))) return BATQ_ERR_ALIGNMENT;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, false, batq::kFmtNvfp4,
+                     static_cast<cudaStream_t>(stream), a_gs_dev, w_gs_dev);
+}
+
+batq_status batq_linear_nvfp4_workspace_size(int S, int N, size_t* bytes) {
+  if (!bytes) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_mn(S, N);
+  if (st != BATQ_OK) return st;
+  *bytes = round_up((size_t)S * (size_t)(N / 2), 256) + nv_scale_bytes_for(S, N, BATQ_SCALES_MMA);
+  return BATQ_OK;
+}
+
+batq_status batq_linear_nvfp4(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
+                              const float* B_dev, const float* ratios_dev, const float* a_gs_dev,
+                              const uint8_t* w_codes, const uint8_t* w_scales, const float* w_gs_dev, int M,
+                              void* workspace, size_t workspace_bytes, batq_dtype out_dtype, void* out, int ldo,
+                              void* stream) {
+  if (!workspace) return BATQ_ERR_INVALID_ARG;
+  size_t need = 0;
+  batq_status st = batq_linear_nvfp4_workspace_size(S, N, &need);
+  if (st != BATQ_OK) return st;
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BATQ_ERR_ALIGNMENT;
+  uint8_t* a_codes = static_cast<uint8_t*>(workspace);
+  uint8_t* a_scales = a_codes + round_up((size_t)S * (size_t)(N / 2), 256);
+  st = check_quant_args(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA,
+                        nullptr);
+  if (st != BATQ_OK) return st;
+  st = check_gemm_args(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo);
+  if (st != BATQ_OK) return st;
+  if ((a_gs_dev && !aligned4(a_gs_dev)) || (w_gs_dev && !aligned4(w_gs_dev))) return BATQ_ERR_ALIGNMENT;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA, nullptr,
+                    batq::kFmtNvfp4, s, a_gs_dev);
+  if (st != BATQ_OK) return st;
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, batq::kFmtNvfp4, s,
+                     a_gs_dev, w_gs_dev);
 }
 
 batq_status batq_selftest_wait_timeout(unsigned int limit_us, void* stream) {

@@ -25,6 +25,11 @@
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator quadrant of each warp,
 //              staged through shared memory and written with TMA stores
 //              (prefill) or stored directly, coalesced along i (decode).
+//
+// The same kernel serves the W4A8 variant (E4M3 bytes, kind::mxf8f6f4, K = 32
+// per MMA) and NVFP4 operands (packed E2M1 with an E4M3 scale per 16 K,
+// kind::mxf4nvf4 block16, four scales per MMA; the epilogue multiplies by
+// fp32(1 / (gs_a gs_w)), the per-tensor encode scales of both operands).
 #include <cstdint>
 
 #include "host_util.h"
@@ -41,12 +46,16 @@ constexpr int kThreads = 224;     // 7 warps: producer, MMA, 4 epilogue, scale c
 constexpr int kSfWarp = 6;
 constexpr int kSfAtom = 512;      // bytes of one 128-row x 4-scale tile
 
-// kFp8: both operands are E4M3 bytes (the W4A8 variant), else packed E2M1.
-template <int BN, bool kSwap, int kStages, bool kFp8>
+// kFmt: operand format (Fmt).
+template <int BN, bool kSwap, int kStages, int kFmt>
 struct GemmCfg {
+  static constexpr bool kFp8 = (kFmt == kFmtMxfp8);
+  static constexpr bool kNv = (kFmt == kFmtNvfp4);
   static constexpr int kBK = kFp8 ? kBKBytes : 2 * kBKBytes;     // K elements per stage
   static constexpr int kKPerMma = kFp8 ? 32 : 64;                // K elements per MMA
-  static constexpr int kAtoms = kBK / 128;                       // 4-scale atoms per row and stage
+  static constexpr int kSfBlock = kNv ? 16 : 32;                 // K elements per scale
+  static constexpr int kSfPerMma = kKPerMma / kSfBlock;          // scales per row and MMA
+  static constexpr int kAtoms = kBK / (4 * kSfBlock);            // 4-scale atoms per row and stage
   static constexpr int kPBytes = kBM * kBKBytes;
   static constexpr int kQBytes = BN * kBKBytes;
   static constexpr int kQRowAtoms = BN > 128 ? 2 : 1;           // 128-row scale atoms covering Q rows
@@ -80,13 +89,16 @@ struct GemmArgs {
   const uint8_t* w_codes;   // the weight operand (P when swapped, else Q), for the L2 prefetch
   int w_rows;               // its valid rows
   int early_w;              // the preceding grid does not write the weights: prefetch them before waiting
+  const float* gs_a;        // NVFP4 per-tensor encode scales (device, nullable: 1)
+  const float* gs_w;
 };
 
-template <int BN, bool kSwap, int kStages, bool kOutBF16, bool kFp8>
+template <int BN, bool kSwap, int kStages, bool kOutBF16, int kFmt>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_mxfp4(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ GemmArgs g) {
-  using C = GemmCfg<BN, kSwap, kStages, kFp8>;
+  using C = GemmCfg<BN, kSwap, kStages, kFmt>;
+  constexpr bool kFp8 = C::kFp8;
   constexpr int kBK = C::kBK, kKPerMma = C::kKPerMma;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -204,14 +216,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dp = sdesc_kmajor_sw128(sp);
         const uint64_t dq = sdesc_kmajor_sw128(sq);
         for (int j = 0; j < nmma; ++j) {
-          // MMA j covers 32-element scale blocks kb.. of the stage: atom kb / 4,
-          // byte kb % 4 of each 4-scale TMEM column.
-          const int kb = j * (kKPerMma / 32);
+          // MMA j covers scale blocks kb.. of the stage: atom kb / 4, byte
+          // kb % 4 of each 4-scale TMEM column (NVFP4: four scales, byte 0).
+          const int kb = j * C::kSfPerMma;
           const int a = kb >> 2;
           const int sf_id = kb & 3;
           // Advance K by 32 bytes inside the 128-byte swizzle atom.
           if constexpr (kFp8)
             tc_mma_mxf8(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc_mxf8(kBM, BN, sf_id, sf_id),
+                        t_sfp + s * C::kSfPCols + a * 4, t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms,
+                        (ks > 0 || j > 0) ? 1u : 0u);
+          else if constexpr (C::kNv)
+            tc_mma_nvf4(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc_nvf4(kBM, BN),
                         t_sfp + s * C::kSfPCols + a * 4, t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms,
                         (ks > 0 || j > 0) ? 1u : 0u);
           else
@@ -243,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ssfq = ssfp + C::kSfPBytes;
         const int kleft = g.N - ks * kBK;
         const int nmma = kleft >= kBK ? kMmasPerStage : kleft / kKPerMma;
-        const int atoms = ((nmma - 1) * (kKPerMma / 32)) / 4 + 1;  // atoms the stage's MMAs read
+        const int atoms = ((nmma - 1) * C::kSfPerMma) / 4 + 1;  // atoms the stage's MMAs read
         for (int a = 0; a < atoms; ++a) {
           tc_cp_32x128b_warpx4(t_sfp + s * C::kSfPCols + a * 4, sdesc_sf_atom(ssfp + a * kSfAtom));
 #pragma unroll
@@ -262,6 +278,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------ epilogue ------------------------------
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31 are this warp's
+    float alpha = 1.0f;
+    if constexpr (C::kNv) {
+      // The scales may come from the preceding grid (the weight preparation).
+      griddep_wait();
+      alpha = __frcp_rn(__fmul_rn(g.gs_a != nullptr ? *g.gs_a : 1.0f, g.gs_w != nullptr ? *g.gs_w : 1.0f));
+    }
+    auto scaled = [&](uint32_t bits) {
+      if constexpr (C::kNv) return __fmul_rn(__uint_as_float(bits), alpha);
+      return __uint_as_float(bits);
+    };
     if (!mbar_wait(acc_full, 0)) set_error(g.err, kErrMmaTimeout);
     tc_fence_after_sync();
     const uint32_t t_row = t_acc + ((uint32_t)(32 * quad) << 16);
@@ -278,10 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int tok = q0 + c0 + j;
           if (tok < g.rows_q && i < g.rows_p) {
             if constexpr (kOutBF16) {
-              const uint32_t pk = pack_bf16x2(__uint_as_float(r[j]), 0.0f);
+              const uint32_t pk = pack_bf16x2(scaled(r[j]), 0.0f);
               reinterpret_cast<uint16_t*>(g.out)[(size_t)tok * g.ldo + i] = (uint16_t)(pk & 0xFFFFu);
             } else {
-              reinterpret_cast<float*>(g.out)[(size_t)tok * g.ldo + i] = __uint_as_float(r[j]);
+              reinterpret_cast<float*>(g.out)[(size_t)tok * g.ldo + i] = scaled(r[j]);
             }
           }
         }
@@ -305,10 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 8; ++c) {
             const uint32_t* r = c < 4 ? r0 : r1;
             const int o = (c & 3) * 8;
-            uint4 v = make_uint4(pack_bf16x2(__uint_as_float(r[o + 0]), __uint_as_float(r[o + 1])),
-                                 pack_bf16x2(__uint_as_float(r[o + 2]), __uint_as_float(r[o + 3])),
-                                 pack_bf16x2(__uint_as_float(r[o + 4]), __uint_as_float(r[o + 5])),
-                                 pack_bf16x2(__uint_as_float(r[o + 6]), __uint_as_float(r[o + 7])));
+            uint4 v = make_uint4(pack_bf16x2(scaled(r[o + 0]), scaled(r[o + 1])),
+                                 pack_bf16x2(scaled(r[o + 2]), scaled(r[o + 3])),
+                                 pack_bf16x2(scaled(r[o + 4]), scaled(r[o + 5])),
+                                 pack_bf16x2(scaled(r[o + 6]), scaled(r[o + 7])));
             *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) = v;
           }
         } else {
@@ -318,7 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
-                make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+                make_uint4(__float_as_uint(scaled(r[4 * c])), __float_as_uint(scaled(r[4 * c + 1])),
+                           __float_as_uint(scaled(r[4 * c + 2])), __float_as_uint(scaled(r[4 * c + 3])));
           }
         }
       }
@@ -343,9 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BN, bool kSwap, int kStages, bool kOutBF16, bool kFp8>
+template <int BN, bool kSwap, int kStages, bool kOutBF16, int kFmt>
 cudaError_t launch_cfg(const GemmLaunch& L) {
-  using C = GemmCfg<BN, kSwap, kStages, kFp8>;
+  using C = GemmCfg<BN, kSwap, kStages, kFmt>;
+  constexpr bool kFp8 = C::kFp8;
   const int rows_p = kSwap ? L.M : L.S;
   const int rows_q = kSwap ? L.S : L.M;
   const uint8_t* codes_p = kSwap ? L.w_codes : L.a_codes;
@@ -379,16 +407,18 @@ cudaError_t launch_cfg(const GemmLaunch& L) {
   g.rows_p_pad = (rows_p + 127) / 128 * 128;
   g.rows_q_pad = (rows_q + 127) / 128 * 128;
   g.N = L.N;
-  g.kpad = (L.N / 32 + 3) / 4 * 4;
+  g.kpad = C::kNv ? L.N / 16 : (L.N / 32 + 3) / 4 * 4;  // scale columns (NVFP4: N / 16, a multiple of 4)
   g.ldo = L.ldo;
   g.tiles_q = (rows_q + BN - 1) / BN;
   g.num_kstages = (L.N + C::kBK - 1) / C::kBK;
   g.w_codes = L.w_codes;
   g.w_rows = L.M;
   g.early_w = L.weights_ready ? 1 : 0;
+  g.gs_a = L.gs_a;
+  g.gs_w = L.gs_w;
   const int tiles_p = (rows_p + kBM - 1) / kBM;
 
-  auto kern = k_gemm_mxfp4<BN, kSwap, kStages, kOutBF16, kFp8>;
+  auto kern = k_gemm_mxfp4<BN, kSwap, kStages, kOutBF16, kFmt>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -410,20 +440,24 @@ cudaError_t launch_cfg(const GemmLaunch& L) {
   return cudaLaunchKernelEx(&cfg, kern, tm_p, tm_q, tm_out, g);
 }
 
-template <bool kOutBF16, bool kFp8>
+template <bool kOutBF16, int kFmt>
 cudaError_t launch_dtype(const GemmLaunch& L) {
-  if (L.S <= 16) return launch_cfg<16, true, 4, kOutBF16, kFp8>(L);
-  if (L.S <= 32) return launch_cfg<32, true, 4, kOutBF16, kFp8>(L);
-  if (L.S <= 64) return launch_cfg<64, true, 4, kOutBF16, kFp8>(L);
-  if (L.S <= 128) return launch_cfg<256, false, 4, kOutBF16, kFp8>(L);
+  if (L.S <= 16) return launch_cfg<16, true, 4, kOutBF16, kFmt>(L);
+  if (L.S <= 32) return launch_cfg<32, true, 4, kOutBF16, kFmt>(L);
+  if (L.S <= 64) return launch_cfg<64, true, 4, kOutBF16, kFmt>(L);
+  if (L.S <= 128) return launch_cfg<256, false, 4, kOutBF16, kFmt>(L);
   return launch_gemm_pair(L);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_mxfp4(const GemmLaunch& L) {
-  if (L.fp8) return L.out_bf16 ? launch_dtype<true, true>(L) : launch_dtype<false, true>(L);
-  return L.out_bf16 ? launch_dtype<true, false>(L) : launch_dtype<false, false>(L);
+  switch (L.fmt) {
+    case kFmtMxfp4: return L.out_bf16 ? launch_dtype<true, kFmtMxfp4>(L) : launch_dtype<false, kFmtMxfp4>(L);
+    case kFmtMxfp8: return L.out_bf16 ? launch_dtype<true, kFmtMxfp8>(L) : launch_dtype<false, kFmtMxfp8>(L);
+    case kFmtNvfp4: return L.out_bf16 ? launch_dtype<true, kFmtNvfp4>(L) : launch_dtype<false, kFmtNvfp4>(L);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace batq

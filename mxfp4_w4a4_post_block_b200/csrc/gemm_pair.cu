@@ -19,9 +19,15 @@
 //     registers, release TMEM for the next tile at once, and write the output
 //     through a small per-warp shared-memory box (32 rows x 32 bytes) with TMA
 //     stores while the next tile's MMAs run;
-//   * six 35 KB stages keep ~210 KB of operand loads in flight per SM: under
-//     full load the L2-to-SM latency is ~1.5 us, and this tile needs 64 bytes
-//     per SM per tensor-core cycle.
+//   * three 70 KB stages (two 128-byte swizzle tiles of K each, eight MMAs
+//     per stage) keep ~210 KB of operand loads in flight per SM: under full
+//     load the L2-to-SM latency is ~1.5 us, and this tile needs 64 bytes per
+//     SM per tensor-core cycle.  NVFP4 operands (E4M3 scale per 16 K: twice
+//     the scale bytes and TMEM columns per K) use five 38 KB stages of one
+//     swizzle tile each, which fit the 512 TMEM columns;
+//   * formats: MXFP4 (kind::mxf4, E8M0 per 32 K), MXFP8 x MXFP4-in-E4M3 (the
+//     W4A8 variant, kind::mxf8f6f4) and NVFP4 (kind::mxf4nvf4 block16, with
+//     the per-tensor factor fp32(1 / (gs_a gs_w)) applied in the epilogue).
 // Every barrier wait is bounded; on expiry a bit is set in the device error
 // word and the waiting loop ends (TMEM is released and both CTAs still meet
 // at the closing cluster barrier).
@@ -38,28 +44,30 @@ constexpr int kRowsPerCta = 128;       // token rows per CTA (TMEM lanes)
 constexpr int kTileM = 256;            // token rows per pair
 constexpr int kTileN = 256;            // out-features per pair (MMA N)
 constexpr int kHalfN = kTileN / 2;     // weight rows loaded by each CTA
-constexpr int kSwAtoms = 2;            // 128-byte swizzle atoms along K per stage
-constexpr int kBKBytes = 128 * kSwAtoms; // bytes of K per stage and row
-constexpr int kStages = 6 / kSwAtoms;  // ~210 KB of operands in flight per SM (L2 latency ~1.5 us)
 constexpr int kSwTile = 128 * 128;     // one 128-row x 128-byte swizzled operand tile
 constexpr int kSfAtom = 512;           // 128 rows x 4 scales
 constexpr int kEpiWarps = 8;
 constexpr int kSfWarp = 2 + kEpiWarps;          // issues the scale-factor copies
 constexpr int kThreads = (3 + kEpiWarps) * 32;
 
-constexpr int kABytes = kRowsPerCta * kBKBytes;             // 32 KB (kSwAtoms swizzle tiles)
-constexpr int kBBytes = kHalfN * kBKBytes;                  // 32 KB
 constexpr int kBoxBytes = 1024;                             // one epilogue store box: 32 rows x 32 bytes
 constexpr int kStagingBytes = kEpiWarps * kBoxBytes;
 constexpr int kTmemCols = 512;
 
-// Per element format (kFp8: E4M3 bytes, the W4A8 variant; else packed E2M1).
-// A stage always holds 128 bytes of K per row; an MMA consumes 32 of them.
-template <bool kFp8>
+// Per operand format (Fmt).  An MMA consumes 32 bytes of K per row.
+template <int kFmt>
 struct PairCfg {
+  static constexpr bool kFp8 = (kFmt == kFmtMxfp8);
+  static constexpr bool kNv = (kFmt == kFmtNvfp4);
+  static constexpr int kSwAtoms = kNv ? 1 : 2;               // 128-byte swizzle atoms along K per stage
+  static constexpr int kBKBytes = 128 * kSwAtoms;            // bytes of K per stage and row
+  static constexpr int kStages = kNv ? 5 : 3;                // ~190-210 KB of operands in flight per SM
+  static constexpr int kABytes = kRowsPerCta * kBKBytes;     // own activation rows
+  static constexpr int kBBytes = kHalfN * kBKBytes;          // own half of the weight rows
   static constexpr int kBK = kFp8 ? kBKBytes : 2 * kBKBytes;  // K elements per stage
   static constexpr int kKPerMma = kFp8 ? 32 : 64;             // K elements per MMA
-  static constexpr int kAtoms = kBK / 128;                    // 4-scale atoms per row and stage
+  static constexpr int kSfBlock = kNv ? 16 : 32;              // K elements per scale
+  static constexpr int kAtoms = kBK / (4 * kSfBlock);         // 4-scale atoms per row and stage
   static constexpr int kSfaBytes = kAtoms * kSfAtom;          // K atoms of own rows
   static constexpr int kSfbBytes = 2 * kAtoms * kSfAtom;      // 2 row atoms x K atoms
   static constexpr int kStageTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // bytes one CTA's loads deliver
@@ -83,9 +91,11 @@ struct PairArgs {
   int num_kstages;
   int early_weights;        // weights may be read before waiting for the preceding grid
   int sf_box_chunks;        // 256-byte scale chunks per row tile in one stage's box (<= 2 * kAtoms)
+  const float* gs_a;        // NVFP4 per-tensor encode scales (device, nullable: 1)
+  const float* gs_w;
 };
 
-template <bool kOutBF16, bool kFp8>
+template <bool kOutBF16, int kFmt>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfw,
@@ -93,9 +103,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const __grid_constant__ PairArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  using C = PairCfg<kFp8>;
+  using C = PairCfg<kFmt>;
   constexpr int kStageBytes = C::kStageBytes, kSfaBytes = C::kSfaBytes, kSfaCols = C::kSfaCols,
-                kSfbCols = C::kSfbCols, kBK = C::kBK, kKPerMma = C::kKPerMma;
+                kSfbCols = C::kSfbCols, kBK = C::kBK, kKPerMma = C::kKPerMma, kStages = C::kStages,
+                kABytes = C::kABytes, kBBytes = C::kBBytes, kSwAtoms = C::kSwAtoms, kBKBytes = C::kBKBytes,
+                kSfPerMma = C::kKPerMma / C::kSfBlock;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
@@ -236,19 +248,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int kleft = g.N - ks * kBK;
         const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
         for (int j = 0; j < nmma; ++j) {
-          // MMA j covers 32-element scale blocks kb.. of the stage: atom kb / 4,
-          // byte kb % 4 of each 4-scale TMEM column.
-          const int kb = j * (kKPerMma / 32);
+          // MMA j covers scale blocks kb.. of the stage: atom kb / 4, byte
+          // kb % 4 of each 4-scale TMEM column (NVFP4: four scales, byte 0).
+          const int kb = j * kSfPerMma;
           const int a = kb >> 2;
           const int sf_id = kb & 3;
           // Bytes 32j.. of the stage's K: swizzle tile j / 4, then 32 bytes per
           // MMA inside its 128-byte swizzle atom.
           const uint64_t da = sdesc_kmajor_sw128(sa + (j >> 2) * kSwTile) + (uint64_t)((j & 3) * 2);
           const uint64_t db = sdesc_kmajor_sw128(sb + (j >> 2) * kSwTile) + (uint64_t)((j & 3) * 2);
-          if constexpr (kFp8)
+          if constexpr (C::kFp8)
             tc_mma_pair_mxf8(t_acc, da, db, idesc_mxf8(256, kTileN, sf_id, sf_id),
                              t_sfa + st_idx * kSfaCols + a * 4, t_sfb + st_idx * kSfbCols + a * 8,
                              (ks > 0 || j > 0) ? 1u : 0u);
+          else if constexpr (C::kNv)
+            tc_mma_pair_nvf4(t_acc, da, db, idesc_nvf4(256, kTileN), t_sfa + st_idx * kSfaCols + a * 4,
+                             t_sfb + st_idx * kSfbCols + a * 8, (ks > 0 || j > 0) ? 1u : 0u);
           else
             tc_mma_pair_mxf4(t_acc, da, db, idesc_mxf4_m256(kTileN, sf_id, sf_id), t_sfa + st_idx * kSfaCols + a * 4,
                              t_sfb + st_idx * kSfbCols + a * 8, (ks > 0 || j > 0) ? 1u : 0u);
@@ -278,7 +293,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
         const uint32_t ssfa = smem_u32(smem + st_idx * kStageBytes) + kABytes + kBBytes;
         const uint32_t ssfb = ssfa + kSfaBytes;
-        const int atoms = ((nmma - 1) * (kKPerMma / 32)) / 4 + 1;  // atoms the stage's MMAs read
+        const int atoms = ((nmma - 1) * kSfPerMma) / 4 + 1;  // atoms the stage's MMAs read
         for (int a = 0; a < atoms; ++a) {
           tc_cp_pair_32x128b_warpx4(t_sfa + st_idx * kSfaCols + a * 4, sdesc_sf_atom(ssfa + a * kSfAtom));
           // weight-scale box is {2 row tiles} x {sf_box_chunks}: row tile r, atom a at
@@ -299,6 +314,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     uint32_t tile_iter = 0;
     bool store_pending = false;
+    float alpha = 1.0f;
+    if constexpr (C::kNv) {
+      // The scales may come from the preceding grid (the weight preparation).
+      griddep_wait();
+      alpha = __frcp_rn(__fmul_rn(g.gs_a != nullptr ? *g.gs_a : 1.0f, g.gs_w != nullptr ? *g.gs_w : 1.0f));
+    }
+    // accumulator bits -> output value (NVFP4: times the per-tensor factor)
+    auto scaled = [&](uint32_t bits) {
+      if constexpr (C::kNv) return __fmul_rn(__uint_as_float(bits), alpha);
+      return __uint_as_float(bits);
+    };
     for (int t = cluster_id; t < num_tiles; t += num_clusters, ++tile_iter) {
       const int row0 = (t / g.tiles_n) * kTileM + (int)rank * kRowsPerCta + 32 * quad;
       const int n0 = (t % g.tiles_n) * kTileN + col0;
@@ -338,13 +364,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint4 q;
             if constexpr (kOutBF16) {
               const uint32_t* r = v[2 * bx + (c >> 2)] + (c & 3) * 8;
-              q = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                             pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                             pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                             pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+              q = make_uint4(pack_bf16x2(scaled(r[0]), scaled(r[1])), pack_bf16x2(scaled(r[2]), scaled(r[3])),
+                             pack_bf16x2(scaled(r[4]), scaled(r[5])), pack_bf16x2(scaled(r[6]), scaled(r[7])));
             } else {
               const uint32_t* r = v[bx] + 4 * c;
-              q = make_uint4(r[0], r[1], r[2], r[3]);
+              q = make_uint4(__float_as_uint(scaled(r[0])), __float_as_uint(scaled(r[1])),
+                             __float_as_uint(scaled(r[2])), __float_as_uint(scaled(r[3])));
             }
             *reinterpret_cast<uint4*>(wrow + ((c ^ (lane & 7)) << 4)) = q;
           }
@@ -379,17 +404,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 2; ++c) {
             const int o = c * 8;
             *reinterpret_cast<uint4*>(rowp + ((c ^ sw) << 4)) =
-                make_uint4(pack_bf16x2(__uint_as_float(r[o + 0]), __uint_as_float(r[o + 1])),
-                           pack_bf16x2(__uint_as_float(r[o + 2]), __uint_as_float(r[o + 3])),
-                           pack_bf16x2(__uint_as_float(r[o + 4]), __uint_as_float(r[o + 5])),
-                           pack_bf16x2(__uint_as_float(r[o + 6]), __uint_as_float(r[o + 7])));
+                make_uint4(pack_bf16x2(scaled(r[o + 0]), scaled(r[o + 1])),
+                           pack_bf16x2(scaled(r[o + 2]), scaled(r[o + 3])),
+                           pack_bf16x2(scaled(r[o + 4]), scaled(r[o + 5])),
+                           pack_bf16x2(scaled(r[o + 6]), scaled(r[o + 7])));
           }
         } else {
           const uint32_t* r = v[bx >> 2] + (bx & 3) * 8;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             *reinterpret_cast<uint4*>(rowp + ((c ^ sw) << 4)) =
-                make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+                make_uint4(__float_as_uint(scaled(r[4 * c])), __float_as_uint(scaled(r[4 * c + 1])),
+                           __float_as_uint(scaled(r[4 * c + 2])), __float_as_uint(scaled(r[4 * c + 3])));
           }
         }
         fence_proxy_async_smem();
@@ -415,12 +441,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool kOutBF16, bool kFp8>
+template <bool kOutBF16, int kFmt>
 cudaError_t launch_pair_impl(const GemmLaunch& L) {
-  using C = PairCfg<kFp8>;
-  const uint64_t row_bytes = (uint64_t)(kFp8 ? L.N : L.N / 2);
+  using C = PairCfg<kFmt>;
+  const uint64_t row_bytes = (uint64_t)(C::kFp8 ? L.N : L.N / 2);
   // Code tiles: boxes of 128 rows x 128 bytes (one swizzle atom); a stage takes kSwAtoms of them.
-  const int kpad = (L.N / 32 + 3) / 4 * 4;
+  // Scale columns per row: k = N / 32 rounded up to 4 (MX), N / 16 (NVFP4, a multiple of 4).
+  const int kpad = C::kNv ? L.N / 16 : (L.N / 32 + 3) / 4 * 4;
   const uint64_t sf_row_tile_bytes = (uint64_t)(kpad / 4) * kSfAtom;
   const uint64_t a_tiles = (uint64_t)(L.S + 127) / 128;
   const uint64_t w_tiles = (uint64_t)(L.M + 127) / 128;
@@ -462,8 +489,10 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   g.num_kstages = (L.N + C::kBK - 1) / C::kBK;
   g.early_weights = L.weights_ready ? 1 : 0;
   g.sf_box_chunks = box_chunks;
+  g.gs_a = L.gs_a;
+  g.gs_w = L.gs_w;
 
-  auto kern = k_gemm_pair<kOutBF16, kFp8>;
+  auto kern = k_gemm_pair<kOutBF16, kFmt>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -493,8 +522,12 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
 }  // namespace
 
 cudaError_t launch_gemm_pair(const GemmLaunch& L) {
-  if (L.fp8) return L.out_bf16 ? launch_pair_impl<true, true>(L) : launch_pair_impl<false, true>(L);
-  return L.out_bf16 ? launch_pair_impl<true, false>(L) : launch_pair_impl<false, false>(L);
+  switch (L.fmt) {
+    case kFmtMxfp4: return L.out_bf16 ? launch_pair_impl<true, kFmtMxfp4>(L) : launch_pair_impl<false, kFmtMxfp4>(L);
+    case kFmtMxfp8: return L.out_bf16 ? launch_pair_impl<true, kFmtMxfp8>(L) : launch_pair_impl<false, kFmtMxfp8>(L);
+    case kFmtNvfp4: return L.out_bf16 ? launch_pair_impl<true, kFmtNvfp4>(L) : launch_pair_impl<false, kFmtNvfp4>(L);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace batq

@@ -6,6 +6,13 @@
 
 namespace batq {
 
+// Element / scale format of a quantised operand.
+enum Fmt : int {
+  kFmtMxfp4 = 0,  // packed E2M1, one E8M0 scale per 32 elements
+  kFmtMxfp8 = 1,  // E4M3 bytes, one E8M0 scale per 32 elements (the W4A8 variant's activations)
+  kFmtNvfp4 = 2,  // packed E2M1, one E4M3 scale per 16 elements, per-tensor fp32 encode scale
+};
+
 struct QuantLaunch {
   const void* X;
   bool bf16;
@@ -19,7 +26,17 @@ struct QuantLaunch {
   float* y_debug;       // device S x N or nullptr
   unsigned* err;        // device error word
   cudaStream_t stream;
-  bool fp8;             // E4M3 elements (MXFP8, one byte each) instead of packed E2M1
+  int fmt;              // Fmt
+  // NVFP4 only.  The per-tensor encode scale gs comes from gs_amax (device word
+  // holding the fp32 bits of a tensor amax: gs = 448 * 6 / amax) if set, else
+  // from gs (device float), else is 1.  gs_out (device, nullable) receives the
+  // gs used.  With amax_out set the launch only measures: the largest clipped
+  // |y| of every finite block is folded into *amax_out (fp32 bits, atomic max)
+  // and nothing else is written.
+  const float* gs;
+  const unsigned* gs_amax;
+  float* gs_out;
+  unsigned* amax_out;
 };
 
 // Returns cudaErrorInvalidValue when the tensor map cannot be encoded.
@@ -44,9 +61,13 @@ struct GemmLaunch {
   // weights, so they may be read before waiting for it (set by the linear
   // layer, whose preceding grid is its own quantiser).
   bool weights_ready;
-  // Both operands are E4M3 bytes (the W4A8 variant: MXFP8 activations, MXFP4
-  // weights in E4M3 containers) instead of packed E2M1.
-  bool fp8;
+  // kFmtMxfp8: both operands are E4M3 bytes (the W4A8 variant: MXFP8
+  // activations, MXFP4 weights in E4M3 containers); kFmtNvfp4: packed E2M1
+  // with E4M3 scales per 16 K, and the epilogue multiplies by
+  // fp32(1 / fp32(gs_a * gs_w)) read from the device (each nullable: 1).
+  int fmt;
+  const float* gs_a;
+  const float* gs_w;
 };
 
 cudaError_t launch_gemm_mxfp4(const GemmLaunch& L);

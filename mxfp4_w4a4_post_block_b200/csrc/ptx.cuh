@@ -201,6 +201,33 @@ __device__ __forceinline__ uint32_t e4m3x4(float v0, float v1, float v2, float v
   return out;
 }
 
+// Two E4M3 codes of non-negative scales (round to nearest even, saturating at
+// 448): u0 in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_bits(float u0, float u1) {
+  uint32_t out;
+  asm("{\n\t.reg .b16 h;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h, %2, %1;\n\t"
+      "cvt.u32.u16 %0, h;\n\t}"
+      : "=r"(out)
+      : "f"(u0), "f"(u1));
+  return out;
+}
+
+// Exact values of the two E4M3 codes in the low 16 bits of `bits` (low byte
+// -> .x).  Every E4M3 value is an f16 value, so the widening is exact.
+__device__ __forceinline__ float2 e4m3x2_values(uint32_t bits) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 c, l, h;\n\t.reg .b32 hh;\n\t"
+      "cvt.u16.u32 c, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 hh, c;\n\t"
+      "mov.b32 {l, h}, hh;\n\t"
+      "cvt.f32.f16 %0, l;\n\t"
+      "cvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(bits));
+  return make_float2(lo, hi);
+}
+
 // ------------------------------------------------------------ bulk copies
 
 // Prefetch `bytes` of global memory into L2 (16-byte aligned address, size a multiple of 16).
@@ -268,6 +295,19 @@ __device__ __forceinline__ void tc_mma_mxf8(uint32_t tacc, uint64_t adesc, uint6
       : "memory");
 }
 
+// D (TMEM, fp32) (+)= A x B^T for packed E2M1 operands with one unsigned E4M3
+// scale per 16 K (NVFP4; kind::mxf4nvf4, K = 64 per MMA, so the four scales of a
+// row fill one 32-bit TMEM column and the scale id is 0).
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane.
@@ -324,6 +364,13 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(int n, int sf_id_a, int sf_id_
 __host__ __device__ constexpr uint32_t idesc_mxf8(int m, int n, int sf_id_a, int sf_id_b) {
   return ((uint32_t)(sf_id_b & 3) << 4) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(m >> 4) << 24) |
          ((uint32_t)(sf_id_a & 3) << 29);
+}
+
+// Instruction descriptor of kind::mxf4nvf4 with E2M1 A and B (format code 1),
+// unsigned E4M3 scales (bit 23 clear), K-major, M = m, N = n, dense K = 64,
+// scale ids 0.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -425,6 +472,17 @@ __device__ __forceinline__ void tc_mma_pair_mxf8(uint32_t tacc, uint64_t adesc, 
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Pair MMA of kind::mxf4nvf4 (E2M1 x E2M1, E4M3 scale per 16 K), otherwise as tc_mma_pair_mxf4.
+__device__ __forceinline__ void tc_mma_pair_nvf4(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
       : "memory");
 }

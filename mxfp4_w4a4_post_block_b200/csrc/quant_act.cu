@@ -26,6 +26,14 @@
 //   * the block extrema are in-thread (the whole block lives in one thread),
 //     the clipped amax is max(|clamp(min)|, |clamp(max)|) (clamp is
 //     monotone), and the scale comes from the exponent bits of amax.
+//
+// Output formats: MXFP4 (E2M1 + E8M0 per 32), MXFP8 (E4M3 + E8M0 per 32, the
+// W4A8 variant) and NVFP4 (E2M1 + E4M3 per 16 elements with a per-tensor fp32
+// encode scale gs; ARCQuant page, "背景" section, for the 16-element E4M3
+// grouping).  For NVFP4 the transform and the clip still work on the 32-block;
+// each half then gets scale E4M3(fp32(amax_half * gs) / 6) and the elements
+// are multiplied by fp32(gs / scale) before the E2M1 rounding, every step an
+// IEEE fp32 operation.
 #include <cfloat>
 #include <cstdint>
 
@@ -38,7 +46,9 @@ namespace {
 
 constexpr int kRows = 32;         // tokens per tile (one per lane)
 constexpr int kCols = 8;          // 32-blocks per tile (one per warp of a consumer group)
-constexpr uint8_t kPadScale = 0x7F;
+constexpr uint8_t kPadScale = 0x7F;        // E8M0 1.0 in padding rows and columns
+constexpr uint32_t kPadScaleNv = 0x3838u;  // two E4M3 1.0 scales in NVFP4 padding rows
+constexpr float kNvGlobalNumerator = 2688.0f;  // 448 (largest E4M3) x 6 (largest E2M1)
 
 template <bool kBF16>
 struct Tile {
@@ -52,7 +62,7 @@ struct Tile {
   static constexpr int kBOffset = kXBytes;                  // kCols x 16 fp32 B_i
   static constexpr int kROffset = kXBytes + kCols * 64;     // kCols x 2 fp32 clip ratios
   static constexpr int kStageBytes = (kROffset + kCols * 8 + 1023) / 1024 * 1024;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 2 * kStages * 8 + 1024;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 2 * kStages * 8 + 16 + 1024;
 };
 
 struct QuantArgs {
@@ -68,6 +78,11 @@ struct QuantArgs {
   int mma_layout;
   int tiles_r, tiles_c;
   unsigned long long tiles_c_magic;  // ceil(2^40 / tiles_c): t / tiles_c = (t * magic) >> 40 for t < 2^24
+  // NVFP4 per-tensor scale sources and outputs (see QuantLaunch)
+  const float* gs;
+  const unsigned* gs_amax;
+  float* gs_out;
+  unsigned* amax_out;
 };
 
 __device__ __forceinline__ int tile_row(int t, const QuantArgs& p) {
@@ -121,15 +136,18 @@ __device__ __forceinline__ void load_block(uint32_t box, int lane, float x[32]) 
   }
 }
 
-// kFp8: E4M3 elements (MXFP8, the W4A8 variant's activations) instead of E2M1.
-template <bool kBF16, bool kFp8>
+// kFmt: output format (Fmt).
+template <bool kBF16, int kFmt>
 __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
     k_quant_act(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
   using T = Tile<kBF16>;
+  constexpr bool kFp8 = (kFmt == kFmtMxfp8);
+  constexpr bool kNv = (kFmt == kFmtNvfp4);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::kStages * T::kStageBytes);
   uint64_t* empty = full + T::kStages;
+  float* gs_smem = reinterpret_cast<float*>(empty + T::kStages);  // NVFP4 per-tensor encode scale
   // Fetch the TMA descriptors while the barriers and TMEM are set up.
   if (threadIdx.x == 0) {
     tma_prefetch_map(&tmx);
@@ -165,6 +183,22 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
       // Every grid before this one is complete from here on, so the dependent
       // GEMM may start (and fetch weights) while the codes are produced.
       griddep_launch_dependents();
+      if constexpr (kNv) {
+        // Per-tensor encode scale, published to the consumers through the
+        // release of this thread's first arrivals on the stage barriers.
+        float gs = 1.0f;
+        if (p.gs_amax != nullptr) {
+          const float a = __uint_as_float(*p.gs_amax);
+          if (a > 0.0f) {
+            gs = __fdiv_rn(kNvGlobalNumerator, a);
+            if (!(gs <= FLT_MAX)) gs = 1.0f;
+          }
+        } else if (p.gs != nullptr) {
+          gs = *p.gs;
+        }
+        *gs_smem = gs;
+        if (p.gs_out != nullptr && blockIdx.x == 0) *p.gs_out = gs;
+      }
       for (int i = 0; i < nloc; ++i) {
         const int s = i % T::kStages;
         if (!mbar_wait(&empty[s], ((i / T::kStages) & 1) ^ 1)) {
@@ -264,85 +298,131 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
         y[2 * i + 1] = y2[i].y;
       }
 
-      // Block extrema (NaN-propagating), clip bounds, clipped amax.
-      float mn = fmin3_nan(y[0], y[1], y[2]), mx = fmax3_nan(y[0], y[1], y[2]);
+      // Extrema (NaN-propagating) of each 16-element half, and of the block.
+      float mn0 = fmin3_nan(y[0], y[1], y[2]), mx0 = fmax3_nan(y[0], y[1], y[2]);
+      float mn1 = fmin3_nan(y[16], y[17], y[18]), mx1 = fmax3_nan(y[16], y[17], y[18]);
 #pragma unroll
-      for (int j = 3; j < 31; j += 2) {
-        mn = fmin3_nan(mn, y[j], y[j + 1]);
-        mx = fmax3_nan(mx, y[j], y[j + 1]);
+      for (int j = 3; j < 15; j += 2) {
+        mn0 = fmin3_nan(mn0, y[j], y[j + 1]);
+        mx0 = fmax3_nan(mx0, y[j], y[j + 1]);
+        mn1 = fmin3_nan(mn1, y[16 + j], y[17 + j]);
+        mx1 = fmax3_nan(mx1, y[16 + j], y[17 + j]);
       }
-      mn = fmin_nan(mn, y[31]);
-      mx = fmax_nan(mx, y[31]);
+      mn0 = fmin_nan(mn0, y[15]);
+      mx0 = fmax_nan(mx0, y[15]);
+      mn1 = fmin_nan(mn1, y[31]);
+      mx1 = fmax_nan(mx1, y[31]);
+      const float mn = fmin_nan(mn0, mn1), mx = fmax_nan(mx0, mx1);
       const bool finite = (fabsf(mn) <= FLT_MAX) && (fabsf(mx) <= FLT_MAX);
+      // Clip bounds from the whole block; clipped amax = max(|clamp(min)|, |clamp(max)|).
       const float lo = r_min * mn;
       const float hi = r_max * mx;
-      const float cmn = fminf(fmaxf(mn, lo), hi);
-      const float cmx = fminf(fmaxf(mx, lo), hi);
-      const float amax = fmaxf(fabsf(cmn), fabsf(cmx));
+      auto clampf = [&](float v) { return fminf(fmaxf(v, lo), hi); };
 
-      // Shared scale: floor(log2 amax) = biased exponent - 127, so the scale
-      // byte e + 127 = biased exponent - emax (emax = 2 for E2M1, 8 for E4M3;
-      // clamped at 0, which also covers amax == 0 and subnormal amax).  2^-e
-      // is built from exponent bits.
-      constexpr uint32_t kEmax = kFp8 ? 8u : 2u;
-      const uint32_t ebits = __float_as_uint(amax) >> 23;
-      uint32_t sbyte = ebits > kEmax ? ebits - kEmax : 0u;
-      const float inv_scale = __uint_as_float((254u - sbyte) << 23);
-
-      // Clip, then divide by the shared scale (an exact power-of-two multiply,
-      // two elements per packed multiply), then round to E2M1 or E4M3.
-      const float2 inv2 = make_float2(inv_scale, inv_scale);
-      constexpr int kWords = kFp8 ? 8 : 4;  // 32 codes of 4 or 8 bits
-      uint32_t words[kWords];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        float2 q[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 c2 = make_float2(fminf(fmaxf(y[8 * w + 2 * j], lo), hi),
-                                        fminf(fmaxf(y[8 * w + 2 * j + 1], lo), hi));
-          q[j] = __fmul2_rn(c2, inv2);
-        }
-        if constexpr (kFp8) {
-          words[2 * w] = e4m3x4(q[0].x, q[0].y, q[1].x, q[1].y);
-          words[2 * w + 1] = e4m3x4(q[2].x, q[2].y, q[3].x, q[3].y);
+      if (kNv && p.amax_out != nullptr) {
+        // Measuring pass: fold this warp's largest clipped |y| into the tensor amax.
+        const float a = finite ? fmaxf(fmaxf(fabsf(clampf(mn0)), fabsf(clampf(mx0))),
+                                       fmaxf(fabsf(clampf(mn1)), fabsf(clampf(mx1))))
+                               : 0.0f;
+        const unsigned v = __reduce_max_sync(0xffffffffu, row < p.S ? __float_as_uint(a) : 0u);
+        if (lane == 0 && v != 0u) atomicMax(p.amax_out, v);
+      } else {
+        uint32_t sbits;  // scale byte (MX) or two scale bytes (NVFP4, half 0 in the low byte)
+        float2 mult;     // multiplier of the elements of each half
+        if constexpr (kNv) {
+          // Group scale E4M3(fp32(amax * gs) / 6) per half; multiplier fp32(gs / scale).
+          const float gs = *gs_smem;
+          const float a0 = fmaxf(fabsf(clampf(mn0)), fabsf(clampf(mx0)));
+          const float a1 = fmaxf(fabsf(clampf(mn1)), fabsf(clampf(mx1)));
+          sbits = e4m3x2_bits(__fdiv_rn(__fmul_rn(a0, gs), 6.0f), __fdiv_rn(__fmul_rn(a1, gs), 6.0f));
+          const float2 sv = e4m3x2_values(sbits);
+          mult.x = sv.x == 0.0f ? 0.0f : __fdiv_rn(gs, sv.x);
+          mult.y = sv.y == 0.0f ? 0.0f : __fdiv_rn(gs, sv.y);
         } else {
-          words[w] = e2m1x8(q[0].x, q[0].y, q[1].x, q[1].y, q[2].x, q[2].y, q[3].x, q[3].y);
+          // Shared scale: floor(log2 amax) = biased exponent - 127, so the scale
+          // byte e + 127 = biased exponent - emax (emax = 2 for E2M1, 8 for E4M3;
+          // clamped at 0, which also covers amax == 0 and subnormal amax).  2^-e
+          // is built from exponent bits.
+          const float amax = fmaxf(fabsf(clampf(mn)), fabsf(clampf(mx)));
+          constexpr uint32_t kEmax = kFp8 ? 8u : 2u;
+          const uint32_t ebits = __float_as_uint(amax) >> 23;
+          sbits = ebits > kEmax ? ebits - kEmax : 0u;
+          const float inv_scale = __uint_as_float((254u - sbits) << 23);
+          mult = make_float2(inv_scale, inv_scale);
         }
-      }
-      if (!finite) {
-        sbyte = 0xFFu;
-#pragma unroll
-        for (int w = 0; w < kWords; ++w) words[w] = 0u;
-      }
 
-      if (row < p.S) {
-        constexpr int kBlockCodeBytes = kWords * 4;
-        uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (size_t)(kFp8 ? p.N : p.N >> 1) +
-                                              (size_t)b * kBlockCodeBytes);
-        dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-        if constexpr (kFp8) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-        if (p.mma_layout)
-          p.scales[mma_scale_offset(row, b, p.kpad)] = (uint8_t)sbyte;
-        else
-          p.scales[(size_t)row * p.k + b] = (uint8_t)sbyte;
-        if (p.y_debug != nullptr) {
-          float4* yd = reinterpret_cast<float4*>(p.y_debug + (size_t)row * p.N + (size_t)b * 32);
+        // Clip, then divide by the scale (an exact power-of-two multiply for MX,
+        // the fp32 multiplier for NVFP4; two elements per packed multiply), then
+        // round to E2M1 or E4M3.
+        constexpr int kWords = kFp8 ? 8 : 4;  // 32 codes of 4 or 8 bits
+        uint32_t words[kWords];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) yd[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+        for (int w = 0; w < 4; ++w) {
+          const float m = w < 2 ? mult.x : mult.y;
+          const float2 inv2 = make_float2(m, m);
+          float2 q[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 c2 = make_float2(clampf(y[8 * w + 2 * j]), clampf(y[8 * w + 2 * j + 1]));
+            q[j] = __fmul2_rn(c2, inv2);
+          }
+          if constexpr (kFp8) {
+            words[2 * w] = e4m3x4(q[0].x, q[0].y, q[1].x, q[1].y);
+            words[2 * w + 1] = e4m3x4(q[2].x, q[2].y, q[3].x, q[3].y);
+          } else {
+            words[w] = e2m1x8(q[0].x, q[0].y, q[1].x, q[1].y, q[2].x, q[2].y, q[3].x, q[3].y);
+          }
         }
-      } else if (p.mma_layout && row < p.rows_out) {
+        if (!finite) {
+          sbits = kNv ? 0x7F7Fu : 0xFFu;
+#pragma unroll
+          for (int w = 0; w < kWords; ++w) words[w] = 0u;
+        }
+
+        if (row < p.S) {
+          constexpr int kBlockCodeBytes = kWords * 4;
+          uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (size_t)(kFp8 ? p.N : p.N >> 1) +
+                                                (size_t)b * kBlockCodeBytes);
+          dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+          if constexpr (kFp8) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+          if constexpr (kNv) {
+            // scale columns 2b and 2b + 1 are adjacent in both layouts
+            uint8_t* sp = p.mma_layout ? p.scales + mma_scale_offset(row, 2 * b, p.kpad)
+                                       : p.scales + (size_t)row * (size_t)(2 * p.k) + 2 * b;
+            *reinterpret_cast<uint16_t*>(sp) = (uint16_t)sbits;
+          } else if (p.mma_layout) {
+            p.scales[mma_scale_offset(row, b, p.kpad)] = (uint8_t)sbits;
+          } else {
+            p.scales[(size_t)row * p.k + b] = (uint8_t)sbits;
+          }
+          if (p.y_debug != nullptr) {
+            float4* yd = reinterpret_cast<float4*>(p.y_debug + (size_t)row * p.N + (size_t)b * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) yd[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+          }
+        } else if (p.mma_layout && row < p.rows_out) {
+          if constexpr (kNv)
+            *reinterpret_cast<uint16_t*>(p.scales + mma_scale_offset(row, 2 * b, p.kpad)) = (uint16_t)kPadScaleNv;
+          else
+            p.scales[mma_scale_offset(row, b, p.kpad)] = kPadScale;
+        }
+      }
+    } else if (p.mma_layout && row < p.rows_out) {
+      // Padding: rows past S (all formats) and block columns past k (MX only;
+      // the NVFP4 column count 2k is already a multiple of 4).
+      if constexpr (kNv) {
+        if (b < p.k)
+          *reinterpret_cast<uint16_t*>(p.scales + mma_scale_offset(row, 2 * b, p.kpad)) = (uint16_t)kPadScaleNv;
+      } else if (b < p.kpad) {
         p.scales[mma_scale_offset(row, b, p.kpad)] = kPadScale;
       }
-    } else if (p.mma_layout && b < p.kpad && row < p.rows_out) {
-      p.scales[mma_scale_offset(row, b, p.kpad)] = kPadScale;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
 }
 
-template <bool kBF16, bool kFp8>
+template <bool kBF16, int kFmt>
 cudaError_t launch_impl(const QuantLaunch& L) {
   using T = Tile<kBF16>;
   // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
@@ -364,9 +444,14 @@ cudaError_t launch_impl(const QuantLaunch& L) {
   a.S = L.S;
   a.N = L.N;
   a.k = L.N / 32;
-  a.kpad = (a.k + 3) / 4 * 4;
-  a.mma_layout = L.mma_layout ? 1 : 0;
-  a.rows_out = L.mma_layout ? (L.S + 127) / 128 * 128 : L.S;
+  // scale columns of the MMA layout: k rounded up to 4 (MX), 2k (NVFP4, already a multiple of 4)
+  a.kpad = kFmt == kFmtNvfp4 ? 2 * a.k : (a.k + 3) / 4 * 4;
+  a.mma_layout = (L.mma_layout && L.amax_out == nullptr) ? 1 : 0;
+  a.gs = L.gs;
+  a.gs_amax = L.gs_amax;
+  a.gs_out = L.gs_out;
+  a.amax_out = kFmt == kFmtNvfp4 ? L.amax_out : nullptr;
+  a.rows_out = a.mma_layout ? (L.S + 127) / 128 * 128 : L.S;
   a.tiles_r = (a.rows_out + kRows - 1) / kRows;
   a.tiles_c = (a.k + kCols - 1) / kCols;
   a.tiles_c_magic = ((1ull << 40) + (unsigned long long)a.tiles_c - 1) / (unsigned long long)a.tiles_c;
@@ -375,7 +460,7 @@ cudaError_t launch_impl(const QuantLaunch& L) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16, kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          T::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -392,14 +477,18 @@ cudaError_t launch_impl(const QuantLaunch& L) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16, kFp8>, map, a);
+  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16, kFmt>, map, a);
 }
 
 }  // namespace
 
 cudaError_t launch_quant_act(const QuantLaunch& L) {
-  if (L.fp8) return L.bf16 ? launch_impl<true, true>(L) : launch_impl<false, true>(L);
-  return L.bf16 ? launch_impl<true, false>(L) : launch_impl<false, false>(L);
+  switch (L.fmt) {
+    case kFmtMxfp4: return L.bf16 ? launch_impl<true, kFmtMxfp4>(L) : launch_impl<false, kFmtMxfp4>(L);
+    case kFmtMxfp8: return L.bf16 ? launch_impl<true, kFmtMxfp8>(L) : launch_impl<false, kFmtMxfp8>(L);
+    case kFmtNvfp4: return L.bf16 ? launch_impl<true, kFmtNvfp4>(L) : launch_impl<false, kFmtNvfp4>(L);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace batq

@@ -16,6 +16,11 @@ Tolerances:
   carried into scaled units (E4M3 boundaries are 1/16 apart down to the
   subnormals, so an element with cancellation can cross one within the fp32
   error of the transform).
+* NVFP4 (E2M1 codes, E4M3 scale per 16): the same condition-scaled band around
+  each E2M1 midpoint, carried into scaled units by the group's multiplier
+  gs / scale; a whole group may differ in scale when amax * gs / 6 lies within
+  the band of an E4M3 midpoint; for weights, whose gs the CUDA path derives from
+  its own amax, the band also covers the relative difference of the two gs.
 """
 
 from __future__ import annotations
@@ -145,6 +150,67 @@ def assert_quant_parity_e4m3(codes_gpu, scales_gpu_linear, ref, X, A, B, label="
     diff_all = diff | np.repeat(sdiff, 32, axis=1)
     r = {"mismatch": int(diff_all.sum()), "unexplained": int((diff_all & ~ex).sum()),
          "scale_unexplained": int((sdiff & ~ex_blk).sum()), "total": diff.size}
+    assert r["unexplained"] == 0 and r["scale_unexplained"] == 0, f"{label}: {r}"
+    assert r["mismatch"] < 1e-4 * r["total"], f"{label}: too many boundary mismatches {r}"
+    return r
+
+
+# ------------------------------------------------------------ NVFP4 output ----
+
+def condition_scale_weights(W, A, B):
+    """sum_j |w_j| |(P_i^-T)_ji| per fused weight element (fp64), from the oracle's dense inverses."""
+    W = np.abs(np.asarray(W, np.float64))
+    M, N = W.shape
+    out = np.empty_like(W)
+    for i in range(N // 32):
+        pinv_t = O.gauss_jordan_inverse(O.kron_block(A, B[i])).T
+        out[:, 32 * i:32 * (i + 1)] = W[:, 32 * i:32 * (i + 1)] @ np.abs(pinv_t)
+    return out
+
+
+def exempt_mask_nvfp4(ref, cond, gs_rel=0.0):
+    """Elements (rows, N) and groups (rows, N/16) whose NVFP4 code / scale may differ from the oracle's.
+
+    The CUDA path's transformed value differs from the oracle's by at most
+    1e-5 * max(|y|, condition scale) (the Y tolerance), and its per-tensor gs
+    (weights: derived from its own amax) by a relative gs_rel.  An element is
+    exempt when an E2M1 midpoint lies within that error, carried into scaled
+    units, of the oracle's q, or when |y| itself is within it of 0 (the sign of
+    a zero code); a whole group is exempt when fp32(amax gs) / 6 lies within the
+    error of its amax of an E4M3 midpoint (the group scale may flip).
+    """
+    yh = np.abs(ref["Y_hat"].astype(np.float64))
+    rows, N = yh.shape
+    q = np.abs(ref["q"])
+    gs = ref["gs"]
+    sval = O.e4m3_decode(ref["scales"])
+    with np.errstate(divide="ignore", invalid="ignore"):
+        mult = np.where(sval > 0, gs / np.where(sval > 0, sval, 1.0), 0.0)
+    mult = np.repeat(np.nan_to_num(mult), 16, axis=1)
+    err_y = REL * np.maximum(yh, cond)
+    band = err_y * mult + 2.0 * gs_rel * q
+    near = yh <= err_y
+    for m in MIDPOINTS:
+        near |= np.abs(q - m) <= band
+    amax = yh.reshape(rows, N // 16, 16).max(axis=2)
+    cmax = cond.reshape(rows, N // 16, 16).max(axis=2)
+    u = amax * gs / 6.0
+    band_u = REL * np.maximum(amax, cmax) * gs / 6.0 + 2.0 * gs_rel * u + 1e-300
+    idx = np.clip(np.searchsorted(E4M3_MIDPOINTS, u), 1, len(E4M3_MIDPOINTS) - 1)
+    du = np.minimum(np.abs(u - E4M3_MIDPOINTS[idx - 1]), np.abs(u - E4M3_MIDPOINTS[idx]))
+    near_u = du <= band_u
+    return near | np.repeat(near_u, 16, axis=1), near_u
+
+
+def assert_quant_parity_nvfp4(codes_gpu, scales_gpu_linear, ref, cond, gs_rel=0.0, label=""):
+    """Codes and E4M3 group scales bit-exact outside the exemptions; exempt mismatches < 1e-4."""
+    ex, ex_grp = exempt_mask_nvfp4(ref, cond, gs_rel)
+    diff = O.unpack_nibbles(codes_gpu) != O.unpack_nibbles(ref["codes"])
+    sdiff = np.asarray(scales_gpu_linear) != ref["scales"]
+    diff_all = diff | np.repeat(sdiff, 16, axis=1)
+    r = {"mismatch": int(diff_all.sum()), "unexplained": int((diff_all & ~ex).sum()),
+         "scale_mismatch": int(sdiff.sum()), "scale_unexplained": int((sdiff & ~ex_grp).sum()),
+         "total": diff.size}
     assert r["unexplained"] == 0 and r["scale_unexplained"] == 0, f"{label}: {r}"
     assert r["mismatch"] < 1e-4 * r["total"], f"{label}: too many boundary mismatches {r}"
     return r
