@@ -27,6 +27,8 @@ Recipes (numpy ``default_rng(seed)``, drawn in the order listed):
   q_proj.
 * ``layer``     seeds 500+j for the seven linears of one decoder layer at
   S=8192 (q, k, v, o, gate, up, down); X as q_proj.
+* ``with_block_hadamard(w)``: w's X and W with P_i = H_32 / sqrt(32) (Sylvester) for every
+  block and no clip, the block-rotation baseline as an input.
 """
 
 from __future__ import annotations
@@ -180,6 +182,31 @@ def custom(S: int, N: int, M: int, seed: int, x_dtype: str = "bf16", sigma: floa
     rng = np.random.default_rng(seed)
     x = _student_t_outliers(rng, S, N, outlier_frac, outlier_mult)
     return _finish(f"custom_{S}x{N}x{M}", seed, rng, x, x_dtype, N, M, sigma, 2.0, 1.0, with_w)
+
+
+def sylvester_hadamard(n: int) -> np.ndarray:
+    """Sylvester's +-1 Hadamard matrix of order n (a power of two): H_1 = [1], H_2m = [[H, H], [H, -H]]."""
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    if h.shape[0] != n:
+        raise ValueError("order must be a power of two")
+    return h
+
+
+def with_block_hadamard(w: Workload) -> Workload:
+    """The same activations and weights with the block Hadamard transform as every P_i and no clip.
+
+    This is the block-rotation baseline the pages compare against (BRQ; thelatestinai.com BATQuant
+    page, Figure 2 caption, panel (a)) given as an input of the method: Sylvester's construction
+    makes H_32 = H_4 (x) H_8, so A = H_8 / sqrt(8) (fp32) and B_i = H_4 / 2 give
+    P_i = H_32 / sqrt(32) up to the fp32 rounding of A; alpha = 40 makes sigma(alpha) = 1 in fp32.
+    """
+    k = w.N // BLOCK
+    A = (sylvester_hadamard(8) / np.sqrt(8.0)).astype(np.float32)
+    B = np.tile((sylvester_hadamard(4) / 2.0).astype(np.float32), (k, 1, 1))
+    big = np.full(k, 40.0, np.float32)
+    return dataclasses.replace(w, name=w.name + "_blockhadamard", A=A, B=B, alpha_min=big, alpha_max=big.copy())
 
 
 CONFIGS = {

@@ -169,3 +169,18 @@ def test_linear_error_vs_unquantised_matches_oracle():
     rel_gpu = np.linalg.norm(out.cpu().numpy() - exact) / np.linalg.norm(exact)
     rel_ref = np.linalg.norm(ref - exact) / np.linalg.norm(exact)
     assert abs(rel_gpu - rel_ref) < 1e-3 * rel_ref + 1e-6, (rel_gpu, rel_ref)
+
+
+def test_linear_with_block_hadamard_transform():
+    """Block Hadamard P_i (orthogonal, so the fused weights are W P_i) through batq_linear matches
+    the oracle, and its distance from x W^T is the oracle's."""
+    w = WL.with_block_hadamard(WL.custom(96, 512, 256, 77))
+    out, wc, wsc = _linear(w)
+    ref, T, act, wp = O.linear(w.x, w.A, w.B, w.alpha_min, w.alpha_max, w.W)
+    lin = O.scales_from_mma_layout(wsc.cpu().numpy(), w.M, w.k)
+    PT.assert_quant_parity(wc.cpu().numpy(), lin, {"q": wp["q"], "Y_hat": wp["W_fused"], "codes": wp["codes"],
+                                                    "scales": wp["scales"]}, "hadamard weights")
+    exact = w.x.astype(np.float64) @ w.W.astype(np.float64).T
+    rel_gpu = np.linalg.norm(out.cpu().numpy() - exact) / np.linalg.norm(exact)
+    rel_ref = np.linalg.norm(ref - exact) / np.linalg.norm(exact)
+    assert abs(rel_gpu - rel_ref) < 2e-3 * rel_ref + 1e-6, (rel_gpu, rel_ref)

@@ -186,3 +186,13 @@ def test_subnormal_blocks_and_smallest_scale():
     assert (ref["scales"] == 0).all()
     np.testing.assert_array_equal(scales, ref["scales"])
     np.testing.assert_array_equal(codes, ref["codes"])
+
+
+@pytest.mark.parametrize("maker", [WL.tiny, lambda: WL.custom(200, 320, 16, 76),
+                                   lambda: WL.q_proj(S=512, with_w=False)])
+def test_block_hadamard_as_transform(maker):
+    """The block-rotation baseline (every P_i = H32 / sqrt(32), no clip) given as the method's
+    input runs through the same kernel and matches the oracle."""
+    w = WL.with_block_hadamard(maker())
+    codes, scales, y, _ = GU.gpu_quant(w)
+    _check_all(w, codes, scales, y, label="block hadamard")

@@ -771,3 +771,35 @@ def test_nvfp4_error_below_mxfp4_on_gaussian_blocks():
     e_mx = np.mean((O.dequantize(c4, s4) - V) ** 2)
     e_nv = np.mean((O.dequantize_nvfp4(cn, sn) - V) ** 2)
     assert e_nv < 0.8 * e_mx, (e_nv, e_mx)
+
+
+# ------------------------------------------------ block Hadamard as P_i ----
+
+def test_block_hadamard_factors_give_h32_over_sqrt32():
+    """A = H8/sqrt(8), B_i = H4/2 (Sylvester) give P_i = H32/sqrt(32): checked against scipy's
+    independent Hadamard construction; P_i is orthogonal, so the fused weights use P_i itself."""
+    from scipy.linalg import hadamard
+    w = WL.with_block_hadamard(WL.tiny())
+    P = O.dense_blocks(w.A, w.B)
+    ref = hadamard(32) / np.sqrt(32.0)
+    assert np.abs(P - ref[None]).max() < 1e-7
+    np.testing.assert_allclose(P[0] @ P[0].T, np.eye(32), atol=1e-6)
+    np.testing.assert_allclose(O.gauss_jordan_inverse(P[0]), P[0].T, atol=1e-6)
+    assert (O.clip_ratios(w.alpha_min) == 1.0).all()
+
+
+def test_block_hadamard_of_a_unit_vector_is_a_sign_row():
+    """x = e_j gives y = row j of H32 / sqrt(32): every |y| = 2^-2.5, scale exponent -5, every
+    scaled value +-5.66 -> magnitude 6, with the signs of row j of scipy's H32."""
+    from scipy.linalg import hadamard
+    w = WL.with_block_hadamard(WL.tiny(with_w=False))
+    X = np.zeros((32, 256), np.float32)
+    for j in range(32):
+        X[j, 32 + j] = 1.0                      # block column 1
+    act = O.quant_act(X, w.A, w.B, w.alpha_min, w.alpha_max)
+    codes = O.unpack_nibbles(act["codes"])
+    assert (act["scales"][:, 1] == 127 - 5).all()
+    H = hadamard(32)
+    for j in range(32):
+        assert ((codes[j, 32:64] & 7) == 7).all()
+        np.testing.assert_array_equal(codes[j, 32:64] >> 3, (H[j] < 0).astype(np.uint8))
