@@ -308,6 +308,28 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t tacc, uint64_t adesc, uint6
       : "memory");
 }
 
+// True in exactly one active lane of the warp (the lowest); all lanes must call it.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// D (TMEM, fp32) (+)= A (smem, bf16) x B (smem, bf16)^T, kind::f16, K = 16.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tacc),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane.
@@ -343,6 +365,18 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor: K-major operand tile with 64-byte rows
+// written with the 64-byte swizzle (16-byte chunk c of row r at c ^ ((r >> 1) & 3);
+// 8-row groups 512 bytes apart).  The tile must start on a 512-byte boundary.
+__device__ __forceinline__ uint64_t sdesc_kmajor_sw64(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;             // leading-dimension offset (unused with this swizzle)
+  d |= (uint64_t)(512u >> 4) << 32;    // stride between 8-row groups
+  d |= (uint64_t)1u << 46;             // descriptor version (sm_100)
+  d |= (uint64_t)4u << 61;             // 64-byte swizzle
+  return d;
+}
+
 // Descriptor of a 32-row x 16-byte scale-factor atom (no swizzle, rows 16 bytes apart).
 __device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
   uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
@@ -364,6 +398,12 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(int n, int sf_id_a, int sf_id_
 __host__ __device__ constexpr uint32_t idesc_mxf8(int m, int n, int sf_id_a, int sf_id_b) {
   return ((uint32_t)(sf_id_b & 3) << 4) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(m >> 4) << 24) |
          ((uint32_t)(sf_id_a & 3) << 29);
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B (format code 1 in bits
+// 7-9 and 10-12), fp32 D (1 in bits 4-5), K-major, M = m, N = n.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
 // Instruction descriptor of kind::mxf4nvf4 with E2M1 A and B (format code 1),

@@ -40,15 +40,13 @@
 #include "host_util.h"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "quant_common.cuh"
 
 namespace batq {
 namespace {
 
 constexpr int kRows = 32;         // tokens per tile (one per lane)
 constexpr int kCols = 8;          // 32-blocks per tile (one per warp of a consumer group)
-constexpr uint8_t kPadScale = 0x7F;        // E8M0 1.0 in padding rows and columns
-constexpr uint32_t kPadScaleNv = 0x3838u;  // two E4M3 1.0 scales in NVFP4 padding rows
-constexpr float kNvGlobalNumerator = 2688.0f;  // 448 (largest E4M3) x 6 (largest E2M1)
 
 template <bool kBF16>
 struct Tile {
@@ -64,45 +62,6 @@ struct Tile {
   static constexpr int kStageBytes = (kROffset + kCols * 8 + 1023) / 1024 * 1024;
   static constexpr int kSmemBytes = kStages * kStageBytes + 2 * kStages * 8 + 16 + 1024;
 };
-
-struct QuantArgs {
-  float A[64];
-  const float* B;
-  const float* ratios;
-  uint8_t* codes;
-  uint8_t* scales;
-  float* y_debug;
-  unsigned* err;
-  int S, N, k, kpad;
-  int rows_out;  // rows whose scales are written (S, or S rounded up to 128 in MMA layout)
-  int mma_layout;
-  int tiles_r, tiles_c;
-  unsigned long long tiles_c_magic;  // ceil(2^40 / tiles_c): t / tiles_c = (t * magic) >> 40 for t < 2^24
-  // NVFP4 per-tensor scale sources and outputs (see QuantLaunch)
-  const float* gs;
-  const unsigned* gs_amax;
-  float* gs_out;
-  unsigned* amax_out;
-};
-
-__device__ __forceinline__ int tile_row(int t, const QuantArgs& p) {
-  return (int)(((unsigned long long)(unsigned)t * p.tiles_c_magic) >> 40);
-}
-
-__device__ __forceinline__ uint32_t mma_scale_offset(int row, int kb, int kpad) {
-  return (uint32_t)(((row >> 7) * (kpad >> 2) + (kb >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (kb & 3));
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ float2 lds64f(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
-}
 
 // One token's 32-element block from the swizzled tile (box = shared address of its slab).  bf16 boxes use the
 // 64-byte swizzle (16-byte chunk c of row t stored at chunk c ^ ((t >> 1) & 3)),
@@ -141,7 +100,6 @@ template <bool kBF16, int kFmt>
 __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
     k_quant_act(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
   using T = Tile<kBF16>;
-  constexpr bool kFp8 = (kFmt == kFmtMxfp8);
   constexpr bool kNv = (kFmt == kFmtNvfp4);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -186,16 +144,7 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
       if constexpr (kNv) {
         // Per-tensor encode scale, published to the consumers through the
         // release of this thread's first arrivals on the stage barriers.
-        float gs = 1.0f;
-        if (p.gs_amax != nullptr) {
-          const float a = __uint_as_float(*p.gs_amax);
-          if (a > 0.0f) {
-            gs = __fdiv_rn(kNvGlobalNumerator, a);
-            if (!(gs <= FLT_MAX)) gs = 1.0f;
-          }
-        } else if (p.gs != nullptr) {
-          gs = *p.gs;
-        }
+        const float gs = nv_encode_scale(p);
         *gs_smem = gs;
         if (p.gs_out != nullptr && blockIdx.x == 0) *p.gs_out = gs;
       }
@@ -298,141 +247,16 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
         y[2 * i + 1] = y2[i].y;
       }
 
-      // Extrema (NaN-propagating) of each 16-element half, and of the block.
-      float mn0 = fmin3_nan(y[0], y[1], y[2]), mx0 = fmax3_nan(y[0], y[1], y[2]);
-      float mn1 = fmin3_nan(y[16], y[17], y[18]), mx1 = fmax3_nan(y[16], y[17], y[18]);
-#pragma unroll
-      for (int j = 3; j < 15; j += 2) {
-        mn0 = fmin3_nan(mn0, y[j], y[j + 1]);
-        mx0 = fmax3_nan(mx0, y[j], y[j + 1]);
-        mn1 = fmin3_nan(mn1, y[16 + j], y[17 + j]);
-        mx1 = fmax3_nan(mx1, y[16 + j], y[17 + j]);
-      }
-      mn0 = fmin_nan(mn0, y[15]);
-      mx0 = fmax_nan(mx0, y[15]);
-      mn1 = fmin_nan(mn1, y[31]);
-      mx1 = fmax_nan(mx1, y[31]);
-      const float mn = fmin_nan(mn0, mn1), mx = fmax_nan(mx0, mx1);
-      const bool finite = (fabsf(mn) <= FLT_MAX) && (fabsf(mx) <= FLT_MAX);
-      // Clip bounds from the whole block; clipped amax = max(|clamp(min)|, |clamp(max)|).
-      const float lo = r_min * mn;
-      const float hi = r_max * mx;
-      auto clampf = [&](float v) { return fminf(fmaxf(v, lo), hi); };
-
-      if (kNv && p.amax_out != nullptr) {
-        // Measuring pass: fold this warp's largest clipped |y| into the tensor amax.
-        const float a = finite ? fmaxf(fmaxf(fabsf(clampf(mn0)), fabsf(clampf(mx0))),
-                                       fmaxf(fabsf(clampf(mn1)), fabsf(clampf(mx1))))
-                               : 0.0f;
-        const unsigned v = __reduce_max_sync(0xffffffffu, row < p.S ? __float_as_uint(a) : 0u);
-        if (lane == 0 && v != 0u) atomicMax(p.amax_out, v);
-      } else {
-        uint32_t sbits;  // scale byte (MX) or two scale bytes (NVFP4, half 0 in the low byte)
-        float2 mult;     // multiplier of the elements of each half
-        if constexpr (kNv) {
-          // Group scale E4M3(fp32(amax * gs) / 6) per half; multiplier fp32(gs / scale).
-          const float gs = *gs_smem;
-          const float a0 = fmaxf(fabsf(clampf(mn0)), fabsf(clampf(mx0)));
-          const float a1 = fmaxf(fabsf(clampf(mn1)), fabsf(clampf(mx1)));
-          sbits = e4m3x2_bits(__fdiv_rn(__fmul_rn(a0, gs), 6.0f), __fdiv_rn(__fmul_rn(a1, gs), 6.0f));
-          const float2 sv = e4m3x2_values(sbits);
-          mult.x = sv.x == 0.0f ? 0.0f : __fdiv_rn(gs, sv.x);
-          mult.y = sv.y == 0.0f ? 0.0f : __fdiv_rn(gs, sv.y);
-        } else {
-          // Shared scale: floor(log2 amax) = biased exponent - 127, so the scale
-          // byte e + 127 = biased exponent - emax (emax = 2 for E2M1, 8 for E4M3;
-          // clamped at 0, which also covers amax == 0 and subnormal amax).  2^-e
-          // is built from exponent bits.
-          const float amax = fmaxf(fabsf(clampf(mn)), fabsf(clampf(mx)));
-          constexpr uint32_t kEmax = kFp8 ? 8u : 2u;
-          const uint32_t ebits = __float_as_uint(amax) >> 23;
-          sbits = ebits > kEmax ? ebits - kEmax : 0u;
-          const float inv_scale = __uint_as_float((254u - sbits) << 23);
-          mult = make_float2(inv_scale, inv_scale);
-        }
-
-        // Clip, then divide by the scale (an exact power-of-two multiply for MX,
-        // the fp32 multiplier for NVFP4; two elements per packed multiply), then
-        // round to E2M1 or E4M3.
-        constexpr int kWords = kFp8 ? 8 : 4;  // 32 codes of 4 or 8 bits
-        uint32_t words[kWords];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float m = w < 2 ? mult.x : mult.y;
-          const float2 inv2 = make_float2(m, m);
-          float2 q[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 c2 = make_float2(clampf(y[8 * w + 2 * j]), clampf(y[8 * w + 2 * j + 1]));
-            q[j] = __fmul2_rn(c2, inv2);
-          }
-          if constexpr (kFp8) {
-            words[2 * w] = e4m3x4(q[0].x, q[0].y, q[1].x, q[1].y);
-            words[2 * w + 1] = e4m3x4(q[2].x, q[2].y, q[3].x, q[3].y);
-          } else {
-            words[w] = e2m1x8(q[0].x, q[0].y, q[1].x, q[1].y, q[2].x, q[2].y, q[3].x, q[3].y);
-          }
-        }
-        if (!finite) {
-          sbits = kNv ? 0x7F7Fu : 0xFFu;
-#pragma unroll
-          for (int w = 0; w < kWords; ++w) words[w] = 0u;
-        }
-
-        if (row < p.S) {
-          constexpr int kBlockCodeBytes = kWords * 4;
-          uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (size_t)(kFp8 ? p.N : p.N >> 1) +
-                                                (size_t)b * kBlockCodeBytes);
-          dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-          if constexpr (kFp8) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-          if constexpr (kNv) {
-            // scale columns 2b and 2b + 1 are adjacent in both layouts
-            uint8_t* sp = p.mma_layout ? p.scales + mma_scale_offset(row, 2 * b, p.kpad)
-                                       : p.scales + (size_t)row * (size_t)(2 * p.k) + 2 * b;
-            *reinterpret_cast<uint16_t*>(sp) = (uint16_t)sbits;
-          } else if (p.mma_layout) {
-            p.scales[mma_scale_offset(row, b, p.kpad)] = (uint8_t)sbits;
-          } else {
-            p.scales[(size_t)row * p.k + b] = (uint8_t)sbits;
-          }
-          if (p.y_debug != nullptr) {
-            float4* yd = reinterpret_cast<float4*>(p.y_debug + (size_t)row * p.N + (size_t)b * 32);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) yd[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
-          }
-        } else if (p.mma_layout && row < p.rows_out) {
-          if constexpr (kNv)
-            *reinterpret_cast<uint16_t*>(p.scales + mma_scale_offset(row, 2 * b, p.kpad)) = (uint16_t)kPadScaleNv;
-          else
-            p.scales[mma_scale_offset(row, b, p.kpad)] = kPadScale;
-        }
-      }
-    } else if (p.mma_layout && row < p.rows_out) {
-      // Padding: rows past S (all formats) and block columns past k (MX only;
-      // the NVFP4 column count 2k is already a multiple of 4).
-      if constexpr (kNv) {
-        if (b < p.k)
-          *reinterpret_cast<uint16_t*>(p.scales + mma_scale_offset(row, 2 * b, p.kpad)) = (uint16_t)kPadScaleNv;
-      } else if (b < p.kpad) {
-        p.scales[mma_scale_offset(row, b, p.kpad)] = kPadScale;
-      }
+      encode_block<kFmt>(y, r_min, r_max, kNv ? *gs_smem : 1.0f, row, b, lane, p);
+    } else {
+      pad_scales<kFmt>(row, b, p);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
 }
 
-template <bool kBF16, int kFmt>
-cudaError_t launch_impl(const QuantLaunch& L) {
-  using T = Tile<kBF16>;
-  // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
-  CUtensorMap map;
-  const uint64_t esz = kBF16 ? 2u : 4u;
-  if (!make_map_3d_swizzled(&map, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.X,
-                            32, (uint64_t)L.S, (uint64_t)(L.N / 32), (uint64_t)L.ldx * esz, 32 * esz, 32, kRows,
-                            kCols, kBF16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) {
-    return cudaErrorInvalidValue;
-  }
+QuantArgs make_args(const QuantLaunch& L) {
   QuantArgs a;
   for (int i = 0; i < 64; ++i) a.A[i] = L.A[i];
   a.B = L.B;
@@ -445,17 +269,30 @@ cudaError_t launch_impl(const QuantLaunch& L) {
   a.N = L.N;
   a.k = L.N / 32;
   // scale columns of the MMA layout: k rounded up to 4 (MX), 2k (NVFP4, already a multiple of 4)
-  a.kpad = kFmt == kFmtNvfp4 ? 2 * a.k : (a.k + 3) / 4 * 4;
+  a.kpad = L.fmt == kFmtNvfp4 ? 2 * a.k : (a.k + 3) / 4 * 4;
   a.mma_layout = (L.mma_layout && L.amax_out == nullptr) ? 1 : 0;
   a.gs = L.gs;
   a.gs_amax = L.gs_amax;
   a.gs_out = L.gs_out;
-  a.amax_out = kFmt == kFmtNvfp4 ? L.amax_out : nullptr;
+  a.amax_out = L.fmt == kFmtNvfp4 ? L.amax_out : nullptr;
   a.rows_out = a.mma_layout ? (L.S + 127) / 128 * 128 : L.S;
   a.tiles_r = (a.rows_out + kRows - 1) / kRows;
   a.tiles_c = (a.k + kCols - 1) / kCols;
   a.tiles_c_magic = ((1ull << 40) + (unsigned long long)a.tiles_c - 1) / (unsigned long long)a.tiles_c;
+  return a;
+}
 
+template <bool kBF16, int kFmt>
+cudaError_t launch_impl(const QuantLaunch& L, const QuantArgs& a) {
+  using T = Tile<kBF16>;
+  // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
+  CUtensorMap map;
+  const uint64_t esz = kBF16 ? 2u : 4u;
+  if (!make_map_3d_swizzled(&map, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.X,
+                            32, (uint64_t)L.S, (uint64_t)(L.N / 32), (uint64_t)L.ldx * esz, 32 * esz, 32, kRows,
+                            kCols, kBF16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) {
+    return cudaErrorInvalidValue;
+  }
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -483,10 +320,18 @@ cudaError_t launch_impl(const QuantLaunch& L) {
 }  // namespace
 
 cudaError_t launch_quant_act(const QuantLaunch& L) {
+  const QuantArgs a = make_args(L);
+  // bf16 activations are exact tensor-core operands.  When every SM gets at
+  // least six of its 128-token x 128-element tiles, the tensor-core kernel
+  // (quant_act_tc.cu) is faster: its per-tile cost is lower but its pipeline
+  // takes longer to fill.  Smaller bf16 problems and fp32 activations take the
+  // CUDA-core kernel above.
+  const long long tc_tiles = (long long)((a.k + 3) / 4) * ((L.S + 127) / 128);
+  if (L.bf16 && tc_tiles >= 6LL * sm_count()) return launch_quant_act_tc(L, a);
   switch (L.fmt) {
-    case kFmtMxfp4: return L.bf16 ? launch_impl<true, kFmtMxfp4>(L) : launch_impl<false, kFmtMxfp4>(L);
-    case kFmtMxfp8: return L.bf16 ? launch_impl<true, kFmtMxfp8>(L) : launch_impl<false, kFmtMxfp8>(L);
-    case kFmtNvfp4: return L.bf16 ? launch_impl<true, kFmtNvfp4>(L) : launch_impl<false, kFmtNvfp4>(L);
+    case kFmtMxfp4: return L.bf16 ? launch_impl<true, kFmtMxfp4>(L, a) : launch_impl<false, kFmtMxfp4>(L, a);
+    case kFmtMxfp8: return L.bf16 ? launch_impl<true, kFmtMxfp8>(L, a) : launch_impl<false, kFmtMxfp8>(L, a);
+    case kFmtNvfp4: return L.bf16 ? launch_impl<true, kFmtNvfp4>(L, a) : launch_impl<false, kFmtNvfp4>(L, a);
   }
   return cudaErrorInvalidValue;
 }

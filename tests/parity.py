@@ -5,10 +5,14 @@ Tolerances:
   (the condition-scaled reading of "within 1e-5 relative": a plain relative
   error is ill-posed for entries near cancellation);
 * FP4 codes and E8M0 scales bit-exact, except elements whose pre-rounding value
-  q lies within 1e-5 relative of an E2M1 rounding boundary (midpoints 0.25,
-  0.75, 1.25, 1.75, 2.5, 3.5, 5) and whole blocks whose clipped amax lies
-  within 1e-5 relative of a power of two (the shared exponent may flip); the
-  mismatching elements must number fewer than 1e-4 of all elements;
+  q lies within the Y tolerance 1e-5 * max(|y|, sum_j |x_j| |P_ji|), carried
+  into scaled units (and never less than 1e-5 of q), of an E2M1 rounding
+  boundary (midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5), values within the
+  tolerance of zero (the sign of a zero code), and whole blocks whose clipped
+  amax lies within the tolerance of a power of two (the shared exponent may
+  flip); the mismatching elements must number fewer than 1e-4 of all elements.
+  Weight codes use the condition scale of the fused weights,
+  sum_j |w_j| |(P_i^-T)_ji|;
 * GEMM: |out_gpu - out_ref| <= 1e-4 * sum_n |a_n| |w_n| against the oracle's
   fp64 product of the same codes.
 * W4A8 (E4M3 codes): as for FP4, except that the band around each rounding
@@ -49,26 +53,47 @@ def check_y(y_gpu, X, A, B, y_ref):
     return int(bad.sum()), float(np.max(err / np.maximum(scale, 1e-300)))
 
 
-def exempt_mask(ref):
-    """Boolean (S, N): elements whose code may legitimately differ."""
+def exempt_mask(ref, cond=None):
+    """Boolean (S, N): elements whose code may legitimately differ.
+
+    Without ``cond``: q within 1e-5 relative of a midpoint, blocks whose amax is
+    within 1e-5 relative of a power of two.  With ``cond`` (the condition scale
+    sum_j |x_j| |P_ji| of each element, for values that went through the
+    transform): the band is the Y tolerance 1e-5 * max(|y|, cond) carried into
+    scaled units, which also covers values with cancellation (|y| << cond),
+    together with the sign of values within the tolerance of 0, and blocks
+    whose amax lies within 1e-5 * max(amax, largest cond of the block) of a
+    power of two.
+    """
     q = np.abs(ref["q"])
-    near_mid = np.zeros(q.shape, dtype=bool)
-    for m in MIDPOINTS:
-        near_mid |= np.abs(q - m) <= REL * m
     S, N = q.shape
     k = N // 32
-    amax = np.abs(ref["Y_hat"].astype(np.float64)).reshape(S, k, 32).max(axis=2)
+    yh = np.abs(ref["Y_hat"].astype(np.float64))
+    near_mid = np.zeros(q.shape, dtype=bool)
+    if cond is None:
+        for m in MIDPOINTS:
+            near_mid |= np.abs(q - m) <= REL * m
+    else:
+        e = ref["scales"].astype(np.int64) - 127
+        inv = np.repeat(np.exp2(-np.clip(e, -127, 127).astype(np.float64)), 32, axis=1)
+        err_y = REL * np.maximum(yh, cond)
+        band = np.maximum(err_y * inv, REL * q)
+        for m in MIDPOINTS:
+            near_mid |= np.abs(q - m) <= band
+        near_mid |= yh <= err_y
+    amax = yh.reshape(S, k, 32).max(axis=2)
     with np.errstate(divide="ignore", invalid="ignore"):
         p2 = np.exp2(np.round(np.log2(np.where(amax > 0, amax, 1.0))))
-    near_pow2 = (amax > 0) & (np.abs(amax - p2) <= REL * p2)
+    tol = REL * p2 if cond is None else REL * np.maximum(p2, cond.reshape(S, k, 32).max(axis=2))
+    near_pow2 = (amax > 0) & (np.abs(amax - p2) <= tol)
     return near_mid | np.repeat(near_pow2, 32, axis=1), near_pow2
 
 
-def compare_codes(codes_gpu, scales_gpu_linear, ref):
+def compare_codes(codes_gpu, scales_gpu_linear, ref, cond=None):
     """Returns dict(mismatch, unexplained, scale_mismatch, scale_unexplained, total)."""
     cg = O.unpack_nibbles(codes_gpu)
     cr = O.unpack_nibbles(ref["codes"])
-    ex, ex_blk = exempt_mask(ref)
+    ex, ex_blk = exempt_mask(ref, cond)
     diff = cg != cr
     sdiff = np.asarray(scales_gpu_linear) != ref["scales"]
     S, N = cg.shape
@@ -83,8 +108,8 @@ def compare_codes(codes_gpu, scales_gpu_linear, ref):
     }
 
 
-def assert_quant_parity(codes_gpu, scales_gpu_linear, ref, label=""):
-    r = compare_codes(codes_gpu, scales_gpu_linear, ref)
+def assert_quant_parity(codes_gpu, scales_gpu_linear, ref, label="", cond=None):
+    r = compare_codes(codes_gpu, scales_gpu_linear, ref, cond)
     assert r["unexplained"] == 0 and r["scale_unexplained"] == 0, f"{label}: {r}"
     assert r["mismatch"] < 1e-4 * r["total"], f"{label}: too many boundary mismatches {r}"
     return r

@@ -104,7 +104,7 @@ def test_prepare_weights_parity(maker):
     lin = O.scales_from_mma_layout(scales.cpu().numpy(), w.M, w.k)
     r = PT.assert_quant_parity(codes.cpu().numpy(), lin, {"q": ref["q"], "Y_hat": ref["W_fused"],
                                                           "codes": ref["codes"], "scales": ref["scales"]},
-                               "prepare")
+                               "prepare", cond=PT.condition_scale_weights(w.W, w.A, w.B))
     print("prepare mismatches", r)
 
 
@@ -115,7 +115,7 @@ def test_prepare_weights_q_proj():
     lin = O.scales_from_mma_layout(scales.cpu().numpy(), w.M, w.k)
     r = PT.assert_quant_parity(codes.cpu().numpy(), lin, {"q": ref["q"], "Y_hat": ref["W_fused"],
                                                           "codes": ref["codes"], "scales": ref["scales"]},
-                               "prepare q_proj")
+                               "prepare q_proj", cond=PT.condition_scale_weights(w.W, w.A, w.B))
     print("prepare q_proj mismatches", r)
 
 
@@ -157,7 +157,7 @@ def test_linear_matches_quant_then_gemm_and_oracle(maker):
     PT.assert_gemm_parity(out.cpu().numpy()[rows], ref, T, "linear")
     # and the activations themselves match the oracle's (boundary exemptions only)
     act = O.quant_act(w.x[rows], w.A, w.B, w.alpha_min, w.alpha_max)
-    PT.assert_quant_parity(codes[rows], lin[rows], act, "linear act")
+    PT.assert_quant_parity(codes[rows], lin[rows], act, "linear act", cond=PT.condition_scale(w.x[rows], w.A, w.B))
 
 
 def test_linear_error_vs_unquantised_matches_oracle():
@@ -179,7 +179,8 @@ def test_linear_with_block_hadamard_transform():
     ref, T, act, wp = O.linear(w.x, w.A, w.B, w.alpha_min, w.alpha_max, w.W)
     lin = O.scales_from_mma_layout(wsc.cpu().numpy(), w.M, w.k)
     PT.assert_quant_parity(wc.cpu().numpy(), lin, {"q": wp["q"], "Y_hat": wp["W_fused"], "codes": wp["codes"],
-                                                    "scales": wp["scales"]}, "hadamard weights")
+                                                    "scales": wp["scales"]}, "hadamard weights",
+                           cond=PT.condition_scale_weights(w.W, w.A, w.B))
     exact = w.x.astype(np.float64) @ w.W.astype(np.float64).T
     rel_gpu = np.linalg.norm(out.cpu().numpy() - exact) / np.linalg.norm(exact)
     rel_ref = np.linalg.norm(ref - exact) / np.linalg.norm(exact)

@@ -231,3 +231,40 @@ def test_linear_nvfp4_error_matches_oracle_and_beats_mxfp4():
     BQ.batq_linear(X, w.A, B, ratios, wc4, ws4, w.M, ws, out4)
     rel_mx = np.linalg.norm(out4.cpu().numpy() - exact) / np.linalg.norm(exact)
     assert rel_gpu < rel_mx, (rel_gpu, rel_mx)
+
+
+def test_quant_nvfp4_tensor_core_transform_large():
+    """A shape large enough for the tensor-core transform (sampled rows, gs from the device)."""
+    w = WL.custom(4173, 8192, 16, 78, with_w=False)
+    codes, lin, y, raw = _quant_nv(w, 5.0)
+    rows = np.unique(np.concatenate([np.random.default_rng(78).choice(w.S, 128, replace=False),
+                                     np.arange(w.S - 20, w.S)]))
+    ref = O.quant_act_nvfp4(w.x[rows], w.A, w.B, w.alpha_min, w.alpha_max, 5.0)
+    bad, worst = PT.check_y(y[rows], w.x[rows], w.A, w.B, ref["Y"])
+    assert bad == 0, worst
+    PT.assert_quant_parity_nvfp4(codes[rows], lin[rows], ref, PT.condition_scale(w.x[rows], w.A, w.B),
+                                 label="nvfp4 tc")
+    own = O.nvfp4_quantize(O.clip_blocks(y[rows], O.clip_ratios(w.alpha_min), O.clip_ratios(w.alpha_max))[0], 5.0)
+    np.testing.assert_array_equal(codes[rows], own[0])
+    np.testing.assert_array_equal(lin[rows], own[1])
+
+
+def test_prepare_weights_nvfp4_tensor_core_measuring_pass():
+    """bf16 weights large enough for the tensor-core transform: both passes (amax, then codes)."""
+    w = WL.custom(16, 4096, 8192, 79)
+    Wb = torch.from_numpy(np.ascontiguousarray(w.W)).cuda().to(torch.bfloat16)
+    Wv = Wb.float().cpu().numpy()
+    codes, scales = BQ.empty_nvfp4_buffers(w.M, w.N)
+    gs = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty(BQ.batq_prepare_weights_nvfp4_workspace_size(w.N), dtype=torch.uint8, device="cuda")
+    BQ.batq_prepare_weights_nvfp4(Wb, w.A, w.B, codes, scales, gs, ws)
+    assert BQ.batq_device_error() == 0
+    rows = np.sort(np.random.default_rng(79).choice(w.M, 96, replace=False))
+    ref_all = O.prepare_weights_nvfp4(Wv, w.A, w.B)
+    gs_rel = abs(float(gs.item()) - ref_all["gs"]) / ref_all["gs"]
+    assert gs_rel <= 1e-5
+    lin = O.scales_from_mma_layout(scales.cpu().numpy(), w.M, w.N // 16)[rows]
+    ref = {"q": ref_all["q"][rows], "Y_hat": ref_all["W_fused"][rows], "codes": ref_all["codes"][rows],
+           "scales": ref_all["scales"][rows], "gs": ref_all["gs"]}
+    PT.assert_quant_parity_nvfp4(codes.cpu().numpy()[rows], lin, ref, PT.condition_scale_weights(Wv[rows], w.A, w.B),
+                                 gs_rel=max(gs_rel, 1e-7), label="prepare nvfp4 tc")

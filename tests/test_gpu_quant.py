@@ -32,7 +32,7 @@ def _check_all(w, codes, scales, y, rows=None, label=""):
         strict = O.encode_from_transformed(y, r[0], r[1])
         np.testing.assert_array_equal(scales, strict["scales"], err_msg=label + " scales (strict)")
         np.testing.assert_array_equal(codes, strict["codes"], err_msg=label + " codes (strict)")
-    return PT.assert_quant_parity(codes, scales, ref, label)
+    return PT.assert_quant_parity(codes, scales, ref, label, cond=PT.condition_scale(x, w.A, w.B))
 
 
 @pytest.mark.parametrize("layout", [BQ.BATQ_SCALES_LINEAR, BQ.BATQ_SCALES_MMA])
@@ -196,3 +196,19 @@ def test_block_hadamard_as_transform(maker):
     w = WL.with_block_hadamard(maker())
     codes, scales, y, _ = GU.gpu_quant(w)
     _check_all(w, codes, scales, y, label="block hadamard")
+
+
+@pytest.mark.parametrize("S,N,seed", [(3001, 12288, 21), (8192, 4096, 22)])
+def test_tensor_core_transform_large_ragged(S, N, seed):
+    """Shapes with at least six 128 x 128 tiles per SM take the tensor-core transform; ragged S
+    leaves a partial last tile.  Sampled rows (including the last ones) against the oracle, the
+    GPU's own Y re-encoded bit-exact, and the padding rows of the last 128-row scale tile."""
+    w = WL.custom(S, N, 16, seed, with_w=False)
+    codes, scales, y, raw = GU.gpu_quant(w)
+    rows = np.unique(np.concatenate([np.random.default_rng(seed).choice(S, 200, replace=False),
+                                     np.arange(S - 40, S)]))
+    _check_all(w, codes, scales, y, rows=rows, label=f"tc {S}x{N}")
+    pad_rows = np.arange(S, (S + 127) // 128 * 128)
+    if len(pad_rows):
+        r, c = np.meshgrid(pad_rows, np.arange(w.k), indexing="ij")
+        assert (raw[O.mma_scale_offset(r, c, w.k)] == 0x7F).all()

@@ -140,3 +140,15 @@ def test_linear_w4a8_matches_quant_then_gemm_and_oracle(maker):
         e8 = np.linalg.norm(out.cpu().numpy() - exact)
         e4 = np.linalg.norm(o4 - exact)
         assert e8 < e4, (e8, e4)
+
+
+def test_quant_mxfp8_tensor_core_transform_large():
+    """A shape large enough for the tensor-core transform (sampled rows)."""
+    w = WL.custom(4173, 8192, 16, 63, with_w=False)
+    codes, lin, y, _ = _quant8(w)
+    rows = np.unique(np.concatenate([np.random.default_rng(63).choice(w.S, 128, replace=False),
+                                     np.arange(w.S - 20, w.S)]))
+    ref = O.quant_act_mxfp8(w.x[rows], w.A, w.B, w.alpha_min, w.alpha_max)
+    bad, worst = PT.check_y(y[rows], w.x[rows], w.A, w.B, ref["Y"])
+    assert bad == 0, worst
+    PT.assert_quant_parity_e4m3(codes[rows], lin[rows], ref, w.x[rows], w.A, w.B, "mxfp8 tc")
