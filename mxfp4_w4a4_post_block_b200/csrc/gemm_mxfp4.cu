@@ -197,82 +197,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
-    if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      for (int ks = 0; ks < nks && ok; ++ks) {
-        if (!mbar_wait(&sf_ready[s], ph)) {
-          set_error(g.err, kErrDataTimeout);
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        uint8_t* st = smem + s * C::kStageBytes;
-        const uint32_t sp = smem_u32(st);
-        const uint32_t sq = sp + C::kPBytes;
-        const int kleft = g.N - ks * kBK;
-        const int nmma = kleft >= kBK ? kMmasPerStage : kleft / kKPerMma;
-        const uint64_t dp = sdesc_kmajor_sw128(sp);
-        const uint64_t dq = sdesc_kmajor_sw128(sq);
+    // The whole warp runs the loop (warp-uniform state: a loop run by one lane
+    // spends many more instructions per MMA); one elected lane issues.
+    const bool issuer = elect_one();
+    int s = 0;
+    uint32_t ph = 0;
+    for (int ks = 0; ks < nks; ++ks) {
+      if (!mbar_wait_warp(&sf_ready[s], ph)) {
+        if (issuer) set_error(g.err, kErrDataTimeout);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint64_t dp = sdesc_kmajor_sw128(smem_u32(smem + s * C::kStageBytes));
+      const uint64_t dq = dp + (uint64_t)(C::kPBytes >> 4);  // addresses < 2^18: no carry out of the field
+      const uint32_t tsfp = t_sfp + s * C::kSfPCols, tsfq = t_sfq + s * C::kSfQCols;
+      const int kleft = g.N - ks * kBK;
+      const int nmma = kleft >= kBK ? kMmasPerStage : kleft / kKPerMma;
+      if (issuer) {
         for (int j = 0; j < nmma; ++j) {
           // MMA j covers scale blocks kb.. of the stage: atom kb / 4, byte
           // kb % 4 of each 4-scale TMEM column (NVFP4: four scales, byte 0).
           const int kb = j * C::kSfPerMma;
           const int a = kb >> 2;
           const int sf_id = kb & 3;
+          const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
           // Advance K by 32 bytes inside the 128-byte swizzle atom.
           if constexpr (kFp8)
             tc_mma_mxf8(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc_mxf8(kBM, BN, sf_id, sf_id),
-                        t_sfp + s * C::kSfPCols + a * 4, t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms,
-                        (ks > 0 || j > 0) ? 1u : 0u);
+                        tsfp + a * 4, tsfq + a * 4 * C::kQRowAtoms, acc);
           else if constexpr (C::kNv)
-            tc_mma_nvf4(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc_nvf4(kBM, BN),
-                        t_sfp + s * C::kSfPCols + a * 4, t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms,
-                        (ks > 0 || j > 0) ? 1u : 0u);
+            tc_mma_nvf4(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc_nvf4(kBM, BN), tsfp + a * 4,
+                        tsfq + a * 4 * C::kQRowAtoms, acc);
           else
             tc_mma_mxf4(t_acc, dp + (uint64_t)(j * 2), dq + (uint64_t)(j * 2), idesc_mxf4(BN, sf_id, sf_id),
-                        t_sfp + s * C::kSfPCols + a * 4, t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms,
-                        (ks > 0 || j > 0) ? 1u : 0u);
+                        tsfp + a * 4, tsfq + a * 4 * C::kQRowAtoms, acc);
         }
         tc_commit(&empty[s]);
-        if (++s == kStages) {
-          s = 0;
-          ph ^= 1;
-        }
       }
-      // Signal the epilogue once every issued MMA has completed (also on error).
-      tc_commit(acc_full);
+      __syncwarp();
+      if (++s == kStages) {
+        s = 0;
+        ph ^= 1;
+      }
     }
+    // Signal the epilogue once every issued MMA has completed (also on error).
+    if (issuer) tc_commit(acc_full);
+    __syncwarp();
   } else if (warp == kSfWarp) {
     // ------------------------------ scale copies ------------------------------
-    if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      for (int ks = 0; ks < nks; ++ks) {
-        if (!mbar_wait(&full[s], ph)) {
-          set_error(g.err, kErrDataTimeout);
-          break;
-        }
-        tc_fence_after_sync();
-        const uint32_t ssfp = smem_u32(smem + s * C::kStageBytes) + C::kPBytes + C::kQBytes;
-        const uint32_t ssfq = ssfp + C::kSfPBytes;
-        const int kleft = g.N - ks * kBK;
-        const int nmma = kleft >= kBK ? kMmasPerStage : kleft / kKPerMma;
-        const int atoms = ((nmma - 1) * C::kSfPerMma) / 4 + 1;  // atoms the stage's MMAs read
+    // Warp-wide loop, one elected issuer (as the MMA warp).
+    const bool issuer = elect_one();
+    int s = 0;
+    uint32_t ph = 0;
+    for (int ks = 0; ks < nks; ++ks) {
+      if (!mbar_wait_warp(&full[s], ph)) {
+        if (issuer) set_error(g.err, kErrDataTimeout);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint64_t dsfp = sdesc_sf_atom(smem_u32(smem + s * C::kStageBytes) + C::kPBytes + C::kQBytes);
+      const uint64_t dsfq = dsfp + (uint64_t)(C::kSfPBytes >> 4);
+      const uint32_t tsfp = t_sfp + s * C::kSfPCols, tsfq = t_sfq + s * C::kSfQCols;
+      const int kleft = g.N - ks * kBK;
+      const int nmma = kleft >= kBK ? kMmasPerStage : kleft / kKPerMma;
+      const int atoms = ((nmma - 1) * C::kSfPerMma) / 4 + 1;  // atoms the stage's MMAs read
+      if (issuer) {
         for (int a = 0; a < atoms; ++a) {
-          tc_cp_32x128b_warpx4(t_sfp + s * C::kSfPCols + a * 4, sdesc_sf_atom(ssfp + a * kSfAtom));
+          tc_cp_32x128b_warpx4(tsfp + a * 4, dsfp + (uint64_t)(a * (kSfAtom >> 4)));
 #pragma unroll
           for (int r = 0; r < C::kQRowAtoms; ++r) {
-            tc_cp_32x128b_warpx4(t_sfq + s * C::kSfQCols + a * 4 * C::kQRowAtoms + r * 4,
-                                 sdesc_sf_atom(ssfq + (r * C::kAtoms + a) * kSfAtom));
+            tc_cp_32x128b_warpx4(tsfq + a * 4 * C::kQRowAtoms + r * 4,
+                                 dsfq + (uint64_t)((r * C::kAtoms + a) * (kSfAtom >> 4)));
           }
         }
         tc_commit(&sf_ready[s]);
-        if (++s == kStages) {
-          s = 0;
-          ph ^= 1;
-        }
+      }
+      __syncwarp();
+      if (++s == kStages) {
+        s = 0;
+        ph ^= 1;
       }
     }
   } else {

@@ -224,53 +224,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------ MMA issuer (leader only) ------------------------------
     // The stages of all of this cluster's tiles form one sequence g = 0, 1, ...;
     // stage g's scales are already in TMEM slot g % kStages when sf_ready fires.
-    if (leader && lane == 0) {
+    // The whole warp runs the loop, so its state stays warp-uniform (a loop run
+    // by one lane spends many more instructions per MMA), and one elected lane
+    // issues the MMAs and commits.
+    if (leader) {
+      const bool issuer = elect_one();
       const int total = my_tiles * nks;
       for (int gi = 0; gi < total; ++gi) {
         const int ks = gi % nks;
         const uint32_t tile_iter = (uint32_t)(gi / nks);
         if (ks == 0) {
           // The accumulator must have been drained by both CTAs' epilogues.
-          if (!mbar_wait(acc_empty, (tile_iter & 1) ^ 1)) {
-            set_error(g.err, kErrDrainTimeout);
+          if (!mbar_wait_warp(acc_empty, (tile_iter & 1) ^ 1)) {
+            if (issuer) set_error(g.err, kErrDrainTimeout);
             break;
           }
           tc_fence_after_sync();
         }
         const int st_idx = gi % kStages;
-        if (!mbar_wait(&sf_ready[st_idx], (uint32_t)((gi / kStages) & 1))) {
-          set_error(g.err, kErrDataTimeout);
+        if (!mbar_wait_warp(&sf_ready[st_idx], (uint32_t)((gi / kStages) & 1))) {
+          if (issuer) set_error(g.err, kErrDataTimeout);
           break;
         }
         tc_fence_after_sync();
-        const uint32_t sa = smem_u32(smem + st_idx * kStageBytes);
-        const uint32_t sb = sa + kABytes;
+        // Shared addresses stay below 2^18, so the descriptor of base + off is
+        // the base descriptor + off / 16.
+        const uint64_t da0 = sdesc_kmajor_sw128(smem_u32(smem + st_idx * kStageBytes));
+        const uint64_t db0 = da0 + (uint64_t)(kABytes >> 4);
+        const uint32_t tsfa = t_sfa + st_idx * kSfaCols, tsfb = t_sfb + st_idx * kSfbCols;
         const int kleft = g.N - ks * kBK;
         const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
-        for (int j = 0; j < nmma; ++j) {
-          // MMA j covers scale blocks kb.. of the stage: atom kb / 4, byte
-          // kb % 4 of each 4-scale TMEM column (NVFP4: four scales, byte 0).
-          const int kb = j * kSfPerMma;
-          const int a = kb >> 2;
-          const int sf_id = kb & 3;
-          // Bytes 32j.. of the stage's K: swizzle tile j / 4, then 32 bytes per
-          // MMA inside its 128-byte swizzle atom.
-          const uint64_t da = sdesc_kmajor_sw128(sa + (j >> 2) * kSwTile) + (uint64_t)((j & 3) * 2);
-          const uint64_t db = sdesc_kmajor_sw128(sb + (j >> 2) * kSwTile) + (uint64_t)((j & 3) * 2);
-          if constexpr (C::kFp8)
-            tc_mma_pair_mxf8(t_acc, da, db, idesc_mxf8(256, kTileN, sf_id, sf_id),
-                             t_sfa + st_idx * kSfaCols + a * 4, t_sfb + st_idx * kSfbCols + a * 8,
-                             (ks > 0 || j > 0) ? 1u : 0u);
-          else if constexpr (C::kNv)
-            tc_mma_pair_nvf4(t_acc, da, db, idesc_nvf4(256, kTileN), t_sfa + st_idx * kSfaCols + a * 4,
-                             t_sfb + st_idx * kSfbCols + a * 8, (ks > 0 || j > 0) ? 1u : 0u);
-          else
-            tc_mma_pair_mxf4(t_acc, da, db, idesc_mxf4_m256(kTileN, sf_id, sf_id), t_sfa + st_idx * kSfaCols + a * 4,
-                             t_sfb + st_idx * kSfbCols + a * 8, (ks > 0 || j > 0) ? 1u : 0u);
+        if (issuer) {
+          for (int j = 0; j < nmma; ++j) {
+            // MMA j covers scale blocks kb.. of the stage: atom kb / 4, byte
+            // kb % 4 of each 4-scale TMEM column (NVFP4: four scales, byte 0).
+            const int kb = j * kSfPerMma;
+            const int a = kb >> 2;
+            const int sf_id = kb & 3;
+            // Bytes 32j.. of the stage's K: swizzle tile j / 4, then 32 bytes per
+            // MMA inside its 128-byte swizzle atom.
+            const uint64_t off = (uint64_t)((j >> 2) * (kSwTile >> 4) + (j & 3) * 2);
+            const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
+            if constexpr (C::kFp8)
+              tc_mma_pair_mxf8(t_acc, da0 + off, db0 + off, idesc_mxf8(256, kTileN, sf_id, sf_id), tsfa + a * 4,
+                               tsfb + a * 8, acc);
+            else if constexpr (C::kNv)
+              tc_mma_pair_nvf4(t_acc, da0 + off, db0 + off, idesc_nvf4(256, kTileN), tsfa + a * 4, tsfb + a * 8, acc);
+            else
+              tc_mma_pair_mxf4(t_acc, da0 + off, db0 + off, idesc_mxf4_m256(kTileN, sf_id, sf_id), tsfa + a * 4,
+                               tsfb + a * 8, acc);
+          }
+          tc_commit_pair(&empty[st_idx], 0x3);
+          // Both epilogues may read the accumulator once every MMA of the tile has completed.
+          if (ks == nks - 1) tc_commit_pair(acc_full, 0x3);
         }
-        tc_commit_pair(&empty[st_idx], 0x3);
-        // Both epilogues may read the accumulator once every MMA of the tile has completed.
-        if (ks == nks - 1) tc_commit_pair(acc_full, 0x3);
+        __syncwarp();
       }
     }
   } else if (warp == kSfWarp) {
@@ -278,31 +286,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Stage g's data has landed (full) -> copy its scale tiles into TMEM slot
     // g % kStages in both CTAs -> sf_ready.  The slot's previous contents were
     // consumed by the MMAs of stage g - kStages, which completed before the
-    // producer could refill the stage.
-    if (leader && lane == 0) {
+    // producer could refill the stage.  Warp-wide loop, one elected issuer.
+    if (leader) {
+      const bool issuer = elect_one();
       const int total = my_tiles * nks;
       for (int gi = 0; gi < total; ++gi) {
         const int st_idx = gi % kStages;
-        if (!mbar_wait(&full[st_idx], (uint32_t)((gi / kStages) & 1))) {
-          set_error(g.err, kErrDataTimeout);
+        if (!mbar_wait_warp(&full[st_idx], (uint32_t)((gi / kStages) & 1))) {
+          if (issuer) set_error(g.err, kErrDataTimeout);
           break;
         }
         tc_fence_after_sync();
         const int ks = gi % nks;
         const int kleft = g.N - ks * kBK;
         const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
-        const uint32_t ssfa = smem_u32(smem + st_idx * kStageBytes) + kABytes + kBBytes;
-        const uint32_t ssfb = ssfa + kSfaBytes;
+        const uint64_t dsfa = sdesc_sf_atom(smem_u32(smem + st_idx * kStageBytes) + kABytes + kBBytes);
+        const uint64_t dsfb = dsfa + (uint64_t)(kSfaBytes >> 4);
+        const uint64_t dsfb1 = dsfb + (uint64_t)((g.sf_box_chunks * 256) >> 4);
+        const uint32_t tsfa = t_sfa + st_idx * kSfaCols, tsfb = t_sfb + st_idx * kSfbCols;
         const int atoms = ((nmma - 1) * kSfPerMma) / 4 + 1;  // atoms the stage's MMAs read
-        for (int a = 0; a < atoms; ++a) {
-          tc_cp_pair_32x128b_warpx4(t_sfa + st_idx * kSfaCols + a * 4, sdesc_sf_atom(ssfa + a * kSfAtom));
-          // weight-scale box is {2 row tiles} x {sf_box_chunks}: row tile r, atom a at
-          // r * sf_box_chunks * 256 + a * 512
-          tc_cp_pair_32x128b_warpx4(t_sfb + st_idx * kSfbCols + a * 8, sdesc_sf_atom(ssfb + a * kSfAtom));
-          tc_cp_pair_32x128b_warpx4(t_sfb + st_idx * kSfbCols + a * 8 + 4,
-                                    sdesc_sf_atom(ssfb + g.sf_box_chunks * 256 + a * kSfAtom));
+        if (issuer) {
+          for (int a = 0; a < atoms; ++a) {
+            const uint64_t off = (uint64_t)(a * (kSfAtom >> 4));
+            tc_cp_pair_32x128b_warpx4(tsfa + a * 4, dsfa + off);
+            // weight-scale box is {2 row tiles} x {sf_box_chunks}: row tile r, atom a at
+            // r * sf_box_chunks * 256 + a * 512
+            tc_cp_pair_32x128b_warpx4(tsfb + a * 8, dsfb + off);
+            tc_cp_pair_32x128b_warpx4(tsfb + a * 8 + 4, dsfb1 + off);
+          }
+          tc_commit_pair_local(&sf_ready[st_idx]);
         }
-        tc_commit_pair_local(&sf_ready[st_idx]);
+        __syncwarp();
       }
     }
   } else if (warp >= 2 && warp < 2 + kEpiWarps) {
@@ -328,8 +342,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int t = cluster_id; t < num_tiles; t += num_clusters, ++tile_iter) {
       const int row0 = (t / g.tiles_n) * kTileM + (int)rank * kRowsPerCta + 32 * quad;
       const int n0 = (t % g.tiles_n) * kTileN + col0;
-      if (!mbar_wait(acc_full, tile_iter & 1)) {
-        set_error(g.err, kErrMmaTimeout);
+      if (!mbar_wait_warp(acc_full, tile_iter & 1)) {
+        if (lane == 0) set_error(g.err, kErrMmaTimeout);
         break;
       }
       __syncwarp();

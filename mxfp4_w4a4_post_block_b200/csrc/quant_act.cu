@@ -186,8 +186,8 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
     const int c0 = (t - tr * p.tiles_c) * kCols;
     const int b = c0 + wc;
     const int row = r0 + lane;
-    if (!mbar_wait(&full[s], (i / T::kStages) & 1)) {
-      set_error(p.err, kErrDataTimeout);
+    if (!mbar_wait_warp(&full[s], (i / T::kStages) & 1)) {
+      if (lane == 0) set_error(p.err, kErrDataTimeout);
       break;
     }
     if (r0 < p.S && b < p.k) {

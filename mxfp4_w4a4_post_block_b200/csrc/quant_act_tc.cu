@@ -179,18 +179,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < total; ++g) {
       if (g == 0 || (i0 + g) % tiles_r == 0) {
         // The new strip's P_i parts are in shared memory.
-        if (!mbar_wait(p_ready, strip_count & 1)) {
+        if (!mbar_wait_warp(p_ready, strip_count & 1)) {
           if (leader) set_error(p.err, kErrDataTimeout);
           break;
         }
         ++strip_count;
       }
       const int st = g % kStages, buf = g % kAccBufs;
-      if (!mbar_wait(&acc_empty[buf], ((g / kAccBufs) & 1) ^ 1)) {
+      if (!mbar_wait_warp(&acc_empty[buf], ((g / kAccBufs) & 1) ^ 1)) {
         if (leader) set_error(p.err, kErrDrainTimeout);
         break;
       }
-      if (!mbar_wait(&full[st], (g / kStages) & 1)) {
+      if (!mbar_wait_warp(&full[st], (g / kStages) & 1)) {
         if (leader) set_error(p.err, kErrDataTimeout);
         break;
       }
@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const int buf = g % kAccBufs;
-      if (!mbar_wait(&acc_full[buf], (g / kAccBufs) & 1)) {
-        set_error(p.err, kErrMmaTimeout);
+      if (!mbar_wait_warp(&acc_full[buf], (g / kAccBufs) & 1)) {
+        if (lane == 0) set_error(p.err, kErrMmaTimeout);
         break;
       }
       __syncwarp();
