@@ -330,6 +330,37 @@ BATQ_API batq_status batq_linear_nvfp4(const void* X, batq_dtype x_dtype, int S,
                               const float* w_gs_dev, int M, void* workspace, size_t workspace_bytes,
                               batq_dtype out_dtype, void* out, int ldo, void* stream);
 
+/* ------------------------------------------------------------------------
+ * BAT on the KV cache (the pages' KV8 / KV4 settings: BATQuant thelatestinai.com
+ * page, Table 2 caption, W4A8KV8 and W4A8KV4; gist.science summary, §2.D: the
+ * transforms also apply to the KV cache).  New key (or value) rows -- N =
+ * kv_heads x head_dim elements per token, N % 64 == 0 -- go through the same
+ * block transform, clip and MX quantisation as batq_quant_act (A, B_i and the
+ * clip ratios are the cache's own) and are written into a paged cache at the
+ * rows slot_mapping names.  The attention side (the inverse transform folded
+ * into the queries or the output projection) is not part of this call.
+ * ------------------------------------------------------------------------ */
+
+typedef enum {
+  BATQ_KV_MXFP4 = 0, /* KV4: packed E2M1 codes, num_slots x N/2 bytes */
+  BATQ_KV_MXFP8 = 1  /* KV8: E4M3 codes, num_slots x N bytes */
+} batq_kv_format;
+
+/*
+ * slot_mapping_dev: device int32[S], the cache row of each new token; tokens
+ * with a negative slot, or one >= num_slots, are skipped (padding tokens); two
+ * tokens must not share a slot.  cache_codes: device num_slots x (N/2 or N)
+ * bytes, 16-byte aligned; cache_scales: device num_slots x N/32 E8M0 bytes
+ * (LINEAR layout).  Rows not named are left as they were.  Stream-ordered,
+ * asynchronous.  Errors: BATQ_ERR_INVALID_ARG (null pointers, num_slots < 1,
+ * unknown format), BATQ_ERR_SHAPE, BATQ_ERR_ALIGNMENT, BATQ_ERR_ARCH,
+ * BATQ_ERR_CUDA.
+ */
+BATQ_API batq_status batq_quant_kv_cache(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                                const float* A_host, const float* B_dev, const float* ratios_dev,
+                                const int* slot_mapping_dev, int num_slots, batq_kv_format kv_format,
+                                uint8_t* cache_codes, uint8_t* cache_scales, void* stream);
+
 /*
  * batq_linear without a caller-provided workspace, for callers that cannot
  * allocate device memory (for example a plugin running in a process whose

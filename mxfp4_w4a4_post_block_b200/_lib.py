@@ -23,6 +23,8 @@ BATQ_F32 = 0
 BATQ_BF16 = 1
 BATQ_SCALES_LINEAR = 0
 BATQ_SCALES_MMA = 1
+BATQ_KV_MXFP4 = 0
+BATQ_KV_MXFP8 = 1
 
 _c_int, _c_size_p, _vp, _fp = ctypes.c_int, ctypes.POINTER(ctypes.c_size_t), ctypes.c_void_p, ctypes.c_void_p
 
@@ -62,6 +64,8 @@ SIGNATURES = {
     "batq_linear_nvfp4_workspace_size": (_c_int, [_c_int, _c_int, _c_size_p]),
     "batq_linear_nvfp4": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
                                    _vp, ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
+    "batq_quant_kv_cache": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _c_int, _vp,
+                                     _vp, _vp]),
     "batq_selftest_wait_timeout": (_c_int, [ctypes.c_uint, _vp]),
     "batq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint)]),
 }

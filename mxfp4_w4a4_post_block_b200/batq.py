@@ -13,7 +13,8 @@ import ctypes
 import numpy as np
 
 from . import _lib
-from ._lib import (BATQ_BF16, BATQ_F32, BATQ_OK, BATQ_SCALES_LINEAR, BATQ_SCALES_MMA)  # noqa: F401
+from ._lib import (BATQ_BF16, BATQ_F32, BATQ_KV_MXFP4, BATQ_KV_MXFP8, BATQ_OK, BATQ_SCALES_LINEAR,  # noqa: F401
+                   BATQ_SCALES_MMA)
 
 
 class BatqError(RuntimeError):
@@ -288,6 +289,21 @@ def batq_linear_nvfp4(X, A, B, ratios, a_gs, w_codes, w_scales, w_gs, M, workspa
                                          _dev_ptr(w_gs, "w_gs"), M, _dev_ptr(workspace, "workspace"),
                                          workspace.numel() * workspace.element_size(), _dtype_code(out),
                                          _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_linear_nvfp4")
+
+
+# -------------------------------------------------------------- KV cache
+
+def batq_quant_kv_cache(X, A, B, ratios, slot_mapping, cache_codes, cache_scales, kv_format=BATQ_KV_MXFP4,
+                        stream=None):
+    """Transform + clip + MXFP4 / MXFP8 of new K or V rows X (S x N) into cache rows slot_mapping (int32 CUDA)."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    num_slots = cache_codes.shape[0]
+    _check(_lib.load().batq_quant_kv_cache(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0), a.ctypes.data,
+                                           _dev_ptr(B, "B"), _dev_ptr(ratios, "ratios"),
+                                           _dev_ptr(slot_mapping, "slot_mapping"), num_slots, kv_format,
+                                           _dev_ptr(cache_codes, "cache_codes"), _dev_ptr(cache_scales, "cache_scales"),
+                                           _stream(stream)), "batq_quant_kv_cache")
 
 
 def batq_selftest_wait_timeout(limit_us: int, stream=None):

@@ -583,6 +583,43 @@ batq_status batq_linear_nvfp4(const void* X, batq_dtype x_dtype, int S, int N, i
                      a_gs_dev, w_gs_dev);
 }
 
+// ------------------------------------------------------------------ KV cache
+
+batq_status batq_quant_kv_cache(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_host,
+                                const float* B_dev, const float* ratios_dev, const int* slot_mapping_dev,
+                                int num_slots, batq_kv_format kv_format, uint8_t* cache_codes,
+                                uint8_t* cache_scales, void* stream) {
+  if (!slot_mapping_dev || num_slots < 1) return BATQ_ERR_INVALID_ARG;
+  if (kv_format != BATQ_KV_MXFP4 && kv_format != BATQ_KV_MXFP8) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_quant_args(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, cache_codes, cache_scales,
+                                    BATQ_SCALES_LINEAR, nullptr);
+  if (st != BATQ_OK) return st;
+  if (!aligned4(slot_mapping_dev)) return BATQ_ERR_ALIGNMENT;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  batq::QuantLaunch L;
+  L.X = X;
+  L.bf16 = (x_dtype == BATQ_BF16);
+  L.S = S;
+  L.N = N;
+  L.ldx = ldx;
+  std::memcpy(L.A, A_host, sizeof(L.A));
+  L.B = B_dev;
+  L.ratios = ratios_dev;
+  L.codes = cache_codes;
+  L.scales = cache_scales;
+  L.mma_layout = false;
+  L.y_debug = nullptr;
+  L.err = error_word();
+  L.stream = static_cast<cudaStream_t>(stream);
+  L.fmt = kv_format == BATQ_KV_MXFP8 ? batq::kFmtMxfp8 : batq::kFmtMxfp4;
+  L.row_map = slot_mapping_dev;
+  L.num_slots = num_slots;
+  cudaError_t e = batq::launch_quant_act(L);
+  if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
+  return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
+}
+
 batq_status batq_selftest_wait_timeout(unsigned int limit_us, void* stream) {
   if (limit_us == 0 || limit_us > 1000000u) return BATQ_ERR_INVALID_ARG;
   batq_status st = check_arch();

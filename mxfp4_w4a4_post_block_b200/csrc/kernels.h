@@ -33,10 +33,14 @@ struct QuantLaunch {
   // gs used.  With amax_out set the launch only measures: the largest clipped
   // |y| of every finite block is folded into *amax_out (fp32 bits, atomic max)
   // and nothing else is written.
-  const float* gs;
-  const unsigned* gs_amax;
-  float* gs_out;
-  unsigned* amax_out;
+  const float* gs = nullptr;
+  const unsigned* gs_amax = nullptr;
+  float* gs_out = nullptr;
+  unsigned* amax_out = nullptr;
+  // Output row of token r: row_map[r] (device int32[S]; rows < 0 or >= num_slots
+  // are skipped), e.g. the slot of a paged KV cache.  Linear scale layout only.
+  const int* row_map = nullptr;
+  int num_slots = 0;
 };
 
 // Returns cudaErrorInvalidValue when the tensor map cannot be encoded.

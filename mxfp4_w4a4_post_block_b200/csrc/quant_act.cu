@@ -275,6 +275,8 @@ QuantArgs make_args(const QuantLaunch& L) {
   a.gs_amax = L.gs_amax;
   a.gs_out = L.gs_out;
   a.amax_out = L.fmt == kFmtNvfp4 ? L.amax_out : nullptr;
+  a.row_map = L.row_map;
+  a.rows_cap = L.row_map != nullptr ? L.num_slots : L.S;
   a.rows_out = a.mma_layout ? (L.S + 127) / 128 * 128 : L.S;
   a.tiles_r = (a.rows_out + kRows - 1) / kRows;
   a.tiles_c = (a.k + kCols - 1) / kCols;

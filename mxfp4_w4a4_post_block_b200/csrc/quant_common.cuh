@@ -35,6 +35,10 @@ struct QuantArgs {
   const unsigned* gs_amax;
   float* gs_out;
   unsigned* amax_out;
+  // Output row of token r: row_map[r] (skipped when < 0 or >= rows_cap), or r
+  // itself when row_map is null (then rows_cap = S).  Linear scale layout only.
+  const int* row_map;
+  int rows_cap;
 };
 
 __device__ __forceinline__ int tile_row(int t, const QuantArgs& p) {
@@ -162,28 +166,29 @@ __device__ __forceinline__ void encode_block(const float (&y)[32], float r_min, 
       for (int w = 0; w < kWords; ++w) words[w] = 0u;
     }
 
-    if (row < p.S) {
+    const int orow = (row < p.S && p.row_map != nullptr) ? p.row_map[row] : row;
+    if (row < p.S && orow >= 0 && orow < p.rows_cap) {
       constexpr int kBlockCodeBytes = kWords * 4;
-      uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (size_t)(kFp8 ? p.N : p.N >> 1) +
+      uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)orow * (size_t)(kFp8 ? p.N : p.N >> 1) +
                                             (size_t)b * kBlockCodeBytes);
       dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
       if constexpr (kFp8) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
       if constexpr (kNv) {
         // scale columns 2b and 2b + 1 are adjacent in both layouts
-        uint8_t* sp = p.mma_layout ? p.scales + mma_scale_offset(row, 2 * b, p.kpad)
-                                   : p.scales + (size_t)row * (size_t)(2 * p.k) + 2 * b;
+        uint8_t* sp = p.mma_layout ? p.scales + mma_scale_offset(orow, 2 * b, p.kpad)
+                                   : p.scales + (size_t)orow * (size_t)(2 * p.k) + 2 * b;
         *reinterpret_cast<uint16_t*>(sp) = (uint16_t)sbits;
       } else if (p.mma_layout) {
-        p.scales[mma_scale_offset(row, b, p.kpad)] = (uint8_t)sbits;
+        p.scales[mma_scale_offset(orow, b, p.kpad)] = (uint8_t)sbits;
       } else {
-        p.scales[(size_t)row * p.k + b] = (uint8_t)sbits;
+        p.scales[(size_t)orow * p.k + b] = (uint8_t)sbits;
       }
       if (p.y_debug != nullptr) {
         float4* yd = reinterpret_cast<float4*>(p.y_debug + (size_t)row * p.N + (size_t)b * 32);
 #pragma unroll
         for (int j = 0; j < 8; ++j) yd[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
       }
-    } else if (p.mma_layout && row < p.rows_out) {
+    } else if (row >= p.S && p.mma_layout && row < p.rows_out) {
       if constexpr (kNv)
         *reinterpret_cast<uint16_t*>(p.scales + mma_scale_offset(row, 2 * b, p.kpad)) = (uint16_t)kPadScaleNv;
       else

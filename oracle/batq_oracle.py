@@ -66,6 +66,11 @@ share one E4M3 scale; the pages give no other rule, so these are readings):
   zero codes.
 * GEMM: out = fp32(1 / fp32(gs_a * gs_w)) * sum (code_a s_a)(code_w s_w).
 
+KV cache (the pages' KV8 / KV4 settings): new key or value rows (kv_heads x
+head_dim elements per token) take the same transform, clip and MXFP4 / MXFP8
+encoding and are written to the cache rows a slot mapping names; negative slots
+are skipped.  The attention side is not part of the path.
+
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 closed forms, brute force and the pages' Table 1.
 """
@@ -668,3 +673,27 @@ def gemm_nvfp4(a_codes, a_scales, w_codes, w_scales, alpha: float = 1.0):
     Dw = dequantize_nvfp4(w_codes, w_scales)
     al = float(np.float32(alpha))
     return al * (Da @ Dw.T), abs(al) * (np.abs(Da) @ np.abs(Dw).T)
+
+
+# ---------------------------------------------------------------------------
+# BAT on the KV cache: new key / value rows quantised into a paged cache
+# [thelatestinai.com BATQuant page, Table 2 caption (W4A8KV8, W4A8KV4);
+#  gist.science summary, section 2.D (the transforms also cover the KV cache)]
+# ---------------------------------------------------------------------------
+
+def quant_kv_cache(X, A, B, alpha_min, alpha_max, slots, cache_codes, cache_scales, kv_format="mxfp4"):
+    """Transform, clip and MXFP4 (KV4) or MXFP8 (KV8) of new rows X, written into copies of the cache.
+
+    Row r of X goes to cache row slots[r]; a slot below 0 or past the cache is skipped, and rows the
+    mapping does not name keep their contents.  Returns (codes, scales, the per-token result).
+    """
+    act = quant_act(X, A, B, alpha_min, alpha_max) if kv_format == "mxfp4" else \
+        quant_act_mxfp8(X, A, B, alpha_min, alpha_max)
+    codes = np.array(cache_codes, dtype=np.uint8, copy=True)
+    scales = np.array(cache_scales, dtype=np.uint8, copy=True)
+    n = codes.shape[0]
+    for r, s in enumerate(np.asarray(slots).tolist()):
+        if 0 <= s < n:
+            codes[s] = act["codes"][r]
+            scales[s] = act["scales"][r]
+    return codes, scales, act

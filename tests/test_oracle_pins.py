@@ -803,3 +803,36 @@ def test_block_hadamard_of_a_unit_vector_is_a_sign_row():
     for j in range(32):
         assert ((codes[j, 32:64] & 7) == 7).all()
         np.testing.assert_array_equal(codes[j, 32:64] >> 3, (H[j] < 0).astype(np.uint8))
+
+
+# ------------------------------------------------------------- KV cache ----
+
+def test_kv_cache_scatter_invariants():
+    """A skipped token changes nothing, the cache does not depend on the order of the new tokens,
+    and each written row depends only on its own token (rows of another token perturbed: unchanged)."""
+    w = WL.custom(12, 256, 16, 41, x_dtype="f32", with_w=False)
+    rng = np.random.default_rng(41)
+    n = 20
+    cc0 = rng.integers(0, 256, (n, 128), dtype=np.uint8)
+    cs0 = rng.integers(0, 256, (n, 8), dtype=np.uint8)
+    slots = rng.permutation(n)[:12]
+    slots[3] = -1
+    slots[7] = n + 5
+    for fmt in ("mxfp4", "mxfp8"):
+        width = 128 if fmt == "mxfp4" else 256
+        cc = rng.integers(0, 256, (n, width), dtype=np.uint8)
+        c1, s1, act = O.quant_kv_cache(w.x, w.A, w.B, w.alpha_min, w.alpha_max, slots, cc, cs0, fmt)
+        untouched = np.setdiff1d(np.arange(n), slots[(slots >= 0) & (slots < n)])
+        np.testing.assert_array_equal(c1[untouched], cc[untouched])
+        np.testing.assert_array_equal(s1[untouched], cs0[untouched])
+        perm = rng.permutation(12)
+        c2, s2, _ = O.quant_kv_cache(w.x[perm], w.A, w.B, w.alpha_min, w.alpha_max, slots[perm], cc, cs0, fmt)
+        np.testing.assert_array_equal(c1, c2)
+        np.testing.assert_array_equal(s1, s2)
+        x3 = w.x.copy()
+        x3[5] *= 7.0
+        c3, s3, _ = O.quant_kv_cache(x3, w.A, w.B, w.alpha_min, w.alpha_max, slots, cc, cs0, fmt)
+        others = np.array([s for r, s in enumerate(slots) if r != 5 and 0 <= s < n])
+        np.testing.assert_array_equal(c3[others], c1[others])
+        np.testing.assert_array_equal(s3[others], s1[others])
+        assert not np.array_equal(c3[slots[5]], c1[slots[5]]) or not np.array_equal(s3[slots[5]], s1[slots[5]])
