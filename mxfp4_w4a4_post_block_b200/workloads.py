@@ -27,6 +27,7 @@ Recipes (numpy ``default_rng(seed)``, drawn in the order listed):
   q_proj.
 * ``layer``     seeds 500+j for the seven linears of one decoder layer at
   S=8192 (q, k, v, o, gate, up, down); X as q_proj.
+* ``with_naive_kronecker(w, seed)``: w's inputs with one A_i = I + 0.1 N per block.
 * ``with_block_hadamard(w)``: w's X and W with P_i = H_32 / sqrt(32) (Sylvester) for every
   block and no clip, the block-rotation baseline as an input.
 """
@@ -207,6 +208,15 @@ def with_block_hadamard(w: Workload) -> Workload:
     B = np.tile((sylvester_hadamard(4) / 2.0).astype(np.float32), (k, 1, 1))
     big = np.full(k, 40.0, np.float32)
     return dataclasses.replace(w, name=w.name + "_blockhadamard", A=A, B=B, alpha_min=big, alpha_max=big.copy())
+
+
+def with_naive_kronecker(w: Workload, seed: int = 0, sigma: float = 0.1) -> Workload:
+    """The same inputs with one 8x8 factor per block, A_i = I + sigma N(0, 1) (the "naive Kronecker"
+    decomposition of Table 1, P_i = B_i (x) A_i), drawn from default_rng(seed)."""
+    k = w.N // BLOCK
+    rng = np.random.default_rng(seed)
+    A = _near_identity(rng, (k, 8, 8), sigma)
+    return dataclasses.replace(w, name=w.name + "_naivekron", A=A)
 
 
 CONFIGS = {

@@ -66,6 +66,10 @@ share one E4M3 scale; the pages give no other rule, so these are readings):
   zero codes.
 * GEMM: out = fp32(1 / fp32(gs_a * gs_w)) * sum (code_a s_a)(code_w s_w).
 
+Naive Kronecker (Table 1's middle row, [p3]): one 8x8 A_i per block instead of
+the shared A, P_i = B_i (x) A_i; every function that takes A accepts either
+shape (8, 8) or (k, 8, 8).
+
 KV cache (the pages' KV8 / KV4 settings): new key or value rows (kv_heads x
 head_dim elements per token) take the same transform, clip and MXFP4 / MXFP8
 encoding and are written to the cache rows a slot mapping names; negative slots
@@ -158,16 +162,19 @@ def dense_blocks(A: np.ndarray, B: np.ndarray) -> np.ndarray:
     """All k dense blocks P_i = B_i (x) A, shape (k, 32, 32), fp64 [p1 BAT: P = diag(P_1..P_k)].
 
     Same entry-by-entry rule as ``kron_block``, applied to every block at once.
+    ``A`` is either the shared 8x8 factor (GPK) or one 8x8 factor per block,
+    shape (k, 8, 8): P_i = B_i (x) A_i, the "naive Kronecker" row of Table 1 [p3].
     """
     A = np.asarray(A, dtype=np.float64)
     B = np.asarray(B, dtype=np.float64)
     k = B.shape[0]
+    Ak = A if A.ndim == 3 else np.broadcast_to(A, (k, G1, G1))
     P = np.zeros((k, G, G), dtype=np.float64)
     for r in range(G2):
         for c in range(G2):
             for a in range(G1):
                 for b in range(G1):
-                    P[:, G1 * r + a, G1 * c + b] = B[:, r, c] * A[a, b]
+                    P[:, G1 * r + a, G1 * c + b] = B[:, r, c] * Ak[:, a, b]
     return P
 
 
@@ -394,7 +401,7 @@ def fuse_weights_f64(W: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
     k = N // G
     out = np.empty_like(W)
     for i in range(k):
-        Pinv = gauss_jordan_inverse(kron_block(A, B[i]))
+        Pinv = gauss_jordan_inverse(kron_block(A[i] if np.ndim(A) == 3 else A, B[i]))
         out[:, G * i:G * (i + 1)] = W[:, G * i:G * (i + 1)] @ Pinv.T
     return out
 

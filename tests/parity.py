@@ -188,7 +188,7 @@ def condition_scale_weights(W, A, B):
     M, N = W.shape
     out = np.empty_like(W)
     for i in range(N // 32):
-        pinv_t = O.gauss_jordan_inverse(O.kron_block(A, B[i])).T
+        pinv_t = O.gauss_jordan_inverse(O.kron_block(A[i] if np.ndim(A) == 3 else A, B[i])).T
         out[:, 32 * i:32 * (i + 1)] = W[:, 32 * i:32 * (i + 1)] @ np.abs(pinv_t)
     return out
 

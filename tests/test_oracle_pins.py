@@ -836,3 +836,42 @@ def test_kv_cache_scatter_invariants():
         np.testing.assert_array_equal(c3[others], c1[others])
         np.testing.assert_array_equal(s3[others], s1[others])
         assert not np.array_equal(c3[slots[5]], c1[slots[5]]) or not np.array_equal(s3[slots[5]], s1[slots[5]])
+
+
+# ---------------------------------------------- naive Kronecker (per-block A_i) ----
+
+def test_naive_kronecker_blocks_are_numpy_kron_of_the_pair():
+    """P_i = B_i (x) A_i against numpy's Kronecker product, block by block."""
+    w = WL.with_naive_kronecker(WL.tiny(with_w=False), 5)
+    P = O.dense_blocks(w.A, w.B)
+    for i in range(w.k):
+        np.testing.assert_array_equal(P[i], np.kron(w.B[i].astype(np.float64), w.A[i].astype(np.float64)))
+    assert O.param_counts(4096)["naive_kronecker"] == 128 * (64 + 16)
+
+
+def test_naive_kronecker_with_equal_factors_is_gpk():
+    """A_i = A for every block reproduces the GPK path bit for bit (activations and weights)."""
+    w = WL.tiny()
+    Ak = np.repeat(w.A[None], w.k, axis=0)
+    a1 = O.quant_act(w.x, w.A, w.B, w.alpha_min, w.alpha_max)
+    a2 = O.quant_act(w.x, Ak, w.B, w.alpha_min, w.alpha_max)
+    np.testing.assert_array_equal(a1["codes"], a2["codes"])
+    np.testing.assert_array_equal(a1["scales"], a2["scales"])
+    np.testing.assert_array_equal(a1["Y"], a2["Y"])
+    w1, w2 = O.prepare_weights(w.W, w.A, w.B), O.prepare_weights(w.W, Ak, w.B)
+    np.testing.assert_array_equal(w1["codes"], w2["codes"])
+
+
+def test_naive_kronecker_block_locality_and_fusion_invariance():
+    """Changing A_j changes block j only; (x P)(P^-1 W^T) = x W^T with per-block factors."""
+    w = WL.with_naive_kronecker(WL.tiny(), 6)
+    Y = O.transform_f64(w.x, w.A, w.B)
+    A2 = w.A.copy()
+    A2[3] = A2[3] * 1.5 + 0.1
+    Y2 = O.transform_f64(w.x, A2, w.B)
+    changed = np.abs(Y2 - Y).reshape(w.S, w.k, 32).max(axis=(0, 2)) > 0
+    assert changed.tolist() == [j == 3 for j in range(w.k)]
+    Wf = O.fuse_weights_f64(w.W, w.A, w.B)
+    ref = w.x.astype(np.float64) @ w.W.astype(np.float64).T
+    got = Y @ Wf.T
+    assert np.abs(got - ref).max() <= 1e-12 * np.abs(w.x).sum(1).max() * np.abs(w.W).max() * 10
