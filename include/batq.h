@@ -331,6 +331,36 @@ BATQ_API batq_status batq_linear_nvfp4(const void* X, batq_dtype x_dtype, int S,
                               batq_dtype out_dtype, void* out, int ldo, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Naive Kronecker decomposition (BATQuant thelatestinai.com page, Table 1,
+ * middle row: P_i = B_i (x) A_i with an 8x8 A_i per block, k (g1^2 + g2^2)
+ * parameters, 10,240 at N = 4096, against GPK's shared A).  The same path as
+ * batq_quant_act / batq_prepare_weights / batq_linear with MXFP4 output,
+ * except that A is replaced by one 8x8 row-major A_i per block column:
+ * A_blocks k x 64 floats (device, 16-byte aligned, for the activation calls;
+ * host for the weight preparation, which inverts every A_i in fp64 and returns
+ * BATQ_ERR_SINGULAR as batq_prepare_weights does).
+ * ------------------------------------------------------------------------ */
+
+BATQ_API batq_status batq_quant_act_kron(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                                const float* A_blocks_dev, const float* B_dev, const float* ratios_dev,
+                                uint8_t* codes, uint8_t* scales, batq_scale_layout layout, float* y_debug,
+                                void* stream);
+
+/* Device workspace bytes batq_prepare_weights_kron needs (B'_i and A'_i). Host only. */
+BATQ_API batq_status batq_prepare_weights_kron_workspace_size(int N, size_t* bytes);
+
+BATQ_API batq_status batq_prepare_weights_kron(const void* W, batq_dtype w_dtype, int M, int N, int ldw,
+                                      const float* A_blocks_host, const float* B_host, uint8_t* w_codes,
+                                      uint8_t* w_scales, batq_scale_layout layout, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
+/* Whole linear with per-block A_i; workspace as batq_linear_workspace_size. */
+BATQ_API batq_status batq_linear_kron(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                             const float* A_blocks_dev, const float* B_dev, const float* ratios_dev,
+                             const uint8_t* w_codes, const uint8_t* w_scales, int M, void* workspace,
+                             size_t workspace_bytes, batq_dtype out_dtype, void* out, int ldo, void* stream);
+
+/* ------------------------------------------------------------------------
  * BAT on the KV cache (the pages' KV8 / KV4 settings: BATQuant thelatestinai.com
  * page, Table 2 caption, W4A8KV8 and W4A8KV4; gist.science summary, §2.D: the
  * transforms also apply to the KV cache).  New key (or value) rows -- N =

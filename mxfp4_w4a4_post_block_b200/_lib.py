@@ -64,6 +64,13 @@ SIGNATURES = {
     "batq_linear_nvfp4_workspace_size": (_c_int, [_c_int, _c_int, _c_size_p]),
     "batq_linear_nvfp4": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
                                    _vp, ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
+    "batq_quant_act_kron": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
+                                     _vp]),
+    "batq_prepare_weights_kron_workspace_size": (_c_int, [_c_int, _c_size_p]),
+    "batq_prepare_weights_kron": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _vp,
+                                           ctypes.c_size_t, _vp]),
+    "batq_linear_kron": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
+                                  ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
     "batq_quant_kv_cache": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _c_int, _vp,
                                      _vp, _vp]),
     "batq_selftest_wait_timeout": (_c_int, [ctypes.c_uint, _vp]),

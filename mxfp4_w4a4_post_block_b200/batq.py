@@ -291,6 +291,51 @@ def batq_linear_nvfp4(X, A, B, ratios, a_gs, w_codes, w_scales, w_gs, M, workspa
                                          _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_linear_nvfp4")
 
 
+# ------------------------------------------------- naive Kronecker (per-block A_i)
+
+def batq_prepare_weights_kron_workspace_size(N: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_lib.load().batq_prepare_weights_kron_workspace_size(N, ctypes.byref(b)),
+           "batq_prepare_weights_kron_workspace_size")
+    return b.value
+
+
+def batq_quant_act_kron(X, A_blocks, B, ratios, codes, scales, layout=BATQ_SCALES_MMA, y_debug=None, stream=None):
+    """As batq_quant_act with one 8x8 A_i per block (A_blocks: CUDA float tensor, k x 64)."""
+    S, N = X.shape
+    _check(_lib.load().batq_quant_act_kron(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0),
+                                           _dev_ptr(A_blocks, "A_blocks"), _dev_ptr(B, "B"),
+                                           _dev_ptr(ratios, "ratios"), _dev_ptr(codes, "codes"),
+                                           _dev_ptr(scales, "scales"), layout, _dev_ptr(y_debug, "y_debug"),
+                                           _stream(stream)), "batq_quant_act_kron")
+
+
+def batq_prepare_weights_kron(W, A_blocks_host, B_host, w_codes, w_scales, workspace, layout=BATQ_SCALES_MMA,
+                              stream=None):
+    """Offline weight side with one A_i per block (host arrays: A_blocks k x 8 x 8, B k x 4 x 4)."""
+    M, N = W.shape
+    k = N // 32
+    a = _host_f32(A_blocks_host, k * 64, "A_blocks")
+    b = _host_f32(B_host, k * 16, "B")
+    _check(_lib.load().batq_prepare_weights_kron(_dev_ptr(W, "W"), _dtype_code(W), M, N, W.stride(0),
+                                                 a.ctypes.data, b.ctypes.data, _dev_ptr(w_codes, "w_codes"),
+                                                 _dev_ptr(w_scales, "w_scales"), layout,
+                                                 _dev_ptr(workspace, "workspace"),
+                                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "batq_prepare_weights_kron")
+
+
+def batq_linear_kron(X, A_blocks, B, ratios, w_codes, w_scales, M, workspace, out, stream=None):
+    """Whole W4A4 linear with one A_i per block (A_blocks: CUDA float tensor, k x 64)."""
+    S, N = X.shape
+    _check(_lib.load().batq_linear_kron(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0),
+                                        _dev_ptr(A_blocks, "A_blocks"), _dev_ptr(B, "B"), _dev_ptr(ratios, "ratios"),
+                                        _dev_ptr(w_codes, "w_codes"), _dev_ptr(w_scales, "w_scales"), M,
+                                        _dev_ptr(workspace, "workspace"),
+                                        workspace.numel() * workspace.element_size(), _dtype_code(out),
+                                        _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_linear_kron")
+
+
 # -------------------------------------------------------------- KV cache
 
 def batq_quant_kv_cache(X, A, B, ratios, slot_mapping, cache_codes, cache_scales, kv_format=BATQ_KV_MXFP4,

@@ -112,7 +112,7 @@ batq_status launch_quant(const void* X, batq_dtype x_dtype, int S, int N, int ld
                          const float* B_dev, const float* ratios_dev, uint8_t* codes, uint8_t* scales,
                          batq_scale_layout layout, float* y_debug, int fmt, cudaStream_t stream,
                          const float* gs = nullptr, const unsigned* gs_amax = nullptr, float* gs_out = nullptr,
-                         unsigned* amax_out = nullptr) {
+                         unsigned* amax_out = nullptr, const float* A_blocks = nullptr) {
   batq::QuantLaunch L;
   L.X = X;
   L.bf16 = (x_dtype == BATQ_BF16);
@@ -133,6 +133,7 @@ batq_status launch_quant(const void* X, batq_dtype x_dtype, int S, int N, int ld
   L.gs_amax = gs_amax;
   L.gs_out = gs_out;
   L.amax_out = amax_out;
+  L.A_blocks = A_blocks;
   cudaError_t e = batq::launch_quant_act(L);
   if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
   return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
@@ -231,6 +232,34 @@ size_t nv_scale_bytes_for(int rows, int N, batq_scale_layout layout) {
 }
 
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Stand-in for the shared A where the naive Kronecker calls pass one A_i per block instead.
+const float kUnusedA[64] = {};
+
+// Naive Kronecker weight side: A'_i = A_i^-T (k x 64 floats) for every block, and B'_i as in
+// fused_transform, both copied into the workspace: B' at 0, A' at a_offset.
+batq_status fused_transform_kron(const float* A_blocks_host, const float* B_host, int N, void* workspace,
+                                 size_t a_offset, cudaStream_t s) {
+  const int k = N / 32;
+  float unused[64];
+  // B'_i and the transfer to the workspace's start: the shared-A routine with an identity A.
+  float eye[64] = {};
+  for (int i = 0; i < 8; ++i) eye[i * 9] = 1.0f;
+  batq_status st = fused_transform(eye, B_host, N, workspace, unused, s);
+  if (st != BATQ_OK) return st;
+  std::vector<float> a_fused((size_t)k * 64);
+  for (int i = 0; i < k; ++i) {
+    double a[64], ainv[64];
+    for (int j = 0; j < 64; ++j) a[j] = A_blocks_host[(size_t)i * 64 + j];
+    if (!invert(a, ainv, 8)) return BATQ_ERR_SINGULAR;
+    for (int r = 0; r < 8; ++r)
+      for (int c = 0; c < 8; ++c) a_fused[(size_t)i * 64 + r * 8 + c] = (float)ainv[c * 8 + r];
+  }
+  if (cudaMemcpyAsync(static_cast<uint8_t*>(workspace) + a_offset, a_fused.data(), a_fused.size() * sizeof(float),
+                      cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return BATQ_ERR_CUDA;
+  return BATQ_OK;
+}
 
 }  // namespace
 
@@ -581,6 +610,80 @@ batq_status batq_linear_nvfp4(const void* X, batq_dtype x_dtype, int S, int N, i
   if (st != BATQ_OK) return st;
   return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, batq::kFmtNvfp4, s,
                      a_gs_dev, w_gs_dev);
+}
+
+// ------------------------------------------------------------------ naive Kronecker (per-block A_i)
+
+batq_status batq_quant_act_kron(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_blocks_dev,
+                                const float* B_dev, const float* ratios_dev, uint8_t* codes, uint8_t* scales,
+                                batq_scale_layout layout, float* y_debug, void* stream) {
+  if (!A_blocks_dev) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_quant_args(X, x_dtype, S, N, ldx, kUnusedA, B_dev, ratios_dev, codes, scales, layout,
+                                    y_debug);
+  if (st != BATQ_OK) return st;
+  if (!aligned16(A_blocks_dev)) return BATQ_ERR_ALIGNMENT;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  return launch_quant(X, x_dtype, S, N, ldx, kUnusedA, B_dev, ratios_dev, codes, scales, layout, y_debug,
+                      batq::kFmtMxfp4, static_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, nullptr,
+                      A_blocks_dev);
+}
+
+batq_status batq_prepare_weights_kron_workspace_size(int N, size_t* bytes) {
+  if (!bytes) return BATQ_ERR_INVALID_ARG;
+  size_t base = 0;
+  batq_status st = batq_prepare_workspace_size(N, &base);
+  if (st != BATQ_OK) return st;
+  *bytes = base + round_up((size_t)(N / 32) * 64 * sizeof(float), 256);
+  return BATQ_OK;
+}
+
+batq_status batq_prepare_weights_kron(const void* W, batq_dtype w_dtype, int M, int N, int ldw,
+                                      const float* A_blocks_host, const float* B_host, uint8_t* w_codes,
+                                      uint8_t* w_scales, batq_scale_layout layout, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!A_blocks_host || !B_host || !workspace) return BATQ_ERR_INVALID_ARG;
+  batq_status st = check_quant_args(W, w_dtype, M, N, ldw, kUnusedA, reinterpret_cast<const float*>(workspace),
+                                    nullptr, w_codes, w_scales, layout, nullptr);
+  if (st != BATQ_OK) return st;
+  size_t need = 0, base = 0;
+  batq_prepare_weights_kron_workspace_size(N, &need);
+  batq_prepare_workspace_size(N, &base);
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = fused_transform_kron(A_blocks_host, B_host, N, workspace, base, s);
+  if (st != BATQ_OK) return st;
+  const float* a_fused = reinterpret_cast<const float*>(static_cast<uint8_t*>(workspace) + base);
+  return launch_quant(W, w_dtype, M, N, ldw, kUnusedA, reinterpret_cast<const float*>(workspace), nullptr, w_codes,
+                      w_scales, layout, nullptr, batq::kFmtMxfp4, s, nullptr, nullptr, nullptr, nullptr, a_fused);
+}
+
+batq_status batq_linear_kron(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* A_blocks_dev,
+                             const float* B_dev, const float* ratios_dev, const uint8_t* w_codes,
+                             const uint8_t* w_scales, int M, void* workspace, size_t workspace_bytes,
+                             batq_dtype out_dtype, void* out, int ldo, void* stream) {
+  if (!workspace || !A_blocks_dev) return BATQ_ERR_INVALID_ARG;
+  size_t need = 0;
+  batq_status st = batq_linear_workspace_size(S, N, &need);
+  if (st != BATQ_OK) return st;
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  if (!aligned16(workspace) || !aligned16(A_blocks_dev)) return BATQ_ERR_ALIGNMENT;
+  uint8_t* a_codes = static_cast<uint8_t*>(workspace);
+  uint8_t* a_scales = a_codes + round_up((size_t)S * (N / 2), 256);
+  st = check_quant_args(X, x_dtype, S, N, ldx, kUnusedA, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA,
+                        nullptr);
+  if (st != BATQ_OK) return st;
+  st = check_gemm_args(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo);
+  if (st != BATQ_OK) return st;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_quant(X, x_dtype, S, N, ldx, kUnusedA, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA, nullptr,
+                    batq::kFmtMxfp4, s, nullptr, nullptr, nullptr, nullptr, A_blocks_dev);
+  if (st != BATQ_OK) return st;
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, batq::kFmtMxfp4, s);
 }
 
 // ------------------------------------------------------------------ KV cache

@@ -41,6 +41,9 @@ struct QuantLaunch {
   // are skipped), e.g. the slot of a paged KV cache.  Linear scale layout only.
   const int* row_map = nullptr;
   int num_slots = 0;
+  // Naive Kronecker decomposition: one 8x8 A_i per block (device, k x 64
+  // floats, 16-byte aligned) replaces A; MXFP4 output only.
+  const float* A_blocks = nullptr;
 };
 
 // Returns cudaErrorInvalidValue when the tensor map cannot be encoded.

@@ -48,7 +48,8 @@ namespace {
 constexpr int kRows = 32;         // tokens per tile (one per lane)
 constexpr int kCols = 8;          // 32-blocks per tile (one per warp of a consumer group)
 
-template <bool kBF16>
+// kNaive: one A_i per block column, staged with the tile (naive Kronecker).
+template <bool kBF16, bool kNaive = false>
 struct Tile {
   static constexpr int kGroups = kBF16 ? 3 : 1;          // consumer groups per CTA
   static constexpr int kStages = kGroups * (kBF16 ? 3 : 4);  // ring depth (a multiple of kGroups)
@@ -59,7 +60,8 @@ struct Tile {
   static constexpr int kXBytes = kCols * kBoxBytes;         // activations of one tile
   static constexpr int kBOffset = kXBytes;                  // kCols x 16 fp32 B_i
   static constexpr int kROffset = kXBytes + kCols * 64;     // kCols x 2 fp32 clip ratios
-  static constexpr int kStageBytes = (kROffset + kCols * 8 + 1023) / 1024 * 1024;
+  static constexpr int kAOffset = kROffset + kCols * 8;     // kCols x 64 fp32 A_i (naive Kronecker)
+  static constexpr int kStageBytes = (kAOffset + (kNaive ? kCols * 256 : 0) + 1023) / 1024 * 1024;
   static constexpr int kSmemBytes = kStages * kStageBytes + 2 * kStages * 8 + 16 + 1024;
 };
 
@@ -95,11 +97,11 @@ __device__ __forceinline__ void load_block(uint32_t box, int lane, float x[32]) 
   }
 }
 
-// kFmt: output format (Fmt).
-template <bool kBF16, int kFmt>
-__global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
+// kFmt: output format (Fmt); kNaive: per-block A_i from p.A_blocks.
+template <bool kBF16, int kFmt, bool kNaive>
+__global__ void __launch_bounds__(Tile<kBF16, kNaive>::kThreads, 1)
     k_quant_act(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
-  using T = Tile<kBF16>;
+  using T = Tile<kBF16, kNaive>;
   constexpr bool kNv = (kFmt == kFmtNvfp4);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -161,12 +163,14 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
         if (r0 < p.S) {
           const int nb = min(kCols, p.k - c0);  // even: k is even and c0 a multiple of 8
           uint8_t* dst = smem + s * T::kStageBytes;
-          const uint32_t pbytes = (uint32_t)nb * 64u + (p.ratios != nullptr ? (uint32_t)nb * 8u : 0u);
+          const uint32_t pbytes = (uint32_t)nb * 64u + (p.ratios != nullptr ? (uint32_t)nb * 8u : 0u) +
+                                  (kNaive ? (uint32_t)nb * 256u : 0u);
           // the box always delivers all 8 block columns (zero-filled past k)
           mbar_arrive_expect_tx(&full[s], (uint32_t)T::kXBytes + pbytes);
           tma_load_3d(dst, &tmx, &full[s], 0, r0, c0);
           bulk_load(dst + T::kBOffset, p.B + (size_t)c0 * 16, (uint32_t)nb * 64u, &full[s]);
           if (p.ratios != nullptr) bulk_load(dst + T::kROffset, p.ratios + (size_t)c0 * 2, (uint32_t)nb * 8u, &full[s]);
+          if constexpr (kNaive) bulk_load(dst + T::kAOffset, p.A_blocks + (size_t)c0 * 64, (uint32_t)nb * 256u, &full[s]);
         } else {
           mbar_arrive(&full[s]);  // padding rows only: nothing to load
         }
@@ -220,7 +224,9 @@ __global__ void __launch_bounds__(Tile<kBF16>::kThreads, 1)
 #pragma unroll
           for (int a = 0; a < 8; ++a) {
             const float xv = x[8 * r + a];
-            acc = __ffma2_rn(make_float2(xv, xv), make_float2(p.A[8 * a + 2 * j], p.A[8 * a + 2 * j + 1]), acc);
+            const float2 ap = kNaive ? lds64f(st + T::kAOffset + wc * 256 + (8 * a + 2 * j) * 4)
+                                     : make_float2(p.A[8 * a + 2 * j], p.A[8 * a + 2 * j + 1]);
+            acc = __ffma2_rn(make_float2(xv, xv), ap, acc);
           }
           tm[4 * r + j] = acc;
         }
@@ -277,6 +283,7 @@ QuantArgs make_args(const QuantLaunch& L) {
   a.amax_out = L.fmt == kFmtNvfp4 ? L.amax_out : nullptr;
   a.row_map = L.row_map;
   a.rows_cap = L.row_map != nullptr ? L.num_slots : L.S;
+  a.A_blocks = L.A_blocks;
   a.rows_out = a.mma_layout ? (L.S + 127) / 128 * 128 : L.S;
   a.tiles_r = (a.rows_out + kRows - 1) / kRows;
   a.tiles_c = (a.k + kCols - 1) / kCols;
@@ -284,9 +291,9 @@ QuantArgs make_args(const QuantLaunch& L) {
   return a;
 }
 
-template <bool kBF16, int kFmt>
+template <bool kBF16, int kFmt, bool kNaive = false>
 cudaError_t launch_impl(const QuantLaunch& L, const QuantArgs& a) {
-  using T = Tile<kBF16>;
+  using T = Tile<kBF16, kNaive>;
   // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
   CUtensorMap map;
   const uint64_t esz = kBF16 ? 2u : 4u;
@@ -299,7 +306,7 @@ cudaError_t launch_impl(const QuantLaunch& L, const QuantArgs& a) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16, kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16, kFmt, kNaive>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          T::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -316,7 +323,7 @@ cudaError_t launch_impl(const QuantLaunch& L, const QuantArgs& a) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16, kFmt>, map, a);
+  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16, kFmt, kNaive>, map, a);
 }
 
 }  // namespace
@@ -330,6 +337,10 @@ cudaError_t launch_quant_act(const QuantLaunch& L) {
   // CUDA-core kernel above.
   const long long tc_tiles = (long long)((a.k + 3) / 4) * ((L.S + 127) / 128);
   if (L.bf16 && tc_tiles >= 6LL * sm_count()) return launch_quant_act_tc(L, a);
+  if (L.A_blocks != nullptr) {  // naive Kronecker: MXFP4 output
+    if (L.fmt != kFmtMxfp4) return cudaErrorInvalidValue;
+    return L.bf16 ? launch_impl<true, kFmtMxfp4, true>(L, a) : launch_impl<false, kFmtMxfp4, true>(L, a);
+  }
   switch (L.fmt) {
     case kFmtMxfp4: return L.bf16 ? launch_impl<true, kFmtMxfp4>(L, a) : launch_impl<false, kFmtMxfp4>(L, a);
     case kFmtMxfp8: return L.bf16 ? launch_impl<true, kFmtMxfp8>(L, a) : launch_impl<false, kFmtMxfp8>(L, a);

@@ -70,8 +70,9 @@ __device__ __forceinline__ double bf16_value(uint32_t bits) {
 
 // Encoder thread tid (0..511) writes the three parts of 8 entries of P_i for
 // block column cb = tid / 128 of strip s: output element n, input elements
-// 8 jc .. 8 jc + 7, i.e. P[8 jc + a][n] = B_i[jc][n / 8] A[a][n % 8] for a = 0..7,
-// as one 16-byte chunk per part at its 64-byte-swizzle position.
+// 8 jc .. 8 jc + 7, i.e. P[8 jc + a][n] = B_i[jc][n / 8] A[a][n % 8] for a = 0..7
+// (A_i[a][n % 8] with the naive Kronecker decomposition), as one 16-byte chunk
+// per part at its 64-byte-swizzle position.
 __device__ __forceinline__ void build_p_chunk(uint8_t* sp, int tid, int s, const QuantArgs& p) {
   const int cb = tid >> 7;
   const int n = (tid >> 2) & 31;
@@ -84,7 +85,9 @@ __device__ __forceinline__ void build_p_chunk(uint8_t* sp, int tid, int s, const
     uint32_t pr[kParts][2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const double v = bv * (double)p.A[(a + h) * 8 + (n & 7)];  // exact in fp64
+      const int ai = (a + h) * 8 + (n & 7);
+      const float av = p.A_blocks == nullptr ? p.A[ai] : (b < p.k ? p.A_blocks[(size_t)b * 64 + ai] : 0.0f);
+      const double v = bv * (double)av;  // exact in fp64
       const uint32_t hi = bf16_bits((float)v);
       const double r1 = v - bf16_value(hi);
       const uint32_t mid = bf16_bits((float)r1);

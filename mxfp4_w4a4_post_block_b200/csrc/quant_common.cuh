@@ -39,6 +39,8 @@ struct QuantArgs {
   // itself when row_map is null (then rows_cap = S).  Linear scale layout only.
   const int* row_map;
   int rows_cap;
+  // Naive Kronecker: one 8x8 A_i per block (device, k x 64 floats) instead of A.
+  const float* A_blocks;
 };
 
 __device__ __forceinline__ int tile_row(int t, const QuantArgs& p) {
