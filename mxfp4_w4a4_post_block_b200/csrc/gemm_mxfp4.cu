@@ -22,6 +22,7 @@
 //   warp 6     copies each stage's scales into TMEM (tcgen05.cp 32x128b.warpx4)
 //              and signals the MMA thread (copies issued by the MMA thread
 //              itself would serialise with its MMAs);
+//   (warps 1 and 6 run their stage loops warp-wide, one elected lane issuing)
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator quadrant of each warp,
 //              staged through shared memory and written with TMA stores
 //              (prefill) or stored directly, coalesced along i (decode).

@@ -11,10 +11,13 @@
 //     leader's stage barrier, and its commits arrive on both CTAs' barriers;
 //   * each CTA keeps the activation scales of its own rows and the weight
 //     scales of all 256 columns in its TMEM (128-row x 4-scale tiles copied
-//     with tcgen05.cp 32x128b.warpx4); a dedicated thread issues those copies
-//     and signals the MMA thread per stage, because copies issued by the MMA
+//     with tcgen05.cp 32x128b.warpx4); a dedicated warp issues those copies
+//     and signals the MMA warp per stage, because copies issued by the MMA
 //     thread itself serialise with its MMAs in the tensor pipe (a stage of
 //     six copies and four MMAs takes ~990 cycles inline, ~700 when split);
+//   * the MMA and scale-copy warps run their stage loops warp-wide (the loop
+//     state stays warp-uniform) and one elected lane issues; a loop run by
+//     lane 0 alone spent several more instructions per MMA or copy;
 //   * eight epilogue warps per CTA read their 128 accumulator columns into
 //     registers, release TMEM for the next tile at once, and write the output
 //     through a small per-warp shared-memory box (32 rows x 32 bytes) with TMA

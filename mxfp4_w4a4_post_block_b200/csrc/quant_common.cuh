@@ -28,6 +28,7 @@ struct QuantArgs {
   int S, N, k, kpad;
   int rows_out;  // rows whose scales are written (S, or S rounded up to 128 in MMA layout)
   int mma_layout;
+  // Tiling of the CUDA-core kernel (32 tokens x 8 blocks); the tensor-core kernel tiles itself.
   int tiles_r, tiles_c;
   unsigned long long tiles_c_magic;  // ceil(2^40 / tiles_c): t / tiles_c = (t * magic) >> 40 for t < 2^24
   // NVFP4 per-tensor scale sources and outputs (see QuantLaunch)
