@@ -75,6 +75,10 @@ head_dim elements per token) take the same transform, clip and MXFP4 / MXFP8
 encoding and are written to the cache rows a slot mapping names; negative slots
 are skipped.  The attention side is not part of the path.
 
+RMSNorm fused ahead of the transform (a reading of the ARCQuant page's fused
+reorder -> RMSNorm -> quantise kernel applied to this path): z = x / sqrt(mean
+over the token of x^2 + eps) * gamma in fp64, not rounded before the transform.
+
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 closed forms, brute force and the pages' Table 1.
 """
@@ -704,3 +708,27 @@ def quant_kv_cache(X, A, B, alpha_min, alpha_max, slots, cache_codes, cache_scal
             codes[s] = act["codes"][r]
             scales[s] = act["scales"][r]
     return codes, scales, act
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm ahead of the transform (the normalisation before each linear; the
+# ARCQuant page's fused kernel runs reorder -> RMSNorm -> quantise in one pass)
+# ---------------------------------------------------------------------------
+
+def rmsnorm(X, gamma, eps: float):
+    """Per token: z = x / sqrt(mean(x^2) + eps) * gamma, in fp64 (no intermediate rounding)."""
+    X = np.asarray(X, dtype=np.float64)
+    g = np.asarray(gamma, dtype=np.float64)
+    ms = np.mean(X * X, axis=1, keepdims=True)
+    return X / np.sqrt(ms + float(eps)) * g[None, :]
+
+
+def rmsnorm_quant_act(X, gamma, eps, A, B, alpha_min, alpha_max) -> dict:
+    """RMSNorm fused ahead of the activation path: the normalised values are transformed directly
+    (they never leave the kernel, so they are not rounded to bf16), then clip and MXFP4."""
+    Z = rmsnorm(X, gamma, eps)
+    Y = transform(Z, A, B)
+    r_min, r_max = clip_ratios(alpha_min), clip_ratios(alpha_max)
+    Yh, lo, hi, nonfinite = clip_blocks(Y, r_min, r_max)
+    codes, scales, q = mxfp4_quantize(Yh, nonfinite)
+    return {"Z": Z, "Y": Y, "Y_hat": Yh, "codes": codes, "scales": scales, "q": q, "nonfinite": nonfinite}

@@ -875,3 +875,44 @@ def test_naive_kronecker_block_locality_and_fusion_invariance():
     ref = w.x.astype(np.float64) @ w.W.astype(np.float64).T
     got = Y @ Wf.T
     assert np.abs(got - ref).max() <= 1e-12 * np.abs(w.x).sum(1).max() * np.abs(w.W).max() * 10
+
+
+# ------------------------------------------------- RMSNorm ahead of the transform ----
+
+def test_rmsnorm_matches_torch_rms_norm():
+    """Against torch's own RMSNorm (fp64 CPU), with a non-trivial weight and eps."""
+    import torch
+    rng = np.random.default_rng(51)
+    X = rng.standard_normal((9, 256)) * np.exp2(rng.integers(-4, 4, (9, 1)))
+    g = rng.uniform(0.5, 1.5, 256)
+    for eps in (0.0, 1e-6, 0.3):
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(X), (256,), torch.from_numpy(g), eps).numpy()
+        np.testing.assert_allclose(O.rmsnorm(X, g, eps), ref, rtol=1e-13, atol=0)
+
+
+def test_rmsnorm_quant_closed_forms_and_invariances():
+    """A constant row c normalises to sign(c) gamma exactly (eps = 0): with P = I, no clip and
+    gamma = 1 every value is +-1, scale exponent -2, code magnitude 6 (value 4).  Scaling a row by a
+    power of two changes nothing (eps = 0); a zero row with eps > 0 gives zero blocks; rows are
+    independent."""
+    k = 8
+    A, B = np.eye(8), np.tile(np.eye(4), (k, 1, 1))
+    big = np.full(k, 40.0)
+    X = np.full((2, 256), 3.25)
+    X[1] *= -1
+    r = O.rmsnorm_quant_act(X, np.ones(256), 0.0, A, B, big, big)
+    codes = O.unpack_nibbles(r["codes"])
+    assert (r["scales"] == 127 - 2).all()
+    assert (codes[0] == 6).all() and (codes[1] == 14).all()
+    w = WL.custom(6, 256, 16, 52, x_dtype="f32", with_w=False)
+    g = np.random.default_rng(52).uniform(0.5, 1.5, 256)
+    r1 = O.rmsnorm_quant_act(w.x, g, 0.0, w.A, w.B, w.alpha_min, w.alpha_max)
+    r2 = O.rmsnorm_quant_act(w.x * 8.0, g, 0.0, w.A, w.B, w.alpha_min, w.alpha_max)
+    np.testing.assert_array_equal(r1["codes"], r2["codes"])
+    np.testing.assert_array_equal(r1["scales"], r2["scales"])
+    Xz = w.x.copy()
+    Xz[2] = 0.0
+    rz = O.rmsnorm_quant_act(Xz, g, 1e-6, w.A, w.B, w.alpha_min, w.alpha_max)
+    assert (rz["scales"][2] == 0).all() and (rz["codes"][2] == 0).all()
+    np.testing.assert_array_equal(rz["codes"][[0, 1, 3, 4, 5]], O.rmsnorm_quant_act(
+        w.x[[0, 1, 3, 4, 5]], g, 1e-6, w.A, w.B, w.alpha_min, w.alpha_max)["codes"])
