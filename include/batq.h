@@ -341,6 +341,13 @@ BATQ_API batq_status batq_linear_nvfp4(const void* X, batq_dtype x_dtype, int S,
  * BATQ_ERR_SINGULAR as batq_prepare_weights does).
  * ------------------------------------------------------------------------ */
 
+/*
+ * As batq_quant_act (MXFP4 codes, scales in either layout, optional y_debug)
+ * with A_blocks_dev (device, k x 64 floats, A_i row-major at 64 i, 16-byte
+ * aligned) in place of the shared A.  Errors as batq_quant_act;
+ * BATQ_ERR_INVALID_ARG for a NULL A_blocks_dev, BATQ_ERR_ALIGNMENT for a
+ * misaligned one.
+ */
 BATQ_API batq_status batq_quant_act_kron(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
                                 const float* A_blocks_dev, const float* B_dev, const float* ratios_dev,
                                 uint8_t* codes, uint8_t* scales, batq_scale_layout layout, float* y_debug,
@@ -349,12 +356,26 @@ BATQ_API batq_status batq_quant_act_kron(const void* X, batq_dtype x_dtype, int 
 /* Device workspace bytes batq_prepare_weights_kron needs (B'_i and A'_i). Host only. */
 BATQ_API batq_status batq_prepare_weights_kron_workspace_size(int N, size_t* bytes);
 
+/*
+ * As batq_prepare_weights with A_blocks_host (host, k x 64 floats) in place
+ * of A: W'_mat = B_i^-1 W_mat A_i^-T per block, MXFP4 without clip.  The fp64
+ * inverses of every A_i and B_i are formed on the host (BATQ_ERR_SINGULAR if
+ * any is singular or has 1-norm condition number above 1e8) and copied into
+ * `workspace` (batq_prepare_weights_kron_workspace_size bytes, device,
+ * 16-byte aligned) before the quantiser runs.  Other errors as
+ * batq_prepare_weights.
+ */
 BATQ_API batq_status batq_prepare_weights_kron(const void* W, batq_dtype w_dtype, int M, int N, int ldw,
                                       const float* A_blocks_host, const float* B_host, uint8_t* w_codes,
                                       uint8_t* w_scales, batq_scale_layout layout, void* workspace,
                                       size_t workspace_bytes, void* stream);
 
-/* Whole linear with per-block A_i; workspace as batq_linear_workspace_size. */
+/*
+ * Whole linear with per-block A_i: batq_quant_act_kron into the workspace
+ * (batq_linear_workspace_size bytes) followed by the MXFP4 GEMM on the same
+ * stream, with the weights from batq_prepare_weights_kron.  Arguments and
+ * errors otherwise as batq_linear.
+ */
 BATQ_API batq_status batq_linear_kron(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
                              const float* A_blocks_dev, const float* B_dev, const float* ratios_dev,
                              const uint8_t* w_codes, const uint8_t* w_scales, int M, void* workspace,
