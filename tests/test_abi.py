@@ -120,3 +120,64 @@ def test_prepare_checks(L):
     B = np.tile(np.eye(4, dtype=np.float32), (8, 1, 1))
     st = L.batq_prepare_weights(FAKE, 0, 128, 256, 256, A.ctypes.data, B.ctypes.data, FAKE, FAKE, 1, FAKE, 1, None)
     assert st == _lib.BATQ_ERR_WORKSPACE
+
+
+def test_variant_buffer_and_workspace_sizes(L):
+    cb, sb, b = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    # MXFP8: one byte per element, the MXFP4 scale layouts
+    assert L.batq_mxfp8_buffer_sizes(200, 320, 1, ctypes.byref(cb), ctypes.byref(sb)) == 0
+    assert cb.value == 200 * 320 and sb.value == O.mma_layout_bytes(200, 10)
+    # NVFP4: packed codes, one scale per 16 elements (N/16 columns, a multiple of 4)
+    assert L.batq_nvfp4_buffer_sizes(200, 320, 1, ctypes.byref(cb), ctypes.byref(sb)) == 0
+    assert cb.value == 200 * 160 and sb.value == 256 * 20 == O.mma_layout_bytes(200, 20)
+    assert L.batq_nvfp4_buffer_sizes(200, 320, 0, ctypes.byref(cb), ctypes.byref(sb)) == 0
+    assert sb.value == 200 * 20
+    assert L.batq_nvfp4_buffer_sizes(200, 100, 0, ctypes.byref(cb), ctypes.byref(sb)) == _lib.BATQ_ERR_SHAPE
+    base = ctypes.c_size_t()
+    assert L.batq_prepare_workspace_size(4096, ctypes.byref(base)) == 0
+    assert L.batq_prepare_weights_nvfp4_workspace_size(4096, ctypes.byref(b)) == 0 and b.value == base.value + 256
+    assert L.batq_prepare_weights_kron_workspace_size(4096, ctypes.byref(b)) == 0
+    assert b.value == base.value + 128 * 64 * 4
+    assert L.batq_linear_nvfp4_workspace_size(2048, 4096, ctypes.byref(b)) == 0
+    assert b.value == 2048 * 2048 + 2048 * 256
+    assert L.batq_linear_w4a8_workspace_size(2048, 4096, ctypes.byref(b)) == 0
+    assert b.value == 2048 * 4096 + 2048 * 128
+    assert L.batq_prepare_weights_w4a8_workspace_size(4096, 4096, ctypes.byref(b)) == 0
+    assert b.value == base.value + 4096 * 2048
+
+
+def test_variant_argument_checks_fail_before_any_launch(L):
+    A = np.eye(8, dtype=np.float32)
+    B = np.tile(np.eye(4, dtype=np.float32), (8, 1, 1))
+    err = _lib
+    # NVFP4: misaligned per-tensor scale pointers, missing gs output
+    assert L.batq_quant_act_nvfp4(FAKE, 1, 16, 256, 256, A.ctypes.data, FAKE, None, FAKE + 2, FAKE, FAKE, 1, None,
+                                  None) == err.BATQ_ERR_ALIGNMENT
+    assert L.batq_gemm_nvfp4(FAKE, FAKE, FAKE + 1, FAKE, FAKE, None, 16, 128, 256, 0, FAKE, 128,
+                             None) == err.BATQ_ERR_ALIGNMENT
+    assert L.batq_prepare_weights_nvfp4(FAKE, 0, 128, 256, 256, A.ctypes.data, B.ctypes.data, FAKE, FAKE, 1, None,
+                                        FAKE, 1 << 20, None) == err.BATQ_ERR_INVALID_ARG
+    assert L.batq_linear_nvfp4(FAKE, 1, 16, 256, 256, A.ctypes.data, FAKE, None, None, FAKE, FAKE, None, 128, FAKE, 16,
+                               0, FAKE, 128, None) == err.BATQ_ERR_WORKSPACE
+    # KV cache: slot mapping, slot count, format, alignment
+    kv = L.batq_quant_kv_cache
+    assert kv(FAKE, 1, 16, 1024, 1024, A.ctypes.data, FAKE, None, None, 100, 0, FAKE, FAKE,
+              None) == err.BATQ_ERR_INVALID_ARG
+    assert kv(FAKE, 1, 16, 1024, 1024, A.ctypes.data, FAKE, None, FAKE, 0, 0, FAKE, FAKE,
+              None) == err.BATQ_ERR_INVALID_ARG
+    assert kv(FAKE, 1, 16, 1024, 1024, A.ctypes.data, FAKE, None, FAKE, 100, 2, FAKE, FAKE,
+              None) == err.BATQ_ERR_INVALID_ARG
+    assert kv(FAKE, 1, 16, 1024, 1024, A.ctypes.data, FAKE, None, FAKE + 2, 100, 1, FAKE, FAKE,
+              None) == err.BATQ_ERR_ALIGNMENT
+    assert kv(FAKE, 1, 16, 1000, 1024, A.ctypes.data, FAKE, None, FAKE, 100, 1, FAKE, FAKE,
+              None) == err.BATQ_ERR_SHAPE
+    # naive Kronecker: per-block factors required and 16-byte aligned; workspaces checked
+    assert L.batq_quant_act_kron(FAKE, 1, 16, 256, 256, None, FAKE, None, FAKE, FAKE, 1, None,
+                                 None) == err.BATQ_ERR_INVALID_ARG
+    assert L.batq_quant_act_kron(FAKE, 1, 16, 256, 256, FAKE + 4, FAKE, None, FAKE, FAKE, 1, None,
+                                 None) == err.BATQ_ERR_ALIGNMENT
+    Ak = np.tile(np.eye(8, dtype=np.float32), (8, 1, 1))
+    assert L.batq_prepare_weights_kron(FAKE, 0, 128, 256, 256, Ak.ctypes.data, B.ctypes.data, FAKE, FAKE, 1, FAKE,
+                                       64, None) == err.BATQ_ERR_WORKSPACE
+    assert L.batq_linear_kron(FAKE, 1, 16, 256, 256, FAKE, FAKE, None, FAKE, FAKE, 128, FAKE, 16, 0, FAKE, 128,
+                              None) == err.BATQ_ERR_WORKSPACE
