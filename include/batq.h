@@ -64,7 +64,7 @@ extern "C" {
 typedef enum {
   BATQ_OK = 0,
   BATQ_ERR_INVALID_ARG = 1, /* null pointer, bad enum, negative size */
-  BATQ_ERR_SHAPE = 2,       /* N % 64 != 0, S < 1, M % 16 != 0, ld < row length */
+  BATQ_ERR_SHAPE = 2,       /* N % 64 != 0, S < 1, M % 16 != 0, ld < row length, rows x N/32 >= 2^31 */
   BATQ_ERR_ALIGNMENT = 3,   /* a device pointer or row stride not 16-byte aligned */
   BATQ_ERR_SINGULAR = 4,    /* A or some B_i singular / condition number > 1e8 */
   BATQ_ERR_ARCH = 5,        /* current device is not sm_100 */

@@ -55,8 +55,11 @@ size_t scale_bytes_for(int rows, int N, batq_scale_layout layout) {
   return (size_t)rows * k;
 }
 
+// rows x N/32 below 2^31 keeps every tile index, scale offset and scale
+// buffer inside the kernels' 32-bit arithmetic (N = 4096: up to 16.7 M rows).
 batq_status check_mn(int rows, int N) {
   if (rows < 1 || N < 64 || (N % 64) != 0) return BATQ_ERR_SHAPE;
+  if ((long long)rows * (N / 32) >= (1LL << 31)) return BATQ_ERR_SHAPE;
   return BATQ_OK;
 }
 

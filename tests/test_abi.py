@@ -181,3 +181,13 @@ def test_variant_argument_checks_fail_before_any_launch(L):
                                        64, None) == err.BATQ_ERR_WORKSPACE
     assert L.batq_linear_kron(FAKE, 1, 16, 256, 256, FAKE, FAKE, None, FAKE, FAKE, 128, FAKE, 16, 0, FAKE, 128,
                               None) == err.BATQ_ERR_WORKSPACE
+
+
+def test_sizes_beyond_the_32_bit_index_range_are_rejected(L):
+    """rows x N/32 must stay below 2^31 (the kernels' tile indices and scale offsets are 32-bit)."""
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.batq_act_buffer_sizes((1 << 31) // 128 - 1, 4096, 1, ctypes.byref(cb), ctypes.byref(sb)) == 0
+    assert L.batq_act_buffer_sizes((1 << 31) // 128, 4096, 1, ctypes.byref(cb), ctypes.byref(sb)) == _lib.BATQ_ERR_SHAPE
+    A = np.eye(8, dtype=np.float32)
+    assert L.batq_quant_act(FAKE, 1, 1 << 24, 4096, 4096, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, None,
+                            None) == _lib.BATQ_ERR_SHAPE
