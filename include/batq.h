@@ -424,9 +424,18 @@ BATQ_API batq_status batq_quant_kv_cache(const void* X, batq_dtype x_dtype, int 
  * library's own device memory; every GPU that loads the library holds it
  * until the process exits.  Problems whose batq_linear_workspace_size exceeds
  * it return BATQ_ERR_SCRATCH_LIMIT before anything is launched (for N = 4096,
- * up to 7704 tokens fit).  The call allocates nothing.  The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture.  All calls
+ * up to 7704 tokens fit).  The call allocates nothing itself, but CUDA
+ * creates the array on a device when it loads the library's device code there,
+ * which with the default lazy module loading happens at the first call on
+ * that device (or at any earlier libbatq call that ran there).  A process
+ * whose device memory another allocator reserves up front should therefore
+ * make one small, valid batq_linear_no_alloc call on each device before that
+ * allocator reserves the memory (a call refused with BATQ_ERR_SCRATCH_LIMIT
+ * returns before touching the device and does not create it), or set
+ * CUDA_MODULE_LOADING=EAGER so the array is created when the CUDA context is.
+ * The first call on a device also looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls
  * share the one array and it keeps the last call's contents (every byte the
  * GEMM reads is rewritten by each call, so stale contents are never used), so
  * calls that can overlap on the GPU (different streams, or several host

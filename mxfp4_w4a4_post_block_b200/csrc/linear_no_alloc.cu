@@ -10,6 +10,7 @@
 // in the library's own device memory instead.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
@@ -18,25 +19,30 @@
 namespace {
 
 // The scratch array.  Every device that loads this library's module holds it
-// until the process exits.  In host code its name is only a host-side handle,
-// never a device address: the address comes from cudaGetSymbolAddress below.
+// until the process exits.  With CUDA's default lazy module loading the array
+// is created on a device when the module is first used there (at the latest by
+// the address lookup below), so it needs 16 MiB of free device memory at that
+// moment.  In host code its name is only a host-side handle, never a device
+// address: the address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) uint8_t g_linear_scratch[BATQ_NO_ALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
 
 // Device address of the scratch array on the current device, looked up once
-// per device with that device current.
+// per device with that device current.  Host threads may make their first
+// call on a device at the same time: the cache slots are atomics, and two
+// threads that both look the address up store the same value.
 batq_status scratch_address(void** out) {
-  static void* cached[kMaxDevices] = {nullptr};
+  static std::atomic<void*> cached[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BATQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return BATQ_ERR_INVALID_ARG;
-  if (cached[dev] == nullptr) {
-    void* p = nullptr;
+  void* p = cached[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
     if (cudaGetSymbolAddress(&p, g_linear_scratch) != cudaSuccess || p == nullptr) return BATQ_ERR_CUDA;
-    cached[dev] = p;
+    cached[dev].store(p, std::memory_order_release);
   }
-  *out = cached[dev];
+  *out = p;
   return BATQ_OK;
 }
 

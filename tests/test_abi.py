@@ -191,3 +191,21 @@ def test_sizes_beyond_the_32_bit_index_range_are_rejected(L):
     A = np.eye(8, dtype=np.float32)
     assert L.batq_quant_act(FAKE, 1, 1 << 24, 4096, 4096, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, None,
                             None) == _lib.BATQ_ERR_SHAPE
+
+
+def test_no_alloc_scratch_limit_edge(L):
+    """The fixed scratch of batq_linear_no_alloc holds exactly the workspace of 7704 tokens at
+    N = 4096 (codes 7704 x 2048 bytes plus MMA-layout scales 7808 x 128 bytes = 16 MiB); one token
+    more is refused with BATQ_ERR_SCRATCH_LIMIT before any CUDA call, so this runs without a GPU."""
+    ws = ctypes.c_size_t()
+    assert L.batq_linear_workspace_size(7704, 4096, ctypes.byref(ws)) == 0
+    assert ws.value == _lib.NO_ALLOC_SCRATCH_BYTES
+    assert L.batq_linear_workspace_size(7705, 4096, ctypes.byref(ws)) == 0
+    assert ws.value > _lib.NO_ALLOC_SCRATCH_BYTES
+    A = np.eye(8, dtype=np.float32)
+    buf = (ctypes.c_uint8 * 256)()
+    p = (ctypes.addressof(buf) + 15) // 16 * 16  # never dereferenced: the size check comes first
+    st = L.batq_linear_no_alloc(p, _lib.BATQ_BF16, 7705, 4096, 4096, A.ctypes.data, p, p, p, p, 4096,
+                                _lib.BATQ_F32, p, 4096, None)
+    assert st == _lib.BATQ_ERR_SCRATCH_LIMIT
+    assert b"scratch" in L.batq_status_string(st)

@@ -8,17 +8,14 @@ its scratch for the quantised activations from a fixed array inside the
 library instead of a caller workspace.  These tests call it through the C-ABI
 and check that its output matches batq_linear's (which uses a caller-allocated
 workspace) within the GEMM tolerance the other tests use, on two calls in a
-row with different inputs, and that problems too large for the array are
-refused before anything runs.
+row with different inputs.  The refusal of problems too large for the array
+happens before any CUDA call and is tested without a GPU (tests/test_abi.py).
 """
-
-import ctypes
 
 import numpy as np
 import pytest
 import torch
 
-from mxfp4_w4a4_post_block_b200 import _lib
 from mxfp4_w4a4_post_block_b200 import batq as BQ
 from mxfp4_w4a4_post_block_b200 import workloads as WL
 from oracle import batq_oracle as O
@@ -60,13 +57,3 @@ def test_no_alloc_matches_workspace_linear_on_two_calls_in_a_row():
         assert np.all(err <= 1e-4 * T), f"{w.name}: worst {np.max(err / np.maximum(T, 1e-300))}"
         assert np.array_equal(na, ref), f"{w.name}: outputs differ"
 
-
-def test_no_alloc_refuses_problems_larger_than_its_scratch():
-    L = _lib.load()
-    A = np.eye(8, dtype=np.float32)
-    dummy = torch.zeros(64, dtype=torch.uint8, device="cuda")
-    p = dummy.data_ptr()
-    st = L.batq_linear_no_alloc(p, _lib.BATQ_BF16, 7705, 4096, 4096, A.ctypes.data, p, p, p, p, 4096,
-                                _lib.BATQ_F32, p, 4096, None)
-    assert st == _lib.BATQ_ERR_SCRATCH_LIMIT
-    assert b"scratch" in L.batq_status_string(st)
