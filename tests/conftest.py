@@ -17,3 +17,18 @@ def lib():
     """The loaded C-ABI library (GPU tests only)."""
     from mxfp4_w4a4_post_block_b200 import _lib
     return _lib.load()
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With BATQ_PARITY_REPORT set to a path, write the code/scale mismatch counts of every
+    quantiser parity check of the session there (JSON, by check label)."""
+    path = os.environ.get("BATQ_PARITY_REPORT")
+    if not path:
+        return
+    try:
+        import parity
+    except ImportError:
+        return
+    import json
+    with open(path, "w") as f:
+        json.dump(parity.REPORT, f, indent=1, sort_keys=True)

@@ -90,10 +90,19 @@ def exempt_mask(ref, cond=None):
 
 
 def compare_codes(codes_gpu, scales_gpu_linear, ref, cond=None):
-    """Returns dict(mismatch, unexplained, scale_mismatch, scale_unexplained, total)."""
+    """Returns dict(mismatch, unexplained, scale_mismatch, scale_unexplained, outside_literal,
+    scale_outside_literal, total).
+
+    ``unexplained`` counts mismatches outside the band in use (the condition-scaled band when
+    ``cond`` is given); ``outside_literal`` counts mismatching elements outside the literal band
+    of the stated tolerance (pre-rounding q within 1e-5 relative of an E2M1 midpoint, or a block
+    amax within 1e-5 relative of a power of two), whatever band the test uses, so that the
+    widening of that band for values with cancellation stays visible and bounded.
+    """
     cg = O.unpack_nibbles(codes_gpu)
     cr = O.unpack_nibbles(ref["codes"])
     ex, ex_blk = exempt_mask(ref, cond)
+    lit, lit_blk = exempt_mask(ref, None) if cond is not None else (ex, ex_blk)
     diff = cg != cr
     sdiff = np.asarray(scales_gpu_linear) != ref["scales"]
     S, N = cg.shape
@@ -104,14 +113,35 @@ def compare_codes(codes_gpu, scales_gpu_linear, ref, cond=None):
         "unexplained": int((diff_all & ~ex).sum()),
         "scale_mismatch": int(sdiff.sum()),
         "scale_unexplained": int((sdiff & ~ex_blk).sum()),
+        "outside_literal": int((diff_all & ~lit).sum()),
+        "scale_outside_literal": int((sdiff & ~lit_blk).sum()),
         "total": S * N,
     }
 
 
-def assert_quant_parity(codes_gpu, scales_gpu_linear, ref, label="", cond=None):
+# Counts of every assert_quant_parity call of the session, by label (written out by conftest.py
+# when BATQ_PARITY_REPORT names a file).
+REPORT = {}
+
+
+# Mismatches allowed outside the literal 1e-5-of-q band, as a fraction of the elements.  None for
+# the GPK transforms of the workloads (every mismatch there lies within 1e-5 relative of an E2M1
+# midpoint or of a power of two); the block Hadamard as P_i (every entry +-1/sqrt(32), so blocks
+# cancel heavily) moves a few codes whose fp32 error, bounded by the condition scale, crosses a
+# midpoint from further away: 1 of 64,000 and 4 of 2,097,152 elements on the test shapes.
+LITERAL_LIMIT = 0.0
+LITERAL_LIMIT_HADAMARD = 3e-5
+
+
+def assert_quant_parity(codes_gpu, scales_gpu_linear, ref, label="", cond=None, literal_limit=LITERAL_LIMIT):
+    """Codes and scales bit-exact outside the exemption band, exempt mismatches below 1e-4 of the
+    elements, and mismatches outside the literal 1e-5-of-q band at most ``literal_limit`` of them."""
     r = compare_codes(codes_gpu, scales_gpu_linear, ref, cond)
+    REPORT.setdefault(label, []).append(r)
+    print(f"parity {label}: {r}")
     assert r["unexplained"] == 0 and r["scale_unexplained"] == 0, f"{label}: {r}"
     assert r["mismatch"] < 1e-4 * r["total"], f"{label}: too many boundary mismatches {r}"
+    assert r["outside_literal"] <= literal_limit * r["total"], f"{label}: outside the literal band {r}"
     return r
 
 

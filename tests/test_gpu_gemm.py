@@ -44,13 +44,50 @@ def _run(a, sa, w, sw, out_dtype=torch.float32):
     (300, 1024, 768),
     (129, 256, 256),    # smallest CTA-pair path, second CTA nearly empty
     (1000, 1280, 512),  # several pair tiles per cluster row
-    (520, 4096, 256),   # more pair tiles than co-resident clusters
+    (520, 4096, 256),   # 3 x 16 = 48 pair tiles (one per cluster), ragged last row band
+    (2048, 4096, 256),  # 8 x 16 = 128 pair tiles on 74 clusters: 54 clusters run two
 ])
 def test_gemm_random_operands(S, M, N):
     a, sa, w, sw = _random_operands(S, M, N, S * 7 + M + N)
     out = _run(a, sa, w, sw)
     ref, T = O.gemm(a, sa, w, sw)
     PT.assert_gemm_parity(out, ref, T, f"{S}x{M}x{N}")
+
+
+def band_rows(S, seed):
+    """Two rows from every 256-row band of pair tiles, one in each CTA's 128 rows, in 32-row quarters
+    that rotate from band to band (each quarter is drained by its own epilogue warp), and the last
+    row.  With all M columns these rows touch every output tile of the pair GEMM, so every tile of
+    every cluster's persistent sequence, its last tile included, is compared."""
+    rng = np.random.default_rng(seed)
+    rows = [S - 1]
+    for b in range(-(-S // 256)):
+        for half in (0, 1):
+            r = b * 256 + half * 128 + ((b + 2 * half) % 4) * 32 + int(rng.integers(0, 32))
+            if r < S:
+                rows.append(r)
+    return np.unique(np.array(rows, dtype=np.int64))
+
+
+@pytest.mark.parametrize("S,M,N", [
+    (4096, 4096, 12288),   # down_proj: K = 12288 (24 K stages), 16 x 16 = 256 pair tiles (3-4 per cluster)
+    (8192, 12288, 4096),   # layer gate / up: 32 x 48 = 1536 pair tiles (20-21 per cluster)
+    (8192, 1024, 4096),    # layer k / v: 32 x 4 = 128 pair tiles
+    (8192, 4096, 12288),   # layer down: 512 pair tiles, K = 12288
+    (3000, 8192, 128),     # one partial K stage per tile, 12 x 32 = 384 pair tiles, ragged last band
+])
+def test_gemm_large_shapes_every_pair_tile(S, M, N):
+    """The persistent pair GEMM at the prefill shapes of the down_proj and layer workloads (random
+    operands over every code value), compared on rows that touch every pair tile."""
+    a, sa, w, sw = _random_operands(S, M, N, S + 3 * M + 7 * N)
+    k = N // 32
+    out = GU.gpu_gemm(GU.to_dev_u8(a), GU.to_dev_u8(PT.to_mma_layout(sa, S, k)), GU.to_dev_u8(w),
+                      GU.to_dev_u8(PT.to_mma_layout(sw, M, k)), S, M, N)
+    rows = band_rows(S, S + M)
+    got = out[torch.from_numpy(rows).cuda()].cpu().numpy()
+    del out
+    ref, T = O.gemm_rows(a, sa, w, sw, rows)
+    PT.assert_gemm_parity(got, ref, T, f"{S}x{M}x{N}")
 
 
 @pytest.mark.parametrize("S", [16, 200])
@@ -180,8 +217,46 @@ def test_linear_with_block_hadamard_transform():
     lin = O.scales_from_mma_layout(wsc.cpu().numpy(), w.M, w.k)
     PT.assert_quant_parity(wc.cpu().numpy(), lin, {"q": wp["q"], "Y_hat": wp["W_fused"], "codes": wp["codes"],
                                                     "scales": wp["scales"]}, "hadamard weights",
-                           cond=PT.condition_scale_weights(w.W, w.A, w.B))
+                           cond=PT.condition_scale_weights(w.W, w.A, w.B), literal_limit=PT.LITERAL_LIMIT_HADAMARD)
     exact = w.x.astype(np.float64) @ w.W.astype(np.float64).T
     rel_gpu = np.linalg.norm(out.cpu().numpy() - exact) / np.linalg.norm(exact)
     rel_ref = np.linalg.norm(ref - exact) / np.linalg.norm(exact)
     assert abs(rel_gpu - rel_ref) < 2e-3 * rel_ref + 1e-6, (rel_gpu, rel_ref)
+
+
+@pytest.mark.parametrize("maker", [lambda: WL.down_proj(), lambda: WL.layer_linear(1), lambda: WL.layer_linear(4),
+                                   lambda: WL.layer_linear(6)],
+                         ids=["down_proj", "layer_k", "layer_gate", "layer_down"])
+def test_linear_large_end_to_end(maker):
+    """batq_linear at the down_proj shape and three linears of the S = 8192 layer, checked stage by
+    stage against the oracle: the activation codes and scales it left in its workspace on rows that
+    touch every pair tile, the prepared weights on sampled rows, and the GEMM output on the same
+    activation rows and every output column (the oracle's fp64 product of the linear's own codes)."""
+    w = maker()
+    X = GU.x_tensor(w)
+    B, ratios = GU.params(w)
+    wc, wsc = GU.gpu_prepare(w)
+    ws = torch.empty(BQ.batq_linear_workspace_size(w.S, w.N), dtype=torch.uint8, device="cuda")
+    out = torch.empty((w.S, w.M), dtype=torch.float32, device="cuda")
+    BQ.batq_linear(X, w.A, B, ratios, wc, wsc, w.M, ws, out)
+    assert BQ.batq_device_error() == 0
+    rows = band_rows(w.S, w.seed)
+    got = out[torch.from_numpy(rows).cuda()].cpu().numpy()
+    del out, X
+    ws_h = ws.cpu().numpy()
+    ncode = w.S * w.N // 2
+    codes = ws_h[:ncode].reshape(w.S, w.N // 2)
+    off = -(-ncode // 256) * 256
+    a_sc = O.scales_from_mma_layout(ws_h[off:off + O.mma_layout_bytes(w.S, w.k)], w.S, w.k)
+    act = O.quant_act(w.x[rows], w.A, w.B, w.alpha_min, w.alpha_max)
+    PT.assert_quant_parity(codes[rows], a_sc[rows], act, f"{w.name} activations",
+                           cond=PT.condition_scale(w.x[rows], w.A, w.B))
+    wc_h = wc.cpu().numpy()
+    w_sc = O.scales_from_mma_layout(wsc.cpu().numpy(), w.M, w.k)
+    wrows = np.unique(np.concatenate([np.random.default_rng(w.seed).choice(w.M, 48, replace=False), [w.M - 1]]))
+    wp = O.prepare_weights(w.W[wrows], w.A, w.B)
+    PT.assert_quant_parity(wc_h[wrows], w_sc[wrows], {"q": wp["q"], "Y_hat": wp["W_fused"], "codes": wp["codes"],
+                                                      "scales": wp["scales"]}, f"{w.name} weights",
+                           cond=PT.condition_scale_weights(w.W[wrows], w.A, w.B))
+    ref, T = O.gemm_rows(codes, a_sc, wc_h, w_sc, rows)
+    PT.assert_gemm_parity(got, ref, T, f"{w.name} linear")
