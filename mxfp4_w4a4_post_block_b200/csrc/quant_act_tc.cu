@@ -16,19 +16,27 @@
 // token), a tile 128 tokens of a strip; tiles are ordered strip by strip and
 // each CTA (one per SM) takes an equal contiguous share, so it meets at most
 // a few strips and builds each strip's P_i parts once in shared memory (24 KB,
-// 64-byte swizzled K-major rows, as the MMA reads them).
+// 64-byte swizzled K-major rows, as the MMA reads them).  The three parts of
+// one P_i are 96 consecutive rows, so one MMA with N = 96 multiplies the
+// activations by all three at once: per tile and block column two MMAs
+// (M = 128 tokens, N = 96, K = 16) write three 32-column partial results
+// X hi, X mid, X lo side by side in TMEM, and the encoders add them in fp32
+// (hi + (mid + lo)).  That is 8 MMAs per tile where three separate N = 32
+// accumulations took 24, each of which re-read the 4 KB activation slice
+// from shared memory.
 //   warp 0      TMA producer: one 3-D box per tile (128 tokens x 4 blocks of
 //               bf16, 32 KB, 64-byte swizzle = the MMA's K-major operand
 //               layout) into a 4-stage ring;
-//   warp 1      TMEM allocation (512 columns: four 128-column accumulators)
-//               and the MMAs, issued by one elected lane while the whole
-//               warp runs the loop: per tile and block column three parts
-//               x two K steps of M = 128, N = 32, K = 16, then a commit;
+//   warp 1      TMEM allocation (512 columns: one 96-column accumulator per
+//               block column, 128 columns apart) and the MMAs, issued by one
+//               elected lane while the whole warp runs the loop: per tile and
+//               block column two MMAs, then a commit to that column's
+//               accumulator barrier;
 //   warps 2-17  encoders: warp w reads TMEM lane quadrant w % 4 (its 32
-//               tokens) and block column (w - 2) / 4 of the tile with one
-//               tcgen05.ld of 32 columns, releases the accumulator, then
-//               clips, scales, encodes and stores; they also build the P_i
-//               parts at the start of every strip.
+//               tokens) and block column (w - 2) / 4 of the tile with three
+//               tcgen05.ld of 32 columns, releases the accumulator, sums the
+//               parts, then clips, scales, encodes and stores; they also build
+//               the P_i parts of their block column at the start of every strip.
 // Every barrier wait is bounded; on expiry a bit is set in the device error
 // word and the loop ends.
 #include <cuda_bf16.h>
@@ -51,9 +59,9 @@ constexpr int kSlab = kTok * 64;                 // one block column of a tile: 
 constexpr int kXBytes = kCB * kSlab;             // 32 KB
 constexpr int kPPart = 32 * 64;                  // one part of one P_i: 32 output rows x 32 bf16
 constexpr int kPBytes = kCB * kParts * kPPart;   // 24 KB
-constexpr int kAccCols = kCB * 32;               // TMEM columns of one tile's Y
-constexpr int kAccBufs = 4;
-constexpr int kTmemCols = kAccCols * kAccBufs;   // 512 (the 154 KB of shared memory keeps one CTA per SM)
+constexpr int kAccN = kParts * 32;               // MMA N: the three parts' outputs side by side
+constexpr int kAccStride = 128;                  // TMEM columns between block columns' accumulators
+constexpr int kTmemCols = kCB * kAccStride;      // 512 (the 154 KB of shared memory keeps one CTA per SM)
 constexpr int kEncWarps = 4 * kCB;               // one per (TMEM lane quadrant, block column)
 constexpr int kThreads = (2 + kEncWarps) * 32;   // 576
 constexpr int kPOffset = kStages * kXBytes;
@@ -72,7 +80,10 @@ __device__ __forceinline__ double bf16_value(uint32_t bits) {
 // block column cb = tid / 128 of strip s: output element n, input elements
 // 8 jc .. 8 jc + 7, i.e. P[8 jc + a][n] = B_i[jc][n / 8] A[a][n % 8] for a = 0..7
 // (A_i[a][n % 8] with the naive Kronecker decomposition), as one 16-byte chunk
-// per part at its 64-byte-swizzle position.
+// per part at its 64-byte-swizzle position.  With the RMSNorm ahead of the
+// transform (kNorm) row 8 jc + a of P_i is scaled by gamma of that input
+// element, so the MMA computes (x gamma) P_i.
+template <bool kNorm>
 __device__ __forceinline__ void build_p_chunk(uint8_t* sp, int tid, int s, const QuantArgs& p) {
   const int cb = tid >> 7;
   const int n = (tid >> 2) & 31;
@@ -87,7 +98,8 @@ __device__ __forceinline__ void build_p_chunk(uint8_t* sp, int tid, int s, const
     for (int h = 0; h < 2; ++h) {
       const int ai = (a + h) * 8 + (n & 7);
       const float av = p.A_blocks == nullptr ? p.A[ai] : (b < p.k ? p.A_blocks[(size_t)b * 64 + ai] : 0.0f);
-      const double v = bv * (double)av;  // exact in fp64
+      double v = bv * (double)av;  // exact in fp64
+      if constexpr (kNorm) v *= b < p.k ? (double)p.gamma[(size_t)b * 32 + jc * 8 + a + h] : 0.0;
       const uint32_t hi = bf16_bits((float)v);
       const double r1 = v - bf16_value(hi);
       const uint32_t mid = bf16_bits((float)r1);
@@ -106,16 +118,18 @@ __device__ __forceinline__ void build_p_chunk(uint8_t* sp, int tid, int s, const
         make_uint4(w[q][0], w[q][1], w[q][2], w[q][3]);
 }
 
-template <int kFmt>
+// kNorm: RMSNorm ahead of the transform (gamma folded into P_i, the token's
+// 1 / rms from p.row_scale applied to the transformed values).
+template <int kFmt, bool kNorm = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_quant_act_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
   uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
-  uint64_t* acc_empty = acc_full + kAccBufs;
-  uint64_t* p_ready = acc_empty + kAccBufs;
+  uint64_t* acc_full = empty + kStages;   // per block column: its MMAs of the tile completed
+  uint64_t* acc_empty = acc_full + kCB;   // per block column: its four encoder warps read TMEM
+  uint64_t* p_ready = acc_empty + kCB;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(p_ready + 1);
   if (threadIdx.x == 0) tma_prefetch_map(&tmx);
   const int warp = threadIdx.x >> 5;
@@ -128,9 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
 #pragma unroll
-    for (int b = 0; b < kAccBufs; ++b) {
+    for (int b = 0; b < kCB; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kEncWarps);
+      mbar_init(&acc_empty[b], 4);
     }
     mbar_init(p_ready, kEncWarps);
     fence_barrier_init();
@@ -175,11 +189,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ MMA warp ------------------------------
     // The whole warp runs the loop (its state stays warp-uniform) and one
     // elected lane issues the MMAs and their commits.
-    constexpr uint32_t kIdesc = idesc_bf16(kTok, 32);
+    constexpr uint32_t kIdesc = idesc_bf16(kTok, kAccN);
     const uint64_t db = sdesc_kmajor_sw64(smem_u32(smem + kPOffset));
     const bool leader = elect_one();
     uint32_t strip_count = 0;
-    for (int g = 0; g < total; ++g) {
+    bool ok = true;
+    for (int g = 0; g < total && ok; ++g) {
       if (g == 0 || (i0 + g) % tiles_r == 0) {
         // The new strip's P_i parts are in shared memory.
         if (!mbar_wait_warp(p_ready, strip_count & 1)) {
@@ -188,11 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++strip_count;
       }
-      const int st = g % kStages, buf = g % kAccBufs;
-      if (!mbar_wait_warp(&acc_empty[buf], ((g / kAccBufs) & 1) ^ 1)) {
-        if (leader) set_error(p.err, kErrDrainTimeout);
-        break;
-      }
+      const int st = g % kStages;
       if (!mbar_wait_warp(&full[st], (g / kStages) & 1)) {
         if (leader) set_error(p.err, kErrDataTimeout);
         break;
@@ -202,24 +213,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       // field never carries: the descriptor of base + off is the base
       // descriptor + off / 16, one add per operand and MMA.
       const uint64_t da = sdesc_kmajor_sw64(smem_u32(smem + st * kXBytes));
-      const uint32_t tacc = tmem + (uint32_t)(buf * kAccCols);
-      if (leader) {
 #pragma unroll
-        for (int cb = 0; cb < kCB; ++cb) {
-#pragma unroll
-          for (int q = 0; q < kParts; ++q) {
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              // K step kk = bytes 32 kk .. 32 kk + 31 of each 64-byte row
-              tc_mma_bf16(tacc + (uint32_t)(cb * 32), da + (uint64_t)((cb * kSlab + kk * 32) >> 4),
-                          db + (uint64_t)(((cb * kParts + q) * kPPart + kk * 32) >> 4), kIdesc,
-                          (q | kk) ? 1u : 0u);
-            }
-          }
+      for (int cb = 0; cb < kCB; ++cb) {
+        // The block column's accumulator must have been read by its encoders.
+        if (!mbar_wait_warp(&acc_empty[cb], (g & 1) ^ 1)) {
+          if (leader) set_error(p.err, kErrDrainTimeout);
+          ok = false;
+          break;
         }
-        tc_commit(&empty[st]);      // the stage may be refilled once these MMAs have read it
-        tc_commit(&acc_full[buf]);  // and the encoders may read the accumulator
+        tc_fence_after_sync();
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            // K step kk = bytes 32 kk .. 32 kk + 31 of each 64-byte row; B = the
+            // 96 rows of the three parts of this block column's P_i.
+            tc_mma_bf16(tmem + (uint32_t)(cb * kAccStride), da + (uint64_t)((cb * kSlab + kk * 32) >> 4),
+                        db + (uint64_t)((cb * kParts * kPPart + kk * 32) >> 4), kIdesc, kk ? 1u : 0u);
+          }
+          tc_commit(&acc_full[cb]);  // the encoders may read this block column's results
+        }
+        __syncwarp();
       }
+      if (!ok) break;
+      if (leader) tc_commit(&empty[st]);  // the stage may be refilled once these MMAs have read it
       __syncwarp();
     }
   } else {
@@ -241,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g == 0 || t == 0) {
         // Every MMA of the previous strip has completed (this warp saw its
         // last accumulator), so the parts may be overwritten.
-        build_p_chunk(sp, e * 32 + lane, s, p);
+        build_p_chunk<kNorm>(sp, e * 32 + lane, s, p);
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor cores
         __syncwarp();
         if (lane == 0) mbar_arrive(p_ready);
@@ -252,24 +268,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           r_max = p.ratios[2 * b + 1];
         }
       }
-      const int buf = g % kAccBufs;
-      if (!mbar_wait_warp(&acc_full[buf], (g / kAccBufs) & 1)) {
+      if (!mbar_wait_warp(&acc_full[cb], g & 1)) {
         if (lane == 0) set_error(p.err, kErrMmaTimeout);
         break;
       }
       __syncwarp();
       tc_fence_after_sync();
-      uint32_t r[32];
-      tmem_ld_32cols(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(buf * kAccCols + cb * 32), r);
+      // The three partial results X hi, X mid, X lo of this block column,
+      // summed as hi + (mid + lo).
+      const uint32_t tacc = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(cb * kAccStride);
+      uint32_t ra[32], rb[32];
+      tmem_ld_32cols(tacc + 32, ra);
+      tmem_ld_32cols(tacc + 64, rb);
+      tmem_ld_wait();
+      float y[32];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float2 sv = __fadd2_rn(make_float2(__uint_as_float(ra[j]), __uint_as_float(ra[j + 1])),
+                                     make_float2(__uint_as_float(rb[j]), __uint_as_float(rb[j + 1])));
+        y[j] = sv.x;
+        y[j + 1] = sv.y;
+      }
+      tmem_ld_32cols(tacc, ra);
       tmem_ld_wait();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      const int row = t * kTok + 32 * quad + lane;
-      if (b < p.k) {
-        float y[32];
+      if (lane == 0) mbar_arrive(&acc_empty[cb]);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(r[j]);
+      for (int j = 0; j < 32; j += 2) {
+        const float2 sv = __fadd2_rn(make_float2(__uint_as_float(ra[j]), __uint_as_float(ra[j + 1])),
+                                     make_float2(y[j], y[j + 1]));
+        y[j] = sv.x;
+        y[j + 1] = sv.y;
+      }
+      const int row = t * kTok + 32 * quad + lane;
+      if constexpr (kNorm) {
+        const float rs = row < p.S ? p.row_scale[row] : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float2 sv = __fmul2_rn(make_float2(y[j], y[j + 1]), make_float2(rs, rs));
+          y[j] = sv.x;
+          y[j + 1] = sv.y;
+        }
+      }
+      if (b < p.k) {
         encode_block<kFmt>(y, r_min, r_max, gs, row, b, lane, p);
       } else {
         pad_scales<kFmt>(row, b, p);
@@ -285,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kFmt>
+template <int kFmt, bool kNorm = false>
 cudaError_t launch_tc_impl(const QuantLaunch& L, const QuantArgs& a) {
   // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
   CUtensorMap map;
@@ -297,7 +339,7 @@ cudaError_t launch_tc_impl(const QuantLaunch& L, const QuantArgs& a) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_quant_act_tc<kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_quant_act_tc<kFmt, kNorm>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -315,12 +357,16 @@ cudaError_t launch_tc_impl(const QuantLaunch& L, const QuantArgs& a) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_quant_act_tc<kFmt>, map, a);
+  return cudaLaunchKernelEx(&cfg, k_quant_act_tc<kFmt, kNorm>, map, a);
 }
 
 }  // namespace
 
 cudaError_t launch_quant_act_tc(const QuantLaunch& L, const QuantArgs& a) {
+  if (L.gamma != nullptr) {  // RMSNorm ahead of the transform: MXFP4 output, shared A
+    if (L.fmt != kFmtMxfp4 || L.A_blocks != nullptr || L.row_scale == nullptr) return cudaErrorInvalidValue;
+    return launch_tc_impl<kFmtMxfp4, true>(L, a);
+  }
   switch (L.fmt) {
     case kFmtMxfp4: return launch_tc_impl<kFmtMxfp4>(L, a);
     case kFmtMxfp8: return launch_tc_impl<kFmtMxfp8>(L, a);
