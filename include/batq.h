@@ -412,6 +412,53 @@ BATQ_API batq_status batq_quant_kv_cache(const void* X, batq_dtype x_dtype, int 
                                 const int* slot_mapping_dev, int num_slots, batq_kv_format kv_format,
                                 uint8_t* cache_codes, uint8_t* cache_scales, void* stream);
 
+/* ------------------------------------------------------------------------
+ * RMSNorm fused ahead of the activation path (the step before every linear:
+ * BATQuant transforms the activations online before each linear,
+ * thelatestinai.com page, Figure 3 caption; the pages' only kernel design,
+ * ARCQuant's reading notes, section "融合核函数设计", fuses RMSNorm with the
+ * quantisation).  Per token s: z = x_s / sqrt(mean_j x_sj^2 + eps) * gamma,
+ * then y = z P_i, the clip and MXFP4 exactly as batq_quant_act.  z never
+ * leaves the library's kernels and is not rounded to bf16: a first kernel
+ * computes each token's 1 / sqrt(mean x^2 + eps) (sum of squares in fp64,
+ * rounded to fp32 once) into the workspace, and the quantiser applies gamma
+ * to the elements and that factor to the transformed values.
+ * ------------------------------------------------------------------------ */
+
+/* Device workspace bytes batq_rmsnorm_quant_act needs (S floats, rounded up to 256). Host only. */
+BATQ_API batq_status batq_rmsnorm_workspace_size(int S, size_t* bytes);
+
+/*
+ * As batq_quant_act (MXFP4 codes, scales in either layout, optional y_debug:
+ * the transformed values of z) with the RMSNorm ahead of the transform.
+ * gamma_dev: device, N floats, 16-byte aligned; eps: finite, >= 0.
+ * workspace: device, >= batq_rmsnorm_workspace_size(S) bytes, 16-byte
+ * aligned; it receives the per-token factors (the caller owns it).  Errors as
+ * batq_quant_act, plus BATQ_ERR_INVALID_ARG (NULL gamma or workspace, eps
+ * negative or not finite), BATQ_ERR_WORKSPACE, BATQ_ERR_ALIGNMENT.
+ */
+BATQ_API batq_status batq_rmsnorm_quant_act(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                                            const float* gamma_dev, float eps, const float* A_host,
+                                            const float* B_dev, const float* ratios_dev, uint8_t* codes,
+                                            uint8_t* scales, batq_scale_layout layout, void* workspace,
+                                            size_t workspace_bytes, float* y_debug, void* stream);
+
+/* Device workspace bytes batq_rmsnorm_linear needs: batq_linear's plus the per-token factors. Host only. */
+BATQ_API batq_status batq_rmsnorm_linear_workspace_size(int S, int N, size_t* bytes);
+
+/*
+ * Whole linear with the RMSNorm ahead of the transform: batq_rmsnorm_quant_act
+ * into the workspace (codes and MMA scales laid out as for batq_linear, the
+ * per-token factors after them) followed by the MXFP4 GEMM against weights
+ * prepared by batq_prepare_weights, on the same stream.  Arguments and errors
+ * otherwise as batq_linear and batq_rmsnorm_quant_act.
+ */
+BATQ_API batq_status batq_rmsnorm_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx,
+                                         const float* gamma_dev, float eps, const float* A_host,
+                                         const float* B_dev, const float* ratios_dev, const uint8_t* w_codes,
+                                         const uint8_t* w_scales, int M, void* workspace, size_t workspace_bytes,
+                                         batq_dtype out_dtype, void* out, int ldo, void* stream);
+
 /*
  * batq_linear without a caller-provided workspace, for callers that cannot
  * allocate device memory (for example a plugin running in a process whose

@@ -73,6 +73,12 @@ SIGNATURES = {
                                   ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
     "batq_quant_kv_cache": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _c_int, _vp,
                                      _vp, _vp]),
+    "batq_rmsnorm_workspace_size": (_c_int, [_c_int, _c_size_p]),
+    "batq_rmsnorm_quant_act": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, ctypes.c_float, _vp, _vp, _vp,
+                                        _vp, _vp, _c_int, _vp, ctypes.c_size_t, _vp, _vp]),
+    "batq_rmsnorm_linear_workspace_size": (_c_int, [_c_int, _c_int, _c_size_p]),
+    "batq_rmsnorm_linear": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, ctypes.c_float, _vp, _vp, _vp, _vp,
+                                     _vp, _c_int, _vp, ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
     "batq_selftest_wait_timeout": (_c_int, [ctypes.c_uint, _vp]),
     "batq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint)]),
 }

@@ -351,6 +351,45 @@ def batq_quant_kv_cache(X, A, B, ratios, slot_mapping, cache_codes, cache_scales
                                            _stream(stream)), "batq_quant_kv_cache")
 
 
+# ------------------------------------------------- RMSNorm ahead of the transform
+
+def batq_rmsnorm_workspace_size(S: int) -> int:
+    v = ctypes.c_size_t()
+    _check(_lib.load().batq_rmsnorm_workspace_size(S, ctypes.byref(v)), "batq_rmsnorm_workspace_size")
+    return v.value
+
+
+def batq_rmsnorm_linear_workspace_size(S: int, N: int) -> int:
+    v = ctypes.c_size_t()
+    _check(_lib.load().batq_rmsnorm_linear_workspace_size(S, N, ctypes.byref(v)), "batq_rmsnorm_linear_workspace_size")
+    return v.value
+
+
+def batq_rmsnorm_quant_act(X, gamma, eps, A, B, ratios, codes, scales, workspace, layout=BATQ_SCALES_MMA,
+                           y_debug=None, stream=None):
+    """RMSNorm (gamma: CUDA float tensor of N, eps) fused ahead of the transform, clip and MXFP4 of X."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    _check(_lib.load().batq_rmsnorm_quant_act(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0),
+                                              _dev_ptr(gamma, "gamma"), float(eps), a.ctypes.data, _dev_ptr(B, "B"),
+                                              _dev_ptr(ratios, "ratios"), _dev_ptr(codes, "codes"),
+                                              _dev_ptr(scales, "scales"), layout, _dev_ptr(workspace, "workspace"),
+                                              workspace.numel() * workspace.element_size(),
+                                              _dev_ptr(y_debug, "y_debug"), _stream(stream)), "batq_rmsnorm_quant_act")
+
+
+def batq_rmsnorm_linear(X, gamma, eps, A, B, ratios, w_codes, w_scales, M, workspace, out, stream=None):
+    """Whole W4A4 linear with the RMSNorm fused ahead of the online quantisation."""
+    S, N = X.shape
+    a = _host_f32(A, 64, "A")
+    _check(_lib.load().batq_rmsnorm_linear(_dev_ptr(X, "X"), _dtype_code(X), S, N, X.stride(0),
+                                           _dev_ptr(gamma, "gamma"), float(eps), a.ctypes.data, _dev_ptr(B, "B"),
+                                           _dev_ptr(ratios, "ratios"), _dev_ptr(w_codes, "w_codes"),
+                                           _dev_ptr(w_scales, "w_scales"), M, _dev_ptr(workspace, "workspace"),
+                                           workspace.numel() * workspace.element_size(), _dtype_code(out),
+                                           _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_rmsnorm_linear")
+
+
 def batq_selftest_wait_timeout(limit_us: int, stream=None):
     """Launch the bounded-wait self-test kernel (its wait always expires)."""
     _check(_lib.load().batq_selftest_wait_timeout(limit_us, _stream(stream)), "batq_selftest_wait_timeout")

@@ -115,7 +115,8 @@ batq_status launch_quant(const void* X, batq_dtype x_dtype, int S, int N, int ld
                          const float* B_dev, const float* ratios_dev, uint8_t* codes, uint8_t* scales,
                          batq_scale_layout layout, float* y_debug, int fmt, cudaStream_t stream,
                          const float* gs = nullptr, const unsigned* gs_amax = nullptr, float* gs_out = nullptr,
-                         unsigned* amax_out = nullptr, const float* A_blocks = nullptr) {
+                         unsigned* amax_out = nullptr, const float* A_blocks = nullptr,
+                         const float* gamma = nullptr, const float* row_scale = nullptr) {
   batq::QuantLaunch L;
   L.X = X;
   L.bf16 = (x_dtype == BATQ_BF16);
@@ -137,6 +138,8 @@ batq_status launch_quant(const void* X, batq_dtype x_dtype, int S, int N, int ld
   L.gs_out = gs_out;
   L.amax_out = amax_out;
   L.A_blocks = A_blocks;
+  L.gamma = gamma;
+  L.row_scale = row_scale;
   cudaError_t e = batq::launch_quant_act(L);
   if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
   return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
@@ -262,6 +265,27 @@ batq_status fused_transform_kron(const float* A_blocks_host, const float* B_host
                       cudaMemcpyHostToDevice, s) != cudaSuccess)
     return BATQ_ERR_CUDA;
   return BATQ_OK;
+}
+
+size_t rms_bytes_for(int S) { return round_up((size_t)S * sizeof(float), 256); }
+
+// Checks of the RMSNorm arguments beyond the quantiser's own.
+batq_status check_rmsnorm_args(const float* gamma_dev, float eps) {
+  if (!gamma_dev) return BATQ_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return BATQ_ERR_INVALID_ARG;
+  if (!aligned16(gamma_dev)) return BATQ_ERR_ALIGNMENT;
+  return BATQ_OK;
+}
+
+// RMSNorm factors of every token into rms (device, S floats), then the
+// quantiser with gamma and those factors, on one stream.
+batq_status launch_rmsnorm_quant(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* gamma_dev,
+                                 float eps, const float* A_host, const float* B_dev, const float* ratios_dev,
+                                 uint8_t* codes, uint8_t* scales, batq_scale_layout layout, float* rms,
+                                 float* y_debug, cudaStream_t s) {
+  if (batq::launch_row_rms(X, x_dtype == BATQ_BF16, S, N, ldx, eps, rms, s) != cudaSuccess) return BATQ_ERR_CUDA;
+  return launch_quant(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout, y_debug,
+                      batq::kFmtMxfp4, s, nullptr, nullptr, nullptr, nullptr, nullptr, gamma_dev, rms);
 }
 
 }  // namespace
@@ -750,6 +774,78 @@ batq_status batq_device_error(void* stream, unsigned int* flags_out) {
   }
   *flags_out = v;
   return v ? BATQ_ERR_TIMEOUT : BATQ_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------ RMSNorm ahead of the transform
+
+extern "C" {
+
+batq_status batq_rmsnorm_workspace_size(int S, size_t* bytes) {
+  if (!bytes) return BATQ_ERR_INVALID_ARG;
+  if (S < 1) return BATQ_ERR_SHAPE;
+  *bytes = rms_bytes_for(S);
+  return BATQ_OK;
+}
+
+batq_status batq_rmsnorm_quant_act(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* gamma_dev,
+                                   float eps, const float* A_host, const float* B_dev, const float* ratios_dev,
+                                   uint8_t* codes, uint8_t* scales, batq_scale_layout layout, void* workspace,
+                                   size_t workspace_bytes, float* y_debug, void* stream) {
+  batq_status st = check_quant_args(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, codes, scales, layout,
+                                    y_debug);
+  if (st != BATQ_OK) return st;
+  st = check_rmsnorm_args(gamma_dev, eps);
+  if (st != BATQ_OK) return st;
+  if (!workspace) return BATQ_ERR_INVALID_ARG;
+  if (workspace_bytes < rms_bytes_for(S)) return BATQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BATQ_ERR_ALIGNMENT;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  return launch_rmsnorm_quant(X, x_dtype, S, N, ldx, gamma_dev, eps, A_host, B_dev, ratios_dev, codes, scales,
+                              layout, static_cast<float*>(workspace), y_debug, static_cast<cudaStream_t>(stream));
+}
+
+batq_status batq_rmsnorm_linear_workspace_size(int S, int N, size_t* bytes) {
+  if (!bytes) return BATQ_ERR_INVALID_ARG;
+  size_t lin = 0;
+  batq_status st = batq_linear_workspace_size(S, N, &lin);
+  if (st != BATQ_OK) return st;
+  *bytes = round_up(lin, 256) + rms_bytes_for(S);
+  return BATQ_OK;
+}
+
+batq_status batq_rmsnorm_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx, const float* gamma_dev,
+                                float eps, const float* A_host, const float* B_dev, const float* ratios_dev,
+                                const uint8_t* w_codes, const uint8_t* w_scales, int M, void* workspace,
+                                size_t workspace_bytes, batq_dtype out_dtype, void* out, int ldo, void* stream) {
+  if (!workspace) return BATQ_ERR_INVALID_ARG;
+  size_t need = 0, lin = 0;
+  batq_status st = batq_rmsnorm_linear_workspace_size(S, N, &need);
+  if (st != BATQ_OK) return st;
+  batq_linear_workspace_size(S, N, &lin);
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BATQ_ERR_ALIGNMENT;
+  uint8_t* a_codes = static_cast<uint8_t*>(workspace);
+  uint8_t* a_scales = a_codes + round_up((size_t)S * (N / 2), 256);
+  float* rms = reinterpret_cast<float*>(a_codes + round_up(lin, 256));
+  st = check_quant_args(X, x_dtype, S, N, ldx, A_host, B_dev, ratios_dev, a_codes, a_scales, BATQ_SCALES_MMA,
+                        nullptr);
+  if (st != BATQ_OK) return st;
+  st = check_rmsnorm_args(gamma_dev, eps);
+  if (st != BATQ_OK) return st;
+  st = check_gemm_args(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo);
+  if (st != BATQ_OK) return st;
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_rmsnorm_quant(X, x_dtype, S, N, ldx, gamma_dev, eps, A_host, B_dev, ratios_dev, a_codes, a_scales,
+                            BATQ_SCALES_MMA, rms, nullptr, s);
+  if (st != BATQ_OK) return st;
+  // As in batq_linear: the quantiser writes only the workspace, so the GEMM
+  // may fetch weights while it runs.
+  return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, batq::kFmtMxfp4, s);
 }
 
 }  // extern "C"

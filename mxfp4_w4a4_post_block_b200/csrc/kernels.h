@@ -44,6 +44,12 @@ struct QuantLaunch {
   // Naive Kronecker decomposition: one 8x8 A_i per block (device, k x 64
   // floats, 16-byte aligned) replaces A; MXFP4 output only.
   const float* A_blocks = nullptr;
+  // RMSNorm ahead of the transform (both set or both null): gamma (device, N
+  // floats, 16-byte aligned) scales element j of every token before the
+  // transform, row_scale (device, S floats: 1 / rms of each token, from
+  // launch_row_rms) scales the transformed values of the token.
+  const float* gamma = nullptr;
+  const float* row_scale = nullptr;
 };
 
 // Returns cudaErrorInvalidValue when the tensor map cannot be encoded.
@@ -86,6 +92,11 @@ cudaError_t launch_gemm_pair(const GemmLaunch& L);
 // element holding the same value; packed_bytes must be a multiple of 16 and
 // both pointers 16-byte aligned.
 cudaError_t launch_e2m1_to_e4m3(const uint8_t* packed, uint8_t* out, size_t packed_bytes, cudaStream_t stream);
+
+// r_out[s] = fp32(1 / sqrt(sum_j x_sj^2 / N + eps)) for every token s (sum in
+// fp64); X as for the quantisers (16-byte aligned rows).
+cudaError_t launch_row_rms(const void* X, bool bf16, int S, int N, int ldx, float eps, float* r_out,
+                           cudaStream_t stream);
 
 // One-thread kernel whose barrier wait always expires after limit_ns.
 cudaError_t launch_wait_selftest(uint64_t limit_ns, unsigned* err, cudaStream_t stream);

@@ -48,8 +48,9 @@ namespace {
 constexpr int kRows = 32;         // tokens per tile (one per lane)
 constexpr int kCols = 8;          // 32-blocks per tile (one per warp of a consumer group)
 
-// kNaive: one A_i per block column, staged with the tile (naive Kronecker).
-template <bool kBF16, bool kNaive = false>
+// kNaive: one A_i per block column, staged with the tile (naive Kronecker);
+// kNorm: the RMSNorm gamma of the tile's block columns staged too.
+template <bool kBF16, bool kNaive = false, bool kNorm = false>
 struct Tile {
   static constexpr int kGroups = kBF16 ? 3 : 1;          // consumer groups per CTA
   static constexpr int kStages = kGroups * (kBF16 ? 3 : 4);  // ring depth (a multiple of kGroups)
@@ -61,7 +62,8 @@ struct Tile {
   static constexpr int kBOffset = kXBytes;                  // kCols x 16 fp32 B_i
   static constexpr int kROffset = kXBytes + kCols * 64;     // kCols x 2 fp32 clip ratios
   static constexpr int kAOffset = kROffset + kCols * 8;     // kCols x 64 fp32 A_i (naive Kronecker)
-  static constexpr int kStageBytes = (kAOffset + (kNaive ? kCols * 256 : 0) + 1023) / 1024 * 1024;
+  static constexpr int kGOffset = kAOffset + (kNaive ? kCols * 256 : 0);  // kCols x 32 fp32 RMSNorm gamma
+  static constexpr int kStageBytes = (kGOffset + (kNorm ? kCols * 128 : 0) + 1023) / 1024 * 1024;
   static constexpr int kSmemBytes = kStages * kStageBytes + 2 * kStages * 8 + 16 + 1024;
 };
 
@@ -97,11 +99,12 @@ __device__ __forceinline__ void load_block(uint32_t box, int lane, float x[32]) 
   }
 }
 
-// kFmt: output format (Fmt); kNaive: per-block A_i from p.A_blocks.
-template <bool kBF16, int kFmt, bool kNaive>
-__global__ void __launch_bounds__(Tile<kBF16, kNaive>::kThreads, 1)
+// kFmt: output format (Fmt); kNaive: per-block A_i from p.A_blocks; kNorm:
+// RMSNorm ahead of the transform (p.gamma and p.row_scale).
+template <bool kBF16, int kFmt, bool kNaive, bool kNorm = false>
+__global__ void __launch_bounds__(Tile<kBF16, kNaive, kNorm>::kThreads, 1)
     k_quant_act(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
-  using T = Tile<kBF16, kNaive>;
+  using T = Tile<kBF16, kNaive, kNorm>;
   constexpr bool kNv = (kFmt == kFmtNvfp4);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -164,13 +167,14 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive>::kThreads, 1)
           const int nb = min(kCols, p.k - c0);  // even: k is even and c0 a multiple of 8
           uint8_t* dst = smem + s * T::kStageBytes;
           const uint32_t pbytes = (uint32_t)nb * 64u + (p.ratios != nullptr ? (uint32_t)nb * 8u : 0u) +
-                                  (kNaive ? (uint32_t)nb * 256u : 0u);
+                                  (kNaive ? (uint32_t)nb * 256u : 0u) + (kNorm ? (uint32_t)nb * 128u : 0u);
           // the box always delivers all 8 block columns (zero-filled past k)
           mbar_arrive_expect_tx(&full[s], (uint32_t)T::kXBytes + pbytes);
           tma_load_3d(dst, &tmx, &full[s], 0, r0, c0);
           bulk_load(dst + T::kBOffset, p.B + (size_t)c0 * 16, (uint32_t)nb * 64u, &full[s]);
           if (p.ratios != nullptr) bulk_load(dst + T::kROffset, p.ratios + (size_t)c0 * 2, (uint32_t)nb * 8u, &full[s]);
           if constexpr (kNaive) bulk_load(dst + T::kAOffset, p.A_blocks + (size_t)c0 * 64, (uint32_t)nb * 256u, &full[s]);
+          if constexpr (kNorm) bulk_load(dst + T::kGOffset, p.gamma + (size_t)c0 * 32, (uint32_t)nb * 128u, &full[s]);
         } else {
           mbar_arrive(&full[s]);  // padding rows only: nothing to load
         }
@@ -180,6 +184,9 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive>::kThreads, 1)
   }
 
   // ---------------- consumers ----------------
+  // The RMSNorm factors come from the preceding grid (launch_row_rms); the
+  // consumers read them directly, so they too wait for that grid.
+  if constexpr (kNorm) griddep_wait();
   const int grp = warp / kCols;
   const int wc = warp % kCols;  // block column of the tile owned by this warp
   for (int i = grp; i < nloc; i += T::kGroups) {
@@ -198,6 +205,22 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive>::kThreads, 1)
       const uint32_t st = smem_u32(smem) + s * T::kStageBytes;
       float x[32];
       load_block<kBF16>(st + wc * T::kBoxBytes, lane, x);
+      if constexpr (kNorm) {
+        // RMSNorm: x gamma (the block's 32 gamma values are the same for the whole warp)
+        const uint32_t gp = st + T::kGOffset + wc * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 gv = lds128(gp + c * 16);
+          const float2 g01 = __fmul2_rn(make_float2(x[4 * c], x[4 * c + 1]),
+                                        make_float2(__uint_as_float(gv.x), __uint_as_float(gv.y)));
+          const float2 g23 = __fmul2_rn(make_float2(x[4 * c + 2], x[4 * c + 3]),
+                                        make_float2(__uint_as_float(gv.z), __uint_as_float(gv.w)));
+          x[4 * c] = g01.x;
+          x[4 * c + 1] = g01.y;
+          x[4 * c + 2] = g23.x;
+          x[4 * c + 3] = g23.y;
+        }
+      }
 
       // B_i (row-major 4x4) and the clip ratios: the same for the whole warp.
       const uint32_t bp = st + T::kBOffset + wc * 64;
@@ -246,6 +269,12 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive>::kThreads, 1)
           y2[4 * c + j] = acc;
         }
       }
+      if constexpr (kNorm) {
+        // RMSNorm: the token's 1 / rms times the transformed values
+        const float rs = p.row_scale[row];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y2[i] = __fmul2_rn(y2[i], make_float2(rs, rs));
+      }
       float y[32];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -284,6 +313,8 @@ QuantArgs make_args(const QuantLaunch& L) {
   a.row_map = L.row_map;
   a.rows_cap = L.row_map != nullptr ? L.num_slots : L.S;
   a.A_blocks = L.A_blocks;
+  a.gamma = L.gamma;
+  a.row_scale = L.row_scale;
   a.rows_out = a.mma_layout ? (L.S + 127) / 128 * 128 : L.S;
   a.tiles_r = (a.rows_out + kRows - 1) / kRows;
   a.tiles_c = (a.k + kCols - 1) / kCols;
@@ -291,9 +322,9 @@ QuantArgs make_args(const QuantLaunch& L) {
   return a;
 }
 
-template <bool kBF16, int kFmt, bool kNaive = false>
+template <bool kBF16, int kFmt, bool kNaive = false, bool kNorm = false>
 cudaError_t launch_impl(const QuantLaunch& L, const QuantArgs& a) {
-  using T = Tile<kBF16, kNaive>;
+  using T = Tile<kBF16, kNaive, kNorm>;
   // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
   CUtensorMap map;
   const uint64_t esz = kBF16 ? 2u : 4u;
@@ -306,7 +337,7 @@ cudaError_t launch_impl(const QuantLaunch& L, const QuantArgs& a) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16, kFmt, kNaive>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16, kFmt, kNaive, kNorm>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          T::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -323,7 +354,7 @@ cudaError_t launch_impl(const QuantLaunch& L, const QuantArgs& a) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16, kFmt, kNaive>, map, a);
+  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16, kFmt, kNaive, kNorm>, map, a);
 }
 
 }  // namespace
@@ -337,6 +368,10 @@ cudaError_t launch_quant_act(const QuantLaunch& L) {
   // CUDA-core kernel above.
   const long long tc_tiles = (long long)((a.k + 3) / 4) * ((L.S + 127) / 128);
   if (L.bf16 && tc_tiles >= 6LL * sm_count()) return launch_quant_act_tc(L, a);
+  if (L.gamma != nullptr) {  // RMSNorm ahead of the transform: MXFP4 output, shared A
+    if (L.fmt != kFmtMxfp4 || L.A_blocks != nullptr || L.row_scale == nullptr) return cudaErrorInvalidValue;
+    return L.bf16 ? launch_impl<true, kFmtMxfp4, false, true>(L, a) : launch_impl<false, kFmtMxfp4, false, true>(L, a);
+  }
   if (L.A_blocks != nullptr) {  // naive Kronecker: MXFP4 output
     if (L.fmt != kFmtMxfp4) return cudaErrorInvalidValue;
     return L.bf16 ? launch_impl<true, kFmtMxfp4, true>(L, a) : launch_impl<false, kFmtMxfp4, true>(L, a);

@@ -42,6 +42,10 @@ struct QuantArgs {
   int rows_cap;
   // Naive Kronecker: one 8x8 A_i per block (device, k x 64 floats) instead of A.
   const float* A_blocks;
+  // RMSNorm ahead of the transform (both null without it): per-element gamma
+  // (N floats) and per-token 1 / rms (S floats).
+  const float* gamma;
+  const float* row_scale;
 };
 
 __device__ __forceinline__ int tile_row(int t, const QuantArgs& p) {

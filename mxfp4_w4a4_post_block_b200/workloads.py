@@ -30,6 +30,8 @@ Recipes (numpy ``default_rng(seed)``, drawn in the order listed):
 * ``with_naive_kronecker(w, seed)``: w's inputs with one A_i = I + 0.1 N per block.
 * ``with_block_hadamard(w)``: w's X and W with P_i = H_32 / sqrt(32) (Sylvester) for every
   block and no clip, the block-rotation baseline as an input.
+* ``rmsnorm_gamma(N, seed)``: RMSNorm weights 1 + 0.2 N(0, 1) for the fused norm ahead of the
+  transform (eps = 1e-6 in the tests).
 """
 
 from __future__ import annotations
@@ -217,6 +219,13 @@ def with_naive_kronecker(w: Workload, seed: int = 0, sigma: float = 0.1) -> Work
     rng = np.random.default_rng(seed)
     A = _near_identity(rng, (k, 8, 8), sigma)
     return dataclasses.replace(w, name=w.name + "_naivekron", A=A)
+
+
+def rmsnorm_gamma(N: int, seed: int) -> np.ndarray:
+    """RMSNorm weights for the fused norm ahead of the transform: fp32 (N,), 1 + 0.2 N(0, 1) from
+    default_rng(seed) (the norm weight of a trained layer sits around 1; the pages give no values)."""
+    rng = np.random.default_rng(seed)
+    return (1.0 + 0.2 * rng.standard_normal(N)).astype(np.float32)
 
 
 CONFIGS = {

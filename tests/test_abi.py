@@ -183,6 +183,41 @@ def test_variant_argument_checks_fail_before_any_launch(L):
                               None) == err.BATQ_ERR_WORKSPACE
 
 
+def test_rmsnorm_sizes_and_argument_checks_fail_before_any_launch(L):
+    """The fused RMSNorm calls: workspace sizes, and every argument error reported on the host
+    before anything is launched (no GPU needed)."""
+    v = ctypes.c_size_t()
+    assert L.batq_rmsnorm_workspace_size(1000, ctypes.byref(v)) == 0 and v.value == 4096
+    assert L.batq_rmsnorm_workspace_size(0, ctypes.byref(v)) == _lib.BATQ_ERR_SHAPE
+    lin = ctypes.c_size_t()
+    assert L.batq_linear_workspace_size(2048, 4096, ctypes.byref(lin)) == 0
+    assert L.batq_rmsnorm_linear_workspace_size(2048, 4096, ctypes.byref(v)) == 0
+    assert v.value == -(-lin.value // 256) * 256 + 8192
+    A = np.eye(8, dtype=np.float32)
+    q = L.batq_rmsnorm_quant_act
+    # null gamma, negative or non-finite eps, null workspace
+    assert q(FAKE, 1, 16, 256, 256, None, 1e-6, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, FAKE, 256, None,
+             None) == _lib.BATQ_ERR_INVALID_ARG
+    assert q(FAKE, 1, 16, 256, 256, FAKE, -1.0, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, FAKE, 256, None,
+             None) == _lib.BATQ_ERR_INVALID_ARG
+    assert q(FAKE, 1, 16, 256, 256, FAKE, float("nan"), A.ctypes.data, FAKE, None, FAKE, FAKE, 1, FAKE, 256, None,
+             None) == _lib.BATQ_ERR_INVALID_ARG
+    assert q(FAKE, 1, 16, 256, 256, FAKE, 1e-6, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, None, 256, None,
+             None) == _lib.BATQ_ERR_INVALID_ARG
+    # misaligned gamma, short workspace, bad shape
+    assert q(FAKE, 1, 16, 256, 256, FAKE + 4, 1e-6, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, FAKE, 256, None,
+             None) == _lib.BATQ_ERR_ALIGNMENT
+    assert q(FAKE, 1, 16, 256, 256, FAKE, 1e-6, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, FAKE, 16, None,
+             None) == _lib.BATQ_ERR_WORKSPACE
+    assert q(FAKE, 1, 16, 100, 256, FAKE, 1e-6, A.ctypes.data, FAKE, None, FAKE, FAKE, 1, FAKE, 256, None,
+             None) == _lib.BATQ_ERR_SHAPE
+    lr = L.batq_rmsnorm_linear
+    assert lr(FAKE, 1, 16, 256, 256, FAKE, 1e-6, A.ctypes.data, FAKE, None, FAKE, FAKE, 128, FAKE, 64, 0, FAKE, 128,
+              None) == _lib.BATQ_ERR_WORKSPACE
+    assert lr(FAKE, 1, 16, 256, 256, None, 1e-6, A.ctypes.data, FAKE, None, FAKE, FAKE, 128, FAKE, 1 << 20, 0, FAKE,
+              128, None) == _lib.BATQ_ERR_INVALID_ARG
+
+
 def test_sizes_beyond_the_32_bit_index_range_are_rejected(L):
     """rows x N/32 must stay below 2^31 (the kernels' tile indices and scale offsets are 32-bit)."""
     cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
