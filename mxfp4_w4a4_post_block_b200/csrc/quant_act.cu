@@ -236,38 +236,15 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive, kNorm>::kThreads, 1)
         r_max = r.y;
       }
 
-      // T = X A  (X is the row-major 4x8 view of the block): column pairs
-      // (T[r][2j], T[r][2j+1]) += (x[r][a], x[r][a]) * (A[a][2j], A[a][2j+1]).
-      float2 tm[16];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-          for (int a = 0; a < 8; ++a) {
-            const float xv = x[8 * r + a];
-            const float2 ap = kNaive ? lds64f(st + T::kAOffset + wc * 256 + (8 * a + 2 * j) * 4)
-                                     : make_float2(p.A[8 * a + 2 * j], p.A[8 * a + 2 * j + 1]);
-            acc = __ffma2_rn(make_float2(xv, xv), ap, acc);
-          }
-          tm[4 * r + j] = acc;
-        }
-      }
-      // Y = B^T T: (Y[c][2j], Y[c][2j+1]) += (B[r][c], B[r][c]) * (T[r][2j], T[r][2j+1]).
+      // Y = B^T X A (X is the row-major 4x8 view of the block), from A (the
+      // parameter bank) or the staged A_i (naive Kronecker).
       float2 y2[16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const float bv = Bm[4 * r + c];
-            acc = __ffma2_rn(make_float2(bv, bv), tm[4 * r + j], acc);
-          }
-          y2[4 * c + j] = acc;
-        }
+      if constexpr (kNaive) {
+        const uint32_t ap = st + T::kAOffset + wc * 256;
+        gpk_transform(x, [&](int a, int j) { return lds64f(ap + (8 * a + 2 * j) * 4); }, Bm, y2);
+      } else {
+        gpk_transform(x, [&](int a, int j) { return make_float2(p.A[8 * a + 2 * j], p.A[8 * a + 2 * j + 1]); }, Bm,
+                      y2);
       }
       if constexpr (kNorm) {
         // RMSNorm: the token's 1 / rms times the transformed values

@@ -67,6 +67,46 @@ __device__ __forceinline__ float2 lds64f(uint32_t addr) {
   return v;
 }
 
+// The GPK block transform of one token's block on CUDA cores (daily-arxiv
+// summary, "GPK 分解": y = x (B_i (x) A), computed as Y = B_i^T X A with X the
+// row-major 4 x 8 view of x).  T = X A produces column pairs (T[r][2j],
+// T[r][2j+1]) from a duplicated x value and an A row pair, then Y = B^T T
+// reuses those column pairs with a duplicated B entry: 192 packed fp32x2 FMAs
+// per block, accumulated in the order a = 0..7, then r = 0..3.  a_pair(a, j)
+// returns (A[a][2j], A[a][2j + 1]); Bm is B_i row-major.  y2[4 c + j] holds
+// (Y[c][2j], Y[c][2j + 1]).
+template <typename APair>
+__device__ __forceinline__ void gpk_transform(const float (&x)[32], APair a_pair, const float (&Bm)[16],
+                                              float2 (&y2)[16]) {
+  float2 tm[16];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        const float xv = x[8 * r + a];
+        acc = __ffma2_rn(make_float2(xv, xv), a_pair(a, j), acc);
+      }
+      tm[4 * r + j] = acc;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float bv = Bm[4 * r + c];
+        acc = __ffma2_rn(make_float2(bv, bv), tm[4 * r + j], acc);
+      }
+      y2[4 * c + j] = acc;
+    }
+  }
+}
+
 // NVFP4 per-tensor encode scale: 448 * 6 / amax from the measured amax word if
 // given, else the device float, else 1.  Read only after the preceding grid
 // has completed (griddepcontrol.wait).
