@@ -51,8 +51,8 @@ CSRC = os.path.join(ROOT, "mxfp4_w4a4_post_block_b200", "csrc")
 # of `bench.py --only linear --workload layer` (metrics dram__bytes_read.sum, dram__bytes_write.sum),
 # valid only for the kernel sources whose hash is recorded with it: a changed kernel reports null.
 NCU_TRAFFIC = {
-    "k_gemm_pair": {"src": None, "bytes_per_step": None},
-    "k_quant_act_tc": {"src": None, "bytes_per_step": None},
+    "k_gemm_pair": {"src": "dd1feeb072a8e1c3", "bytes_per_step": 357677568 + 929853184},
+    "k_quant_act_tc": {"src": "dbf676ececd9235d", "bytes_per_step": 604858368 + 34938880},
 }
 TRAFFIC_SOURCES = {
     "k_gemm_pair": ("gemm_pair.cu", "ptx.cuh", "kernels.h", "host_util.h", "host_util.cpp"),
@@ -342,6 +342,25 @@ class Timer:
             f()
         return statistics.median(self.once(fns, reps, kernels_per_fn) for _ in range(repeats))
 
+    def each(self, fns, repeats=REPEATS):
+        """ms of each of fns within one back-to-back pass over all of them (events between the
+        launches), median over `repeats` passes."""
+        import torch
+        for f in fns:
+            f()
+        per = [[] for _ in fns]
+        for _ in range(repeats):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+            ev[0].record(self.stream)
+            for i, f in enumerate(fns):
+                f()
+                ev[i + 1].record(self.stream)
+            torch.cuda.synchronize()
+            for i in range(len(fns)):
+                per[i].append(ev[i].elapsed_time(ev[i + 1]))
+            self.launches += len(fns)
+        return [statistics.median(p) for p in per]
+
 
 def per_config(dev, peaks, timer, sp):
     """The other workloads, each timed as the median of five repeats of back-to-back launches whose
@@ -591,8 +610,8 @@ def run_batq(args):
         # (-> per-kernel throughput and roofline)
         q_ms = timer.median([launcher("quant", z, sp) for z in layer])
         g_ms = timer.median([launcher("gemm", z, sp) for z in layer])
-        q_each = [timer.median([launcher("quant", z, sp)]) for z in layer]
-        g_each = [timer.median([launcher("gemm", z, sp)]) for z in layer]
+        q_each = timer.each([launcher("quant", z, sp) for z in layer])
+        g_each = timer.each([launcher("gemm", z, sp) for z in layer])
     if ws > 1:
         dist.barrier()
     local_ms, q_ms, g_ms = max_over_ranks([local_ms, q_ms, g_ms], device=dev)
