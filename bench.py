@@ -47,12 +47,12 @@ FP4_NOMINAL_OVER_BF16 = 9.0 / 2.25         # dense fp4 / dense bf16 nominal rati
 REPEATS = 5                                # every per-kernel loop: median of this many repeats
 CSRC = os.path.join(ROOT, "mxfp4_w4a4_post_block_b200", "csrc")
 
-# DRAM bytes (read + write) of one layer step's seven launches of each kernel, from an ncu capture
-# of `bench.py --only linear --workload layer` (metrics dram__bytes_read.sum, dram__bytes_write.sum),
+# DRAM bytes (read + write) of one layer step's launch of each grouped kernel, from an ncu capture of
+# `bench.py --only group --workload layer` (metrics dram__bytes_read.sum, dram__bytes_write.sum),
 # valid only for the kernel sources whose hash is recorded with it: a changed kernel reports null.
 NCU_TRAFFIC = {
-    "k_gemm_pair": {"src": "dd1feeb072a8e1c3", "bytes_per_step": 357677568 + 929853184},
-    "k_quant_act_tc": {"src": "dbf676ececd9235d", "bytes_per_step": 604858368 + 34938880},
+    "k_gemm_pair": {"src": "68b3d42aeabb992e", "bytes_per_step": 375082496 + 1235126272},
+    "k_quant_act_tc": {"src": "d2f8de9014034f80", "bytes_per_step": 605602048 + 142997760},
 }
 TRAFFIC_SOURCES = {
     "k_gemm_pair": ("gemm_pair.cu", "ptx.cuh", "kernels.h", "host_util.h", "host_util.cpp"),
@@ -61,11 +61,20 @@ TRAFFIC_SOURCES = {
 }
 
 
+def _code_only(text):
+    """Source text without C/C++ comments and whitespace runs, so that a comment edit does not mark a
+    recorded capture stale (the compiled kernel is the same)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_hash(kernel):
     h = hashlib.sha256()
     for f in TRAFFIC_SOURCES[kernel]:
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -547,7 +556,15 @@ def run_only(args):
         for z in sets:
             launcher("quant", z, sp)()
     torch.cuda.synchronize()
+    if args.only == "group":
+        group = [dict(X=z["X"], A=z["A"], B=z["B"], ratios=z["ratios"], w_codes=z["wc"], w_scales=z["wsc"],
+                      M=z["M"], out=z["out"]) for z in sets]
+        gws = torch.empty(BQ.batq_linear_grouped_workspace_size([(z["S"], z["N"]) for z in sets]),
+                          dtype=torch.uint8, device=dev)
     for _ in range(args.launches):
+        if args.only == "group":
+            BQ.batq_linear_grouped(group, gws, stream=sp)
+            continue
         for z in sets:
             launcher(args.only, z, sp)()
     torch.cuda.synchronize()
@@ -581,15 +598,30 @@ def run_batq(args):
     layer = [linear_set(w, dev) for w in workloads]
     flops = sum(2.0 * z["S"] * z["N"] * z["M"] for z in layer)
     qbytes = sum(z["S"] * z["N"] * QUANT_BYTES_PER_ELEM for z in layer)
-    step_fns = [launcher("linear", z, sp) for z in layer]
+    # One step: the seven independent linears through batq_linear_grouped (one quantiser launch over
+    # all activations, one CTA-pair GEMM launch over all products).  For comparison the same step as
+    # seven batq_linear calls.
+    group = [dict(X=z["X"], A=z["A"], B=z["B"], ratios=z["ratios"], w_codes=z["wc"], w_scales=z["wsc"], M=z["M"],
+                  out=z["out"]) for z in layer]
+    gws = torch.empty(BQ.batq_linear_grouped_workspace_size([(z["S"], z["N"]) for z in layer]), dtype=torch.uint8,
+                      device=dev)
+    quant_group = [dict(X=z["X"], A=z["A"], B=z["B"], ratios=z["ratios"], codes=z["codes"], scales=z["scales"])
+                   for z in layer]
+    gemm_group = [dict(a_codes=z["codes"], a_scales=z["scales"], w_codes=z["wc"], w_scales=z["wsc"], S=z["S"],
+                       M=z["M"], N=z["N"], out=z["out"]) for z in layer]
+    per_linear_fns = [launcher("linear", z, sp) for z in layer]
 
     def step():
-        for f in step_fns:
+        BQ.batq_linear_grouped(group, gws, stream=sp)
+
+    def step_per_linear():
+        for f in per_linear_fns:
             f()
 
     warm = max(3, args.warmup)
     for _ in range(warm):
         step()
+        step_per_linear()
     torch.cuda.synchronize()
     assert BQ.batq_device_error() == 0
     timer = Timer(stream)
@@ -606,15 +638,24 @@ def run_batq(args):
         e1.record(stream)
         torch.cuda.synchronize()
         local_ms = e0.elapsed_time(e1) / args.steps
-        # timed region 2: each kernel alone over the seven linears, median of five repeats
-        # (-> per-kernel throughput and roofline)
-        q_ms = timer.median([launcher("quant", z, sp) for z in layer])
-        g_ms = timer.median([launcher("gemm", z, sp) for z in layer])
+        # the same K steps as seven batq_linear calls each (context: what grouping saves)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step_per_linear()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_linear_ms = e0.elapsed_time(e1) / args.steps
+        timer.launches += 2 * len(layer) * args.steps
+        # timed region 2: each grouped kernel alone (one launch covers the seven linears), median of
+        # five repeats of three launches back to back (-> per-kernel throughput and roofline)
+        q_ms = timer.median([lambda: BQ.batq_quant_act_grouped(quant_group, stream=sp)], reps=3)
+        g_ms = timer.median([lambda: BQ.batq_gemm_mxfp4_grouped(gemm_group, stream=sp)], reps=3)
+        # each linear's own kernels, one back-to-back pass with events between the launches
         q_each = timer.each([launcher("quant", z, sp) for z in layer])
         g_each = timer.each([launcher("gemm", z, sp) for z in layer])
     if ws > 1:
         dist.barrier()
-    local_ms, q_ms, g_ms = max_over_ranks([local_ms, q_ms, g_ms], device=dev)
+    local_ms, q_ms, g_ms, per_linear_ms = max_over_ranks([local_ms, q_ms, g_ms, per_linear_ms], device=dev)
     assert BQ.batq_device_error() == 0
 
     # End to end through the public call with host buffers: every step uploads each linear's bf16
@@ -692,15 +733,18 @@ def run_batq(args):
         "quant_ms": q_ms,
         "gemm_tflops": gemm_tflops,
         "gemm_ms": g_ms,
+        "per_linear_calls": {"ms_per_step": per_linear_ms, "value": whole_job_tflops(ws, flops, per_linear_ms),
+                             "note": "the same step as seven batq_linear calls (14 launches) instead of one "
+                                     "batq_linear_grouped call (2 launches)"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp4_peak, "traffic": ncu_traffic("k_gemm_pair", n_lin),
-                     "algorithmic_bytes": alg_gemm_bytes / n_lin, "kernel": "k_gemm_pair",
-                     "per_launch": "averages over the seven GEMM launches of one step",
+                     "frac": gemm_tflops / fp4_peak, "traffic": ncu_traffic("k_gemm_pair", 1),
+                     "algorithmic_bytes": alg_gemm_bytes, "kernel": "k_gemm_pair",
+                     "per_launch": "one grouped launch: the seven GEMMs of one step",
                      "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16)"},
         "roofline_quant": {"bound": "hbm", "achieved": quant_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": quant_gbs / peaks["hbm_gbs"], "traffic": ncu_traffic("k_quant_act_tc", n_lin),
-                           "algorithmic_bytes": qbytes / n_lin, "kernel": "k_quant_act_tc",
-                           "per_launch": "averages over the seven quantiser launches of one step",
+                           "frac": quant_gbs / peaks["hbm_gbs"], "traffic": ncu_traffic("k_quant_act_tc", 1),
+                           "algorithmic_bytes": qbytes, "kernel": "k_quant_act_tc",
+                           "per_launch": "one grouped launch: the seven activations of one step",
                            "peak_note": f"{peaks['source']} HBM copy"},
         "per_linear": {n: {"quant_us": q * 1e3, "quant_gbs": z["S"] * z["N"] * QUANT_BYTES_PER_ELEM / q / 1e6,
                            "gemm_us": g * 1e3, "gemm_tflops": 2.0 * z["S"] * z["N"] * z["M"] / g / 1e9}
@@ -710,17 +754,18 @@ def run_batq(args):
                 "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outh)), "ms_per_step": e2e_ms,
                 "note": "batq_linear on pinned host buffers for all seven linears; upload, compute and download on "
                         "three streams, double-buffered across linears"},
-        "timing": "CUDA events on the launching stream; value: exactly K whole steps back to back (7 batq_linear "
-                  "calls each); quantiser / GEMM figures and roofline: median of 5 repeats of the seven launches "
-                  "back to back; gpu_launches counts every library launch between the first and last timed event",
+        "timing": "CUDA events on the launching stream; value: exactly K whole steps back to back (one "
+                  "batq_linear_grouped call each); quantiser / GEMM figures and roofline: median of 5 repeats of "
+                  "3 grouped launches back to back; per_linear: each linear's own kernels with events between "
+                  "launches; gpu_launches counts the library launches between the two events that time value",
         "clocks": clk.summary(),
     }
     del Xh, outh
     if rank == 0 and not args.no_configs:
         line["per_config"] = per_config(dev, peaks, timer, sp)
-    # library kernels launched between the two events that time `value` (a quantiser and a GEMM
-    # per linear and step); the per-kernel loops launch timer.launches more
-    line["gpu_launches"] = 2 * len(layer) * args.steps
+    # library kernels launched between the two events that time `value` (one grouped quantiser and
+    # one grouped GEMM per step); the other timed loops launch timer.launches more
+    line["gpu_launches"] = 2 * args.steps
     line["gpu_launches_other_timed_loops"] = timer.launches
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         del layer
@@ -742,7 +787,8 @@ def main():
     ap.add_argument("--impl", choices=["batq", "reference"], default="batq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-workload kernel timings")
-    ap.add_argument("--only", choices=["quant", "gemm", "linear"], help="launch one kernel a few times (profiling)")
+    ap.add_argument("--only", choices=["quant", "gemm", "linear", "group"],
+                    help="launch one kernel (group: the grouped linear call) a few times (profiling)")
     ap.add_argument("--workload", default="layer", help="with --only: layer, layer_<q|k|v|o|gate|up|down>, "
                                                         "q_proj, down_proj, decode<1|4|16>")
     ap.add_argument("--launches", type=int, default=2)

@@ -186,6 +186,104 @@ BATQ_API batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N
                         void* workspace, size_t workspace_bytes,
                         batq_dtype out_dtype, void* out, int ldo, void* stream);
 
+/*
+ * One linear of a group: the arguments of batq_linear, with the same meaning,
+ * layout and ownership (A_host: 64 floats on the host, read during the call).
+ */
+typedef struct batq_linear_args {
+  const void* X;
+  batq_dtype x_dtype;
+  int S, N, ldx;
+  const float* A_host;
+  const float* B_dev;
+  const float* ratios_dev;
+  const uint8_t* w_codes;
+  const uint8_t* w_scales;
+  int M;
+  batq_dtype out_dtype;
+  void* out;
+  int ldo;
+} batq_linear_args;
+
+#define BATQ_MAX_LINEAR_GROUP 8
+
+/* One activation of a quantiser group: the arguments of batq_quant_act. */
+typedef struct batq_quant_args {
+  const void* X;
+  batq_dtype x_dtype;
+  int S, N, ldx;
+  const float* A_host;
+  const float* B_dev;
+  const float* ratios_dev;
+  uint8_t* codes;
+  uint8_t* scales;
+  batq_scale_layout layout;
+} batq_quant_args;
+
+/*
+ * `count` (1..8) independent batq_quant_act calls (no y_debug) on one stream.
+ * When every X is bf16, one launch of the tensor-core quantiser covers all of
+ * them (their tiles form one list); otherwise they run one after another.
+ * Codes and scales equal batq_quant_act's wherever that call also takes the
+ * tensor-core transform, and otherwise meet the same parity bound (see
+ * batq_linear_grouped).  Outputs must not overlap one another or any input.
+ * Errors: as batq_quant_act for each (the first failing check's code),
+ * BATQ_ERR_INVALID_ARG for count out of range; nothing is launched when a
+ * check fails.
+ */
+BATQ_API batq_status batq_quant_act_grouped(const batq_quant_args* acts, int count, void* stream);
+
+/* One product of a GEMM group: the arguments of batq_gemm_mxfp4. */
+typedef struct batq_gemm_args {
+  const uint8_t* a_codes;
+  const uint8_t* a_scales;
+  const uint8_t* w_codes;
+  const uint8_t* w_scales;
+  int S, M, N;
+  batq_dtype out_dtype;
+  void* out;
+  int ldo;
+} batq_gemm_args;
+
+/*
+ * `count` (1..8) independent batq_gemm_mxfp4 calls on one stream.  When every
+ * S > 128 and every out_dtype is the same, one launch of the CTA-pair GEMM
+ * covers all of them; otherwise they run one after another.  Results equal
+ * batq_gemm_mxfp4's bit for bit.  Outputs must not overlap one another or any
+ * input.  Errors: as batq_gemm_mxfp4 for each, BATQ_ERR_INVALID_ARG for count
+ * out of range; nothing is launched when a check fails.
+ */
+BATQ_API batq_status batq_gemm_mxfp4_grouped(const batq_gemm_args* gemms, int count, void* stream);
+
+/*
+ * Workspace bytes batq_linear_grouped needs for `count` (1..8) linears: each
+ * linear's batq_linear_workspace_size rounded up to 256 bytes, summed.  Host
+ * only.  Errors: BATQ_ERR_INVALID_ARG (null pointers, count out of range), BATQ_ERR_SHAPE.
+ */
+BATQ_API batq_status batq_linear_grouped_workspace_size(const batq_linear_args* linears, int count,
+                                                        size_t* bytes);
+
+/*
+ * `count` (1..8) independent linears on one stream, each computing what
+ * batq_linear computes with its own arguments (BATQuant thelatestinai.com page,
+ * Figure 2: transform, clip and quantise each linear's activations, then the
+ * W4A4 product).  Linear i's codes and scales go to its 256-byte-aligned part
+ * of the workspace, in order.  When every X is bf16, one tensor-core
+ * quantiser launch covers all activations; when every S > 128 and every
+ * out_dtype is the same, one CTA-pair GEMM launch covers all products, which
+ * saves the per-launch fill and drain of 2 x (count - 1) launches.  Otherwise
+ * the linears' kernels run one after another.  The outputs must not overlap
+ * one another or any input.  GEMM results equal batq_linear's bit for bit;
+ * activation codes equal them wherever batq_linear also uses the tensor-core
+ * transform (bf16 and at least six 128 x 128 tiles per SM), and otherwise
+ * meet the same parity bound (the two transforms round Y in different
+ * orders).  Errors: as batq_linear for each linear (the first failing
+ * check's code), BATQ_ERR_INVALID_ARG for count out of range.  Nothing is
+ * launched when a check fails.
+ */
+BATQ_API batq_status batq_linear_grouped(const batq_linear_args* linears, int count, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------ W4A8 variant
  * The pages' second setting (BATQuant thelatestinai.com page, abstract and
  * Table 2, W4A8 rows): the same transform and clip with MXFP8 activations,

@@ -42,6 +42,10 @@ SIGNATURES = {
     "batq_linear_workspace_size": (_c_int, [_c_int, _c_int, _c_size_p]),
     "batq_linear": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
                              ctypes.c_size_t, _c_int, _vp, _c_int, _vp]),
+    "batq_linear_grouped_workspace_size": (_c_int, [_vp, _c_int, _c_size_p]),
+    "batq_linear_grouped": (_c_int, [_vp, _c_int, _vp, ctypes.c_size_t, _vp]),
+    "batq_quant_act_grouped": (_c_int, [_vp, _c_int, _vp]),
+    "batq_gemm_mxfp4_grouped": (_c_int, [_vp, _c_int, _vp]),
     "batq_linear_no_alloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_int,
                                       _c_int, _vp, _c_int, _vp]),
     "batq_mxfp8_buffer_sizes": (_c_int, [_c_int, _c_int, _c_int, _c_size_p, _c_size_p]),

@@ -145,6 +145,96 @@ def batq_linear(X, A, B, ratios, w_codes, w_scales, M, workspace, out, stream=No
                                    _dev_ptr(out, "out"), out.stride(0), _stream(stream)), "batq_linear")
 
 
+class _LinearArgs(ctypes.Structure):
+    """batq_linear_args of include/batq.h."""
+    _fields_ = [("X", ctypes.c_void_p), ("x_dtype", ctypes.c_int), ("S", ctypes.c_int), ("N", ctypes.c_int),
+                ("ldx", ctypes.c_int), ("A_host", ctypes.c_void_p), ("B_dev", ctypes.c_void_p),
+                ("ratios_dev", ctypes.c_void_p), ("w_codes", ctypes.c_void_p), ("w_scales", ctypes.c_void_p),
+                ("M", ctypes.c_int), ("out_dtype", ctypes.c_int), ("out", ctypes.c_void_p), ("ldo", ctypes.c_int)]
+
+
+def _linear_args(linears):
+    """ctypes array of batq_linear_args from dicts with X, A, B, ratios, w_codes, w_scales, M, out; also
+    returns the host copies of A that must stay alive during the call."""
+    arr = (_LinearArgs * len(linears))()
+    keep = []
+    for i, l in enumerate(linears):
+        X, out = l["X"], l["out"]
+        a = _host_f32(l["A"], 64, "A")
+        keep.append(a)
+        arr[i] = _LinearArgs(_dev_ptr(X, "X"), _dtype_code(X), X.shape[0], X.shape[1], X.stride(0), a.ctypes.data,
+                             _dev_ptr(l["B"], "B"), _dev_ptr(l["ratios"], "ratios"), _dev_ptr(l["w_codes"], "w_codes"),
+                             _dev_ptr(l["w_scales"], "w_scales"), int(l["M"]), _dtype_code(out), _dev_ptr(out, "out"),
+                             out.stride(0))
+    return arr, keep
+
+
+def batq_linear_grouped_workspace_size(shapes):
+    """Workspace bytes for linears of the given (S, N) shapes."""
+    arr = (_LinearArgs * len(shapes))()
+    for i, (S, N) in enumerate(shapes):
+        arr[i].S, arr[i].N = S, N
+    n = ctypes.c_size_t()
+    _check(_lib.load().batq_linear_grouped_workspace_size(ctypes.addressof(arr), len(shapes), ctypes.byref(n)),
+           "batq_linear_grouped_workspace_size")
+    return n.value
+
+
+def batq_linear_grouped(linears, workspace, stream=None):
+    """Independent linears (dicts with X, A, B, ratios, w_codes, w_scales, M, out) in one quantiser launch and one
+    GEMM launch where the shapes allow (see include/batq.h)."""
+    arr, keep = _linear_args(linears)
+    _check(_lib.load().batq_linear_grouped(ctypes.addressof(arr), len(linears), _dev_ptr(workspace, "workspace"),
+                                           workspace.numel() * workspace.element_size(), _stream(stream)),
+           "batq_linear_grouped")
+    del keep
+
+
+class _QuantArgs(ctypes.Structure):
+    """batq_quant_args of include/batq.h."""
+    _fields_ = [("X", ctypes.c_void_p), ("x_dtype", ctypes.c_int), ("S", ctypes.c_int), ("N", ctypes.c_int),
+                ("ldx", ctypes.c_int), ("A_host", ctypes.c_void_p), ("B_dev", ctypes.c_void_p),
+                ("ratios_dev", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("layout", ctypes.c_int)]
+
+
+class _GemmArgs(ctypes.Structure):
+    """batq_gemm_args of include/batq.h."""
+    _fields_ = [("a_codes", ctypes.c_void_p), ("a_scales", ctypes.c_void_p), ("w_codes", ctypes.c_void_p),
+                ("w_scales", ctypes.c_void_p), ("S", ctypes.c_int), ("M", ctypes.c_int), ("N", ctypes.c_int),
+                ("out_dtype", ctypes.c_int), ("out", ctypes.c_void_p), ("ldo", ctypes.c_int)]
+
+
+def batq_quant_act_grouped(acts, layout=BATQ_SCALES_MMA, stream=None):
+    """Independent batq_quant_act calls (dicts with X, A, B, ratios, codes, scales) in one launch of the
+    tensor-core quantiser when every X is bf16 (see include/batq.h)."""
+    arr = (_QuantArgs * len(acts))()
+    keep = []
+    for i, q in enumerate(acts):
+        X = q["X"]
+        a = _host_f32(q["A"], 64, "A")
+        keep.append(a)
+        arr[i] = _QuantArgs(_dev_ptr(X, "X"), _dtype_code(X), X.shape[0], X.shape[1], X.stride(0), a.ctypes.data,
+                            _dev_ptr(q["B"], "B"), _dev_ptr(q["ratios"], "ratios"), _dev_ptr(q["codes"], "codes"),
+                            _dev_ptr(q["scales"], "scales"), int(layout))
+    _check(_lib.load().batq_quant_act_grouped(ctypes.addressof(arr), len(acts), _stream(stream)),
+           "batq_quant_act_grouped")
+    del keep
+
+
+def batq_gemm_mxfp4_grouped(gemms, stream=None):
+    """Independent batq_gemm_mxfp4 calls (dicts with a_codes, a_scales, w_codes, w_scales, S, M, N, out) in one
+    launch of the CTA-pair GEMM when every S > 128 and the output types agree (see include/batq.h)."""
+    arr = (_GemmArgs * len(gemms))()
+    for i, g in enumerate(gemms):
+        out = g["out"]
+        arr[i] = _GemmArgs(_dev_ptr(g["a_codes"], "a_codes"), _dev_ptr(g["a_scales"], "a_scales"),
+                           _dev_ptr(g["w_codes"], "w_codes"), _dev_ptr(g["w_scales"], "w_scales"), int(g["S"]),
+                           int(g["M"]), int(g["N"]), _dtype_code(out), _dev_ptr(out, "out"), out.stride(0))
+    _check(_lib.load().batq_gemm_mxfp4_grouped(ctypes.addressof(arr), len(gemms), _stream(stream)),
+           "batq_gemm_mxfp4_grouped")
+
+
 def batq_linear_no_alloc(X, A, B, ratios, w_codes, w_scales, M, out, stream=None):
     """batq_linear for callers that cannot allocate device memory: the scratch for the
     quantised activations comes from a fixed array inside the library (see

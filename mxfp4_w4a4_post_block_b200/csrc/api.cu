@@ -422,6 +422,165 @@ batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx
   return launch_gemm(a_codes, a_scales, w_codes, w_scales, S, M, N, out_dtype, out, ldo, true, batq::kFmtMxfp4, s);
 }
 
+// ------------------------------------------------------------------ groups of linears
+
+// Launch an already checked quantiser group: one tensor-core launch when every
+// X is bf16, else one launch per activation.
+batq_status quant_group_checked(const batq_quant_args* q, int count, cudaStream_t s) {
+  bool all_bf16 = true;
+  for (int i = 0; i < count; ++i) all_bf16 = all_bf16 && q[i].x_dtype == BATQ_BF16;
+  if (!all_bf16) {
+    for (int i = 0; i < count; ++i) {
+      batq_status st = launch_quant(q[i].X, q[i].x_dtype, q[i].S, q[i].N, q[i].ldx, q[i].A_host, q[i].B_dev,
+                                    q[i].ratios_dev, q[i].codes, q[i].scales, q[i].layout, nullptr,
+                                    batq::kFmtMxfp4, s);
+      if (st != BATQ_OK) return st;
+    }
+    return BATQ_OK;
+  }
+  batq::QuantLaunch Q[BATQ_MAX_LINEAR_GROUP];
+  for (int i = 0; i < count; ++i) {
+    batq::QuantLaunch& L = Q[i];
+    L.X = q[i].X;
+    L.bf16 = true;
+    L.S = q[i].S;
+    L.N = q[i].N;
+    L.ldx = q[i].ldx;
+    std::memcpy(L.A, q[i].A_host, sizeof(L.A));
+    L.B = q[i].B_dev;
+    L.ratios = q[i].ratios_dev;
+    L.codes = q[i].codes;
+    L.scales = q[i].scales;
+    L.mma_layout = (q[i].layout == BATQ_SCALES_MMA);
+    L.y_debug = nullptr;
+    L.err = error_word();
+    L.stream = s;
+    L.fmt = batq::kFmtMxfp4;
+  }
+  cudaError_t e = batq::launch_quant_act_group(Q, count);
+  if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
+  return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
+}
+
+// Launch an already checked GEMM group: one CTA-pair launch when every S > 128
+// and every output type agrees, else one launch per product.  weights_ready:
+// the grid before this call writes no weights.
+batq_status gemm_group_checked(const batq_gemm_args* g, int count, bool weights_ready, cudaStream_t s) {
+  bool all_pair = true;
+  for (int i = 0; i < count; ++i) all_pair = all_pair && g[i].S > 128 && g[i].out_dtype == g[0].out_dtype;
+  if (!all_pair) {
+    for (int i = 0; i < count; ++i) {
+      // After the first, the grid before each launch is an earlier GEMM of the
+      // group, whose output overlaps no input.
+      batq_status st = launch_gemm(g[i].a_codes, g[i].a_scales, g[i].w_codes, g[i].w_scales, g[i].S, g[i].M, g[i].N,
+                                   g[i].out_dtype, g[i].out, g[i].ldo, weights_ready || i > 0, batq::kFmtMxfp4, s);
+      if (st != BATQ_OK) return st;
+    }
+    return BATQ_OK;
+  }
+  batq::GemmLaunch G[BATQ_MAX_LINEAR_GROUP];
+  for (int i = 0; i < count; ++i) {
+    batq::GemmLaunch& L = G[i];
+    L.a_codes = g[i].a_codes;
+    L.a_scales = g[i].a_scales;
+    L.w_codes = g[i].w_codes;
+    L.w_scales = g[i].w_scales;
+    L.S = g[i].S;
+    L.M = g[i].M;
+    L.N = g[i].N;
+    L.out_bf16 = (g[i].out_dtype == BATQ_BF16);
+    L.out = g[i].out;
+    L.ldo = g[i].ldo;
+    L.err = error_word();
+    L.stream = s;
+    L.weights_ready = weights_ready;
+    L.fmt = batq::kFmtMxfp4;
+    L.gs_a = nullptr;
+    L.gs_w = nullptr;
+  }
+  cudaError_t e = batq::launch_gemm_pair_group(G, count);
+  if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
+  return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
+}
+
+batq_status batq_quant_act_grouped(const batq_quant_args* acts, int count, void* stream) {
+  if (!acts || count < 1 || count > BATQ_MAX_LINEAR_GROUP) return BATQ_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const batq_quant_args& q = acts[i];
+    batq_status st = check_quant_args(q.X, q.x_dtype, q.S, q.N, q.ldx, q.A_host, q.B_dev, q.ratios_dev, q.codes,
+                                      q.scales, q.layout, nullptr);
+    if (st != BATQ_OK) return st;
+  }
+  batq_status st = check_arch();
+  if (st != BATQ_OK) return st;
+  return quant_group_checked(acts, count, static_cast<cudaStream_t>(stream));
+}
+
+batq_status batq_gemm_mxfp4_grouped(const batq_gemm_args* gemms, int count, void* stream) {
+  if (!gemms || count < 1 || count > BATQ_MAX_LINEAR_GROUP) return BATQ_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const batq_gemm_args& g = gemms[i];
+    batq_status st = check_gemm_args(g.a_codes, g.a_scales, g.w_codes, g.w_scales, g.S, g.M, g.N, g.out_dtype,
+                                     g.out, g.ldo);
+    if (st != BATQ_OK) return st;
+  }
+  batq_status st = check_arch();
+  if (st != BATQ_OK) return st;
+  return gemm_group_checked(gemms, count, false, static_cast<cudaStream_t>(stream));
+}
+
+batq_status batq_linear_grouped_workspace_size(const batq_linear_args* linears, int count, size_t* bytes) {
+  if (!linears || !bytes || count < 1 || count > BATQ_MAX_LINEAR_GROUP) return BATQ_ERR_INVALID_ARG;
+  size_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    size_t need = 0;
+    batq_status st = batq_linear_workspace_size(linears[i].S, linears[i].N, &need);
+    if (st != BATQ_OK) return st;
+    total += round_up(need, 256);
+  }
+  *bytes = total;
+  return BATQ_OK;
+}
+
+batq_status batq_linear_grouped(const batq_linear_args* linears, int count, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!linears || !workspace || count < 1 || count > BATQ_MAX_LINEAR_GROUP) return BATQ_ERR_INVALID_ARG;
+  size_t need = 0;
+  batq_status st = batq_linear_grouped_workspace_size(linears, count, &need);
+  if (st != BATQ_OK) return st;
+  if (workspace_bytes < need) return BATQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BATQ_ERR_ALIGNMENT;
+  // Every check before any launch; linear i's codes and MMA scales in its
+  // 256-byte-aligned part of the workspace.
+  batq_quant_args q[BATQ_MAX_LINEAR_GROUP];
+  batq_gemm_args g[BATQ_MAX_LINEAR_GROUP];
+  uint8_t* at = static_cast<uint8_t*>(workspace);
+  for (int i = 0; i < count; ++i) {
+    const batq_linear_args& l = linears[i];
+    uint8_t* codes = at;
+    uint8_t* scales = at + round_up((size_t)l.S * (l.N / 2), 256);
+    size_t one = 0;
+    batq_linear_workspace_size(l.S, l.N, &one);
+    at += round_up(one, 256);
+    q[i] = batq_quant_args{l.X, l.x_dtype, l.S, l.N, l.ldx, l.A_host, l.B_dev, l.ratios_dev, codes, scales,
+                           BATQ_SCALES_MMA};
+    g[i] = batq_gemm_args{codes, scales, l.w_codes, l.w_scales, l.S, l.M, l.N, l.out_dtype, l.out, l.ldo};
+    st = check_quant_args(l.X, l.x_dtype, l.S, l.N, l.ldx, l.A_host, l.B_dev, l.ratios_dev, codes, scales,
+                          BATQ_SCALES_MMA, nullptr);
+    if (st != BATQ_OK) return st;
+    st = check_gemm_args(codes, scales, l.w_codes, l.w_scales, l.S, l.M, l.N, l.out_dtype, l.out, l.ldo);
+    if (st != BATQ_OK) return st;
+  }
+  st = check_arch();
+  if (st != BATQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = quant_group_checked(q, count, s);
+  if (st != BATQ_OK) return st;
+  // The quantiser grid(s) just launched write only the workspace, so the GEMM
+  // may fetch weights before they finish.
+  return gemm_group_checked(g, count, true, s);
+}
+
 // ------------------------------------------------------------------ W4A8 variant
 
 batq_status batq_mxfp8_buffer_sizes(int rows, int N, batq_scale_layout layout, size_t* code_bytes,

@@ -2,7 +2,10 @@
 //
 // Same product as k_gemm_mxfp4 (out[s][m] = sum_n deq(a)[s][n] deq(w)[m][n],
 // fp32 accumulation in TMEM), computed by persistent clusters of two CTAs on
-// neighbouring SMs.  A pair owns a 256 (tokens) x 256 (out-features) tile:
+// neighbouring SMs.  One launch runs one to eight independent products (a
+// table of tensor maps and shapes in the kernel parameters; their tiles form
+// one list), so a batch of linears pays the pipeline fill and drain once.
+// A pair owns a 256 (tokens) x 256 (out-features) tile:
 //   * each CTA loads its own 128 token rows of activation codes and its own
 //     128-row half of the weight tile, so one SM moves 64 bytes of operands per
 //     tensor-core cycle instead of the 96 a single-CTA 128x256 tile needs;
@@ -85,25 +88,43 @@ struct PairCfg {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-struct PairArgs {
-  void* out;
-  unsigned* err;
+// One GEMM of a launch: its tensor maps and shape.  A launch runs one to kG
+// of them (independent problems of one format and output type) over a single
+// list of pair tiles: problem p's tiles are tile_begin .. tile_begin +
+// tiles_m * tiles_n - 1, row-major over (token tile, out-feature tile).
+struct PairProblem {
+  CUtensorMap tm_a, tm_w, tm_sfa, tm_sfw, tm_out, tm_out_wide;
   int S, M, N;
-  int ldo;
-  int tiles_m, tiles_n;     // pair tiles along tokens / out-features
-  int num_kstages;
-  int early_weights;        // weights may be read before waiting for the preceding grid
-  int sf_box_chunks;        // 256-byte scale chunks per row tile in one stage's box (<= 2 * kAtoms)
-  const float* gs_a;        // NVFP4 per-tensor encode scales (device, nullable: 1)
+  int tiles_n;         // pair tiles along out-features
+  int tile_begin;      // first tile of this problem in the launch's list
+  int num_kstages;     // K stages per tile
+  int sf_box_chunks;   // 256-byte scale chunks per row tile in one stage's box (<= 2 * kAtoms)
+};
+
+template <int kG>
+struct PairLaunch {
+  PairProblem prob[kG];
+  int count;           // problems in use (1 .. kG)
+  int num_tiles;       // tiles of all problems
+  unsigned* err;
+  int early_weights;   // weights may be read before waiting for the preceding grid
+  const float* gs_a;   // NVFP4 per-tensor encode scales (device, nullable: 1); one problem only
   const float* gs_w;
 };
 
-template <bool kOutBF16, int kFmt>
+// Problem of tile t (tiles are in problem order).
+template <int kG>
+__device__ __forceinline__ int problem_of(const PairLaunch<kG>& g, int t) {
+  int p = 0;
+#pragma unroll
+  for (int q = 1; q < kG; ++q)
+    if (q < g.count && t >= g.prob[q].tile_begin) p = q;
+  return p;
+}
+
+template <bool kOutBF16, int kFmt, int kG>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    k_gemm_pair(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
-                const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfw,
-                const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_out_wide,
-                const __grid_constant__ PairArgs g) {
+    k_gemm_pair(const __grid_constant__ PairLaunch<kG> g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   using C = PairCfg<kFmt>;
@@ -120,12 +141,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   // Fetch the TMA descriptors while the barriers and TMEM are set up.
   if (threadIdx.x == 0) {
-    tma_prefetch_map(&tm_a);
-    tma_prefetch_map(&tm_w);
-    tma_prefetch_map(&tm_sfa);
-    tma_prefetch_map(&tm_sfw);
-    tma_prefetch_map(&tm_out);
-    tma_prefetch_map(&tm_out_wide);
+    for (int p = 0; p < g.count; ++p) {
+      tma_prefetch_map(&g.prob[p].tm_a);
+      tma_prefetch_map(&g.prob[p].tm_w);
+      tma_prefetch_map(&g.prob[p].tm_sfa);
+      tma_prefetch_map(&g.prob[p].tm_sfw);
+      tma_prefetch_map(&g.prob[p].tm_out);
+      tma_prefetch_map(&g.prob[p].tm_out_wide);
+    }
   }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -133,7 +156,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const bool leader = (rank == 0);
   const int cluster_id = blockIdx.x >> 1;
   const int num_clusters = gridDim.x >> 1;
-  const int num_tiles = g.tiles_m * g.tiles_n;
+  const int num_tiles = g.num_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -160,128 +183,158 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t t_acc = tmem;
   const uint32_t t_sfa = tmem + kTileN;
   const uint32_t t_sfb = tmem + kTileN + kStages * kSfaCols;
-  const int nks = g.num_kstages;
-  const int my_tiles = cluster_id < num_tiles ? (num_tiles - 1 - cluster_id) / num_clusters + 1 : 0;
 
+  // Every role walks this cluster's tiles (cluster_id, cluster_id + num_clusters,
+  // ...) and each tile's K stages in the same order: one sequence of stages
+  // whose ring slot and phase advance by one per stage.
   if (warp == 0) {
     // ------------------------------ producer (both CTAs) ------------------------------
     if (lane == 0) {
+      // Cursor over the sequence: tile t of problem p, K step ks, its first rows.
+      int t = cluster_id, ks = 0, p = 0, nks = 0, a_row = 0, w_row = 0;
+      auto enter_tile = [&]() {
+        if (t >= num_tiles) return;
+        p = problem_of(g, t);
+        const int lt = t - g.prob[p].tile_begin;
+        a_row = (lt / g.prob[p].tiles_n) * kTileM + (int)rank * kRowsPerCta;
+        w_row = (lt % g.prob[p].tiles_n) * kTileN;
+        nks = g.prob[p].num_kstages;
+      };
+      auto advance = [&]() {
+        if (++ks == nks) {
+          ks = 0;
+          t += num_clusters;
+          enter_tile();
+        }
+      };
       // Bytes one CTA's loads deliver per stage: the code tiles and the scale boxes
       // (one box of own activation scales, one of two weight row tiles).
-      const uint32_t stage_tx = (uint32_t)(kABytes + kBBytes) + 3u * (uint32_t)g.sf_box_chunks * 256u;
-      // Stage g of this cluster's sequence: tile cluster_id + (g / nks) * num_clusters, K step g % nks.
-      const int total = my_tiles * nks;
-      auto a_row_of = [&](int gi) { return ((cluster_id + (gi / nks) * num_clusters) / g.tiles_n) * kTileM + (int)rank * kRowsPerCta; };
-      auto w_row_of = [&](int gi) { return ((cluster_id + (gi / nks) * num_clusters) % g.tiles_n) * kTileN; };
-      auto issue_weights = [&](int gi) {
-        const int st_idx = gi % kStages;
-        uint8_t* st = smem + st_idx * kStageBytes;
-        const uint32_t bar = mapa_shared(smem_u32(&full[st_idx]), 0);
-        const int ks = gi % nks;
-#pragma unroll
-        for (int t = 0; t < kSwAtoms; ++t)
-          tma_load_2d_pair(st + kABytes + t * kSwTile, &tm_w, bar, ks * kBKBytes + t * 128,
-                           w_row_of(gi) + (int)rank * kHalfN);
-        tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &tm_sfw, bar, 0, ks * 2 * C::kAtoms,
-                         w_row_of(gi) / kRowsPerCta);  // {2 row tiles} x {sf_box_chunks}
+      auto stage_tx = [&](int q) {
+        return (uint32_t)(kABytes + kBBytes) + 3u * (uint32_t)g.prob[q].sf_box_chunks * 256u;
       };
-      auto issue_activations = [&](int gi) {
-        const int st_idx = gi % kStages;
+      auto issue_weights = [&](int st_idx, int q, int k_step, int wr) {
         uint8_t* st = smem + st_idx * kStageBytes;
         const uint32_t bar = mapa_shared(smem_u32(&full[st_idx]), 0);
-        const int ks = gi % nks;
 #pragma unroll
-        for (int t = 0; t < kSwAtoms; ++t)
-          tma_load_2d_pair(st + t * kSwTile, &tm_a, bar, ks * kBKBytes + t * 128, a_row_of(gi));
+        for (int a = 0; a < kSwAtoms; ++a)
+          tma_load_2d_pair(st + kABytes + a * kSwTile, &g.prob[q].tm_w, bar, k_step * kBKBytes + a * 128,
+                           wr + (int)rank * kHalfN);
+        tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &g.prob[q].tm_sfw, bar, 0, k_step * 2 * C::kAtoms,
+                         wr / kRowsPerCta);  // {2 row tiles} x {sf_box_chunks}
+      };
+      auto issue_activations = [&](int st_idx, int q, int k_step, int ar) {
+        uint8_t* st = smem + st_idx * kStageBytes;
+        const uint32_t bar = mapa_shared(smem_u32(&full[st_idx]), 0);
+#pragma unroll
+        for (int a = 0; a < kSwAtoms; ++a)
+          tma_load_2d_pair(st + a * kSwTile, &g.prob[q].tm_a, bar, k_step * kBKBytes + a * 128, ar);
         // scale tiles: {256-byte chunk, K chunk (2 per 4-scale atom), 128-row tile}
-        tma_load_3d_pair(st + kABytes + kBBytes, &tm_sfa, bar, 0, ks * 2 * C::kAtoms, a_row_of(gi) / kRowsPerCta);
+        tma_load_3d_pair(st + kABytes + kBBytes, &g.prob[q].tm_sfa, bar, 0, k_step * 2 * C::kAtoms,
+                         ar / kRowsPerCta);
       };
+      enter_tile();
       // When the preceding grid is known not to write the weights (the linear
       // layer's own quantiser), the first ring's weights are loaded before
       // waiting for that grid; the activations always come after the wait.
-      const int prologue = total < kStages ? total : kStages;
+      int pro_p[kStages], pro_ks[kStages], pro_a[kStages];
+      int npro = 0;
       if (!g.early_weights) griddep_wait();
-      for (int gi = 0; gi < prologue; ++gi) {
-        if (leader) mbar_arrive_expect_tx(&full[gi], 2u * stage_tx);
-        issue_weights(gi);
+      while (npro < kStages && t < num_tiles) {
+        if (leader) mbar_arrive_expect_tx(&full[npro], 2u * stage_tx(p));
+        issue_weights(npro, p, ks, w_row);
+        pro_p[npro] = p;
+        pro_ks[npro] = ks;
+        pro_a[npro] = a_row;
+        ++npro;
+        advance();
       }
       if (g.early_weights) griddep_wait();
-      for (int gi = 0; gi < prologue; ++gi) issue_activations(gi);
-      int s = prologue % kStages;
-      uint32_t ph = prologue == kStages ? 1u : 0u;
-      for (int gi = prologue; gi < total; ++gi) {
+      for (int i = 0; i < npro; ++i) issue_activations(i, pro_p[i], pro_ks[i], pro_a[i]);
+      int s = npro % kStages;
+      uint32_t ph = npro == kStages ? 1u : 0u;
+      while (t < num_tiles) {
         if (!mbar_wait(&empty[s], ph ^ 1)) {
           set_error(g.err, kErrReleaseTimeout);
           break;
         }
-        if (leader) mbar_arrive_expect_tx(&full[s], 2u * stage_tx);
-        issue_weights(gi);
-        issue_activations(gi);
+        if (leader) mbar_arrive_expect_tx(&full[s], 2u * stage_tx(p));
+        issue_weights(s, p, ks, w_row);
+        issue_activations(s, p, ks, a_row);
         if (++s == kStages) {
           s = 0;
           ph ^= 1;
         }
+        advance();
       }
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer (leader only) ------------------------------
-    // The stages of all of this cluster's tiles form one sequence g = 0, 1, ...;
-    // stage g's scales are already in TMEM slot g % kStages when sf_ready fires.
+    // Stage g's scales are already in TMEM slot g % kStages when sf_ready fires.
     // The whole warp runs the loop, so its state stays warp-uniform (a loop run
     // by one lane spends many more instructions per MMA), and one elected lane
     // issues the MMAs and commits.
     if (leader) {
       const bool issuer = elect_one();
-      const int total = my_tiles * nks;
-      for (int gi = 0; gi < total; ++gi) {
-        const int ks = gi % nks;
-        const uint32_t tile_iter = (uint32_t)(gi / nks);
-        if (ks == 0) {
-          // The accumulator must have been drained by both CTAs' epilogues.
-          if (!mbar_wait_warp(acc_empty, (tile_iter & 1) ^ 1)) {
-            if (issuer) set_error(g.err, kErrDrainTimeout);
+      int st_idx = 0;
+      uint32_t sph = 0, tile_iter = 0;
+      bool ok = true;
+      for (int t = cluster_id; t < num_tiles && ok; t += num_clusters, ++tile_iter) {
+        const int p = problem_of(g, t);
+        const int nks = g.prob[p].num_kstages, N = g.prob[p].N;
+        for (int ks = 0; ks < nks; ++ks) {
+          if (ks == 0) {
+            // The accumulator must have been drained by both CTAs' epilogues.
+            if (!mbar_wait_warp(acc_empty, (tile_iter & 1) ^ 1)) {
+              if (issuer) set_error(g.err, kErrDrainTimeout);
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+          }
+          if (!mbar_wait_warp(&sf_ready[st_idx], sph)) {
+            if (issuer) set_error(g.err, kErrDataTimeout);
+            ok = false;
             break;
           }
           tc_fence_after_sync();
-        }
-        const int st_idx = gi % kStages;
-        if (!mbar_wait_warp(&sf_ready[st_idx], (uint32_t)((gi / kStages) & 1))) {
-          if (issuer) set_error(g.err, kErrDataTimeout);
-          break;
-        }
-        tc_fence_after_sync();
-        // Shared addresses stay below 2^18, so the descriptor of base + off is
-        // the base descriptor + off / 16.
-        const uint64_t da0 = sdesc_kmajor_sw128(smem_u32(smem + st_idx * kStageBytes));
-        const uint64_t db0 = da0 + (uint64_t)(kABytes >> 4);
-        const uint32_t tsfa = t_sfa + st_idx * kSfaCols, tsfb = t_sfb + st_idx * kSfbCols;
-        const int kleft = g.N - ks * kBK;
-        const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
-        if (issuer) {
-          for (int j = 0; j < nmma; ++j) {
-            // MMA j covers scale blocks kb.. of the stage: atom kb / 4, byte
-            // kb % 4 of each 4-scale TMEM column (NVFP4: four scales, byte 0).
-            const int kb = j * kSfPerMma;
-            const int a = kb >> 2;
-            const int sf_id = kb & 3;
-            // Bytes 32j.. of the stage's K: swizzle tile j / 4, then 32 bytes per
-            // MMA inside its 128-byte swizzle atom.
-            const uint64_t off = (uint64_t)((j >> 2) * (kSwTile >> 4) + (j & 3) * 2);
-            const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
-            if constexpr (C::kFp8)
-              tc_mma_pair_mxf8(t_acc, da0 + off, db0 + off, idesc_mxf8(256, kTileN, sf_id, sf_id), tsfa + a * 4,
-                               tsfb + a * 8, acc);
-            else if constexpr (C::kNv)
-              tc_mma_pair_nvf4(t_acc, da0 + off, db0 + off, idesc_nvf4(256, kTileN), tsfa + a * 4, tsfb + a * 8, acc);
-            else
-              tc_mma_pair_mxf4(t_acc, da0 + off, db0 + off, idesc_mxf4_m256(kTileN, sf_id, sf_id), tsfa + a * 4,
-                               tsfb + a * 8, acc);
+          // Shared addresses stay below 2^18, so the descriptor of base + off is
+          // the base descriptor + off / 16.
+          const uint64_t da0 = sdesc_kmajor_sw128(smem_u32(smem + st_idx * kStageBytes));
+          const uint64_t db0 = da0 + (uint64_t)(kABytes >> 4);
+          const uint32_t tsfa = t_sfa + st_idx * kSfaCols, tsfb = t_sfb + st_idx * kSfbCols;
+          const int kleft = N - ks * kBK;
+          const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
+          if (issuer) {
+            for (int j = 0; j < nmma; ++j) {
+              // MMA j covers scale blocks kb.. of the stage: atom kb / 4, byte
+              // kb % 4 of each 4-scale TMEM column (NVFP4: four scales, byte 0).
+              const int kb = j * kSfPerMma;
+              const int a = kb >> 2;
+              const int sf_id = kb & 3;
+              // Bytes 32j.. of the stage's K: swizzle tile j / 4, then 32 bytes per
+              // MMA inside its 128-byte swizzle atom.
+              const uint64_t off = (uint64_t)((j >> 2) * (kSwTile >> 4) + (j & 3) * 2);
+              const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
+              if constexpr (C::kFp8)
+                tc_mma_pair_mxf8(t_acc, da0 + off, db0 + off, idesc_mxf8(256, kTileN, sf_id, sf_id), tsfa + a * 4,
+                                 tsfb + a * 8, acc);
+              else if constexpr (C::kNv)
+                tc_mma_pair_nvf4(t_acc, da0 + off, db0 + off, idesc_nvf4(256, kTileN), tsfa + a * 4, tsfb + a * 8,
+                                 acc);
+              else
+                tc_mma_pair_mxf4(t_acc, da0 + off, db0 + off, idesc_mxf4_m256(kTileN, sf_id, sf_id), tsfa + a * 4,
+                                 tsfb + a * 8, acc);
+            }
+            tc_commit_pair(&empty[st_idx], 0x3);
+            // Both epilogues may read the accumulator once every MMA of the tile has completed.
+            if (ks == nks - 1) tc_commit_pair(acc_full, 0x3);
           }
-          tc_commit_pair(&empty[st_idx], 0x3);
-          // Both epilogues may read the accumulator once every MMA of the tile has completed.
-          if (ks == nks - 1) tc_commit_pair(acc_full, 0x3);
+          __syncwarp();
+          if (++st_idx == kStages) {
+            st_idx = 0;
+            sph ^= 1u;
+          }
         }
-        __syncwarp();
       }
     }
   } else if (warp == kSfWarp) {
@@ -292,34 +345,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // producer could refill the stage.  Warp-wide loop, one elected issuer.
     if (leader) {
       const bool issuer = elect_one();
-      const int total = my_tiles * nks;
-      for (int gi = 0; gi < total; ++gi) {
-        const int st_idx = gi % kStages;
-        if (!mbar_wait_warp(&full[st_idx], (uint32_t)((gi / kStages) & 1))) {
-          if (issuer) set_error(g.err, kErrDataTimeout);
-          break;
-        }
-        tc_fence_after_sync();
-        const int ks = gi % nks;
-        const int kleft = g.N - ks * kBK;
-        const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
-        const uint64_t dsfa = sdesc_sf_atom(smem_u32(smem + st_idx * kStageBytes) + kABytes + kBBytes);
-        const uint64_t dsfb = dsfa + (uint64_t)(kSfaBytes >> 4);
-        const uint64_t dsfb1 = dsfb + (uint64_t)((g.sf_box_chunks * 256) >> 4);
-        const uint32_t tsfa = t_sfa + st_idx * kSfaCols, tsfb = t_sfb + st_idx * kSfbCols;
-        const int atoms = ((nmma - 1) * kSfPerMma) / 4 + 1;  // atoms the stage's MMAs read
-        if (issuer) {
-          for (int a = 0; a < atoms; ++a) {
-            const uint64_t off = (uint64_t)(a * (kSfAtom >> 4));
-            tc_cp_pair_32x128b_warpx4(tsfa + a * 4, dsfa + off);
-            // weight-scale box is {2 row tiles} x {sf_box_chunks}: row tile r, atom a at
-            // r * sf_box_chunks * 256 + a * 512
-            tc_cp_pair_32x128b_warpx4(tsfb + a * 8, dsfb + off);
-            tc_cp_pair_32x128b_warpx4(tsfb + a * 8 + 4, dsfb1 + off);
+      int st_idx = 0;
+      uint32_t fph = 0;
+      bool ok = true;
+      for (int t = cluster_id; t < num_tiles && ok; t += num_clusters) {
+        const int p = problem_of(g, t);
+        const int nks = g.prob[p].num_kstages, N = g.prob[p].N, box_chunks = g.prob[p].sf_box_chunks;
+        for (int ks = 0; ks < nks; ++ks) {
+          if (!mbar_wait_warp(&full[st_idx], fph)) {
+            if (issuer) set_error(g.err, kErrDataTimeout);
+            ok = false;
+            break;
           }
-          tc_commit_pair_local(&sf_ready[st_idx]);
+          tc_fence_after_sync();
+          const int kleft = N - ks * kBK;
+          const int nmma = kleft >= kBK ? kBK / kKPerMma : kleft / kKPerMma;
+          const uint64_t dsfa = sdesc_sf_atom(smem_u32(smem + st_idx * kStageBytes) + kABytes + kBBytes);
+          const uint64_t dsfb = dsfa + (uint64_t)(kSfaBytes >> 4);
+          const uint64_t dsfb1 = dsfb + (uint64_t)((box_chunks * 256) >> 4);
+          const uint32_t tsfa = t_sfa + st_idx * kSfaCols, tsfb = t_sfb + st_idx * kSfbCols;
+          const int atoms = ((nmma - 1) * kSfPerMma) / 4 + 1;  // atoms the stage's MMAs read
+          if (issuer) {
+            for (int a = 0; a < atoms; ++a) {
+              const uint64_t off = (uint64_t)(a * (kSfAtom >> 4));
+              tc_cp_pair_32x128b_warpx4(tsfa + a * 4, dsfa + off);
+              // weight-scale box is {2 row tiles} x {sf_box_chunks}: row tile r, atom a at
+              // r * sf_box_chunks * 256 + a * 512
+              tc_cp_pair_32x128b_warpx4(tsfb + a * 8, dsfb + off);
+              tc_cp_pair_32x128b_warpx4(tsfb + a * 8 + 4, dsfb1 + off);
+            }
+            tc_commit_pair_local(&sf_ready[st_idx]);
+          }
+          __syncwarp();
+          if (++st_idx == kStages) {
+            st_idx = 0;
+            fph ^= 1u;
+          }
         }
-        __syncwarp();
       }
     }
   } else if (warp >= 2 && warp < 2 + kEpiWarps) {
@@ -343,8 +405,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       return __uint_as_float(bits);
     };
     for (int t = cluster_id; t < num_tiles; t += num_clusters, ++tile_iter) {
-      const int row0 = (t / g.tiles_n) * kTileM + (int)rank * kRowsPerCta + 32 * quad;
-      const int n0 = (t % g.tiles_n) * kTileN + col0;
+      const PairProblem& P = g.prob[problem_of(g, t)];
+      const int lt = t - P.tile_begin;
+      const int row0 = (lt / P.tiles_n) * kTileM + (int)rank * kRowsPerCta + 32 * quad;
+      const int n0 = (lt % P.tiles_n) * kTileN + col0;
       if (!mbar_wait_warp(acc_full, tile_iter & 1)) {
         if (lane == 0) set_error(g.err, kErrMmaTimeout);
         break;
@@ -393,10 +457,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && row0 < g.S) {
+        if (lane == 0 && row0 < P.S) {
           for (int bx = 0; bx < kWideBoxes; ++bx) {
             const int x = n0 + bx * kWideCols;
-            if (x < g.M) tma_store_2d(&tm_out_wide, wide + bx * 4096, x, row0);
+            if (x < P.M) tma_store_2d(&P.tm_out_wide, wide + bx * 4096, x, row0);
           }
           tma_store_commit();
         }
@@ -438,8 +502,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         const int x = n0 + bx * kColsPerBox;
-        if (lane == 0 && row0 < g.S && x < g.M) {
-          tma_store_2d(&tm_out, box, x, row0);
+        if (lane == 0 && row0 < P.S && x < P.M) {
+          tma_store_2d(&P.tm_out, box, x, row0);
           tma_store_commit();
         }
         store_pending = true;
@@ -458,8 +522,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
+// Tensor maps and shape of one problem; false when a map cannot be encoded.
 template <bool kOutBF16, int kFmt>
-cudaError_t launch_pair_impl(const GemmLaunch& L) {
+bool fill_problem(const GemmLaunch& L, int tile_begin, PairProblem* P) {
   using C = PairCfg<kFmt>;
   const uint64_t row_bytes = (uint64_t)(C::kFp8 ? L.N : L.N / 2);
   // Code tiles: boxes of 128 rows x 128 bytes (one swizzle atom); a stage takes kSwAtoms of them.
@@ -468,48 +533,60 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   const uint64_t sf_row_tile_bytes = (uint64_t)(kpad / 4) * kSfAtom;
   const uint64_t a_tiles = (uint64_t)(L.S + 127) / 128;
   const uint64_t w_tiles = (uint64_t)(L.M + 127) / 128;
-
-  CUtensorMap tm_a, tm_w, tm_sfa, tm_sfw, tm_out, tm_out_wide;
-  if (!make_map_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_codes, row_bytes, (uint64_t)L.S, row_bytes, 128,
+  if (!make_map_2d(&P->tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_codes, row_bytes, (uint64_t)L.S, row_bytes, 128,
                    kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  if (!make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_codes, row_bytes, (uint64_t)L.M, row_bytes, 128,
+    return false;
+  if (!make_map_2d(&P->tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_codes, row_bytes, (uint64_t)L.M, row_bytes, 128,
                    kHalfN, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+    return false;
   // Scale tiles as {256-byte chunks, chunks per row tile, row tiles}; one box = the stage's K
   // atoms (x 2 row tiles for the weights), clamped to the row tile when all of K is shorter.
   const uint64_t chunks = sf_row_tile_bytes / 256;
   const int box_chunks = (int)(chunks < (uint64_t)(2 * C::kAtoms) ? chunks : (uint64_t)(2 * C::kAtoms));
-  if (!make_map_3d(&tm_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_scales, 256, chunks, a_tiles, 256,
+  if (!make_map_3d(&P->tm_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.a_scales, 256, chunks, a_tiles, 256,
                    sf_row_tile_bytes, 256, box_chunks, 1))
-    return cudaErrorInvalidValue;
-  if (!make_map_3d(&tm_sfw, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_scales, 256, chunks, w_tiles, 256,
+    return false;
+  if (!make_map_3d(&P->tm_sfw, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_scales, 256, chunks, w_tiles, 256,
                    sf_row_tile_bytes, 256, box_chunks, 2))
-    return cudaErrorInvalidValue;
+    return false;
   const uint32_t esz = kOutBF16 ? 2 : 4;
-  if (!make_map_2d(&tm_out, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
+  if (!make_map_2d(&P->tm_out, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
                    (uint64_t)L.M, (uint64_t)L.S, (uint64_t)L.ldo * esz, 32 / esz, 32, CU_TENSOR_MAP_SWIZZLE_32B))
-    return cudaErrorInvalidValue;
-  if (!make_map_2d(&tm_out_wide, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
-                   (uint64_t)L.M, (uint64_t)L.S, (uint64_t)L.ldo * esz, 128 / esz, 32, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+    return false;
+  if (!make_map_2d(&P->tm_out_wide, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   L.out, (uint64_t)L.M, (uint64_t)L.S, (uint64_t)L.ldo * esz, 128 / esz, 32,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return false;
+  P->S = L.S;
+  P->M = L.M;
+  P->N = L.N;
+  P->tiles_n = (L.M + kTileN - 1) / kTileN;
+  P->tile_begin = tile_begin;
+  P->num_kstages = (L.N + C::kBK - 1) / C::kBK;
+  P->sf_box_chunks = box_chunks;
+  return true;
+}
 
-  PairArgs g;
-  g.out = L.out;
-  g.err = L.err;
-  g.S = L.S;
-  g.M = L.M;
-  g.N = L.N;
-  g.ldo = L.ldo;
-  g.tiles_m = (L.S + kTileM - 1) / kTileM;
-  g.tiles_n = (L.M + kTileN - 1) / kTileN;
-  g.num_kstages = (L.N + C::kBK - 1) / C::kBK;
-  g.early_weights = L.weights_ready ? 1 : 0;
-  g.sf_box_chunks = box_chunks;
-  g.gs_a = L.gs_a;
-  g.gs_w = L.gs_w;
+// Ls[0 .. count-1]: problems of one format and output type on one stream;
+// the first supplies the launch-wide fields (error word, weights_ready, NVFP4 scales).
+template <bool kOutBF16, int kFmt, int kG>
+cudaError_t launch_pair_impl(const GemmLaunch* Ls, int count) {
+  using C = PairCfg<kFmt>;
+  if (count < 1 || count > kG) return cudaErrorInvalidValue;
+  PairLaunch<kG> g = {};
+  int tiles = 0;
+  for (int p = 0; p < count; ++p) {
+    if (!fill_problem<kOutBF16, kFmt>(Ls[p], tiles, &g.prob[p])) return cudaErrorInvalidValue;
+    tiles += ((Ls[p].S + kTileM - 1) / kTileM) * g.prob[p].tiles_n;
+  }
+  g.count = count;
+  g.num_tiles = tiles;
+  g.err = Ls[0].err;
+  g.early_weights = Ls[0].weights_ready ? 1 : 0;
+  g.gs_a = Ls[0].gs_a;
+  g.gs_w = Ls[0].gs_w;
 
-  auto kern = k_gemm_pair<kOutBF16, kFmt>;
+  auto kern = k_gemm_pair<kOutBF16, kFmt, kG>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -518,7 +595,6 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int tiles = g.tiles_m * g.tiles_n;
   const int max_clusters = sm_count() / 2;
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
   // Launched as a programmatic dependent of the preceding grid: set-up and
@@ -527,24 +603,35 @@ cudaError_t launch_pair_impl(const GemmLaunch& L) {
   cfg.gridDim = dim3(2 * clusters);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = L.stream;
+  cfg.stream = Ls[0].stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tm_a, tm_w, tm_sfa, tm_sfw, tm_out, tm_out_wide, g);
+  return cudaLaunchKernelEx(&cfg, kern, g);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_pair(const GemmLaunch& L) {
   switch (L.fmt) {
-    case kFmtMxfp4: return L.out_bf16 ? launch_pair_impl<true, kFmtMxfp4>(L) : launch_pair_impl<false, kFmtMxfp4>(L);
-    case kFmtMxfp8: return L.out_bf16 ? launch_pair_impl<true, kFmtMxfp8>(L) : launch_pair_impl<false, kFmtMxfp8>(L);
-    case kFmtNvfp4: return L.out_bf16 ? launch_pair_impl<true, kFmtNvfp4>(L) : launch_pair_impl<false, kFmtNvfp4>(L);
+    case kFmtMxfp4:
+      return L.out_bf16 ? launch_pair_impl<true, kFmtMxfp4, 1>(&L, 1) : launch_pair_impl<false, kFmtMxfp4, 1>(&L, 1);
+    case kFmtMxfp8:
+      return L.out_bf16 ? launch_pair_impl<true, kFmtMxfp8, 1>(&L, 1) : launch_pair_impl<false, kFmtMxfp8, 1>(&L, 1);
+    case kFmtNvfp4:
+      return L.out_bf16 ? launch_pair_impl<true, kFmtNvfp4, 1>(&L, 1) : launch_pair_impl<false, kFmtNvfp4, 1>(&L, 1);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_pair_group(const GemmLaunch* Ls, int count) {
+  if (count < 1 || count > kMaxGemmGroup) return cudaErrorInvalidValue;
+  for (int p = 0; p < count; ++p)
+    if (Ls[p].fmt != kFmtMxfp4 || Ls[p].out_bf16 != Ls[0].out_bf16 || Ls[p].S <= 128) return cudaErrorInvalidValue;
+  return Ls[0].out_bf16 ? launch_pair_impl<true, kFmtMxfp4, kMaxGemmGroup>(Ls, count)
+                        : launch_pair_impl<false, kFmtMxfp4, kMaxGemmGroup>(Ls, count);
 }
 
 }  // namespace batq

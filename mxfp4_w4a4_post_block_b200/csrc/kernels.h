@@ -59,6 +59,13 @@ struct QuantLaunch {
 // lets its own dependents start early.
 cudaError_t launch_quant_act(const QuantLaunch& L);
 
+// Up to kMaxQuantGroup independent activations quantised in one launch of
+// the tensor-core kernel (bf16, MXFP4, MMA or linear scale layout, no
+// RMSNorm, naive Kronecker or row map), on Ls[0]'s stream with Ls[0]'s error
+// word.  Refuses (cudaErrorInvalidValue) what it does not cover.
+constexpr int kMaxQuantGroup = 8;
+cudaError_t launch_quant_act_group(const QuantLaunch* Ls, int count);
+
 struct GemmLaunch {
   const uint8_t* a_codes;
   const uint8_t* a_scales;  // MMA layout, S rows
@@ -87,6 +94,12 @@ cudaError_t launch_gemm_mxfp4(const GemmLaunch& L);
 
 // Prefill-shape GEMM on CTA pairs (tcgen05 cta_group::2); used for S > 128.
 cudaError_t launch_gemm_pair(const GemmLaunch& L);
+
+// Up to kMaxGemmGroup independent prefill GEMMs (MXFP4, S > 128 each, one
+// output type, one stream: Ls[0]'s) in one launch of the pair kernel over all
+// of their tiles; Ls[0] also gives the error word and weights_ready.
+constexpr int kMaxGemmGroup = 8;
+cudaError_t launch_gemm_pair_group(const GemmLaunch* Ls, int count);
 
 // Widen packed E2M1 codes (element 2j in the low nibble) to one E4M3 byte per
 // element holding the same value; packed_bytes must be a multiple of 16 and

@@ -361,4 +361,18 @@ cudaError_t launch_quant_act(const QuantLaunch& L) {
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_quant_act_group(const QuantLaunch* Ls, int count) {
+  if (count < 1 || count > kMaxQuantGroup) return cudaErrorInvalidValue;
+  QuantArgs as[kMaxQuantGroup];
+  for (int q = 0; q < count; ++q) {
+    const QuantLaunch& L = Ls[q];
+    if (!L.bf16 || L.fmt != kFmtMxfp4 || L.gamma != nullptr || L.row_scale != nullptr || L.A_blocks != nullptr ||
+        L.row_map != nullptr || L.amax_out != nullptr)
+      return cudaErrorInvalidValue;
+    as[q] = make_args(L);
+    as[q].err = Ls[0].err;
+  }
+  return launch_quant_act_tc_group(Ls, as, count);
+}
+
 }  // namespace batq

@@ -13,7 +13,9 @@
 // is taken with the same instructions.
 //
 // Layout of the work: a strip is 4 block columns (128 elements of every
-// token), a tile 128 tokens of a strip; tiles are ordered strip by strip and
+// token), a tile 128 tokens of a strip; tiles are ordered strip by strip (one
+// launch may cover up to eight independent activations, problem after
+// problem, each with its own tensor map and arguments) and
 // each CTA (one per SM) takes an equal contiguous share, so it meets at most
 // a few strips and builds each strip's P_i parts once in shared memory (24 KB,
 // 64-byte swizzled K-major rows, as the MMA reads them).  The three parts of
@@ -118,11 +120,33 @@ __device__ __forceinline__ void build_p_chunk(uint8_t* sp, int tid, int s, const
         make_uint4(w[q][0], w[q][1], w[q][2], w[q][3]);
 }
 
+// One launch: 1 .. kG independent activations (same format), each with its
+// tensor map and arguments.  The tiles of all of them form one list, problem
+// by problem, each strip-major; CTAs take contiguous shares of it.
+template <int kG>
+struct TcLaunch {
+  CUtensorMap tmx[kG];
+  QuantArgs args[kG];
+  int tile_begin[kG];  // first tile of each problem in the list
+  int count;           // problems in use
+  int num_tiles;       // tiles of all problems
+};
+
+// Problem of list tile i (tiles are in problem order).
+template <int kG>
+__device__ __forceinline__ int tc_problem_of(const TcLaunch<kG>& L, int i) {
+  int q = 0;
+#pragma unroll
+  for (int r = 1; r < kG; ++r)
+    if (r < L.count && i >= L.tile_begin[r]) q = r;
+  return q;
+}
+
 // kNorm: RMSNorm ahead of the transform (gamma folded into P_i, the token's
 // 1 / rms from p.row_scale applied to the transformed values).
-template <int kFmt, bool kNorm = false>
+template <int kFmt, bool kNorm, int kG>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_quant_act_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
+    k_quant_act_tc(const __grid_constant__ TcLaunch<kG> L) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
@@ -131,7 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_empty = acc_full + kCB;   // per block column: its four encoder warps read TMEM
   uint64_t* p_ready = acc_empty + kCB;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(p_ready + 1);
-  if (threadIdx.x == 0) tma_prefetch_map(&tmx);
+  if (threadIdx.x == 0)
+    for (int q = 0; q < L.count; ++q) tma_prefetch_map(&L.tmx[q]);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -158,13 +183,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
-  // This CTA's share of the tiles, strip-major: tile i is token tile
-  // i % tiles_r of strip i / tiles_r; a new strip starts at i % tiles_r == 0.
-  const int strips = (p.k + kCB - 1) / kCB;
-  const int tiles_r = (p.S + kTok - 1) / kTok;
-  const long long ntiles = (long long)strips * tiles_r;
+  // This CTA's share of the list.  Within problem q, tile li = i -
+  // tile_begin[q] is token tile li % tiles_r of strip li / tiles_r (tiles_r =
+  // the problem's 128-token tiles); a new strip starts at li % tiles_r == 0.
+  const long long ntiles = L.num_tiles;
   const int i0 = (int)((long long)blockIdx.x * ntiles / gridDim.x);
   const int total = (int)((long long)(blockIdx.x + 1) * ntiles / gridDim.x) - i0;
+  struct TileAt {
+    int q, s, t;  // problem, strip, token tile
+  };
+  auto tile_at = [&](int g) {
+    TileAt a;
+    a.q = tc_problem_of(L, i0 + g);
+    const int tiles_r = (L.args[a.q].S + kTok - 1) / kTok;
+    const int li = i0 + g - L.tile_begin[a.q];
+    a.s = li / tiles_r;
+    a.t = li - a.s * tiles_r;
+    return a;
+  };
+  unsigned* const err_word = L.args[0].err;
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
@@ -177,12 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 0; g < total; ++g) {
         const int st = g % kStages;
         if (!mbar_wait(&empty[st], ((g / kStages) & 1) ^ 1)) {
-          set_error(p.err, kErrReleaseTimeout);
+          set_error(err_word, kErrReleaseTimeout);
           break;
         }
-        const int s = (i0 + g) / tiles_r, t = (i0 + g) % tiles_r;
+        const TileAt a = tile_at(g);
         mbar_arrive_expect_tx(&full[st], (uint32_t)kXBytes);  // the box always delivers all of it (zero fill)
-        tma_load_3d(smem + st * kXBytes, &tmx, &full[st], 0, t * kTok, s * kCB);
+        tma_load_3d(smem + st * kXBytes, &L.tmx[a.q], &full[st], 0, a.t * kTok, a.s * kCB);
       }
     }
   } else if (warp == 1) {
@@ -195,17 +232,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t strip_count = 0;
     bool ok = true;
     for (int g = 0; g < total && ok; ++g) {
-      if (g == 0 || (i0 + g) % tiles_r == 0) {
+      if (g == 0 || tile_at(g).t == 0) {
         // The new strip's P_i parts are in shared memory.
         if (!mbar_wait_warp(p_ready, strip_count & 1)) {
-          if (leader) set_error(p.err, kErrDataTimeout);
+          if (leader) set_error(err_word, kErrDataTimeout);
           break;
         }
         ++strip_count;
       }
       const int st = g % kStages;
       if (!mbar_wait_warp(&full[st], (g / kStages) & 1)) {
-        if (leader) set_error(p.err, kErrDataTimeout);
+        if (leader) set_error(err_word, kErrDataTimeout);
         break;
       }
       tc_fence_after_sync();
@@ -217,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cb = 0; cb < kCB; ++cb) {
         // The block column's accumulator must have been read by its encoders.
         if (!mbar_wait_warp(&acc_empty[cb], (g & 1) ^ 1)) {
-          if (leader) set_error(p.err, kErrDrainTimeout);
+          if (leader) set_error(err_word, kErrDrainTimeout);
           ok = false;
           break;
         }
@@ -246,14 +283,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     griddep_wait();             // parameters and the NVFP4 scale may come from the preceding grid
     float gs = 1.0f;
     if constexpr (kFmt == kFmtNvfp4) {
-      gs = nv_encode_scale(p);
-      if (p.gs_out != nullptr && blockIdx.x == 0 && e == 0 && lane == 0) *p.gs_out = gs;
+      gs = nv_encode_scale(L.args[0]);
+      if (L.args[0].gs_out != nullptr && blockIdx.x == 0 && e == 0 && lane == 0) *L.args[0].gs_out = gs;
     }
     uint8_t* sp = smem + kPOffset;
     float r_min = 1.0f, r_max = 1.0f;
     int b = 0;
     for (int g = 0; g < total; ++g) {
-      const int s = (i0 + g) / tiles_r, t = (i0 + g) % tiles_r;
+      const TileAt at = tile_at(g);
+      const int s = at.s, t = at.t;
+      const QuantArgs& p = L.args[at.q];
       if (g == 0 || t == 0) {
         // Every MMA of the previous strip has completed (this warp saw its
         // last accumulator), so the parts may be overwritten.
@@ -327,37 +366,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kFmt, bool kNorm = false>
-cudaError_t launch_tc_impl(const QuantLaunch& L, const QuantArgs& a) {
-  // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
-  CUtensorMap map;
-  if (!make_map_3d_swizzled(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.X, 32, (uint64_t)L.S, (uint64_t)(L.N / 32),
-                            (uint64_t)L.ldx * 2u, 64, 32, kTok, kCB, CU_TENSOR_MAP_SWIZZLE_64B)) {
-    return cudaErrorInvalidValue;
+// Ls / as [0 .. count-1]: one format, bf16 activations, one stream (Ls[0]'s).
+template <int kFmt, bool kNorm, int kG>
+cudaError_t launch_tc_impl(const QuantLaunch* Ls, const QuantArgs* as, int count) {
+  if (count < 1 || count > kG) return cudaErrorInvalidValue;
+  TcLaunch<kG> T = {};
+  long long tiles = 0;
+  for (int q = 0; q < count; ++q) {
+    const QuantLaunch& L = Ls[q];
+    // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
+    if (!make_map_3d_swizzled(&T.tmx[q], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.X, 32, (uint64_t)L.S,
+                              (uint64_t)(L.N / 32), (uint64_t)L.ldx * 2u, 64, 32, kTok, kCB,
+                              CU_TENSOR_MAP_SWIZZLE_64B)) {
+      return cudaErrorInvalidValue;
+    }
+    T.args[q] = as[q];
+    T.tile_begin[q] = (int)tiles;
+    tiles += (long long)((as[q].k + kCB - 1) / kCB) * ((as[q].S + kTok - 1) / kTok);
   }
+  if (tiles >= (1LL << 31)) return cudaErrorInvalidValue;
+  T.count = count;
+  T.num_tiles = (int)tiles;
+  auto kern = k_quant_act_tc<kFmt, kNorm, kG>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_quant_act_tc<kFmt, kNorm>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const long long strips = (a.k + kCB - 1) / kCB;
-  const long long tiles = strips * ((a.S + kTok - 1) / kTok);
   const int grid = tiles < sm_count() ? (int)tiles : sm_count();  // one CTA per SM
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = L.stream;
+  cfg.stream = Ls[0].stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_quant_act_tc<kFmt, kNorm>, map, a);
+  return cudaLaunchKernelEx(&cfg, kern, T);
 }
 
 }  // namespace
@@ -365,14 +415,18 @@ cudaError_t launch_tc_impl(const QuantLaunch& L, const QuantArgs& a) {
 cudaError_t launch_quant_act_tc(const QuantLaunch& L, const QuantArgs& a) {
   if (L.gamma != nullptr) {  // RMSNorm ahead of the transform: MXFP4 output, shared A
     if (L.fmt != kFmtMxfp4 || L.A_blocks != nullptr || L.row_scale == nullptr) return cudaErrorInvalidValue;
-    return launch_tc_impl<kFmtMxfp4, true>(L, a);
+    return launch_tc_impl<kFmtMxfp4, true, 1>(&L, &a, 1);
   }
   switch (L.fmt) {
-    case kFmtMxfp4: return launch_tc_impl<kFmtMxfp4>(L, a);
-    case kFmtMxfp8: return launch_tc_impl<kFmtMxfp8>(L, a);
-    case kFmtNvfp4: return launch_tc_impl<kFmtNvfp4>(L, a);
+    case kFmtMxfp4: return launch_tc_impl<kFmtMxfp4, false, 1>(&L, &a, 1);
+    case kFmtMxfp8: return launch_tc_impl<kFmtMxfp8, false, 1>(&L, &a, 1);
+    case kFmtNvfp4: return launch_tc_impl<kFmtNvfp4, false, 1>(&L, &a, 1);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_quant_act_tc_group(const QuantLaunch* Ls, const QuantArgs* as, int count) {
+  return launch_tc_impl<kFmtMxfp4, false, kMaxQuantGroup>(Ls, as, count);
 }
 
 }  // namespace batq

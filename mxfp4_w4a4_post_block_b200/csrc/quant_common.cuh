@@ -260,5 +260,8 @@ __device__ __forceinline__ void pad_scales(int row, int b, const QuantArgs& p) {
 
 // The tensor-core quantiser for bf16 activations (quant_act_tc.cu).
 cudaError_t launch_quant_act_tc(const QuantLaunch& L, const QuantArgs& a);
+// The same kernel over 1 .. kMaxQuantGroup activations in one launch (MXFP4,
+// bf16, plain GPK: no RMSNorm, naive Kronecker or row map), Ls[0]'s stream.
+cudaError_t launch_quant_act_tc_group(const QuantLaunch* Ls, const QuantArgs* as, int count);
 
 }  // namespace batq

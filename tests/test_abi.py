@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 
 from mxfp4_w4a4_post_block_b200 import _lib
+from mxfp4_w4a4_post_block_b200 import batq as BQ
 from oracle import batq_oracle as O
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -113,6 +114,64 @@ def test_linear_workspace_checks(L):
     st = L.batq_linear(FAKE, 1, 16, 256, 256, A.ctypes.data, FAKE, None, FAKE, FAKE, 128, FAKE, 16, 0, FAKE, 128,
                        None)
     assert st == _lib.BATQ_ERR_WORKSPACE
+
+
+def _group(shapes):
+    arr = (BQ._LinearArgs * len(shapes))()
+    for i, (S, N) in enumerate(shapes):
+        arr[i].S, arr[i].N = S, N
+    return arr
+
+
+def test_grouped_workspace_size_is_the_256_aligned_sum(L):
+    shapes = [(16, 256), (300, 1024), (4096, 12288), (1, 64)]
+    want = 0
+    for S, N in shapes:
+        one = ctypes.c_size_t()
+        assert L.batq_linear_workspace_size(S, N, ctypes.byref(one)) == _lib.BATQ_OK
+        want += -(-one.value // 256) * 256
+    got = ctypes.c_size_t()
+    arr = _group(shapes)
+    assert L.batq_linear_grouped_workspace_size(ctypes.addressof(arr), len(shapes), ctypes.byref(got)) == _lib.BATQ_OK
+    assert got.value == want
+    assert BQ.batq_linear_grouped_workspace_size(shapes) == want
+
+
+def test_grouped_argument_checks_fail_before_any_launch(L):
+    n = ctypes.c_size_t()
+    arr = _group([(16, 256)] * 9)
+    assert L.batq_linear_grouped_workspace_size(ctypes.addressof(arr), 0, ctypes.byref(n)) == _lib.BATQ_ERR_INVALID_ARG
+    assert L.batq_linear_grouped_workspace_size(ctypes.addressof(arr), 9, ctypes.byref(n)) == _lib.BATQ_ERR_INVALID_ARG
+    assert L.batq_linear_grouped_workspace_size(None, 1, ctypes.byref(n)) == _lib.BATQ_ERR_INVALID_ARG
+    bad = _group([(16, 256), (16, 100)])  # N % 64 != 0
+    assert L.batq_linear_grouped_workspace_size(ctypes.addressof(bad), 2, ctypes.byref(n)) == _lib.BATQ_ERR_SHAPE
+    one = _group([(16, 256)])
+    assert L.batq_linear_grouped(ctypes.addressof(one), 1, None, 1 << 20, None) == _lib.BATQ_ERR_INVALID_ARG
+    assert L.batq_linear_grouped(ctypes.addressof(one), 9, FAKE, 1 << 20, None) == _lib.BATQ_ERR_INVALID_ARG
+    assert L.batq_linear_grouped(ctypes.addressof(one), 1, FAKE, 16, None) == _lib.BATQ_ERR_WORKSPACE
+    # enough workspace, but X is null: the quantiser's argument check refuses it
+    assert L.batq_linear_grouped(ctypes.addressof(one), 1, FAKE, 1 << 20, None) == _lib.BATQ_ERR_INVALID_ARG
+
+
+def test_grouped_quant_and_gemm_checks_fail_before_any_launch(L):
+    A = np.eye(8, dtype=np.float32)
+    q = (BQ._QuantArgs * 2)()
+    q[0] = BQ._QuantArgs(FAKE, 1, 16, 256, 256, A.ctypes.data, FAKE, 0, FAKE, FAKE, 1)
+    q[1] = BQ._QuantArgs(FAKE, 1, 16, 256, 256, A.ctypes.data, FAKE, 0, FAKE, FAKE, 1)
+    assert L.batq_quant_act_grouped(ctypes.addressof(q), 0, None) == _lib.BATQ_ERR_INVALID_ARG
+    assert L.batq_quant_act_grouped(ctypes.addressof(q), 9, None) == _lib.BATQ_ERR_INVALID_ARG
+    assert L.batq_quant_act_grouped(None, 1, None) == _lib.BATQ_ERR_INVALID_ARG
+    q[1].N = 100  # second activation's shape is refused although the first is valid
+    assert L.batq_quant_act_grouped(ctypes.addressof(q), 2, None) == _lib.BATQ_ERR_SHAPE
+    q[1].N, q[1].layout = 256, 7
+    assert L.batq_quant_act_grouped(ctypes.addressof(q), 2, None) == _lib.BATQ_ERR_INVALID_ARG
+    g = (BQ._GemmArgs * 2)()
+    g[0] = BQ._GemmArgs(FAKE, FAKE, FAKE, FAKE, 16, 128, 256, 0, FAKE, 128)
+    g[1] = BQ._GemmArgs(FAKE, FAKE, FAKE, FAKE, 16, 120, 256, 0, FAKE, 128)  # M % 16 != 0
+    assert L.batq_gemm_mxfp4_grouped(ctypes.addressof(g), 0, None) == _lib.BATQ_ERR_INVALID_ARG
+    assert L.batq_gemm_mxfp4_grouped(ctypes.addressof(g), 2, None) == _lib.BATQ_ERR_SHAPE
+    g[1].M, g[1].a_codes = 128, 0
+    assert L.batq_gemm_mxfp4_grouped(ctypes.addressof(g), 2, None) == _lib.BATQ_ERR_INVALID_ARG
 
 
 def test_prepare_checks(L):
