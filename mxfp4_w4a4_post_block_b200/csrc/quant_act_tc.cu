@@ -293,6 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileAt at = tile_at(g);
       const int s = at.s, t = at.t;
       const QuantArgs& p = L.args[at.q];
+      // With several problems per launch, the tile's problem as register
+      // values, fetched before the waits below (its table entry is indexed at
+      // run time); a single-problem launch reads its parameters directly.
+      [[maybe_unused]] const BlockOut o = kG > 1 ? block_out(p) : BlockOut{};
       if (g == 0 || t == 0) {
         // Every MMA of the previous strip has completed (this warp saw its
         // last accumulator), so the parts may be overwritten.
@@ -350,10 +354,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           y[j + 1] = sv.y;
         }
       }
-      if (b < p.k) {
-        encode_block<kFmt>(y, r_min, r_max, gs, row, b, lane, p);
+      if constexpr (kG == 1) {
+        if (b < p.k) {
+          encode_block<kFmt>(y, r_min, r_max, gs, row, b, lane, p);
+        } else {
+          pad_scales<kFmt>(row, b, p);
+        }
       } else {
-        pad_scales<kFmt>(row, b, p);
+        if (b < o.k) {
+          encode_block<kFmt>(y, r_min, r_max, gs, row, b, lane, o);
+        } else {
+          pad_scales<kFmt>(row, b, o);
+        }
       }
     }
   }

@@ -124,13 +124,41 @@ __device__ __forceinline__ float nv_encode_scale(const QuantArgs& p) {
   return gs;
 }
 
+// The fields of QuantArgs that encode_block and pad_scales read, held as
+// values, for a launch serving several problems (launch_quant_act_tc_group):
+// it copies its tile's problem into these once per tile instead of indexing
+// the parameter table inside the encode.  Such launches never have a row map,
+// y_debug or a measuring pass, so those are compile-time null.
+struct BlockOut {
+  uint8_t* codes;
+  uint8_t* scales;
+  int S, N, k, kpad, rows_out, rows_cap, mma_layout;
+  static constexpr float* y_debug = nullptr;
+  static constexpr const int* row_map = nullptr;
+  static constexpr unsigned* amax_out = nullptr;
+};
+__device__ __forceinline__ BlockOut block_out(const QuantArgs& p) {
+  BlockOut o;
+  o.codes = p.codes;
+  o.scales = p.scales;
+  o.S = p.S;
+  o.N = p.N;
+  o.k = p.k;
+  o.kpad = p.kpad;
+  o.rows_out = p.rows_out;
+  o.rows_cap = p.rows_cap;
+  o.mma_layout = p.mma_layout;
+  return o;
+}
+
 // Clip, scale, encode and store one token's 32-element block b (y: its
 // transformed values; gs: the NVFP4 encode scale, unused otherwise).  Rows
 // past S only get padding scales (MMA layout).  All 32 lanes of the warp call
-// it together (the measuring pass reduces across the warp).
-template <int kFmt>
+// it together (the measuring pass reduces across the warp).  Args: QuantArgs
+// or BlockOut.
+template <int kFmt, class Args>
 __device__ __forceinline__ void encode_block(const float (&y)[32], float r_min, float r_max, float gs, int row, int b,
-                                             int lane, const QuantArgs& p) {
+                                             int lane, const Args& p) {
   constexpr bool kFp8 = (kFmt == kFmtMxfp8);
   constexpr bool kNv = (kFmt == kFmtNvfp4);
   // Extrema (NaN-propagating) of each 16-element half, and of the block.
@@ -247,8 +275,8 @@ __device__ __forceinline__ void encode_block(const float (&y)[32], float r_min, 
 // Padding scales for (row, block b) when the block holds no data: rows past S
 // (all formats) and block columns past k (MX only; the NVFP4 column count 2k is
 // already a multiple of 4).
-template <int kFmt>
-__device__ __forceinline__ void pad_scales(int row, int b, const QuantArgs& p) {
+template <int kFmt, class Args>
+__device__ __forceinline__ void pad_scales(int row, int b, const Args& p) {
   if (!p.mma_layout || row >= p.rows_out) return;
   if constexpr (kFmt == kFmtNvfp4) {
     if (b < p.k)
