@@ -419,6 +419,29 @@ def per_config(dev, peaks, timer, sp):
     res["decode_note"] = ("launch-bound quantiser; GEMM judged on weight bytes against HBM; linear = batq_linear "
                           "(the GEMM prefetches its weights into L2 while the quantiser runs)")
 
+    # a decode step of the layer's seven linears at S = 16 (102 MB of prepared weights): one
+    # batq_linear_grouped call (one quantiser launch, one single-CTA GEMM launch) against seven
+    # batq_linear calls; two sets rotate (204 MB of weights, more than L2)
+    dsets = [[linear_set(WL.layer_linear(j, S=16, with_w=False), dev, real_weights=False, gen=g)
+              for j in range(len(WL.LAYER_LINEARS))] for _ in range(2)]
+    dwb = sum(z["M"] * z["N"] * (0.5 + 1.0 / 32) for z in dsets[0])
+    dgroups = []
+    for zs in dsets:
+        gl = [dict(X=z["X"], A=z["A"], B=z["B"], ratios=z["ratios"], w_codes=z["wc"], w_scales=z["wsc"],
+                   M=z["M"], out=z["out"]) for z in zs]
+        gws = torch.empty(BQ.batq_linear_grouped_workspace_size([(z["S"], z["N"]) for z in zs]),
+                          dtype=torch.uint8, device=dev)
+        dgroups.append((gl, gws))
+    grp_ms = timer.median([lambda gl=gl, gws=gws: BQ.batq_linear_grouped(gl, gws, stream=sp)
+                           for gl, gws in dgroups], 10, 2) / 2
+    per_ms = timer.median([launcher("linear", z, sp) for zs in dsets for z in zs], 10, 2) / 2
+    res["decode_layer_16x7_linears"] = {
+        "grouped_us": grp_ms * 1e3, "grouped_weight_gbs": dwb / grp_ms / 1e6,
+        "grouped_frac_hbm": dwb / grp_ms / 1e6 / hbm, "per_linear_calls_us": per_ms * 1e3,
+        "per_linear_weight_gbs": dwb / per_ms / 1e6,
+        "note": "q, k, v, o, gate, up, down at 16 tokens; batq_linear_grouped vs seven batq_linear calls"}
+    del dsets, dgroups
+
     w = WL.q_proj(with_w=False)
     S, N, M = w.S, w.N, w.M
     X = _bf16(w, dev)

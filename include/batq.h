@@ -248,7 +248,10 @@ typedef struct batq_gemm_args {
 /*
  * `count` (1..8) independent batq_gemm_mxfp4 calls on one stream.  When every
  * S > 128 and every out_dtype is the same, one launch of the CTA-pair GEMM
- * covers all of them; otherwise they run one after another.  Results equal
+ * covers all of them; when every S <= 128 falls in the same tile
+ * configuration (S <= 16, <= 32, <= 64 or <= 128; decode batches) with one
+ * out_dtype, one launch of the single-CTA GEMM does; otherwise they run one
+ * after another.  Results equal
  * batq_gemm_mxfp4's bit for bit.  Outputs must not overlap one another or any
  * input.  Errors: as batq_gemm_mxfp4 for each, BATQ_ERR_INVALID_ARG for count
  * out of range; nothing is launched when a check fails.
@@ -269,8 +272,9 @@ BATQ_API batq_status batq_linear_grouped_workspace_size(const batq_linear_args* 
  * Figure 2: transform, clip and quantise each linear's activations, then the
  * W4A4 product).  Linear i's codes and scales go to its 256-byte-aligned part
  * of the workspace, in order.  When every X is bf16, one tensor-core
- * quantiser launch covers all activations; when every S > 128 and every
- * out_dtype is the same, one CTA-pair GEMM launch covers all products, which
+ * quantiser launch covers all activations; when the products qualify (see
+ * batq_gemm_mxfp4_grouped: every S > 128, or every S <= 128 in one tile
+ * configuration, with one out_dtype), one GEMM launch covers them all, which
  * saves the per-launch fill and drain of 2 x (count - 1) launches.  Otherwise
  * the linears' kernels run one after another.  The outputs must not overlap
  * one another or any input.  GEMM results equal batq_linear's bit for bit;

@@ -462,13 +462,22 @@ batq_status quant_group_checked(const batq_quant_args* q, int count, cudaStream_
   return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
 }
 
-// Launch an already checked GEMM group: one CTA-pair launch when every S > 128
-// and every output type agrees, else one launch per product.  weights_ready:
-// the grid before this call writes no weights.
+// Tile configuration of the single-CTA GEMM for S <= 128 tokens.
+int small_bucket(int S) { return S <= 16 ? 0 : S <= 32 ? 1 : S <= 64 ? 2 : 3; }
+
+// Launch an already checked GEMM group: one CTA-pair launch when every S > 128,
+// one single-CTA launch when every S <= 128 falls in the same tile
+// configuration (S <= 16 / 32 / 64 / 128), in both cases with one output
+// type; else one launch per product.  weights_ready: the grid before this
+// call writes no weights.
 batq_status gemm_group_checked(const batq_gemm_args* g, int count, bool weights_ready, cudaStream_t s) {
-  bool all_pair = true;
-  for (int i = 0; i < count; ++i) all_pair = all_pair && g[i].S > 128 && g[i].out_dtype == g[0].out_dtype;
-  if (!all_pair) {
+  bool all_pair = true, all_small = true;
+  for (int i = 0; i < count; ++i) {
+    const bool same_out = g[i].out_dtype == g[0].out_dtype;
+    all_pair = all_pair && g[i].S > 128 && same_out;
+    all_small = all_small && g[i].S <= 128 && small_bucket(g[i].S) == small_bucket(g[0].S) && same_out;
+  }
+  if (!all_pair && !all_small) {
     for (int i = 0; i < count; ++i) {
       // After the first, the grid before each launch is an earlier GEMM of the
       // group, whose output overlaps no input.
@@ -498,7 +507,7 @@ batq_status gemm_group_checked(const batq_gemm_args* g, int count, bool weights_
     L.gs_a = nullptr;
     L.gs_w = nullptr;
   }
-  cudaError_t e = batq::launch_gemm_pair_group(G, count);
+  cudaError_t e = all_pair ? batq::launch_gemm_pair_group(G, count) : batq::launch_gemm_mxfp4_small_group(G, count);
   if (e == cudaErrorInvalidValue) return BATQ_ERR_ALIGNMENT;
   return e == cudaSuccess ? BATQ_OK : BATQ_ERR_CUDA;
 }

@@ -94,11 +94,32 @@ struct GemmArgs {
   const float* gs_w;
 };
 
-template <int BN, bool kSwap, int kStages, bool kOutBF16, int kFmt>
+// One product of a launch: its tensor maps and arguments.  A launch runs one
+// to kG of them (same tile configuration), one CTA per output tile; problem
+// p's CTAs are blocks block_begin .. block_begin + its tile count - 1.
+struct MxProblem {
+  CUtensorMap tm_p, tm_q, tm_out;
+  GemmArgs g;
+  int block_begin;
+};
+
+template <int kG>
+struct MxLaunch {
+  MxProblem prob[kG];
+  int count;
+};
+
+template <int BN, bool kSwap, int kStages, bool kOutBF16, int kFmt, int kG>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_gemm_mxfp4(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
-                 const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ GemmArgs g) {
+    k_gemm_mxfp4(const __grid_constant__ MxLaunch<kG> L) {
   using C = GemmCfg<BN, kSwap, kStages, kFmt>;
+  int pi = 0;  // this CTA's problem
+#pragma unroll
+  for (int r = 1; r < kG; ++r)
+    if (r < L.count && (int)blockIdx.x >= L.prob[r].block_begin) pi = r;
+  const MxProblem& P = L.prob[pi];
+  const GemmArgs& g = P.g;
+  const int bid = (int)blockIdx.x - P.block_begin;  // this CTA's tile within its problem
   constexpr bool kFp8 = C::kFp8;
   constexpr int kBK = C::kBK, kKPerMma = C::kKPerMma;
   extern __shared__ uint8_t smem_raw[];
@@ -111,14 +132,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Fetch the TMA descriptors while the barriers and TMEM are set up.
   if (threadIdx.x == 0) {
-    tma_prefetch_map(&tm_p);
-    tma_prefetch_map(&tm_q);
-    tma_prefetch_map(&tm_out);
+    tma_prefetch_map(&P.tm_p);
+    tma_prefetch_map(&P.tm_q);
+    tma_prefetch_map(&P.tm_out);
   }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int tile_p = blockIdx.x / g.tiles_q;
-  const int tile_q = blockIdx.x % g.tiles_q;
+  const int tile_p = bid / g.tiles_q;
+  const int tile_q = bid % g.tiles_q;
   const int p0 = tile_p * kBM;
   const int q0 = tile_q * BN;
 
@@ -181,8 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int katoms = min(C::kAtoms, (g.kpad >> 2) - katom0);
         const uint32_t sf_bytes = (uint32_t)katoms * kSfAtom;
         mbar_arrive_expect_tx(&full[s], (uint32_t)(C::kPBytes + C::kQBytes) + sf_bytes * (1 + q_atoms_valid));
-        tma_load_2d(st, &tm_p, &full[s], ks * kBKBytes, p0);
-        tma_load_2d(st + C::kPBytes, &tm_q, &full[s], ks * kBKBytes, q0);
+        tma_load_2d(st, &P.tm_p, &full[s], ks * kBKBytes, p0);
+        tma_load_2d(st + C::kPBytes, &P.tm_q, &full[s], ks * kBKBytes, q0);
         const size_t row_stride = (size_t)(g.kpad >> 2) * kSfAtom;
         bulk_load(st + C::kPBytes + C::kQBytes, g.p_scales + (size_t)p_tile_atom * row_stride + katom0 * kSfAtom,
                   sf_bytes, &full[s]);
@@ -357,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         for (int bx = 0; bx < kBoxes; ++bx) {
-          tma_store_2d(&tm_out, stage_out + bx * 4096, q0 + bx * kColsPerBox, p0 + 32 * quad);
+          tma_store_2d(&P.tm_out, stage_out + bx * 4096, q0 + bx * kColsPerBox, p0 + 32 * quad);
         }
         tma_store_commit();
         tma_store_wait_read_all();
@@ -374,8 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Tensor maps and arguments of one product; its CTA count, or -1 when a map
+// cannot be encoded.
 template <int BN, bool kSwap, int kStages, bool kOutBF16, int kFmt>
-cudaError_t launch_cfg(const GemmLaunch& L) {
+int fill_problem(const GemmLaunch& L, int block_begin, MxProblem* P) {
   using C = GemmCfg<BN, kSwap, kStages, kFmt>;
   constexpr bool kFp8 = C::kFp8;
   const int rows_p = kSwap ? L.M : L.S;
@@ -383,25 +406,22 @@ cudaError_t launch_cfg(const GemmLaunch& L) {
   const uint8_t* codes_p = kSwap ? L.w_codes : L.a_codes;
   const uint8_t* codes_q = kSwap ? L.a_codes : L.w_codes;
   const uint64_t row_bytes = (uint64_t)(kFp8 ? L.N : L.N / 2);
-
-  CUtensorMap tm_p, tm_q, tm_out;
-  if (!make_map_2d(&tm_p, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_p, row_bytes, (uint64_t)rows_p, row_bytes, kBKBytes,
+  if (!make_map_2d(&P->tm_p, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_p, row_bytes, (uint64_t)rows_p, row_bytes, kBKBytes,
                    kBM, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  if (!make_map_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_q, row_bytes, (uint64_t)rows_q, row_bytes, kBKBytes,
+    return -1;
+  if (!make_map_2d(&P->tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_q, row_bytes, (uint64_t)rows_q, row_bytes, kBKBytes,
                    BN, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+    return -1;
   if (!kSwap) {
     const uint32_t esz = kOutBF16 ? 2 : 4;
-    if (!make_map_2d(&tm_out, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
+    if (!make_map_2d(&P->tm_out, kOutBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.out,
                      (uint64_t)L.M, (uint64_t)L.S, (uint64_t)L.ldo * esz, 128 / esz, 32,
                      CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
+      return -1;
   } else {
-    tm_out = tm_q;  // unused in the decode epilogue
+    P->tm_out = P->tm_q;  // unused in the decode epilogue
   }
-
-  GemmArgs g;
+  GemmArgs& g = P->g;
   g.p_scales = kSwap ? L.w_scales : L.a_scales;
   g.q_scales = kSwap ? L.a_scales : L.w_scales;
   g.out = L.out;
@@ -420,9 +440,26 @@ cudaError_t launch_cfg(const GemmLaunch& L) {
   g.early_w = L.weights_ready ? 1 : 0;
   g.gs_a = L.gs_a;
   g.gs_w = L.gs_w;
-  const int tiles_p = (rows_p + kBM - 1) / kBM;
+  P->block_begin = block_begin;
+  return ((rows_p + kBM - 1) / kBM) * g.tiles_q;
+}
 
-  auto kern = k_gemm_mxfp4<BN, kSwap, kStages, kOutBF16, kFmt>;
+// Ls[0 .. count-1]: products of one tile configuration, format and output
+// type on Ls[0]'s stream.
+template <int BN, bool kSwap, int kStages, bool kOutBF16, int kFmt, int kG>
+cudaError_t launch_cfg(const GemmLaunch* Ls, int count) {
+  using C = GemmCfg<BN, kSwap, kStages, kFmt>;
+  if (count < 1 || count > kG) return cudaErrorInvalidValue;
+  MxLaunch<kG> T = {};
+  long long blocks = 0;
+  for (int q = 0; q < count; ++q) {
+    const int n = fill_problem<BN, kSwap, kStages, kOutBF16, kFmt>(Ls[q], (int)blocks, &T.prob[q]);
+    if (n < 0) return cudaErrorInvalidValue;
+    blocks += n;
+  }
+  if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
+  T.count = count;
+  auto kern = k_gemm_mxfp4<BN, kSwap, kStages, kOutBF16, kFmt, kG>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -432,28 +469,50 @@ cudaError_t launch_cfg(const GemmLaunch& L) {
     attr_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(tiles_p * g.tiles_q);
+  cfg.gridDim = dim3((unsigned)blocks);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = L.stream;
+  cfg.stream = Ls[0].stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tm_p, tm_q, tm_out, g);
+  return cudaLaunchKernelEx(&cfg, kern, T);
 }
 
 template <bool kOutBF16, int kFmt>
 cudaError_t launch_dtype(const GemmLaunch& L) {
-  if (L.S <= 16) return launch_cfg<16, true, 4, kOutBF16, kFmt>(L);
-  if (L.S <= 32) return launch_cfg<32, true, 4, kOutBF16, kFmt>(L);
-  if (L.S <= 64) return launch_cfg<64, true, 4, kOutBF16, kFmt>(L);
-  if (L.S <= 128) return launch_cfg<256, false, 4, kOutBF16, kFmt>(L);
+  if (L.S <= 16) return launch_cfg<16, true, 4, kOutBF16, kFmt, 1>(&L, 1);
+  if (L.S <= 32) return launch_cfg<32, true, 4, kOutBF16, kFmt, 1>(&L, 1);
+  if (L.S <= 64) return launch_cfg<64, true, 4, kOutBF16, kFmt, 1>(&L, 1);
+  if (L.S <= 128) return launch_cfg<256, false, 4, kOutBF16, kFmt, 1>(&L, 1);
   return launch_gemm_pair(L);
 }
 
+// Tile configuration of a product with S tokens (0: S <= 16, 1: <= 32, 2: <= 64, 3: <= 128).
+int small_s_bucket(int S) { return S <= 16 ? 0 : S <= 32 ? 1 : S <= 64 ? 2 : 3; }
+
+template <bool kOutBF16>
+cudaError_t launch_small_group(const GemmLaunch* Ls, int count) {
+  switch (small_s_bucket(Ls[0].S)) {
+    case 0: return launch_cfg<16, true, 4, kOutBF16, kFmtMxfp4, kMaxGemmGroup>(Ls, count);
+    case 1: return launch_cfg<32, true, 4, kOutBF16, kFmtMxfp4, kMaxGemmGroup>(Ls, count);
+    case 2: return launch_cfg<64, true, 4, kOutBF16, kFmtMxfp4, kMaxGemmGroup>(Ls, count);
+    default: return launch_cfg<256, false, 4, kOutBF16, kFmtMxfp4, kMaxGemmGroup>(Ls, count);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_gemm_mxfp4_small_group(const GemmLaunch* Ls, int count) {
+  if (count < 1 || count > kMaxGemmGroup) return cudaErrorInvalidValue;
+  for (int q = 0; q < count; ++q)
+    if (Ls[q].fmt != kFmtMxfp4 || Ls[q].out_bf16 != Ls[0].out_bf16 || Ls[q].S > 128 ||
+        small_s_bucket(Ls[q].S) != small_s_bucket(Ls[0].S))
+      return cudaErrorInvalidValue;
+  return Ls[0].out_bf16 ? launch_small_group<true>(Ls, count) : launch_small_group<false>(Ls, count);
+}
 
 cudaError_t launch_gemm_mxfp4(const GemmLaunch& L) {
   switch (L.fmt) {

@@ -101,6 +101,11 @@ cudaError_t launch_gemm_pair(const GemmLaunch& L);
 constexpr int kMaxGemmGroup = 8;
 cudaError_t launch_gemm_pair_group(const GemmLaunch* Ls, int count);
 
+// Up to kMaxGemmGroup independent small-S GEMMs (MXFP4, all S in the same one
+// of the tile configurations S <= 16 / 32 / 64 / 128, one output type, Ls[0]'s
+// stream) in one launch of the single-CTA kernel, one CTA per output tile.
+cudaError_t launch_gemm_mxfp4_small_group(const GemmLaunch* Ls, int count);
+
 // Widen packed E2M1 codes (element 2j in the low nibble) to one E4M3 byte per
 // element holding the same value; packed_bytes must be a multiple of 16 and
 // both pointers 16-byte aligned.

@@ -199,3 +199,80 @@ def test_grouped_gemm_equals_batq_gemm_mxfp4(case):
     assert BQ.batq_device_error() == 0
     for i, (gm, ref) in enumerate(zip(gemms, refs)):
         assert torch.equal(gm["out"], ref), f"product {i} {shapes[i]}"
+
+
+def test_layer_workload_as_the_bench_runs_it():
+    """The seven S = 8192 linears of the layer workload (q, k, v, o, gate, up, down) through one grouped
+    call, as the bench times them: every output, code and scale equals batq_linear's bit for bit (each
+    of these shapes takes the tensor-core transform in batq_linear too), and rows of the down linear
+    match the oracle."""
+    linears = []
+    for j in range(len(WL.LAYER_LINEARS)):
+        w = WL.layer_linear(j, with_w=False)
+        g = torch.Generator(device="cuda").manual_seed(900 + j)
+        B, ratios = GU.params(w)
+        wc, wsc = BQ.empty_act_buffers(w.M, w.N)
+        wc.random_(0, 256, generator=g)
+        wsc.random_(118, 134, generator=g)
+        out = torch.full((w.S, w.M), float("nan"), dtype=torch.float32, device="cuda")
+        linears.append(dict(w=w, X=GU.x_tensor(w), A=w.A, B=B, ratios=ratios, w_codes=wc, w_scales=wsc, M=w.M,
+                            out=out))
+    ws = _run_grouped(linears)
+    parts = _workspace_parts(ws, linears)
+    for i, (l, (codes, scales)) in enumerate(zip(linears, parts)):
+        _assert_linear_equal(i, l, codes, scales)
+    # sampled rows of the down linear (K = 12288) against the oracle's fp64 GEMM of the grouped codes
+    l, (codes, scales) = linears[-1], parts[-1]
+    w = l["w"]
+    rows = np.sort(np.random.default_rng(901).choice(w.S, 48, replace=False))
+    c_h = codes.cpu().numpy()
+    a_sc = O.scales_from_mma_layout(scales.cpu().numpy(), w.S, w.k)
+    ref, T = O.gemm_rows(c_h, a_sc, l["w_codes"].cpu().numpy(),
+                         O.scales_from_mma_layout(l["w_scales"].cpu().numpy(), w.M, w.k), rows)
+    PT.assert_gemm_parity(l["out"].cpu().numpy()[rows], ref, T, "layer down, grouped")
+
+
+@pytest.mark.parametrize("shapes", [
+    [(16, 4096, 4096), (16, 1024, 4096), (9, 12288, 4096), (1, 272, 512)],  # S <= 16 (decode, BN = 16)
+    [(32, 1024, 4096), (17, 512, 1024)],                                     # S <= 32
+    [(40, 2048, 4096), (64, 256, 320)],                                      # S <= 64, ragged K stage
+    [(100, 1024, 4096), (128, 256, 512), (65, 512, 1024)],                   # S <= 128 (BN = 256)
+])
+def test_small_S_gemm_group_equals_single_calls(shapes):
+    """Products of one small-S tile configuration share one launch of the single-CTA kernel."""
+    g = torch.Generator(device="cuda").manual_seed(sum(s[0] for s in shapes))
+    gemms, refs = [], []
+    for S, M, N in shapes:
+        a, sa = BQ.empty_act_buffers(S, N)
+        a.random_(0, 256, generator=g)
+        sa.random_(116, 136, generator=g)
+        w, sw = BQ.empty_act_buffers(M, N)
+        w.random_(0, 256, generator=g)
+        sw.random_(116, 136, generator=g)
+        out = torch.full((S, M), float("nan"), dtype=torch.float32, device="cuda")
+        gemms.append(dict(a_codes=a, a_scales=sa, w_codes=w, w_scales=sw, S=S, M=M, N=N, out=out))
+        ref = torch.empty_like(out)
+        BQ.batq_gemm_mxfp4(a, sa, w, sw, S, M, N, ref)
+        refs.append(ref)
+    BQ.batq_gemm_mxfp4_grouped(gemms)
+    torch.cuda.synchronize()
+    assert BQ.batq_device_error() == 0
+    for i, (gm, ref) in enumerate(zip(gemms, refs)):
+        assert torch.equal(gm["out"], ref), f"product {i} {shapes[i]}"
+
+
+def test_decode_layer_group():
+    """A decode step of the layer's seven linears at S = 16 through one grouped call (one quantiser launch,
+    one single-CTA GEMM launch): codes within the oracle's bound, every product equal to the single-call
+    GEMM of the same codes, and the outputs within the oracle's GEMM bound."""
+    linears = []
+    for j, (name, N, M) in enumerate(WL.LAYER_LINEARS):
+        linears.append(_linear(950 + j, 16, N, M))
+    ws = _run_grouped(linears)
+    for i, (l, (codes, scales)) in enumerate(zip(linears, _workspace_parts(ws, linears))):
+        _assert_oracle_parity(f"decode group {i}", l, codes, scales)
+        w = l["w"]
+        ref = torch.empty_like(l["out"])
+        BQ.batq_gemm_mxfp4(codes.contiguous(), scales.contiguous(), l["w_codes"], l["w_scales"], w.S, w.M, w.N, ref)
+        torch.cuda.synchronize()
+        assert torch.equal(l["out"], ref), f"decode group {i}: output differs from the single-call GEMM"
