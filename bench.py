@@ -431,9 +431,8 @@ def per_config(dev, peaks, timer, sp):
                    M=z["M"], out=z["out"]) for z in zs]
         gws = torch.empty(BQ.batq_linear_grouped_workspace_size([(z["S"], z["N"]) for z in zs]),
                           dtype=torch.uint8, device=dev)
-        dgroups.append((gl, gws))
-    grp_ms = timer.median([lambda gl=gl, gws=gws: BQ.batq_linear_grouped(gl, gws, stream=sp)
-                           for gl, gws in dgroups], 10, 2) / 2
+        dgroups.append(BQ.prepare_linear_grouped(gl, gws))  # marshalled once: one ctypes call per step
+    grp_ms = timer.median([lambda f=f: f(sp) for f in dgroups], 10, 2) / 2
     per_ms = timer.median([launcher("linear", z, sp) for zs in dsets for z in zs], 10, 2) / 2
     res["decode_layer_16x7_linears"] = {
         "grouped_us": grp_ms * 1e3, "grouped_weight_gbs": dwb / grp_ms / 1e6,
@@ -633,9 +632,13 @@ def run_batq(args):
     gemm_group = [dict(a_codes=z["codes"], a_scales=z["scales"], w_codes=z["wc"], w_scales=z["wsc"], S=z["S"],
                        M=z["M"], N=z["N"], out=z["out"]) for z in layer]
     per_linear_fns = [launcher("linear", z, sp) for z in layer]
+    # the grouped calls with their arguments marshalled once (one ctypes call per launch)
+    run_group = BQ.prepare_linear_grouped(group, gws)
+    run_quant_group = BQ.prepare_quant_act_grouped(quant_group)
+    run_gemm_group = BQ.prepare_gemm_mxfp4_grouped(gemm_group)
 
     def step():
-        BQ.batq_linear_grouped(group, gws, stream=sp)
+        run_group(sp)
 
     def step_per_linear():
         for f in per_linear_fns:
@@ -671,8 +674,8 @@ def run_batq(args):
         timer.launches += 2 * len(layer) * args.steps
         # timed region 2: each grouped kernel alone (one launch covers the seven linears), median of
         # five repeats of three launches back to back (-> per-kernel throughput and roofline)
-        q_ms = timer.median([lambda: BQ.batq_quant_act_grouped(quant_group, stream=sp)], reps=3)
-        g_ms = timer.median([lambda: BQ.batq_gemm_mxfp4_grouped(gemm_group, stream=sp)], reps=3)
+        q_ms = timer.median([lambda: run_quant_group(sp)], reps=3)
+        g_ms = timer.median([lambda: run_gemm_group(sp)], reps=3)
         # each linear's own kernels, one back-to-back pass with events between the launches
         q_each = timer.each([launcher("quant", z, sp) for z in layer])
         g_each = timer.each([launcher("gemm", z, sp) for z in layer])

@@ -222,11 +222,12 @@ typedef struct batq_quant_args {
 
 /*
  * `count` (1..8) independent batq_quant_act calls (no y_debug) on one stream.
- * When every X is bf16, one launch of the tensor-core quantiser covers all of
- * them (their tiles form one list); otherwise they run one after another.
- * Codes and scales equal batq_quant_act's wherever that call also takes the
- * tensor-core transform, and otherwise meet the same parity bound (see
- * batq_linear_grouped).  Outputs must not overlap one another or any input.
+ * Each activation takes the kernel its own call would take: those for the
+ * tensor-core transform (bf16, at least six 128 x 128 tiles per SM) share one
+ * launch (their tiles form one list); the others get their own launches of
+ * the CUDA-core kernel, which start side by side (each waits for the launch
+ * before it only before finishing).  Codes and scales equal batq_quant_act's
+ * bit for bit.  Outputs must not overlap one another or any input.
  * Errors: as batq_quant_act for each (the first failing check's code),
  * BATQ_ERR_INVALID_ARG for count out of range; nothing is launched when a
  * check fails.
@@ -271,17 +272,14 @@ BATQ_API batq_status batq_linear_grouped_workspace_size(const batq_linear_args* 
  * batq_linear computes with its own arguments (BATQuant thelatestinai.com page,
  * Figure 2: transform, clip and quantise each linear's activations, then the
  * W4A4 product).  Linear i's codes and scales go to its 256-byte-aligned part
- * of the workspace, in order.  When every X is bf16, one tensor-core
- * quantiser launch covers all activations; when the products qualify (see
+ * of the workspace, in order.  The activations are quantised as by
+ * batq_quant_act_grouped; when the products qualify (see
  * batq_gemm_mxfp4_grouped: every S > 128, or every S <= 128 in one tile
  * configuration, with one out_dtype), one GEMM launch covers them all, which
  * saves the per-launch fill and drain of 2 x (count - 1) launches.  Otherwise
- * the linears' kernels run one after another.  The outputs must not overlap
- * one another or any input.  GEMM results equal batq_linear's bit for bit;
- * activation codes equal them wherever batq_linear also uses the tensor-core
- * transform (bf16 and at least six 128 x 128 tiles per SM), and otherwise
- * meet the same parity bound (the two transforms round Y in different
- * orders).  Errors: as batq_linear for each linear (the first failing
+ * the GEMMs run one after another.  The outputs must not overlap one another
+ * or any input.  Codes, scales and outputs equal batq_linear's bit for bit.
+ * Errors: as batq_linear for each linear (the first failing
  * check's code), BATQ_ERR_INVALID_ARG for count out of range.  Nothing is
  * launched when a check fails.
  */

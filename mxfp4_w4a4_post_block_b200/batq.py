@@ -235,6 +235,59 @@ def batq_gemm_mxfp4_grouped(gemms, stream=None):
            "batq_gemm_mxfp4_grouped")
 
 
+def prepare_linear_grouped(linears, workspace):
+    """batq_linear_grouped with its arguments marshalled once: returns run(stream=None), which launches
+    the same call with a single ctypes call (for decode-size steps, where building the argument array
+    on every call would cost more host time than the kernels take)."""
+    arr, keep = _linear_args(linears)
+    lib = _lib.load()
+    ws_ptr, ws_bytes, n = _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(), len(linears)
+    addr = ctypes.addressof(arr)
+
+    def run(stream=None):
+        _check(lib.batq_linear_grouped(addr, n, ws_ptr, ws_bytes, _stream(stream)), "batq_linear_grouped")
+
+    run._keep = (arr, keep, linears, workspace)  # the marshalled arguments and the tensors stay alive
+    return run
+
+
+def prepare_quant_act_grouped(acts, layout=BATQ_SCALES_MMA):
+    """batq_quant_act_grouped with its arguments marshalled once (see prepare_linear_grouped)."""
+    arr = (_QuantArgs * len(acts))()
+    keep = []
+    for i, q in enumerate(acts):
+        X = q["X"]
+        a = _host_f32(q["A"], 64, "A")
+        keep.append(a)
+        arr[i] = _QuantArgs(_dev_ptr(X, "X"), _dtype_code(X), X.shape[0], X.shape[1], X.stride(0), a.ctypes.data,
+                            _dev_ptr(q["B"], "B"), _dev_ptr(q["ratios"], "ratios"), _dev_ptr(q["codes"], "codes"),
+                            _dev_ptr(q["scales"], "scales"), int(layout))
+    lib, addr, n = _lib.load(), ctypes.addressof(arr), len(acts)
+
+    def run(stream=None):
+        _check(lib.batq_quant_act_grouped(addr, n, _stream(stream)), "batq_quant_act_grouped")
+
+    run._keep = (arr, keep, acts)
+    return run
+
+
+def prepare_gemm_mxfp4_grouped(gemms):
+    """batq_gemm_mxfp4_grouped with its arguments marshalled once (see prepare_linear_grouped)."""
+    arr = (_GemmArgs * len(gemms))()
+    for i, g in enumerate(gemms):
+        out = g["out"]
+        arr[i] = _GemmArgs(_dev_ptr(g["a_codes"], "a_codes"), _dev_ptr(g["a_scales"], "a_scales"),
+                           _dev_ptr(g["w_codes"], "w_codes"), _dev_ptr(g["w_scales"], "w_scales"), int(g["S"]),
+                           int(g["M"]), int(g["N"]), _dtype_code(out), _dev_ptr(out, "out"), out.stride(0))
+    lib, addr, n = _lib.load(), ctypes.addressof(arr), len(gemms)
+
+    def run(stream=None):
+        _check(lib.batq_gemm_mxfp4_grouped(addr, n, _stream(stream)), "batq_gemm_mxfp4_grouped")
+
+    run._keep = (arr, gemms)
+    return run
+
+
 def batq_linear_no_alloc(X, A, B, ratios, w_codes, w_scales, M, out, stream=None):
     """batq_linear for callers that cannot allocate device memory: the scratch for the
     quantised activations comes from a fixed array inside the library (see

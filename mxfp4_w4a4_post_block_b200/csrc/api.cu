@@ -424,25 +424,17 @@ batq_status batq_linear(const void* X, batq_dtype x_dtype, int S, int N, int ldx
 
 // ------------------------------------------------------------------ groups of linears
 
-// Launch an already checked quantiser group: one tensor-core launch when every
-// X is bf16, else one launch per activation.
+// Launch an already checked quantiser group.  Each activation takes the
+// kernel its own batq_quant_act call would take, so the codes are the same:
+// those for the tensor-core kernel (bf16, six or more 128 x 128 tiles per SM)
+// share one launch of it, the others one launch of the CUDA-core kernel per
+// input type.
 batq_status quant_group_checked(const batq_quant_args* q, int count, cudaStream_t s) {
-  bool all_bf16 = true;
-  for (int i = 0; i < count; ++i) all_bf16 = all_bf16 && q[i].x_dtype == BATQ_BF16;
-  if (!all_bf16) {
-    for (int i = 0; i < count; ++i) {
-      batq_status st = launch_quant(q[i].X, q[i].x_dtype, q[i].S, q[i].N, q[i].ldx, q[i].A_host, q[i].B_dev,
-                                    q[i].ratios_dev, q[i].codes, q[i].scales, q[i].layout, nullptr,
-                                    batq::kFmtMxfp4, s);
-      if (st != BATQ_OK) return st;
-    }
-    return BATQ_OK;
-  }
   batq::QuantLaunch Q[BATQ_MAX_LINEAR_GROUP];
   for (int i = 0; i < count; ++i) {
     batq::QuantLaunch& L = Q[i];
     L.X = q[i].X;
-    L.bf16 = true;
+    L.bf16 = (q[i].x_dtype == BATQ_BF16);
     L.S = q[i].S;
     L.N = q[i].N;
     L.ldx = q[i].ldx;

@@ -59,10 +59,12 @@ struct QuantLaunch {
 // lets its own dependents start early.
 cudaError_t launch_quant_act(const QuantLaunch& L);
 
-// Up to kMaxQuantGroup independent activations quantised in one launch of
-// the tensor-core kernel (bf16, MXFP4, MMA or linear scale layout, no
-// RMSNorm, naive Kronecker or row map), on Ls[0]'s stream with Ls[0]'s error
-// word.  Refuses (cudaErrorInvalidValue) what it does not cover.
+// Up to kMaxQuantGroup independent activations (MXFP4, MMA or linear scale
+// layout, no RMSNorm, naive Kronecker or row map) on Ls[0]'s stream with
+// Ls[0]'s error word: each takes the kernel launch_quant_act would give it,
+// and those of one kernel and input type share a launch (at most three:
+// tensor-core, CUDA-core bf16, CUDA-core fp32).  Refuses
+// (cudaErrorInvalidValue) what it does not cover.
 constexpr int kMaxQuantGroup = 8;
 cudaError_t launch_quant_act_group(const QuantLaunch* Ls, int count);
 

@@ -99,11 +99,25 @@ __device__ __forceinline__ void load_block(uint32_t box, int lane, float x[32]) 
   }
 }
 
+// One launch: 1 .. kG independent activations (one format and input type),
+// each with its tensor map and arguments; their tiles (32 tokens x 8 blocks,
+// row-major within each) form one list, problem after problem.
+template <int kG>
+struct CcLaunch {
+  CUtensorMap tmx[kG];
+  QuantArgs args[kG];
+  int tile_begin[kG];  // first tile of each problem in the list
+  int count;           // problems in use
+  int num_tiles;       // tiles of all problems
+};
+
 // kFmt: output format (Fmt); kNaive: per-block A_i from p.A_blocks; kNorm:
-// RMSNorm ahead of the transform (p.gamma and p.row_scale).
-template <bool kBF16, int kFmt, bool kNaive, bool kNorm = false>
+// RMSNorm ahead of the transform (p.gamma and p.row_scale); kG: problems per
+// launch (with more than one, each problem's A is staged in shared memory at
+// the start and the transform reads it from there, as for kNaive).
+template <bool kBF16, int kFmt, bool kNaive, bool kNorm, int kG>
 __global__ void __launch_bounds__(Tile<kBF16, kNaive, kNorm>::kThreads, 1)
-    k_quant_act(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ QuantArgs p) {
+    k_quant_act(const __grid_constant__ CcLaunch<kG> L) {
   using T = Tile<kBF16, kNaive, kNorm>;
   constexpr bool kNv = (kFmt == kFmtNvfp4);
   extern __shared__ uint8_t smem_raw[];
@@ -111,12 +125,15 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive, kNorm>::kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::kStages * T::kStageBytes);
   uint64_t* empty = full + T::kStages;
   float* gs_smem = reinterpret_cast<float*>(empty + T::kStages);  // NVFP4 per-tensor encode scale
+  // kG > 1: every problem's A (64 floats each) right after the scale word
+  // (16-byte aligned: the stages are 1 KB multiples, the barriers 144 or 192 bytes).
+  float* a_tab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(gs_smem) + 16);
   // Fetch the TMA descriptors while the barriers and TMEM are set up.
-  if (threadIdx.x == 0) {
-    tma_prefetch_map(&tmx);
-  }
+  if (threadIdx.x == 0)
+    for (int q = 0; q < L.count; ++q) tma_prefetch_map(&L.tmx[q]);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const QuantArgs& p0 = L.args[0];  // launch-wide fields: error word, NVFP4 scale sources
 
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -126,15 +143,34 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive, kNorm>::kThreads, 1)
     }
     fence_barrier_init();
   }
+  if constexpr (kG > 1)
+    for (int i = threadIdx.x; i < L.count * 64; i += blockDim.x) a_tab[i] = L.args[i >> 6].A[i & 63];
   __syncthreads();
 
   // This CTA's contiguous share of the tiles (one CTA per SM, shares differ by
   // at most one tile).  Local tile i sits in stage i % kStages; consumer group
   // i % kGroups processes it (kStages is a multiple of kGroups, so each stage
   // always serves the same group).
-  const long long ntiles = (long long)p.tiles_r * p.tiles_c;
+  const long long ntiles = L.num_tiles;
   const int t_begin = (int)((long long)blockIdx.x * ntiles / gridDim.x);
   const int nloc = (int)((long long)(blockIdx.x + 1) * ntiles / gridDim.x) - t_begin;
+  // Problem of list tile t, and t's tile row and first block column within it.
+  struct TileAt {
+    int q, r0, c0;
+  };
+  auto tile_at = [&](int t) {
+    TileAt a;
+    a.q = 0;
+#pragma unroll
+    for (int r = 1; r < kG; ++r)
+      if (r < L.count && t >= L.tile_begin[r]) a.q = r;
+    const QuantArgs& pq = L.args[a.q];
+    const int lt = t - L.tile_begin[a.q];
+    const int tr = tile_row(lt, pq);
+    a.r0 = tr * kRows;
+    a.c0 = (lt - tr * pq.tiles_c) * kCols;
+    return a;
+  };
 
   if (warp == T::kConsumerWarps) {
     // ---------------- producer: one thread issues the TMA boxes ----------------
@@ -149,20 +185,19 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive, kNorm>::kThreads, 1)
       if constexpr (kNv) {
         // Per-tensor encode scale, published to the consumers through the
         // release of this thread's first arrivals on the stage barriers.
-        const float gs = nv_encode_scale(p);
+        const float gs = nv_encode_scale(p0);
         *gs_smem = gs;
-        if (p.gs_out != nullptr && blockIdx.x == 0) *p.gs_out = gs;
+        if (p0.gs_out != nullptr && blockIdx.x == 0) *p0.gs_out = gs;
       }
       for (int i = 0; i < nloc; ++i) {
         const int s = i % T::kStages;
         if (!mbar_wait(&empty[s], ((i / T::kStages) & 1) ^ 1)) {
-          set_error(p.err, kErrReleaseTimeout);
+          set_error(p0.err, kErrReleaseTimeout);
           break;
         }
-        const int t = t_begin + i;
-        const int tr = tile_row(t, p);
-        const int r0 = tr * kRows;
-        const int c0 = (t - tr * p.tiles_c) * kCols;
+        const TileAt at = tile_at(t_begin + i);
+        const QuantArgs& p = L.args[at.q];
+        const int r0 = at.r0, c0 = at.c0;
         if (r0 < p.S) {
           const int nb = min(kCols, p.k - c0);  // even: k is even and c0 a multiple of 8
           uint8_t* dst = smem + s * T::kStageBytes;
@@ -170,7 +205,7 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive, kNorm>::kThreads, 1)
                                   (kNaive ? (uint32_t)nb * 256u : 0u) + (kNorm ? (uint32_t)nb * 128u : 0u);
           // the box always delivers all 8 block columns (zero-filled past k)
           mbar_arrive_expect_tx(&full[s], (uint32_t)T::kXBytes + pbytes);
-          tma_load_3d(dst, &tmx, &full[s], 0, r0, c0);
+          tma_load_3d(dst, &L.tmx[at.q], &full[s], 0, r0, c0);
           bulk_load(dst + T::kBOffset, p.B + (size_t)c0 * 16, (uint32_t)nb * 64u, &full[s]);
           if (p.ratios != nullptr) bulk_load(dst + T::kROffset, p.ratios + (size_t)c0 * 2, (uint32_t)nb * 8u, &full[s]);
           if constexpr (kNaive) bulk_load(dst + T::kAOffset, p.A_blocks + (size_t)c0 * 64, (uint32_t)nb * 256u, &full[s]);
@@ -191,10 +226,9 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive, kNorm>::kThreads, 1)
   const int wc = warp % kCols;  // block column of the tile owned by this warp
   for (int i = grp; i < nloc; i += T::kGroups) {
     const int s = i % T::kStages;
-    const int t = t_begin + i;
-    const int tr = tile_row(t, p);
-    const int r0 = tr * kRows;
-    const int c0 = (t - tr * p.tiles_c) * kCols;
+    const TileAt at = tile_at(t_begin + i);
+    const QuantArgs& p = L.args[at.q];
+    const int r0 = at.r0, c0 = at.c0;
     const int b = c0 + wc;
     const int row = r0 + lane;
     if (!mbar_wait_warp(&full[s], (i / T::kStages) & 1)) {
@@ -241,6 +275,9 @@ __global__ void __launch_bounds__(Tile<kBF16, kNaive, kNorm>::kThreads, 1)
       float2 y2[16];
       if constexpr (kNaive) {
         const uint32_t ap = st + T::kAOffset + wc * 256;
+        gpk_transform(x, [&](int a, int j) { return lds64f(ap + (8 * a + 2 * j) * 4); }, Bm, y2);
+      } else if constexpr (kG > 1) {
+        const uint32_t ap = smem_u32(a_tab) + at.q * 256;
         gpk_transform(x, [&](int a, int j) { return lds64f(ap + (8 * a + 2 * j) * 4); }, Bm, y2);
       } else {
         gpk_transform(x, [&](int a, int j) { return make_float2(p.A[8 * a + 2 * j], p.A[8 * a + 2 * j + 1]); }, Bm,
@@ -299,39 +336,51 @@ QuantArgs make_args(const QuantLaunch& L) {
   return a;
 }
 
-template <bool kBF16, int kFmt, bool kNaive = false, bool kNorm = false>
-cudaError_t launch_impl(const QuantLaunch& L, const QuantArgs& a) {
+// Ls / as [0 .. count-1]: one format and input type on Ls[0]'s stream.
+template <bool kBF16, int kFmt, bool kNaive = false, bool kNorm = false, int kG = 1>
+cudaError_t launch_impl(const QuantLaunch* Ls, const QuantArgs* as, int count) {
   using T = Tile<kBF16, kNaive, kNorm>;
-  // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
-  CUtensorMap map;
-  const uint64_t esz = kBF16 ? 2u : 4u;
-  if (!make_map_3d_swizzled(&map, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.X,
-                            32, (uint64_t)L.S, (uint64_t)(L.N / 32), (uint64_t)L.ldx * esz, 32 * esz, 32, kRows,
-                            kCols, kBF16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) {
-    return cudaErrorInvalidValue;
+  if (count < 1 || count > kG) return cudaErrorInvalidValue;
+  CcLaunch<kG> C = {};
+  long long tiles = 0;
+  for (int q = 0; q < count; ++q) {
+    const QuantLaunch& L = Ls[q];
+    // X viewed as {32 elements of a block, S tokens, k blocks}; one box = one tile.
+    const uint64_t esz = kBF16 ? 2u : 4u;
+    if (!make_map_3d_swizzled(&C.tmx[q], kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                              L.X, 32, (uint64_t)L.S, (uint64_t)(L.N / 32), (uint64_t)L.ldx * esz, 32 * esz, 32,
+                              kRows, kCols, kBF16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) {
+      return cudaErrorInvalidValue;
+    }
+    C.args[q] = as[q];
+    C.tile_begin[q] = (int)tiles;
+    tiles += (long long)as[q].tiles_r * as[q].tiles_c;
   }
+  if (tiles >= (1LL << 31)) return cudaErrorInvalidValue;
+  C.count = count;
+  C.num_tiles = (int)tiles;
+  auto kern = k_quant_act<kBF16, kFmt, kNaive, kNorm, kG>;
+  const int smem_bytes = T::kSmemBytes + (kG > 1 ? kG * 256 : 0);
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_quant_act<kBF16, kFmt, kNaive, kNorm>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         T::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int ntiles = a.tiles_r * a.tiles_c;
-  const int grid = ntiles < sm_count() ? ntiles : sm_count();  // one CTA per SM
+  const int grid = tiles < sm_count() ? (int)tiles : sm_count();  // one CTA per SM
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(T::kThreads);
-  cfg.dynamicSmemBytes = T::kSmemBytes;
-  cfg.stream = L.stream;
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = Ls[0].stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_quant_act<kBF16, kFmt, kNaive, kNorm>, map, a);
+  return cudaLaunchKernelEx(&cfg, kern, C);
 }
 
 }  // namespace
@@ -347,32 +396,46 @@ cudaError_t launch_quant_act(const QuantLaunch& L) {
   if (L.bf16 && tc_tiles >= 6LL * sm_count()) return launch_quant_act_tc(L, a);
   if (L.gamma != nullptr) {  // RMSNorm ahead of the transform: MXFP4 output, shared A
     if (L.fmt != kFmtMxfp4 || L.A_blocks != nullptr || L.row_scale == nullptr) return cudaErrorInvalidValue;
-    return L.bf16 ? launch_impl<true, kFmtMxfp4, false, true>(L, a) : launch_impl<false, kFmtMxfp4, false, true>(L, a);
+    return L.bf16 ? launch_impl<true, kFmtMxfp4, false, true>(&L, &a, 1) : launch_impl<false, kFmtMxfp4, false, true>(&L, &a, 1);
   }
   if (L.A_blocks != nullptr) {  // naive Kronecker: MXFP4 output
     if (L.fmt != kFmtMxfp4) return cudaErrorInvalidValue;
-    return L.bf16 ? launch_impl<true, kFmtMxfp4, true>(L, a) : launch_impl<false, kFmtMxfp4, true>(L, a);
+    return L.bf16 ? launch_impl<true, kFmtMxfp4, true>(&L, &a, 1) : launch_impl<false, kFmtMxfp4, true>(&L, &a, 1);
   }
   switch (L.fmt) {
-    case kFmtMxfp4: return L.bf16 ? launch_impl<true, kFmtMxfp4>(L, a) : launch_impl<false, kFmtMxfp4>(L, a);
-    case kFmtMxfp8: return L.bf16 ? launch_impl<true, kFmtMxfp8>(L, a) : launch_impl<false, kFmtMxfp8>(L, a);
-    case kFmtNvfp4: return L.bf16 ? launch_impl<true, kFmtNvfp4>(L, a) : launch_impl<false, kFmtNvfp4>(L, a);
+    case kFmtMxfp4: return L.bf16 ? launch_impl<true, kFmtMxfp4>(&L, &a, 1) : launch_impl<false, kFmtMxfp4>(&L, &a, 1);
+    case kFmtMxfp8: return L.bf16 ? launch_impl<true, kFmtMxfp8>(&L, &a, 1) : launch_impl<false, kFmtMxfp8>(&L, &a, 1);
+    case kFmtNvfp4: return L.bf16 ? launch_impl<true, kFmtNvfp4>(&L, &a, 1) : launch_impl<false, kFmtNvfp4>(&L, &a, 1);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_quant_act_group(const QuantLaunch* Ls, int count) {
   if (count < 1 || count > kMaxQuantGroup) return cudaErrorInvalidValue;
-  QuantArgs as[kMaxQuantGroup];
+  // Each activation takes the kernel its own launch_quant_act would take, so
+  // the codes are the same: one launch for those of the tensor-core kernel,
+  // one for the bf16 and one for the fp32 ones of the CUDA-core kernel.
+  QuantLaunch part[3][kMaxQuantGroup];
+  QuantArgs args[3][kMaxQuantGroup];
+  int n[3] = {0, 0, 0};
   for (int q = 0; q < count; ++q) {
     const QuantLaunch& L = Ls[q];
-    if (!L.bf16 || L.fmt != kFmtMxfp4 || L.gamma != nullptr || L.row_scale != nullptr || L.A_blocks != nullptr ||
+    if (L.fmt != kFmtMxfp4 || L.gamma != nullptr || L.row_scale != nullptr || L.A_blocks != nullptr ||
         L.row_map != nullptr || L.amax_out != nullptr)
       return cudaErrorInvalidValue;
-    as[q] = make_args(L);
-    as[q].err = Ls[0].err;
+    const long long tc_tiles = (long long)((L.N / 32 + 3) / 4) * ((L.S + 127) / 128);
+    const int k = (L.bf16 && tc_tiles >= 6LL * sm_count()) ? 0 : (L.bf16 ? 1 : 2);
+    part[k][n[k]] = L;
+    part[k][n[k]].stream = Ls[0].stream;
+    args[k][n[k]] = make_args(L);
+    args[k][n[k]].err = Ls[0].err;
+    ++n[k];
   }
-  return launch_quant_act_tc_group(Ls, as, count);
+  cudaError_t e = cudaSuccess;
+  if (n[0] > 0) e = launch_quant_act_tc_group(part[0], args[0], n[0]);
+  if (e == cudaSuccess && n[1] > 0) e = launch_impl<true, kFmtMxfp4, false, false, kMaxQuantGroup>(part[1], args[1], n[1]);
+  if (e == cudaSuccess && n[2] > 0) e = launch_impl<false, kFmtMxfp4, false, false, kMaxQuantGroup>(part[2], args[2], n[2]);
+  return e;
 }
 
 }  // namespace batq

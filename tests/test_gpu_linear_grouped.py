@@ -1,13 +1,13 @@
 """batq_linear_grouped: independent linears in one quantiser launch and one CTA-pair GEMM launch.
 
-* Where batq_linear itself takes the tensor-core transform (bf16, six or more 128 x 128 tiles per SM),
-  the grouped call must give the same workspace codes and scales and the same outputs bit for bit:
-  the same kernels' arithmetic, only the tiles of several problems share one launch.
-* Smaller shapes take the tensor-core transform in the group where batq_linear takes the CUDA-core
-  one: their codes must meet the oracle parity bound, and the outputs must equal the oracle's fp64
-  GEMM of those codes within 1e-4 * sum |a||w|.
-* Groups that do not qualify (fp32 activations, S <= 128, mixed output types) run the linears' own
-  kernels and must equal batq_linear bit for bit.
+* Every activation takes the quantiser kernel its own batq_linear call would take (the tensor-core
+  ones share one launch, the CUDA-core ones run as side-by-side launches), and the GEMMs of one tile
+  configuration share one launch: the grouped call must give the same workspace codes and scales
+  and the same outputs as batq_linear, bit for bit, for every shape.
+* Small shapes are also checked against the oracle (codes within the parity bound, outputs within
+  1e-4 * sum |a||w| of the fp64 GEMM of those codes).
+* Groups whose GEMMs do not share a configuration (mixed S classes, mixed output types) run them
+  one after another and must still equal batq_linear bit for bit.
 """
 
 import numpy as np
@@ -106,14 +106,22 @@ def test_bf16_output_group_equals_batq_linear():
     _assert_equal_to_batq_linear(linears, ws)
 
 
-def test_small_shapes_match_the_oracle():
-    # below six tensor-core tiles per SM: batq_linear would take the CUDA-core transform, the group
-    # takes the tensor-core one; both must meet the oracle's bound
+def test_small_shapes_match_batq_linear_and_the_oracle():
+    # below six tensor-core tiles per SM: the CUDA-core transform, one launch each, side by side
     shapes = [(200, 512, 272), (129, 1024, 256), (300, 768, 1024), (640, 4096, 512), (257, 64, 16)]
     linears = [_linear(20 + i, *shp) for i, shp in enumerate(shapes)]
     ws = _run_grouped(linears)
     for i, (l, (codes, scales)) in enumerate(zip(linears, _workspace_parts(ws, linears))):
         _assert_oracle_parity(f"group linear {i}", l, codes, scales)
+    _assert_equal_to_batq_linear(linears, ws)
+
+
+def test_mixed_quantiser_kernels_in_one_group():
+    # two activations for the tensor-core kernel (one grouped launch) and three for the CUDA-core one
+    shapes = [(4096, 4096, 512), (200, 512, 272), (1280, 12288, 256), (640, 4096, 512), (300, 768, 1024)]
+    linears = [_linear(60 + i, *shp) for i, shp in enumerate(shapes)]
+    ws = _run_grouped(linears)
+    _assert_equal_to_batq_linear(linears, ws)
 
 
 @pytest.mark.parametrize("case", ["fp32_input", "short_S", "mixed_out"])
@@ -125,17 +133,7 @@ def test_groups_that_do_not_qualify_run_the_linears_own_kernels(case):
     else:
         linears = [_linear(35, 4096, 4096, 512), _linear(36, 4096, 4096, 256, out_dtype=torch.bfloat16)]
     ws = _run_grouped(linears)
-    if case == "fp32_input":
-        _assert_equal_to_batq_linear(linears, ws)  # per-linear quantisers and GEMMs
-    else:
-        # bf16 everywhere: one grouped quantiser; the GEMMs run one by one.  The large linears take the
-        # tensor-core transform in batq_linear too, so they compare bit for bit; the short ones against
-        # the oracle
-        for i, (l, (codes, scales)) in enumerate(zip(linears, _workspace_parts(ws, linears))):
-            if l["w"].S == 4096:
-                _assert_linear_equal(i, l, codes, scales)
-            else:
-                _assert_oracle_parity(f"{case} {i}", l, codes, scales)
+    _assert_equal_to_batq_linear(linears, ws)
 
 
 def test_full_group_of_eight_and_repeat():
@@ -154,8 +152,9 @@ def test_full_group_of_eight_and_repeat():
 
 @pytest.mark.parametrize("layout", [BQ.BATQ_SCALES_MMA, BQ.BATQ_SCALES_LINEAR])
 def test_grouped_quantiser_equals_batq_quant_act(layout):
-    """Tensor-core-sized activations: one grouped launch writes what the single calls write."""
-    shapes = [(4096, 4096), (1280, 12288), (3500, 4096)]
+    """Tensor-core-sized activations (one grouped launch) and small ones (side-by-side CUDA-core
+    launches) write what the single calls write."""
+    shapes = [(4096, 4096), (1280, 12288), (3500, 4096), (200, 512), (16, 4096)]
     acts, refs = [], []
     for i, (S, N) in enumerate(shapes):
         l = _linear(70 + i, S, N, 128)
@@ -262,17 +261,19 @@ def test_small_S_gemm_group_equals_single_calls(shapes):
 
 
 def test_decode_layer_group():
-    """A decode step of the layer's seven linears at S = 16 through one grouped call (one quantiser launch,
-    one single-CTA GEMM launch): codes within the oracle's bound, every product equal to the single-call
-    GEMM of the same codes, and the outputs within the oracle's GEMM bound."""
+    """A decode step of the layer's seven linears at S = 16 through one grouped call (side-by-side
+    CUDA-core quantiser launches, one single-CTA GEMM launch): equal to batq_linear bit for bit, and
+    within the oracle's bounds."""
     linears = []
     for j, (name, N, M) in enumerate(WL.LAYER_LINEARS):
         linears.append(_linear(950 + j, 16, N, M))
     ws = _run_grouped(linears)
     for i, (l, (codes, scales)) in enumerate(zip(linears, _workspace_parts(ws, linears))):
         _assert_oracle_parity(f"decode group {i}", l, codes, scales)
-        w = l["w"]
-        ref = torch.empty_like(l["out"])
-        BQ.batq_gemm_mxfp4(codes.contiguous(), scales.contiguous(), l["w_codes"], l["w_scales"], w.S, w.M, w.N, ref)
-        torch.cuda.synchronize()
-        assert torch.equal(l["out"], ref), f"decode group {i}: output differs from the single-call GEMM"
+    _assert_equal_to_batq_linear(linears, ws)
+    # repeated back to back: the side-by-side launches of one call must not overtake the previous call
+    for _ in range(3):
+        BQ.batq_linear_grouped(linears, ws)
+    torch.cuda.synchronize()
+    assert BQ.batq_device_error() == 0
+    _assert_equal_to_batq_linear(linears, ws)
