@@ -12,7 +12,10 @@
 //     D[i][j], tiles of 128 x {16, 32, 64}, so the weight stream fills the
 //     128-row MMA and the narrow activation side sits in N.
 //
-// One CTA computes one output tile:
+// One CTA computes one output tile; one launch may cover up to eight
+// independent products of one tile configuration (a table of tensor maps and
+// arguments, each problem's CTAs a contiguous range of the grid), which is
+// how a decode step's linears share one launch:
 //   warp 0     TMA producer: per stage a 128 x 256-element P tile, a BN x 256
 //              Q tile (both 128-byte swizzled) and their scale atoms (1-D bulk
 //              copies of the 512-byte 128x4 scale tiles);

@@ -25,7 +25,11 @@
 //     entry, so 384 scalar FMAs per block become 192 packed ones;
 //   * the block extrema are in-thread (the whole block lives in one thread),
 //     the clipped amax is max(|clamp(min)|, |clamp(max)|) (clamp is
-//     monotone), and the scale comes from the exponent bits of amax.
+//     monotone), and the scale comes from the exponent bits of amax;
+//   * one launch may cover up to eight independent activations (a table of
+//     tensor maps and arguments; their tiles form one list): A then comes from
+//     a 2 KB shared-memory copy of every problem's A instead of the parameter
+//     bank, with the same values in the same FMA order.
 //
 // Output formats: MXFP4 (E2M1 + E8M0 per 32), MXFP8 (E4M3 + E8M0 per 32, the
 // W4A8 variant) and NVFP4 (E2M1 + E4M3 per 16 elements with a per-tensor fp32
