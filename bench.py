@@ -51,8 +51,8 @@ CSRC = os.path.join(ROOT, "mxfp4_w4a4_post_block_b200", "csrc")
 # `bench.py --only group --workload layer` (metrics dram__bytes_read.sum, dram__bytes_write.sum),
 # valid only for the kernel sources whose hash is recorded with it: a changed kernel reports null.
 NCU_TRAFFIC = {
-    "k_gemm_pair": {"src": "68b3d42aeabb992e", "bytes_per_step": 358029824 + 1235169280},
-    "k_quant_act_tc": {"src": "190c360bddd66df8", "bytes_per_step": 605204224 + 143690240},
+    "k_gemm_pair": {"src": "ca55f85d7e3a22f0", "bytes_per_step": 373376000 + 1235655936},
+    "k_quant_act_tc": {"src": "12c5b9d4cce2b3a7", "bytes_per_step": 605227264 + 144101376},
 }
 TRAFFIC_SOURCES = {
     "k_gemm_pair": ("gemm_pair.cu", "ptx.cuh", "kernels.h", "host_util.h", "host_util.cpp"),
