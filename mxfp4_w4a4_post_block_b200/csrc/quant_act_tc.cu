@@ -19,23 +19,22 @@
 // each CTA (one per SM) takes an equal contiguous share, so it meets at most
 // a few strips and builds each strip's P_i parts once in shared memory (24 KB,
 // 64-byte swizzled K-major rows, as the MMA reads them).  The three parts of
-// one P_i are 96 consecutive rows, so one MMA with N = 96 multiplies the
-// activations by all three at once: per tile and block column two MMAs
-// (M = 128 tokens, N = 96, K = 16) write three 32-column partial results
-// X hi, X mid, X lo side by side in TMEM, and the encoders add them in fp32
-// (hi + (mid + lo)).  That is 8 MMAs per tile where three separate N = 32
-// accumulations took 24, each of which re-read the 4 KB activation slice
-// from shared memory.
+// one P_i are 96 consecutive rows: per tile, block column and K step one MMA
+// with N = 64 (M = 128 tokens, K = 16) writes X hi and X mid side by side in
+// TMEM and one with N = 32 adds X lo onto the mid columns, so the encoders
+// read two 32-column results and add them in fp32 (hi + (mid + lo)).  That
+// is 16 MMAs per tile where three separate N = 32 accumulations took 24, each
+// of which re-read the 4 KB activation slice from shared memory.
 //   warp 0      TMA producer: one 3-D box per tile (128 tokens x 4 blocks of
 //               bf16, 32 KB, 64-byte swizzle = the MMA's K-major operand
 //               layout) into a 4-stage ring;
-//   warp 1      TMEM allocation (512 columns: one 96-column accumulator per
+//   warp 1      TMEM allocation (512 columns: one 64-column accumulator per
 //               block column, 128 columns apart) and the MMAs, issued by one
 //               elected lane while the whole warp runs the loop: per tile and
-//               block column two MMAs, then a commit to that column's
+//               block column four MMAs, then a commit to that column's
 //               accumulator barrier;
 //   warps 2-17  encoders: warp w reads TMEM lane quadrant w % 4 (its 32
-//               tokens) and block column (w - 2) / 4 of the tile with three
+//               tokens) and block column (w - 2) / 4 of the tile with two
 //               tcgen05.ld of 32 columns, releases the accumulator, sums the
 //               parts, then clips, scales, encodes and stores; they also build
 //               the P_i parts of their block column at the start of every strip.
@@ -61,7 +60,6 @@ constexpr int kSlab = kTok * 64;                 // one block column of a tile: 
 constexpr int kXBytes = kCB * kSlab;             // 32 KB
 constexpr int kPPart = 32 * 64;                  // one part of one P_i: 32 output rows x 32 bf16
 constexpr int kPBytes = kCB * kParts * kPPart;   // 24 KB
-constexpr int kAccN = kParts * 32;               // MMA N: the three parts' outputs side by side
 constexpr int kAccStride = 128;                  // TMEM columns between block columns' accumulators
 constexpr int kTmemCols = kCB * kAccStride;      // 512 (the 154 KB of shared memory keeps one CTA per SM)
 constexpr int kEncWarps = 4 * kCB;               // one per (TMEM lane quadrant, block column)
@@ -226,7 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ MMA warp ------------------------------
     // The whole warp runs the loop (its state stays warp-uniform) and one
     // elected lane issues the MMAs and their commits.
-    constexpr uint32_t kIdesc = idesc_bf16(kTok, kAccN);
+    constexpr uint32_t kIdesc64 = idesc_bf16(kTok, 64);  // hi and mid side by side
+    constexpr uint32_t kIdesc32 = idesc_bf16(kTok, 32);  // lo, accumulated onto mid
     const uint64_t db = sdesc_kmajor_sw64(smem_u32(smem + kPOffset));
     const bool leader = elect_one();
     uint32_t strip_count = 0;
@@ -265,7 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // K step kk = bytes 32 kk .. 32 kk + 31 of each 64-byte row; B = the
             // 96 rows of the three parts of this block column's P_i.
             tc_mma_bf16(tmem + (uint32_t)(cb * kAccStride), da + (uint64_t)((cb * kSlab + kk * 32) >> 4),
-                        db + (uint64_t)((cb * kParts * kPPart + kk * 32) >> 4), kIdesc, kk ? 1u : 0u);
+                        db + (uint64_t)((cb * kParts * kPPart + kk * 32) >> 4), kIdesc64, kk ? 1u : 0u);
+            tc_mma_bf16(tmem + (uint32_t)(cb * kAccStride + 32), da + (uint64_t)((cb * kSlab + kk * 32) >> 4),
+                        db + (uint64_t)(((cb * kParts + 2) * kPPart + kk * 32) >> 4), kIdesc32, 1u);
           }
           tc_commit(&acc_full[cb]);  // the encoders may read this block column's results
         }
@@ -317,30 +318,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       tc_fence_after_sync();
-      // The three partial results X hi, X mid, X lo of this block column,
-      // summed as hi + (mid + lo).
+      // X hi and X mid + X lo (added in TMEM) of this block column, summed in fp32.
       const uint32_t tacc = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(cb * kAccStride);
       uint32_t ra[32], rb[32];
-      tmem_ld_32cols(tacc + 32, ra);
-      tmem_ld_32cols(tacc + 64, rb);
+      tmem_ld_32cols(tacc, ra);
+      tmem_ld_32cols(tacc + 32, rb);
       tmem_ld_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[cb]);
       float y[32];
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
         const float2 sv = __fadd2_rn(make_float2(__uint_as_float(ra[j]), __uint_as_float(ra[j + 1])),
                                      make_float2(__uint_as_float(rb[j]), __uint_as_float(rb[j + 1])));
-        y[j] = sv.x;
-        y[j + 1] = sv.y;
-      }
-      tmem_ld_32cols(tacc, ra);
-      tmem_ld_wait();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[cb]);
-#pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 sv = __fadd2_rn(make_float2(__uint_as_float(ra[j]), __uint_as_float(ra[j + 1])),
-                                     make_float2(y[j], y[j + 1]));
         y[j] = sv.x;
         y[j + 1] = sv.y;
       }
