@@ -445,9 +445,14 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA).
+// Arrive on an mbarrier given by its shared::cluster address (possibly in the
+// peer CTA), with the default release at CTA scope.  The one use is the pair
+// GEMM's accumulator hand-over, whose ordering (TMEM reads complete before the
+// leader's next MMAs) comes from tcgen05.wait::ld and the tcgen05 fences around
+// the arrive; a release at cluster scope there waited ~1 us per tile for the
+// SM's operand loads still in flight.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // Tiled TMA loads into this CTA's shared memory whose completion is counted
