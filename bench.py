@@ -51,8 +51,8 @@ CSRC = os.path.join(ROOT, "mxfp4_w4a4_post_block_b200", "csrc")
 # `bench.py --only group --workload layer` (metrics dram__bytes_read.sum, dram__bytes_write.sum),
 # valid only for the kernel sources whose hash is recorded with it: a changed kernel reports null.
 NCU_TRAFFIC = {
-    "k_gemm_pair": {"src": "ca55f85d7e3a22f0", "bytes_per_step": 372391424 + 1235038464},
-    "k_quant_act_tc": {"src": "d0bf26e85803c638", "bytes_per_step": 605475328 + 143213056},
+    "k_gemm_pair": {"src": "a496fbeb3db1df9c", "bytes_per_step": 374014208 + 1235212032},
+    "k_quant_act_tc": {"src": "e53a61cae13ec272", "bytes_per_step": 605399040 + 143117056},
 }
 TRAFFIC_SOURCES = {
     "k_gemm_pair": ("gemm_pair.cu", "ptx.cuh", "kernels.h", "host_util.h", "host_util.cpp"),

@@ -5,7 +5,9 @@
 // neighbouring SMs.  One launch runs one to eight independent products (a
 // table of tensor maps and shapes in the kernel parameters; their tiles form
 // one list), so a batch of linears pays the pipeline fill and drain once.
-// A pair owns a 256 (tokens) x 256 (out-features) tile:
+// A pair owns a 256 (tokens) x 256 (out-features) tile (in a launch whose last
+// round would fill at most half of the clusters, that round's tiles run as
+// 256 x 128 halves on twice as many clusters):
 //   * each CTA loads its own 128 token rows of activation codes and its own
 //     128-row half of the weight tile, so one SM moves 64 bytes of operands per
 //     tensor-core cycle instead of the 96 a single-CTA 128x256 tile needs;
@@ -93,7 +95,7 @@ struct PairCfg {
 // list of pair tiles: problem p's tiles are tile_begin .. tile_begin +
 // tiles_m * tiles_n - 1, row-major over (token tile, out-feature tile).
 struct PairProblem {
-  CUtensorMap tm_a, tm_w, tm_sfa, tm_sfw, tm_out, tm_out_wide;
+  CUtensorMap tm_a, tm_w, tm_w_half, tm_sfa, tm_sfw, tm_out, tm_out_wide;
   int S, M, N;
   int tiles_n;         // pair tiles along out-features
   int tile_begin;      // first tile of this problem in the launch's list
@@ -106,6 +108,8 @@ struct PairLaunch {
   PairProblem prob[kG];
   int count;           // problems in use (1 .. kG)
   int num_tiles;       // tiles of all problems
+  int split_begin;     // tiles from here on run as two 128-column halves (num_tiles: none)
+  int num_units;       // work units: whole tiles before split_begin, then two halves per tile
   unsigned* err;
   int early_weights;   // weights may be read before waiting for the preceding grid
   const float* gs_a;   // NVFP4 per-tensor encode scales (device, nullable: 1); one problem only
@@ -120,6 +124,20 @@ __device__ __forceinline__ int problem_of(const PairLaunch<kG>& g, int t) {
   for (int q = 1; q < kG; ++q)
     if (q < g.count && t >= g.prob[q].tile_begin) p = q;
   return p;
+}
+
+// Work unit u: tile t whole (half < 0), or its out-feature columns
+// [128 half, 128 half + 128) computed as one M=256 x N=128 accumulation.  A
+// launch whose last round of whole tiles would fill at most half of the
+// clusters runs those tiles as halves on twice as many clusters instead.
+struct Unit {
+  int t, half;
+};
+template <int kG>
+__device__ __forceinline__ Unit unit_of(const PairLaunch<kG>& g, int u) {
+  if (u < g.split_begin) return Unit{u, -1};
+  const int v = u - g.split_begin;
+  return Unit{g.split_begin + (v >> 1), v & 1};
 }
 
 template <bool kOutBF16, int kFmt, int kG>
@@ -144,6 +162,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int p = 0; p < g.count; ++p) {
       tma_prefetch_map(&g.prob[p].tm_a);
       tma_prefetch_map(&g.prob[p].tm_w);
+      if (g.split_begin < g.num_tiles) tma_prefetch_map(&g.prob[p].tm_w_half);
       tma_prefetch_map(&g.prob[p].tm_sfa);
       tma_prefetch_map(&g.prob[p].tm_sfw);
       tma_prefetch_map(&g.prob[p].tm_out);
@@ -156,7 +175,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const bool leader = (rank == 0);
   const int cluster_id = blockIdx.x >> 1;
   const int num_clusters = gridDim.x >> 1;
-  const int num_tiles = g.num_tiles;
+  const int num_units = g.num_units;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -184,43 +203,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t t_sfa = tmem + kTileN;
   const uint32_t t_sfb = tmem + kTileN + kStages * kSfaCols;
 
-  // Every role walks this cluster's tiles (cluster_id, cluster_id + num_clusters,
-  // ...) and each tile's K stages in the same order: one sequence of stages
-  // whose ring slot and phase advance by one per stage.
+  // Every role walks this cluster's work units (cluster_id, cluster_id +
+  // num_clusters, ...) and each unit's K stages in the same order: one sequence
+  // of stages whose ring slot and phase advance by one per stage.
   if (warp == 0) {
     // ------------------------------ producer (both CTAs) ------------------------------
     if (lane == 0) {
-      // Cursor over the sequence: tile t of problem p, K step ks, its first rows.
-      int t = cluster_id, ks = 0, p = 0, nks = 0, a_row = 0, w_row = 0;
-      auto enter_tile = [&]() {
-        if (t >= num_tiles) return;
-        p = problem_of(g, t);
-        const int lt = t - g.prob[p].tile_begin;
+      // Cursor over the sequence: unit u (a tile of problem p or its half hf),
+      // K step ks, its first rows.
+      int u = cluster_id, ks = 0, p = 0, hf = -1, nks = 0, a_row = 0, w_row = 0;
+      auto enter_unit = [&]() {
+        if (u >= num_units) return;
+        const Unit w = unit_of(g, u);
+        p = problem_of(g, w.t);
+        hf = w.half;
+        const int lt = w.t - g.prob[p].tile_begin;
         a_row = (lt / g.prob[p].tiles_n) * kTileM + (int)rank * kRowsPerCta;
-        w_row = (lt % g.prob[p].tiles_n) * kTileN;
+        w_row = (lt % g.prob[p].tiles_n) * kTileN + (hf > 0 ? kHalfN : 0);
         nks = g.prob[p].num_kstages;
       };
       auto advance = [&]() {
         if (++ks == nks) {
           ks = 0;
-          t += num_clusters;
-          enter_tile();
+          u += num_clusters;
+          enter_unit();
         }
       };
-      // Bytes one CTA's loads deliver per stage: the code tiles and the scale boxes
-      // (one box of own activation scales, one of two weight row tiles).
-      auto stage_tx = [&](int q) {
-        return (uint32_t)(kABytes + kBBytes) + 3u * (uint32_t)g.prob[q].sf_box_chunks * 256u;
+      // Bytes one CTA's loads deliver per stage: the code tiles (a half unit
+      // loads 64 weight rows per CTA) and the scale boxes (one box of own
+      // activation scales, one of two weight row tiles).
+      auto stage_tx = [&](int q, int h) {
+        return (uint32_t)(kABytes + (h < 0 ? kBBytes : kBBytes / 2)) + 3u * (uint32_t)g.prob[q].sf_box_chunks * 256u;
       };
-      auto issue_weights = [&](int st_idx, int q, int k_step, int wr) {
+      auto issue_weights = [&](int st_idx, int q, int h, int k_step, int wr) {
         uint8_t* st = smem + st_idx * kStageBytes;
         const uint32_t bar = mapa_shared(smem_u32(&full[st_idx]), 0);
+        const CUtensorMap* map = h < 0 ? &g.prob[q].tm_w : &g.prob[q].tm_w_half;
+        const int rows = h < 0 ? kHalfN : kHalfN / 2;
 #pragma unroll
         for (int a = 0; a < kSwAtoms; ++a)
-          tma_load_2d_pair(st + kABytes + a * kSwTile, &g.prob[q].tm_w, bar, k_step * kBKBytes + a * 128,
-                           wr + (int)rank * kHalfN);
+          tma_load_2d_pair(st + kABytes + a * kSwTile, map, bar, k_step * kBKBytes + a * 128, wr + (int)rank * rows);
+        // {2 row tiles} x {sf_box_chunks}; a half unit uses the first row tile
         tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &g.prob[q].tm_sfw, bar, 0, k_step * 2 * C::kAtoms,
-                         wr / kRowsPerCta);  // {2 row tiles} x {sf_box_chunks}
+                         wr / kRowsPerCta);
       };
       auto issue_activations = [&](int st_idx, int q, int k_step, int ar) {
         uint8_t* st = smem + st_idx * kStageBytes;
@@ -232,33 +257,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tma_load_3d_pair(st + kABytes + kBBytes, &g.prob[q].tm_sfa, bar, 0, k_step * 2 * C::kAtoms,
                          ar / kRowsPerCta);
       };
-      enter_tile();
+      enter_unit();
       // When the preceding grid is known not to write the weights (the linear
       // layer's own quantiser), the first ring's weights are loaded before
       // waiting for that grid; the activations always come after the wait.
+      // Otherwise both operands of each stage are requested together, so the
+      // first stage does not queue behind the later stages' weights.
       int pro_p[kStages], pro_ks[kStages], pro_a[kStages];
       int npro = 0;
       if (!g.early_weights) griddep_wait();
-      while (npro < kStages && t < num_tiles) {
-        if (leader) mbar_arrive_expect_tx(&full[npro], 2u * stage_tx(p));
-        issue_weights(npro, p, ks, w_row);
+      while (npro < kStages && u < num_units) {
+        if (leader) mbar_arrive_expect_tx(&full[npro], 2u * stage_tx(p, hf));
+        issue_weights(npro, p, hf, ks, w_row);
+        if (!g.early_weights) issue_activations(npro, p, ks, a_row);
         pro_p[npro] = p;
         pro_ks[npro] = ks;
         pro_a[npro] = a_row;
         ++npro;
         advance();
       }
-      if (g.early_weights) griddep_wait();
-      for (int i = 0; i < npro; ++i) issue_activations(i, pro_p[i], pro_ks[i], pro_a[i]);
+      if (g.early_weights) {
+        griddep_wait();
+        for (int i = 0; i < npro; ++i) issue_activations(i, pro_p[i], pro_ks[i], pro_a[i]);
+      }
       int s = npro % kStages;
       uint32_t ph = npro == kStages ? 1u : 0u;
-      while (t < num_tiles) {
+      while (u < num_units) {
         if (!mbar_wait(&empty[s], ph ^ 1)) {
           set_error(g.err, kErrReleaseTimeout);
           break;
         }
-        if (leader) mbar_arrive_expect_tx(&full[s], 2u * stage_tx(p));
-        issue_weights(s, p, ks, w_row);
+        if (leader) mbar_arrive_expect_tx(&full[s], 2u * stage_tx(p, hf));
+        issue_weights(s, p, hf, ks, w_row);
         issue_activations(s, p, ks, a_row);
         if (++s == kStages) {
           s = 0;
@@ -278,9 +308,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int st_idx = 0;
       uint32_t sph = 0, tile_iter = 0;
       bool ok = true;
-      for (int t = cluster_id; t < num_tiles && ok; t += num_clusters, ++tile_iter) {
-        const int p = problem_of(g, t);
+      for (int u = cluster_id; u < num_units && ok; u += num_clusters, ++tile_iter) {
+        const Unit w = unit_of(g, u);
+        const int p = problem_of(g, w.t);
         const int nks = g.prob[p].num_kstages, N = g.prob[p].N;
+        const int mma_n = w.half < 0 ? kTileN : kTileN / 2;
         for (int ks = 0; ks < nks; ++ks) {
           if (ks == 0) {
             // The accumulator must have been drained by both CTAs' epilogues.
@@ -316,13 +348,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               const uint64_t off = (uint64_t)((j >> 2) * (kSwTile >> 4) + (j & 3) * 2);
               const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
               if constexpr (C::kFp8)
-                tc_mma_pair_mxf8(t_acc, da0 + off, db0 + off, idesc_mxf8(256, kTileN, sf_id, sf_id), tsfa + a * 4,
+                tc_mma_pair_mxf8(t_acc, da0 + off, db0 + off, idesc_mxf8(256, mma_n, sf_id, sf_id), tsfa + a * 4,
                                  tsfb + a * 8, acc);
               else if constexpr (C::kNv)
-                tc_mma_pair_nvf4(t_acc, da0 + off, db0 + off, idesc_nvf4(256, kTileN), tsfa + a * 4, tsfb + a * 8,
+                tc_mma_pair_nvf4(t_acc, da0 + off, db0 + off, idesc_nvf4(256, mma_n), tsfa + a * 4, tsfb + a * 8,
                                  acc);
               else
-                tc_mma_pair_mxf4(t_acc, da0 + off, db0 + off, idesc_mxf4_m256(kTileN, sf_id, sf_id), tsfa + a * 4,
+                tc_mma_pair_mxf4(t_acc, da0 + off, db0 + off, idesc_mxf4_m256(mma_n, sf_id, sf_id), tsfa + a * 4,
                                  tsfb + a * 8, acc);
             }
             tc_commit_pair(&empty[st_idx], 0x3);
@@ -348,9 +380,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int st_idx = 0;
       uint32_t fph = 0;
       bool ok = true;
-      for (int t = cluster_id; t < num_tiles && ok; t += num_clusters) {
-        const int p = problem_of(g, t);
+      for (int u = cluster_id; u < num_units && ok; u += num_clusters) {
+        const Unit w = unit_of(g, u);
+        const int p = problem_of(g, w.t);
         const int nks = g.prob[p].num_kstages, N = g.prob[p].N, box_chunks = g.prob[p].sf_box_chunks;
+        const bool whole = w.half < 0;  // a half unit's N = 128 columns need one weight row tile
         for (int ks = 0; ks < nks; ++ks) {
           if (!mbar_wait_warp(&full[st_idx], fph)) {
             if (issuer) set_error(g.err, kErrDataTimeout);
@@ -372,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               // weight-scale box is {2 row tiles} x {sf_box_chunks}: row tile r, atom a at
               // r * sf_box_chunks * 256 + a * 512
               tc_cp_pair_32x128b_warpx4(tsfb + a * 8, dsfb + off);
-              tc_cp_pair_32x128b_warpx4(tsfb + a * 8 + 4, dsfb1 + off);
+              if (whole) tc_cp_pair_32x128b_warpx4(tsfb + a * 8 + 4, dsfb1 + off);
             }
             tc_commit_pair_local(&sf_ready[st_idx]);
           }
@@ -388,7 +422,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------ epilogue (both CTAs) ------------------------------
     const int ew = warp - 2;
     const int quad = warp & 3;                // TMEM lanes 32*quad .. 32*quad+31
-    const int col0 = (ew >> 2) * 128;          // this warp's 128 accumulator columns
     uint8_t* box = smem + kStages * kStageBytes + ew * kBoxBytes;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     uint32_t tile_iter = 0;
@@ -404,11 +437,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if constexpr (C::kNv) return __fmul_rn(__uint_as_float(bits), alpha);
       return __uint_as_float(bits);
     };
-    for (int t = cluster_id; t < num_tiles; t += num_clusters, ++tile_iter) {
-      const PairProblem& P = g.prob[problem_of(g, t)];
-      const int lt = t - P.tile_begin;
+    for (int u = cluster_id; u < num_units; u += num_clusters, ++tile_iter) {
+      const Unit w = unit_of(g, u);
+      const PairProblem& P = g.prob[problem_of(g, w.t)];
+      const int lt = w.t - P.tile_begin;
+      // This warp's accumulator columns: half of the unit's 256 (whole tile) or 128.
+      const int wcols = w.half < 0 ? 128 : 64;
+      const int col0 = (ew >> 2) * wcols;
       const int row0 = (lt / P.tiles_n) * kTileM + (int)rank * kRowsPerCta + 32 * quad;
-      const int n0 = (lt % P.tiles_n) * kTileN + col0;
+      const int n0 = (lt % P.tiles_n) * kTileN + (w.half > 0 ? kHalfN : 0) + col0;
       if (!mbar_wait_warp(acc_full, tile_iter & 1)) {
         if (lane == 0) set_error(g.err, kErrMmaTimeout);
         break;
@@ -418,16 +455,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t v[4][32];
       const uint32_t taddr = t_acc + ((uint32_t)(32 * quad) << 16) + col0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_32cols(taddr + 32 * c, v[c]);
+      for (int c = 0; c < 4; ++c)
+        if (32 * c < wcols) tmem_ld_32cols(taddr + 32 * c, v[c]);
       tmem_ld_wait();
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // TMEM free for the next tile
 
-      const bool last_tile = (t + num_clusters >= num_tiles);
-      if (last_tile) {
-        // Nothing is loaded after the last tile, and its MMAs have completed,
-        // so the operand stages are idle: each warp stages its whole 32 x 128
+      const bool last_unit = (u + num_clusters >= num_units);
+      if (last_unit) {
+        // Nothing is loaded after the last unit, and its MMAs have completed,
+        // so the operand stages are idle: each warp stages its whole 32-row
         // block there (128-byte rows, 128-byte swizzle) and issues all of its
         // stores at once instead of one small box at a time.
         if (store_pending) {
@@ -439,6 +477,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint8_t* wide = smem + ew * (kWideBoxes * 4096);
 #pragma unroll
         for (int bx = 0; bx < kWideBoxes; ++bx) {
+          if (bx * kWideCols >= wcols) break;
           uint8_t* wrow = wide + bx * 4096 + lane * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -460,7 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0 && row0 < P.S) {
           for (int bx = 0; bx < kWideBoxes; ++bx) {
             const int x = n0 + bx * kWideCols;
-            if (x < P.M) tma_store_2d(&P.tm_out_wide, wide + bx * 4096, x, row0);
+            if (bx * kWideCols < wcols && x < P.M) tma_store_2d(&P.tm_out_wide, wide + bx * 4096, x, row0);
           }
           tma_store_commit();
         }
@@ -475,6 +514,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int sw = (lane >> 2) & 1;
 #pragma unroll
       for (int bx = 0; bx < 128 / kColsPerBox; ++bx) {
+        if (bx * kColsPerBox >= wcols) break;
         if (store_pending) {
           if (lane == 0) tma_store_wait_read_all();
           __syncwarp();
@@ -539,6 +579,10 @@ bool fill_problem(const GemmLaunch& L, int tile_begin, PairProblem* P) {
   if (!make_map_2d(&P->tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_codes, row_bytes, (uint64_t)L.M, row_bytes, 128,
                    kHalfN, CU_TENSOR_MAP_SWIZZLE_128B))
     return false;
+  // Half units: 64 weight rows per CTA.
+  if (!make_map_2d(&P->tm_w_half, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.w_codes, row_bytes, (uint64_t)L.M, row_bytes, 128,
+                   kHalfN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+    return false;
   // Scale tiles as {256-byte chunks, chunks per row tile, row tiles}; one box = the stage's K
   // atoms (x 2 row tiles for the weights), clamped to the row tile when all of K is shorter.
   const uint64_t chunks = sf_row_tile_bytes / 256;
@@ -581,6 +625,15 @@ cudaError_t launch_pair_impl(const GemmLaunch* Ls, int count) {
   }
   g.count = count;
   g.num_tiles = tiles;
+  // A last round of whole tiles that would occupy at most half of the clusters
+  // runs as half tiles (M = 256 x N = 128) on twice as many: that round then
+  // takes the time of half a tile's MMAs and operand stream instead of a whole
+  // one's.  Each output element is still one K accumulation in one MMA chain.
+  const int max_clusters = sm_count() / 2;
+  const int rem = tiles % max_clusters;
+  const bool split = rem > 0 && 2 * rem <= max_clusters;
+  g.split_begin = split ? tiles - rem : tiles;
+  g.num_units = split ? tiles + rem : tiles;
   g.err = Ls[0].err;
   g.early_weights = Ls[0].weights_ready ? 1 : 0;
   g.gs_a = Ls[0].gs_a;
@@ -595,8 +648,7 @@ cudaError_t launch_pair_impl(const GemmLaunch* Ls, int count) {
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int max_clusters = sm_count() / 2;
-  const int clusters = tiles < max_clusters ? tiles : max_clusters;
+  const int clusters = g.num_units < max_clusters ? g.num_units : max_clusters;
   // Launched as a programmatic dependent of the preceding grid: set-up and
   // weight loads overlap the quantiser's tail; activations wait for it.
   cudaLaunchConfig_t cfg = {};

@@ -200,6 +200,45 @@ def test_grouped_gemm_equals_batq_gemm_mxfp4(case):
         assert torch.equal(gm["out"], ref), f"product {i} {shapes[i]}"
 
 
+def _pair_launch_splits(tiles):
+    """The pair GEMM's rule: a last round of whole tiles that fills at most half of the clusters runs
+    as 256 x 128 half tiles."""
+    clusters = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    rem = tiles % clusters
+    return 0 < rem and 2 * rem <= clusters
+
+
+def test_half_tile_last_round_equals_whole_tiles():
+    """down_proj alone (16 x 16 = 256 pair tiles, 34 in the last round on 74 clusters) runs its last
+    round as half tiles; grouped with a 20-tile companion (276 tiles, 54 in the last round) the same
+    tiles run whole.  Each output element is one K accumulation either way: the bits must agree, for
+    the companion (split when alone) too."""
+    g = torch.Generator(device="cuda").manual_seed(81)
+    shapes = [(4096, 4096, 12288), (1024, 1280, 4096)]
+    tiles = [-(-S // 256) * -(-M // 256) for S, M, _ in shapes]
+    assert _pair_launch_splits(tiles[0]) and _pair_launch_splits(tiles[1])
+    assert not _pair_launch_splits(sum(tiles))
+    gemms, refs = [], []
+    for S, M, N in shapes:
+        a, sa = BQ.empty_act_buffers(S, N)
+        a.random_(0, 256, generator=g)
+        sa.random_(116, 136, generator=g)
+        w, sw = BQ.empty_act_buffers(M, N)
+        w.random_(0, 256, generator=g)
+        sw.random_(116, 136, generator=g)
+        out = torch.full((S, M), float("nan"), dtype=torch.float32, device="cuda")
+        gemms.append(dict(a_codes=a, a_scales=sa, w_codes=w, w_scales=sw, S=S, M=M, N=N, out=out))
+        ref = torch.full_like(out, float("nan"))
+        BQ.batq_gemm_mxfp4(a, sa, w, sw, S, M, N, ref)
+        refs.append(ref)
+    BQ.batq_gemm_mxfp4_grouped(gemms)
+    torch.cuda.synchronize()
+    assert BQ.batq_device_error() == 0
+    for i, (gm, ref) in enumerate(zip(gemms, refs)):
+        assert not torch.isnan(ref).any(), f"product {i}: output not fully written"
+        assert torch.equal(gm["out"], ref), f"product {i} {shapes[i]}"
+
+
 def test_layer_workload_as_the_bench_runs_it():
     """The seven S = 8192 linears of the layer workload (q, k, v, o, gate, up, down) through one grouped
     call, as the bench times them: every output, code and scale equals batq_linear's bit for bit (each
