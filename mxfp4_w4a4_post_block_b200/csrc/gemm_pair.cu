@@ -23,8 +23,10 @@
 //   * the MMA and scale-copy warps run their stage loops warp-wide (the loop
 //     state stays warp-uniform) and one elected lane issues; a loop run by
 //     lane 0 alone spent several more instructions per MMA or copy;
-//   * eight epilogue warps per CTA read their 128 accumulator columns into
-//     registers, release TMEM for the next tile at once, and write the output
+//   * eight epilogue warps per CTA read their 128 accumulator columns (64 of a
+//     half tile) into registers, release TMEM for the next tile at once (the
+//     arrive on the leader's barrier is a CTA-scope release: a cluster-scope
+//     one waited for the SM's operand loads in flight), and write the output
 //     through a small per-warp shared-memory box (32 rows x 32 bytes) with TMA
 //     stores while the next tile's MMAs run;
 //   * three 70 KB stages (two 128-byte swizzle tiles of K each, eight MMAs
