@@ -305,6 +305,20 @@ def test_mma_scale_layout_is_a_bijection():
         assert off.max() < O.mma_layout_bytes(rows, k)
 
 
+def test_mma_scale_layout_worked_entries():
+    """Entries worked by hand from the tcgen05 block-scale atom: a 512-byte atom holds 128 rows x 4
+    scales as 32 lines of 16 bytes, line i carrying rows i, i + 32, i + 64, i + 96 (4 bytes each, one
+    per block column); atoms run along K within a 128-row tile, then tile after tile (k padded to a
+    multiple of 4).  A layout that is one-to-one but swaps any of these roles fails here."""
+    worked = [  # (row, kb, k, offset)
+        (0, 0, 8, 0), (1, 0, 8, 16), (32, 0, 8, 4), (33, 2, 8, 22), (96, 3, 8, 15), (127, 3, 8, 511),
+        (0, 4, 8, 512), (5, 7, 8, 512 + 80 + 3), (128, 0, 8, 1024), (130, 5, 8, 1569),
+        (128, 9, 10, 2561), (255, 11, 10, 3 * 512 + 2 * 512 + 511),
+    ]
+    for row, kb, k, off in worked:
+        assert int(O.mma_scale_offset(row, kb, k)) == off, (row, kb, k)
+
+
 # ------------------------------------------------------- weight side ---------
 
 def test_gauss_jordan_inverse_matches_kronecker_inverse():
